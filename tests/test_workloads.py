@@ -1,0 +1,77 @@
+"""The seeded input recipe: deterministic, head-addressable, right shapes and
+distributions."""
+import numpy as np
+import torch
+
+import workloads as W
+
+
+def test_tiny_shapes_and_recipe():
+    w = W.WORKLOADS["tiny_fp32"]
+    x = W.prefill_inputs(w, seed=0)
+    assert x["q"].shape == (256, 2, 64) and x["q"].dtype == torch.float32
+    assert x["v"].shape == (256, 2, 64)
+    assert x["g"].shape == (256, 2) and x["g"].dtype == torch.float32
+    assert x["state_in"] is None
+    assert x["cu_seqlens"].tolist() == [0, 256]
+    n = torch.linalg.norm(x["k"].double(), dim=-1)
+    assert torch.allclose(n, torch.ones_like(n), atol=1e-6)
+    assert float(x["g"].max()) < 0.0
+    a = torch.exp(x["g"].double())
+    # alpha = sigmoid(N(3,1)): mean near E[sigmoid(3 + z)] ~ 0.93
+    assert 0.88 < float(a.mean()) < 0.97
+    b = x["beta"].double()
+    assert 0.0 < float(b.min()) and float(b.max()) < 1.0
+
+
+def test_deterministic_and_head_subsets():
+    w = W.WORKLOADS["prefill_bf16"]
+    w = W.Workload(**{**w.__dict__, "T": 5000})        # ragged vs the 4096 block
+    full = W.prefill_inputs(w, seed=3)
+    again = W.prefill_inputs(w, seed=3)
+    sub = W.prefill_inputs(w, seed=3, heads=[5, 11])
+    for name in ("q", "k", "v", "g", "beta"):
+        assert torch.equal(full[name], again[name])
+        assert torch.equal(full[name][:, [5, 11]], sub[name])
+    other = W.prefill_inputs(w, seed=4, heads=[5])
+    assert not torch.equal(other["q"], sub["q"][:, :1])
+    assert full["q"].dtype == torch.bfloat16
+
+
+def test_logsoftplus_gate_range():
+    w = W.WORKLOADS["prefill_bf16"]
+    x = W.prefill_inputs(W.Workload(**{**w.__dict__, "T": 4096}), seed=0, heads=[0])
+    g = x["g"].double()
+    assert float(g.max()) <= 0.0 and float(g.min()) > -0.5
+    assert abs(float(torch.exp(g).mean()) - 0.965) < 0.01
+
+
+def test_varlen_lengths_and_state():
+    w = W.WORKLOADS["varlen_bf16"]
+    lens = W.seqlens(w, seed=0)
+    assert len(lens) == 8 and lens.min() >= 1024 and lens.max() <= 32768
+    x = W.prefill_inputs(w, seed=0, heads=[0])
+    cu = x["cu_seqlens"].numpy()
+    assert cu[0] == 0 and np.all(np.diff(cu) == lens)
+    assert x["state_in"].shape == (8, 1, 128, 128)
+    assert abs(float(x["state_in"].std()) - 0.02) < 1e-3
+
+
+def test_decode_tokens():
+    w = W.WORKLOADS["decode_bf16"]
+    t0 = W.decode_tokens(w, 0, seed=0)
+    t1 = W.decode_tokens(w, 1, seed=0)
+    assert t0["q"].shape == (64, 16, 128) and t0["q"].dtype == torch.bfloat16
+    assert not torch.equal(t0["k"], t1["k"])
+    sub = W.decode_tokens(w, 1, seed=0, heads=[2, 7])
+    for name in ("q", "k", "v", "g", "beta"):
+        assert torch.equal(t1[name][:, [2, 7]], sub[name])
+    s = W.decode_state(w, seed=0, heads=[3])
+    assert torch.equal(W.decode_state(w, seed=0)[:, [3]], s)
+
+
+def test_random_prefill_allows_empty():
+    x = W.random_prefill([0, 3, 0, 70], H=2, dk=64, dv=64, dtype=torch.float32, seed=1, state_std=0.02)
+    assert x["cu_seqlens"].tolist() == [0, 0, 3, 3, 73]
+    assert x["q"].shape == (73, 2, 64)
+    assert x["state_in"].shape == (4, 2, 64, 64)
