@@ -1,0 +1,386 @@
+#!/usr/bin/env python
+"""Benchmark of the Gated DeltaNet hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+One step = one gdn_prefill call over the bf16 prefill workload (1 sequence,
+16 heads, 8192 tokens, d_k = d_v = 128, chunk 64, zero initial state) with
+its inputs resident in HBM.  The L2 (126 MB) is flushed before every step by
+writing a 512 MiB buffer; only the prefill launches are inside the CUDA-event
+intervals.  The same run also times the decode step (64 sequences x 16 heads,
+fp32 state, one bf16 token each; L2 flushed before every step) and an
+end-to-end prefill through the public API with pinned host buffers (inputs
+copied in and out, result read back, inside the timed region).
+
+Multi-GPU (torchrun): every rank runs its own replica of the workload (the
+units are independent sequences; there is no data-path collective); the
+reported time is the max over ranks and ``value`` counts the tokens of all
+ranks ("scaling": "weak").
+
+``--impl reference`` times the fp64 CPU oracle (the only other implementation
+of the method) on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 512 << 20
+
+PREFILL = W.WORKLOADS["prefill_bf16"]
+DECODE = W.WORKLOADS["decode_bf16"]
+
+
+def peaks():
+    if os.path.exists(PEAKS_FILE):
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ algorithmic work
+
+def prefill_bytes(T, H, dk, dv, num_seqs, with_state_in, elem=2):
+    """Bytes the prefill must move at minimum: q, k, v, g, beta in; out and
+    the final state out (and the initial state in, when given)."""
+    per_tok_head = (2 * dk + dv) * elem + 2 * 4 + dv * elem
+    state = num_seqs * H * dv * dk * 4
+    return T * H * per_tok_head + state * (2 if with_state_in else 1)
+
+
+def prefill_flops(T, H, d, C=64):
+    """Algorithmic flops per token-head of the chunkwise form (triangles
+    counted once): intra-chunk 5 C d, state 6 d^2, solve C^2 / 3."""
+    return T * H * (5 * C * d + 6 * d * d + C * C / 3.0)
+
+
+def decode_bytes(B, H, dk, dv, elem=2):
+    return B * H * (2 * dv * dk * 4 + (2 * dk + dv) * elem + 8 + dv * elem)
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi sampling during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.idx)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            p = [x.strip() for x in ln.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                mx.append(float(p[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, p[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ distributed
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    if world != n_gpus:
+        print("warning: --gpus %d but WORLD_SIZE %d" % (n_gpus, world), file=sys.stderr)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ native arm
+
+def run_native(args):
+    import linear_attention_vlm_b200 as gdn
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    pk, pk_kind = peaks()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # ---- prefill inputs (seed per rank: independent replicas)
+    w = PREFILL
+    host = W.prefill_inputs(w, seed=rank)
+    T, H, dk, dv = w.T, w.H, w.dk, w.dv
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in host.items()}
+    out = torch.empty((T, H, dv), dtype=w.dtype, device=dev)
+    st_out = torch.empty((1, H, dv, dk), dtype=torch.float32, device=dev)
+    ws_bytes = gdn.gdn_prefill_workspace_size(1, T, H, dk, dv, w.chunk, w.dtype)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    launches_per_prefill = gdn.gdn_prefill_kernel_count(1, T, H, dk, dv, w.chunk, w.dtype)
+
+    def prefill_once():
+        gdn.gdn_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], None, None, out=out,
+                        state_out=st_out, workspace=ws)
+
+    # ---- decode inputs
+    dw = DECODE
+    S = W.decode_state(dw, seed=rank).to(dev)
+    ntok = args.steps + args.warmup
+    toks = [{k: v.to(dev) for k, v in W.decode_tokens(dw, i % dw.steps, seed=rank).items()}
+            for i in range(min(ntok, 64))]
+    dout = torch.empty((dw.num_seqs, dw.H, dw.dv), dtype=dw.dtype, device=dev)
+
+    def decode_once(i):
+        t = toks[i % len(toks)]
+        gdn.gdn_decode_step(t["q"], t["k"], t["v"], t["g"], t["beta"], S, S, out=dout)
+
+    # ---- e2e buffers (pinned host, fresh device copies each step)
+    pin = {k: v.pin_memory() for k, v in host.items() if isinstance(v, torch.Tensor) and k != "cu_seqlens"}
+    out_h = torch.empty((T, H, dv), dtype=w.dtype).pin_memory()
+    st_h = torch.empty((1, H, dv, dk), dtype=torch.float32).pin_memory()
+    dbuf = {k: torch.empty_like(v, device=dev) for k, v in pin.items()}
+    h2d = sum(v.numel() * v.element_size() for v in pin.values())
+    d2h = out_h.numel() * out_h.element_size() + st_h.numel() * st_h.element_size()
+
+    def e2e_once():
+        for k, v in pin.items():
+            dbuf[k].copy_(v, non_blocking=True)
+        o, s = gdn.gdn_prefill(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"], None,
+                               None, out=out, state_out=st_out, workspace=ws)
+        out_h.copy_(o, non_blocking=True)
+        st_h.copy_(s, non_blocking=True)
+
+    # ---- warm-up
+    for i in range(args.warmup):
+        prefill_once()
+        decode_once(i)
+        e2e_once()
+    torch.cuda.synchronize()
+
+    def timed(fn, steps, do_flush=True):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        for i in range(steps):
+            if do_flush:
+                flush.zero_()
+            evs[i][0].record(stream)
+            fn(i)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        ms = [a.elapsed_time(b) for a, b in evs]
+        return sum(ms) / len(ms)
+
+    K = args.steps
+    with ClockSampler(local) as clk:
+        t_wall0 = time.time()
+        ms_prefill = timed(lambda i: prefill_once(), K)
+        ms_decode = timed(decode_once, K)
+        ms_e2e = timed(lambda i: e2e_once(), max(3, K // 10), do_flush=False)
+        wall = time.time() - t_wall0
+    ms_prefill = max_over_ranks(ms_prefill, world)
+    ms_decode = max_over_ranks(ms_decode, world)
+    ms_e2e = max_over_ranks(ms_e2e, world)
+
+    tokens = T * world
+    value = tokens / (ms_prefill * 1e-3)
+    pbytes = prefill_bytes(T, H, dk, dv, 1, with_state_in=False)
+    pflops = prefill_flops(T, H, dk)
+    ach_gbs = pbytes / (ms_prefill * 1e-3) / 1e9
+    dbytes = decode_bytes(dw.num_seqs, dw.H, dw.dk, dw.dv)
+    d_gbs = dbytes / (ms_decode * 1e-3) / 1e9
+    hbm = pk["hbm_gbs"]
+    line = {
+        "metric": "GDN prefill tokens/s and decode tokens/s on 1 B200; % of TC / HBM roofline",
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": ms_prefill,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; q,k L2-normalised N(0,1), v N(0,1), beta=sigmoid(N(0,1)), "
+                "log alpha=-0.05 softplus(N(0,1)))",
+        "config": {"workload": "prefill_bf16: B=1, H=16, T=8192, d_k=d_v=128, chunk=64, "
+                               "zero initial state, fp32 state",
+                   "global_batch": world, "seq_len": T, "heads": H, "head_dim": dk,
+                   "parallelism": "replicas x%d (independent sequences)" % world,
+                   "l2": "flushed before every step (512 MiB write)"},
+        "roofline": {"kernel": "gdn_prefill (all %d launches of one call)" % launches_per_prefill,
+                     "bound": "hbm", "achieved": ach_gbs, "peak": hbm, "unit": "GB/s",
+                     "frac": ach_gbs / hbm, "traffic": None,
+                     "peak_source": pk_kind,
+                     "algorithmic_bytes": pbytes, "algorithmic_flops": pflops,
+                     "tensor_frac": (pflops / (ms_prefill * 1e-3) / 1e12) / pk["bf16_tflops"]},
+        "decode": {"metric": "decode tokens/s (64 sequences x 16 heads, one token each)",
+                   "value": dw.num_seqs * world / (ms_decode * 1e-3), "unit": "tokens/s",
+                   "ms_per_step": ms_decode,
+                   "roofline": {"kernel": "gdn_decode_kernel", "bound": "hbm",
+                                "achieved": d_gbs, "peak": hbm, "unit": "GB/s",
+                                "frac": d_gbs / hbm, "traffic": None,
+                                "algorithmic_bytes": dbytes}},
+        "e2e": {"value": tokens / (ms_e2e * 1e-3), "unit": "tokens/s",
+                "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": K * launches_per_prefill + K + max(3, K // 10) * launches_per_prefill,
+        "clocks": clk.summary(),
+        "timed_wall_s": wall,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ oracle arm
+
+def _oracle_sample(tokens, seed=0):
+    w = W.Workload(**{**PREFILL.__dict__, "T": tokens})
+    x = W.prefill_inputs(w, seed=seed)
+    f = lambda t: t.to(torch.float64).numpy()
+    return (f(x["q"]), f(x["k"]), f(x["v"]), f(x["g"]), f(x["beta"]))
+
+
+def cpu_baseline(tokens=8192):
+    import oracle
+    q, k, v, g, b = _oracle_sample(tokens)
+    n = oracle.default_threads()
+    t0 = time.perf_counter()
+    oracle.prefill(q, k, v, g, b, None, None, nthreads=n)
+    dt = time.perf_counter() - t0
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": min(n, PREFILL.H), "kind": "oracle",
+            "sample": "first %d tokens of the prefill_bf16 workload, all 16 heads (%.1f s)" % (tokens, dt)}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    tokens = 256
+    q, k, v, g, b = _oracle_sample(tokens)
+    n = oracle.default_threads()
+    for _ in range(args.warmup):
+        oracle.prefill(q, k, v, g, b, None, None, nthreads=n)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.prefill(q, k, v, g, b, None, None, nthreads=n)
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * sum(times) / len(times)
+    value = tokens / (ms * 1e-3)
+    sample = "first %d tokens of the prefill_bf16 workload, all 16 heads, per step" % tokens
+    line = {
+        "impl": "reference",
+        "metric": "GDN prefill tokens/s and decode tokens/s on 1 B200; % of TC / HBM roofline",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "prefill_bf16: B=1, H=16, T=8192, d_k=d_v=128, chunk=64 "
+                               "(bounded sample per step)", "seq_len": tokens},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": min(n, PREFILL.H),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_native(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,147 @@
+/*
+ * gdn.h -- C ABI of the B200 Gated DeltaNet hot path (libgdn.so).
+ *
+ * The operation.  InfiniteVL's linear-complexity token mixer is Gated
+ * DeltaNet (InfiniteVL explainer page, "Gated DeltaNet" concept box and
+ * "Building Blocks": a fixed-size memory matrix per head, a gate on the old
+ * memory, an erase along the key, a write, a read with the query; 16 heads
+ * per layer, "Step 2").  Per sequence and head, token by token:
+ *
+ *     alpha_t = exp(g_t)
+ *     S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t = S_t q_t                       (read-out after the write)
+ *
+ * S is d_v x d_k (fp32).  Nothing else is applied: no 1/sqrt(d_k) scale, no
+ * L2 norm, no short convolution, no output gate -- the caller passes q, k, v
+ * (normalised as it wishes), g = log(alpha) and beta.
+ *
+ * Streaming with a carried state (InfiniteVL project page, "Accelerated
+ * Streaming Inference": the linear memory state is updated on the fly with a
+ * constant-size cache) is the state_in / state_out pair of gdn_prefill:
+ * running a sequence in segments with the state carried gives the result of
+ * one run.  gdn_decode_step is the same recurrence for one token per
+ * sequence.
+ *
+ * Conventions shared by every entry point:
+ *  - All data pointers are DEVICE pointers (cu_seqlens and the workspace
+ *    included).  The caller owns every buffer; the library allocates nothing
+ *    and keeps no pointer after a call returns.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
+ *    is the legacy default stream).  Host-side argument errors are returned
+ *    before anything is enqueued.  A launch failure returns GDN_ERR_CUDA.
+ *    The library never synchronises the device.
+ *  - Layouts are contiguous and row-major.  Every base pointer must be 16-byte
+ *    aligned (GDN_ERR_INVALID_ARG otherwise).
+ *  - Inputs are never written.
+ *  - The kernels require finite inputs, g <= 0 and beta in [0, 1]; the sum of g
+ *    over any 64 consecutive tokens of a sequence must stay above -80 (the
+ *    chunkwise prefill forms exp(G_r - G_i) inside a chunk).  Nothing on the
+ *    device checks this; results for other inputs are unspecified.
+ *
+ * Thread safety: entry points keep no mutable global state apart from a
+ * one-time per-device kernel attribute set-up, and may be called from several
+ * host threads on different streams.
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes of every entry point. */
+typedef enum gdn_status {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, bad cu_seqlens length */
+    GDN_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement (dk, dv, chunk, dtype) */
+    GDN_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed */
+    GDN_ERR_WORKSPACE = 5      /* workspace NULL or smaller than gdn_prefill_workspace_size() */
+} gdn_status;
+
+/* Storage type of q, k, v and out.  g, beta and the state are always fp32. */
+typedef enum gdn_dtype {
+    GDN_F32 = 0,               /* fp32 in and out; fp32 arithmetic throughout (SIMT) */
+    GDN_BF16 = 1               /* bf16 in and out; bf16 tensor-core operands, fp32 accumulation and state */
+} gdn_dtype;
+
+/*
+ * Bytes of device workspace gdn_prefill needs for these sizes (0 is possible).
+ * Pure host arithmetic; never touches the device.  Returns 0 for arguments
+ * gdn_prefill would reject.
+ */
+size_t gdn_prefill_workspace_size(int num_seqs, int64_t total_tokens, int H,
+                                  int dk, int dv, int chunk, int dtype);
+
+/*
+ * Chunkwise-parallel prefill over a packed batch of num_seqs sequences.
+ *
+ *   q, k        [total_tokens, H, dk]   dtype
+ *   v           [total_tokens, H, dv]   dtype
+ *   g, beta     [total_tokens, H]       fp32  (g = log alpha)
+ *   state_in    [num_seqs, H, dv, dk]   fp32, or NULL for a zero initial state
+ *   out         [total_tokens, H, dv]   dtype (written)
+ *   state_out   [num_seqs, H, dv, dk]   fp32 final states (written), or NULL
+ *   cu_seqlens  [num_seqs + 1]          int32, device; cu_seqlens[0] = 0,
+ *               non-decreasing, cu_seqlens[num_seqs] = total_tokens; empty
+ *               sequences are allowed (their state_out = state_in).  NULL means
+ *               num_seqs sequences of total_tokens / num_seqs tokens each
+ *               (must divide exactly).
+ *   chunk       64 (the only chunk length implemented)
+ *   workspace   device scratch of at least gdn_prefill_workspace_size() bytes
+ *               (may be NULL when that size is 0); contents need not be
+ *               initialised and are garbage afterwards.
+ *
+ * state_out may equal state_in exactly (in-place update); other overlaps, and
+ * any overlap of out with an input, are not allowed.  Supported: dk = dv in
+ * {64, 128}; dtype GDN_F32 or GDN_BF16.  total_tokens may be 0 (nothing is
+ * launched except the state copy).  The device contents of cu_seqlens are
+ * trusted (not validated).
+ */
+int gdn_prefill(const void *q, const void *k, const void *v, const float *g,
+                const float *beta, const float *state_in, void *out,
+                float *state_out, const int32_t *cu_seqlens, int num_seqs,
+                int64_t total_tokens, int H, int dk, int dv, int chunk,
+                int dtype, void *workspace, size_t workspace_bytes,
+                void *stream);
+
+/*
+ * One recurrent decode step: one new token for each of B sequences.
+ *
+ *   q, k        [B, H, dk]   dtype
+ *   v           [B, H, dv]   dtype
+ *   g, beta     [B, H]       fp32
+ *   state_in    [B, H, dv, dk] fp32 (read)
+ *   state_out   [B, H, dv, dk] fp32 (written); may equal state_in (in place)
+ *   out         [B, H, dv]   dtype (written)
+ *
+ * Reads and writes each state exactly once (bandwidth bound).  Supported:
+ * dk = dv in {64, 128}; dtype GDN_F32 or GDN_BF16.  B = 0 is a no-op.
+ */
+int gdn_decode_step(const void *q, const void *k, const void *v,
+                    const float *g, const float *beta, const float *state_in,
+                    float *state_out, void *out, int B, int H, int dk, int dv,
+                    int dtype, void *stream);
+
+/*
+ * Number of kernel launches gdn_prefill makes for these sizes (0 for
+ * arguments it would reject).  Pure host arithmetic; lets callers account
+ * for the library's launches inside a CUDA graph or a timed region.
+ */
+int gdn_prefill_kernel_count(int num_seqs, int64_t total_tokens, int H, int dk, int dv,
+                             int chunk, int dtype);
+
+/* Static, human-readable name of a gdn_status value. */
+const char *gdn_status_string(int status);
+
+/* Text of the most recent CUDA error seen by this host thread inside the
+ * library ("" if none).  Valid until the next call on this thread. */
+const char *gdn_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

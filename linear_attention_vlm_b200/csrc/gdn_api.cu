@@ -1,0 +1,121 @@
+// Host side of the C ABI declared in include/gdn.h: argument validation,
+// workspace sizing and dispatch to the kernels.  No allocation, no device
+// synchronisation.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "gdn.h"
+#include "gdn_internal.h"
+
+namespace {
+
+thread_local char g_last_cuda_error[256] = "";
+
+int cuda_fail(cudaError_t e) {
+    snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(e),
+             cudaGetErrorString(e));
+    return GDN_ERR_CUDA;
+}
+
+bool misaligned(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+bool shape_supported(int dk, int dv) { return dk == dv && (dk == 64 || dk == 128); }
+
+// Common validation of gdn_prefill's arguments (without workspace).
+int check_prefill(const void *q, const void *k, const void *v, const float *g,
+                  const float *beta, const float *state_in, const void *out,
+                  const float *state_out, const int32_t *cu_seqlens, int num_seqs,
+                  int64_t total_tokens, int H, int dk, int dv, int chunk, int dtype) {
+    if (num_seqs < 1 || H < 1 || total_tokens < 0 || dk < 1 || dv < 1) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (chunk != gdn::kChunk || !shape_supported(dk, dv)) return GDN_ERR_UNSUPPORTED;
+    if ((int64_t)num_seqs * H > (int64_t)INT32_MAX / 2) return GDN_ERR_INVALID_ARG;
+    if (total_tokens > 0 && (!q || !k || !v || !g || !beta || !out)) return GDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, state_in, out, state_out, cu_seqlens};
+    for (const void *p : ptrs)
+        if (p && misaligned(p)) return GDN_ERR_INVALID_ARG;
+    if (!cu_seqlens && total_tokens % num_seqs != 0) return GDN_ERR_INVALID_ARG;
+    if (state_out && state_in && state_out != state_in) {
+        const size_t bytes = (size_t)num_seqs * H * dv * dk * sizeof(float);
+        const char *a = reinterpret_cast<const char *>(state_in);
+        const char *b = reinterpret_cast<const char *>(state_out);
+        if (a < b + bytes && b < a + bytes) return GDN_ERR_INVALID_ARG;   // partial overlap
+    }
+    return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *gdn_status_string(int status) {
+    switch (status) {
+        case GDN_OK: return "GDN_OK";
+        case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG: invalid argument";
+        case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: shape, chunk or dtype not implemented";
+        case GDN_ERR_CUDA: return "GDN_ERR_CUDA: CUDA runtime error";
+        case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE: workspace missing or too small";
+        default: return "unknown gdn_status";
+    }
+}
+
+const char *gdn_last_cuda_error(void) { return g_last_cuda_error; }
+
+size_t gdn_prefill_workspace_size(int num_seqs, int64_t total_tokens, int H, int dk, int dv,
+                                  int chunk, int dtype) {
+    if (num_seqs < 1 || H < 1 || total_tokens < 0) return 0;
+    if (chunk != gdn::kChunk || !shape_supported(dk, dv)) return 0;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return 0;
+    return 0;
+}
+
+int gdn_prefill_kernel_count(int num_seqs, int64_t total_tokens, int H, int dk, int dv,
+                             int chunk, int dtype) {
+    if (num_seqs < 1 || H < 1 || total_tokens < 0) return 0;
+    if (chunk != gdn::kChunk || !shape_supported(dk, dv)) return 0;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return 0;
+    return 1;
+}
+
+int gdn_prefill(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                const float *state_in, void *out, float *state_out, const int32_t *cu_seqlens,
+                int num_seqs, int64_t total_tokens, int H, int dk, int dv, int chunk, int dtype,
+                void *workspace, size_t workspace_bytes, void *stream) {
+    int st = check_prefill(q, k, v, g, beta, state_in, out, state_out, cu_seqlens, num_seqs,
+                           total_tokens, H, dk, dv, chunk, dtype);
+    if (st != GDN_OK) return st;
+    const size_t need = gdn_prefill_workspace_size(num_seqs, total_tokens, H, dk, dv, chunk, dtype);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return GDN_ERR_WORKSPACE;
+    if (workspace && misaligned(workspace)) return GDN_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t uniform_len = cu_seqlens ? 0 : total_tokens / num_seqs;
+    cudaError_t e = gdn::launch_prefill_simt(dtype, dk, q, k, v, g, beta, state_in, out,
+                                             state_out, cu_seqlens, uniform_len, num_seqs, H, s);
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e);
+}
+
+int gdn_decode_step(const void *q, const void *k, const void *v, const float *g,
+                    const float *beta, const float *state_in, float *state_out, void *out,
+                    int B, int H, int dk, int dv, int dtype, void *stream) {
+    if (B < 0 || H < 1) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (!shape_supported(dk, dv)) return GDN_ERR_UNSUPPORTED;
+    if (B == 0) return GDN_OK;
+    if ((int64_t)B * H > (int64_t)INT32_MAX) return GDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, state_in, state_out, out};
+    for (const void *p : ptrs)
+        if (!p || misaligned(p)) return GDN_ERR_INVALID_ARG;
+    if (state_out != state_in) {
+        const size_t bytes = (size_t)B * H * dv * dk * sizeof(float);
+        const char *a = reinterpret_cast<const char *>(state_in);
+        const char *b = reinterpret_cast<const char *>(state_out);
+        if (a < b + bytes && b < a + bytes) return GDN_ERR_INVALID_ARG;
+    }
+    cudaError_t e = gdn::launch_decode(dtype, dk, q, k, v, g, beta, state_in, state_out, out, B,
+                                       H, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e);
+}
+
+}  // extern "C"

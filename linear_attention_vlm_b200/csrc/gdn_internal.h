@@ -1,0 +1,47 @@
+// Internal declarations shared by the libgdn.so translation units.
+// Not part of the public ABI (that is include/gdn.h).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdn {
+
+constexpr int kChunk = 64;   // chunk length of the chunkwise prefill
+
+// Sequence bounds of sequence n: from cu_seqlens if given, else uniform.
+struct SeqBounds {
+    const int32_t *cu;   // device, may be null
+    int64_t uniform_len; // used when cu == null
+    __device__ __forceinline__ void get(int n, int64_t &bos, int64_t &eos) const {
+        if (cu) {
+            bos = cu[n];
+            eos = cu[n + 1];
+        } else {
+            bos = (int64_t)n * uniform_len;
+            eos = bos + uniform_len;
+        }
+    }
+};
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Launchers (return cudaError_t of the launch).
+cudaError_t launch_decode(int dtype, int dk, const void *q, const void *k, const void *v,
+                          const float *g, const float *beta, const float *state_in,
+                          float *state_out, void *out, int B, int H, cudaStream_t stream);
+
+cudaError_t launch_prefill_simt(int dtype, int dk, const void *q, const void *k,
+                                const void *v, const float *g, const float *beta,
+                                const float *state_in, void *out, float *state_out,
+                                const int32_t *cu_seqlens, int64_t uniform_len,
+                                int num_seqs, int H, cudaStream_t stream);
+
+}  // namespace gdn

@@ -1,0 +1,92 @@
+"""The C ABI without a GPU: the library loads, exports every function the
+header declares, sizes workspaces, and rejects bad arguments on the host
+before anything is enqueued."""
+import ctypes
+
+import pytest
+
+import linear_attention_vlm_b200 as gdn
+from linear_attention_vlm_b200 import gdn as binding
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return gdn.library()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = gdn.declared_symbols()
+    assert {"gdn_prefill", "gdn_decode_step", "gdn_prefill_workspace_size",
+            "gdn_status_string", "gdn_last_cuda_error"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), "libgdn.so does not export %s" % n
+
+
+def test_status_strings(lib):
+    for code in (0, 1, 2, 3, 5):
+        assert gdn.status_string(code).startswith("GDN_")
+    assert "unknown" in gdn.status_string(99)
+    assert binding._load().gdn_last_cuda_error() == b""
+
+
+def test_workspace_size_is_host_arithmetic():
+    import torch
+    # rejected configurations report 0
+    assert gdn.gdn_prefill_workspace_size(1, 8192, 16, 96, 96) == 0
+    assert gdn.gdn_prefill_workspace_size(1, 8192, 16, 128, 128, chunk=32) == 0
+    assert gdn.gdn_prefill_workspace_size(0, 8192, 16, 128, 128) == 0
+    # supported ones are finite and grow with the token count
+    a = gdn.gdn_prefill_workspace_size(1, 8192, 16, 128, 128, dtype=torch.bfloat16)
+    b = gdn.gdn_prefill_workspace_size(1, 16384, 16, 128, 128, dtype=torch.bfloat16)
+    assert 0 <= a <= b < (1 << 40)
+
+
+def _prefill_raw(lib, **kw):
+    args = dict(q=16, k=16, v=16, g=16, beta=16, state_in=None, out=16, state_out=None,
+                cu=None, N=1, T=64, H=2, dk=64, dv=64, chunk=64, dtype=0, ws=None, wsb=0,
+                stream=None)
+    args.update(kw)
+    return lib.gdn_prefill(args["q"], args["k"], args["v"], args["g"], args["beta"],
+                           args["state_in"], args["out"], args["state_out"], args["cu"],
+                           args["N"], args["T"], args["H"], args["dk"], args["dv"],
+                           args["chunk"], args["dtype"], args["ws"], args["wsb"], args["stream"])
+
+
+def test_prefill_rejects_bad_arguments(lib):
+    assert _prefill_raw(lib, q=None) == binding.GDN_ERR_INVALID_ARG
+    assert _prefill_raw(lib, q=17) == binding.GDN_ERR_INVALID_ARG          # misaligned
+    assert _prefill_raw(lib, N=0) == binding.GDN_ERR_INVALID_ARG
+    assert _prefill_raw(lib, T=-1) == binding.GDN_ERR_INVALID_ARG
+    assert _prefill_raw(lib, dtype=7) == binding.GDN_ERR_INVALID_ARG
+    assert _prefill_raw(lib, N=3, T=64) == binding.GDN_ERR_INVALID_ARG      # T % N != 0 without cu
+    assert _prefill_raw(lib, dk=96, dv=96) == binding.GDN_ERR_UNSUPPORTED
+    assert _prefill_raw(lib, dk=128, dv=64) == binding.GDN_ERR_UNSUPPORTED
+    assert _prefill_raw(lib, chunk=32) == binding.GDN_ERR_UNSUPPORTED
+    # partial overlap of state_in and state_out
+    assert _prefill_raw(lib, state_in=4096, state_out=4096 + 64) == binding.GDN_ERR_INVALID_ARG
+
+
+def test_decode_rejects_bad_arguments(lib):
+    def call(**kw):
+        a = dict(q=16, k=16, v=16, g=16, beta=16, si=4096, so=4096, out=16, B=1, H=1, dk=64,
+                 dv=64, dtype=1)
+        a.update(kw)
+        return lib.gdn_decode_step(a["q"], a["k"], a["v"], a["g"], a["beta"], a["si"], a["so"],
+                                   a["out"], a["B"], a["H"], a["dk"], a["dv"], a["dtype"], None)
+    assert call(B=0) == binding.GDN_OK                                      # no-op
+    assert call(q=None) == binding.GDN_ERR_INVALID_ARG
+    assert call(out=8) == binding.GDN_ERR_INVALID_ARG
+    assert call(B=-1) == binding.GDN_ERR_INVALID_ARG
+    assert call(dk=32, dv=32) == binding.GDN_ERR_UNSUPPORTED
+    assert call(dtype=3) == binding.GDN_ERR_INVALID_ARG
+    assert call(si=4096, so=4096 + 16) == binding.GDN_ERR_INVALID_ARG       # partial overlap
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(64, 2, 64)
+    s = torch.zeros(64, 2)
+    with pytest.raises(ValueError):
+        gdn.gdn_prefill(x, x, x, s, s)
+    with pytest.raises(ValueError):
+        gdn.gdn_decode_step(x[:1], x[:1], x[:1], s[:1], s[:1], torch.zeros(1, 2, 64, 64))

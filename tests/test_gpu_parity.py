@@ -1,0 +1,211 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Error metric, for every compared tensor: max |x - ref| / max |ref| (error
+relative to the max-norm of the reference).  Bars: fp32 inputs 1e-4; bf16
+inputs with fp32 state 2e-2.  The oracle always sees the inputs exactly as
+stored (bf16 values widened to fp64).
+
+Full-size workloads are compared on sampled heads (each head is an
+independent recurrence, so the oracle can run a head on its own); the
+long prefill is also checked segmented-vs-whole on the device.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+import linear_attention_vlm_b200 as gdn
+
+pytestmark = pytest.mark.gpu
+
+TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
+
+
+def rel_err(x, ref):
+    x = np.asarray(x, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert x.shape == ref.shape, (x.shape, ref.shape)
+    if ref.size == 0:
+        return 0.0
+    scale = np.max(np.abs(ref))
+    return float(np.max(np.abs(x - ref)) / (scale if scale > 0 else 1.0))
+
+
+def np64(t):
+    return None if t is None else t.detach().to("cpu", torch.float64).numpy()
+
+
+def run_gpu(inp, dev, **kw):
+    t = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    out, st = gdn.gdn_prefill(t["q"], t["k"], t["v"], t["g"], t["beta"], t.get("state_in"),
+                              t["cu_seqlens"], **kw)
+    torch.cuda.synchronize()
+    return out, st
+
+
+def run_oracle(inp):
+    return oracle.prefill(np64(inp["q"]), np64(inp["k"]), np64(inp["v"]), np64(inp["g"]),
+                          np64(inp["beta"]), np64(inp.get("state_in")),
+                          inp["cu_seqlens"].numpy().astype(np.int64))
+
+
+def check(inp, dev, tol, **kw):
+    out, st = run_gpu(inp, dev, **kw)
+    ro, rs = run_oracle(inp)
+    eo, es = rel_err(np64(out), ro), rel_err(np64(st), rs)
+    assert eo <= tol and es <= tol, "out err %.3g, state err %.3g (tol %.1g)" % (eo, es, tol)
+    return eo, es
+
+
+def test_tiny_fp32(cuda_device):
+    w = W.WORKLOADS["tiny_fp32"]
+    inp = W.prefill_inputs(w, seed=0)
+    check(inp, cuda_device, 1e-4)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("lens", [[1], [63], [64], [65], [200], [0, 1, 130, 0, 64, 77], [0]],
+                         ids=lambda l: "lens" + "-".join(map(str, l)))
+def test_ragged(cuda_device, dtype, d, lens):
+    inp = W.random_prefill(lens, H=3, dk=d, dv=d, dtype=dtype, seed=sum(lens) + d,
+                           state_std=0.02)
+    check(inp, cuda_device, TOL[dtype])
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_zero_initial_state_and_no_state_out(cuda_device, dtype):
+    inp = W.random_prefill([150], H=2, dk=128, dv=128, dtype=dtype, seed=5)
+    out_a, st_a = run_gpu(inp, cuda_device)
+    z = dict(inp, state_in=torch.zeros(1, 2, 128, 128))
+    out_b, st_b = run_gpu(z, cuda_device)
+    assert torch.equal(out_a, out_b) and torch.equal(st_a, st_b)
+    out_c, st_c = run_gpu(inp, cuda_device, want_state=False)
+    assert st_c is None and torch.equal(out_a, out_c)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_uniform_without_cu_seqlens(cuda_device, dtype):
+    inp = W.random_prefill([96, 96, 96], H=2, dk=64, dv=64, dtype=dtype, seed=8, state_std=0.02)
+    t = {k: (v.to(cuda_device) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    o1, s1 = gdn.gdn_prefill(t["q"], t["k"], t["v"], t["g"], t["beta"], t["state_in"], t["cu_seqlens"])
+    o2, s2 = gdn.gdn_prefill(t["q"], t["k"], t["v"], t["g"], t["beta"], t["state_in"], None, num_seqs=3)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
+def test_in_place_state(cuda_device):
+    inp = W.random_prefill([100, 37], H=2, dk=128, dv=128, dtype=torch.bfloat16, seed=9,
+                           state_std=0.02)
+    t = {k: (v.to(cuda_device) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    o1, s1 = gdn.gdn_prefill(t["q"], t["k"], t["v"], t["g"], t["beta"], t["state_in"], t["cu_seqlens"])
+    s = t["state_in"].clone()
+    o2, s2 = gdn.gdn_prefill(t["q"], t["k"], t["v"], t["g"], t["beta"], s, t["cu_seqlens"], state_out=s)
+    torch.cuda.synchronize()
+    assert s2.data_ptr() == s.data_ptr()
+    assert torch.equal(o1, o2) and torch.equal(s1, s)
+
+
+def test_long_horizon_no_decay(cuda_device):
+    """alpha = 1 keeps every write in the state: errors in early chunks are
+    not forgotten, so this pins long state carry."""
+    inp = W.random_prefill([4096], H=2, dk=128, dv=128, dtype=torch.bfloat16, seed=10)
+    inp["g"].zero_()
+    check(inp, cuda_device, 2e-2)
+
+
+def test_prefill_bf16_sampled_heads(cuda_device):
+    w = W.WORKLOADS["prefill_bf16"]
+    full = W.prefill_inputs(w, seed=0)
+    out, st = run_gpu(full, cuda_device)
+    heads = [0, 7, 15]
+    sub = W.prefill_inputs(w, seed=0, heads=heads)
+    ro, rs = run_oracle(sub)
+    assert rel_err(np64(out[:, heads]), ro) <= 2e-2
+    assert rel_err(np64(st[:, heads]), rs) <= 2e-2
+
+
+def test_long_prefill_segmented(cuda_device):
+    w = W.WORKLOADS["long_prefill_bf16"]
+    full = W.prefill_inputs(w, seed=0)
+    t = {k: (v.to(cuda_device) if isinstance(v, torch.Tensor) else v) for k, v in full.items()}
+    T = w.T
+    out_whole, st_whole = gdn.gdn_prefill(t["q"], t["k"], t["v"], t["g"], t["beta"], None, None)
+    seg = T // w.segments
+    st = torch.zeros(1, w.H, w.dv, w.dk, device=cuda_device)
+    outs = []
+    for s0 in range(0, T, seg):
+        sl = slice(s0, s0 + seg)
+        o, st = gdn.gdn_prefill(t["q"][sl], t["k"][sl], t["v"][sl], t["g"][sl], t["beta"][sl],
+                                st, None, state_out=st)
+        outs.append(o[-64:].clone())
+    torch.cuda.synchronize()
+    # chunk-aligned segments with an fp32 state: identical arithmetic
+    assert torch.equal(st, st_whole)
+    assert torch.equal(outs[-1], out_whole[-64:])
+    heads = [5]
+    sub = W.prefill_inputs(w, seed=0, heads=heads)
+    ro, rs = run_oracle(sub)
+    assert rel_err(np64(st_whole[:, heads]), rs) <= 2e-2
+    assert rel_err(np64(out_whole[:, heads]), ro) <= 2e-2
+
+
+def test_varlen_sampled_heads(cuda_device):
+    w = W.WORKLOADS["varlen_bf16"]
+    full = W.prefill_inputs(w, seed=0)
+    out, st = run_gpu(full, cuda_device)
+    heads = [3, 12]
+    sub = W.prefill_inputs(w, seed=0, heads=heads)
+    ro, rs = run_oracle(sub)
+    assert rel_err(np64(out[:, heads]), ro) <= 2e-2
+    assert rel_err(np64(st[:, heads]), rs) <= 2e-2
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("d", [64, 128])
+def test_decode_small(cuda_device, dtype, d):
+    rng = np.random.default_rng(d)
+    B, H = 5, 3
+    x = W.random_prefill([1] * B, H=H, dk=d, dv=d, dtype=dtype, seed=d, state_std=0.02)
+    q, k, v = (x[n].reshape(B, H, d) for n in ("q", "k", "v"))
+    g, b = x["g"].reshape(B, H), x["beta"].reshape(B, H)
+    s = x["state_in"]
+    o, s2 = gdn.gdn_decode_step(q.to(cuda_device), k.to(cuda_device), v.to(cuda_device),
+                                g.to(cuda_device), b.to(cuda_device), s.to(cuda_device).clone())
+    ro, rs = oracle.decode_step(np64(q), np64(k), np64(v), np64(g), np64(b), np64(s))
+    assert rel_err(np64(o), ro) <= TOL[dtype]
+    assert rel_err(np64(s2), rs) <= 1e-5          # the state is fp32 end to end
+
+
+def test_decode_out_of_place_matches_in_place(cuda_device):
+    w = W.WORKLOADS["decode_bf16"]
+    tok = {k: v.to(cuda_device) for k, v in W.decode_tokens(w, 0, seed=0).items()}
+    s0 = W.decode_state(w, seed=0).to(cuda_device)
+    s_a = s0.clone()
+    o_a, _ = gdn.gdn_decode_step(tok["q"], tok["k"], tok["v"], tok["g"], tok["beta"], s_a)
+    s_b = torch.empty_like(s0)
+    o_b, _ = gdn.gdn_decode_step(tok["q"], tok["k"], tok["v"], tok["g"], tok["beta"], s0, s_b)
+    torch.cuda.synchronize()
+    assert torch.equal(o_a, o_b) and torch.equal(s_a, s_b)
+
+
+def test_decode_1024_steps_sampled(cuda_device):
+    """The decode workload: 64 sequences x 16 heads, 1024 one-token steps,
+    compared after every step on sampled (sequence, head) pairs."""
+    w = W.WORKLOADS["decode_bf16"]
+    S = W.decode_state(w, seed=0).to(cuda_device)
+    heads = [0, 9, 15]
+    seqs = [0, 17, 63]
+    ref_s = np64(W.decode_state(w, seed=0, heads=heads))[seqs]
+    worst_o = 0.0
+    for step in range(w.steps):
+        tok = W.decode_tokens(w, step, seed=0)
+        td = {k: v.to(cuda_device, non_blocking=True) for k, v in tok.items()}
+        o, _ = gdn.gdn_decode_step(td["q"], td["k"], td["v"], td["g"], td["beta"], S)
+        sel = {k: np64(v[:, heads][seqs]) for k, v in tok.items()}
+        ro, ref_s = oracle.decode_step(sel["q"], sel["k"], sel["v"], sel["g"], sel["beta"], ref_s)
+        worst_o = max(worst_o, rel_err(np64(o[:, heads][seqs]), ro))
+        if step + 1 in (1, 32, 1024):
+            assert rel_err(np64(S[:, heads][seqs]), ref_s) <= 1e-4, step
+    assert worst_o <= 2e-2
