@@ -8,6 +8,7 @@
 
 #include "gdn.h"
 #include "gdn_internal.h"
+#include "prefill_tc.h"
 
 namespace {
 
@@ -22,6 +23,15 @@ int cuda_fail(cudaError_t e) {
 bool misaligned(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
 
 bool shape_supported(int dk, int dv) { return dk == dv && (dk == 64 || dk == 128); }
+
+// The fused tensor-core kernel covers bf16 with d_k = d_v = 128; everything
+// else (fp32, d = 64, an empty batch) takes the SIMT kernel.
+bool use_tc(int64_t total_tokens, int dk, int dtype) {
+    return dtype == GDN_BF16 && dk == 128 && total_tokens > 0;
+}
+
+constexpr size_t kStatusBytes = 256;       // device status word(s) at the start of the workspace
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s bound on any in-kernel wait
 
 // Common validation of gdn_prefill's arguments (without workspace).
 int check_prefill(const void *q, const void *k, const void *v, const float *g,
@@ -68,7 +78,7 @@ size_t gdn_prefill_workspace_size(int num_seqs, int64_t total_tokens, int H, int
     if (num_seqs < 1 || H < 1 || total_tokens < 0) return 0;
     if (chunk != gdn::kChunk || !shape_supported(dk, dv)) return 0;
     if (dtype != GDN_F32 && dtype != GDN_BF16) return 0;
-    return 0;
+    return use_tc(total_tokens, dk, dtype) ? kStatusBytes : 0;
 }
 
 int gdn_prefill_kernel_count(int num_seqs, int64_t total_tokens, int H, int dk, int dv,
@@ -91,6 +101,15 @@ int gdn_prefill(const void *q, const void *k, const void *v, const float *g, con
     if (workspace && misaligned(workspace)) return GDN_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t uniform_len = cu_seqlens ? 0 : total_tokens / num_seqs;
+    if (use_tc(total_tokens, dk, dtype)) {
+        int *err = static_cast<int *>(workspace);
+        cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), s);
+        if (e != cudaSuccess) return cuda_fail(e);
+        gdn::TcLaunch L{q, k, v, g, beta, state_in, out, state_out, cu_seqlens, nullptr,
+                        uniform_len, total_tokens, num_seqs, H, err, kWaitLimitNs};
+        e = gdn::launch_prefill_tc(L, s);
+        return e == cudaSuccess ? GDN_OK : cuda_fail(e);
+    }
     cudaError_t e = gdn::launch_prefill_simt(dtype, dk, q, k, v, g, beta, state_in, out,
                                              state_out, cu_seqlens, uniform_len, num_seqs, H, s);
     return e == cudaSuccess ? GDN_OK : cuda_fail(e);
