@@ -6,18 +6,19 @@
 //
 //   p1   [K;Q] K^T                     -> KK^T (rows 0-63), QK^T (rows 64-127)
 //   prep A = strict_lower(beta_r exp(G_r - G_i) k_r.k_i);  T = (I + A)^-1
-//        T' = T diag(beta gamma),  T'' = T diag(beta),  Phat = tril(Q K^T)
-//   p2   W^T  = K^T T'^T               (W  = T diag(beta gamma) K)
-//   p3   U^T  = V^T T''^T              (Ut = T diag(beta) V)
-//   a    U^T -= S W^T                  (U  = Ut - W S^T)
+//        T' = diag(D) T diag(beta gamma),  T'' = diag(D) T diag(beta),
+//        Phat = tril(Q K^T)
+//   p2   W^T  = K^T T'^T               (W  = D o T diag(beta gamma) K)
+//   p3   U^T  = V^T T''^T              (Ut = D o T diag(beta) V)
+//   a    U^T -= S W^T                  (U  = D o (Ut - W S^T): the D-scaled residual)
 //   c1   O1   = S Q^T
-//   b    S   += (D o U)^T K            (S was pre-scaled by gamma_C)
-//   c2   O2   = (D o U)^T Phat^T
+//   b    S   += U^T K                  (S was pre-scaled by gamma_C)
+//   c2   O2   = U^T Phat^T
 //   out  o_t  = gamma_t O1[:,t] + exp(G_t - G_C) O2[:,t]
 //
 // which is the token recurrence S_t = a_t S_{t-1}(I - b_t k_t k_t^T) + b_t v_t
 // k_t^T, o_t = S_t q_t unrolled over the chunk (the exp(G_t - G_C) factor
-// undoes the D factor folded into the shared (D o U) operand).  All seven
+// undoes the D factor folded into the shared D-scaled residual operand).  All seven
 // products are M = 128 tcgen05 MMAs (bf16 operands in 128-byte-swizzled
 // shared memory, fp32 accumulators in TMEM); K, Q, V tiles arrive by TMA.
 //
@@ -52,13 +53,13 @@ constexpr uint32_t OFF_KQ = 0;                         // [2 stages][2 kb][128 r
 constexpr uint32_t OFF_V = OFF_KQ + 2 * 32768;         // [2 kb][64 rows][128 B]
 constexpr uint32_t OFF_S = OFF_V + 16384;              // S bf16 [2 kb][128 rows dv][128 B]
 constexpr uint32_t OFF_W = OFF_S + 32768;              // W bf16 [2 kb][64 rows t][128 B]
-constexpr uint32_t OFF_U = OFF_W + 16384;              // (D o U)^T bf16 [128 rows dv][128 B]
+constexpr uint32_t OFF_U = OFF_W + 16384;              // U^T bf16 [128 rows dv][128 B]; output staging
 constexpr uint32_t OFF_TP = OFF_U + 16384;             // T'  bf16 [64 rows t][128 B]
 constexpr uint32_t OFF_TPP = OFF_TP + 8192;            // T'' bf16 [64][128 B]
 constexpr uint32_t OFF_PH = OFF_TPP + 8192;            // Phat bf16 [2 bufs][64][128 B]
 constexpr uint32_t OFF_AF = OFF_PH + 16384;            // A fp32 [64][AP]
 constexpr uint32_t OFF_TF = OFF_AF + 64 * AP * 4;      // T fp32 [64][AP]
-constexpr uint32_t OFF_SCP = OFF_TF + 64 * AP * 4;     // prep scalars: G, beta, gamma [64] each
+constexpr uint32_t OFF_SCP = OFF_TF + 64 * AP * 4;     // prep scalars: G log2(e), beta, beta gamma, D
 constexpr uint32_t OFF_SCE = OFF_SCP + 1024;           // chain scalars [3 bufs]: Dd, gam, invD [64], gC, len
 constexpr uint32_t OFF_MM = OFF_SCE + 3072;            // solve scratch: 4 warps x 16x16 fp32
 constexpr uint32_t OFF_BAR = OFF_MM + 4096;            // mbarriers, TMEM base, abort flag
@@ -66,8 +67,8 @@ constexpr uint32_t SMEM_USED = OFF_BAR + 256;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;      // + alignment slack
 
 // TMEM columns
-constexpr uint32_t TM_C12 = 0;     // p1 output, then W^T (64 cols)
-constexpr uint32_t TM_C3 = 64;     // U^T accumulator (64)
+constexpr uint32_t TM_C12 = 0;     // p1 output (64 cols)
+constexpr uint32_t TM_C3 = 64;     // W^T from p2, then the U^T accumulator (64)
 constexpr uint32_t TM_C4 = 128;    // state S (128)
 constexpr uint32_t TM_C5 = 256;    // O1 [2 bufs] at 256, 384 (64 each)
 constexpr uint32_t TM_C6 = 320;    // O2 [2 bufs] at 320, 448
@@ -80,7 +81,7 @@ enum {
     B_FULL_V = 4,
     B_EMPTY_V = 5,
     B_P1 = 6,
-    B_P23 = 7,
+    B_P2 = 7,
     B_A = 8,
     B_B = 9,
     B_C = 10,
@@ -89,7 +90,8 @@ enum {
     B_SREADY = 13,
     B_UREADY = 14,
     B_FIN = 15,
-    NUM_BARS = 16
+    B_P3 = 16,
+    NUM_BARS = 17
 };
 
 struct ChainScalars {   // per chunk, chain group
@@ -103,25 +105,47 @@ struct ChainScalars {   // per chunk, chain group
 static_assert(sizeof(ChainScalars) == 1024, "scalar block size");
 
 struct PrepScalars {
-    float G[C];
+    float inv[C];       // exp(-G_t) (at most e^80 under the documented gate domain)
     float beta[C];
-    float gam[C];
-    float pad[C];
+    float bg[C];        // beta * gamma
+    float Dd[C];        // exp(G_C - G_t)
 };
+static_assert(sizeof(PrepScalars) == 1024, "scalar block size");
+
 
 __device__ __forceinline__ uint32_t bar_addr(uint8_t *sm, int i) {
     return smem_u32(sm + OFF_BAR + 8 * i);
 }
 
-// Inclusive cumsum of g over one chunk by one warp; lane l owns rows l, l+32.
-__device__ __forceinline__ void chunk_gates(const float *__restrict__ g, const float *__restrict__ beta,
-                                            int64_t t0, int len, int h, int H, int lane, float &G0,
-                                            float &G1, float &b0, float &b1) {
-    const int r0 = lane, r1 = lane + 32;
-    float x0 = r0 < len ? __ldg(g + (size_t)(t0 + r0) * H + h) : 0.f;
-    float x1 = r1 < len ? __ldg(g + (size_t)(t0 + r1) * H + h) : 0.f;
-    b0 = r0 < len ? __ldg(beta + (size_t)(t0 + r0) * H + h) : 0.f;
-    b1 = r1 < len ? __ldg(beta + (size_t)(t0 + r1) * H + h) : 0.f;
+// Raw gates of one chunk held by one warp (lane l owns rows l and l+32),
+// loaded an iteration before use so that the global-load latency is hidden.
+struct GateRegs {
+    float g0, g1, b0, b1;
+};
+
+__device__ __forceinline__ GateRegs load_gates(const float *__restrict__ g, const float *__restrict__ beta,
+                                               int64_t bos, int64_t eos, int m, int nchunks, int h,
+                                               int H, int lane) {
+    GateRegs r{0.f, 0.f, 0.f, 0.f};
+    if (m < nchunks) {
+        const int64_t t0 = bos + (int64_t)m * C;
+        const int64_t rem = eos - t0;
+        const int len = rem < C ? (int)rem : C;
+        if (lane < len) {
+            r.g0 = __ldg(g + (size_t)(t0 + lane) * H + h);
+            r.b0 = __ldg(beta + (size_t)(t0 + lane) * H + h);
+        }
+        if (lane + 32 < len) {
+            r.g1 = __ldg(g + (size_t)(t0 + lane + 32) * H + h);
+            r.b1 = __ldg(beta + (size_t)(t0 + lane + 32) * H + h);
+        }
+    }
+    return r;
+}
+
+// Inclusive cumsum of the gates inside the chunk (rows past the end are 0).
+__device__ __forceinline__ void scan_gates(const GateRegs &r, int lane, float &G0, float &G1) {
+    float x0 = r.g0, x1 = r.g1;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const float y0 = __shfl_up_sync(0xffffffffu, x0, o);
@@ -205,8 +229,9 @@ __device__ __forceinline__ void solve_block(const float *Af, float *Tf, float *s
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_prefill_tc_kernel(const __grid_constant__ TcParams p) {
     extern __shared__ uint8_t smraw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
-                                              ~static_cast<uintptr_t>(1023));
+    // align to 1024 B by pointer arithmetic on the __shared__ array itself, so
+    // that the compiler keeps shared-space (LDS/STS) addressing for `sm`
+    uint8_t *sm = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);
     uint32_t *tmem_base_ptr = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 8 * NUM_BARS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_BAR + 8 * NUM_BARS + 4);
 
@@ -295,15 +320,22 @@ gdn_prefill_tc_kernel(const __grid_constant__ TcParams p) {
             const uint32_t id_a = idesc_bf16(128, 64, false, false, true);
             const uint32_t id_c1 = idesc_bf16(128, 64, false, false);
             const uint32_t id_b = idesc_bf16(128, 128, false, true);
-            const uint32_t sKQ = smem_u32(sm + OFF_KQ), sV = smem_u32(sm + OFF_V);
+            const uint32_t sKQ = smem_u32(sm + OFF_KQ), sV = smem_u32(sm + OFF_V);  // tile bases
             const uint32_t sS = smem_u32(sm + OFF_S), sW = smem_u32(sm + OFF_W);
             const uint32_t sU = smem_u32(sm + OFF_U), sTP = smem_u32(sm + OFF_TP);
             const uint32_t sTPP = smem_u32(sm + OFF_TPP), sPH = smem_u32(sm + OFF_PH);
+            // descriptors are built once; a byte offset `o` inside a tile adds o >> 4
+            const uint64_t dKQk = desc_sw128(sKQ, 16, 1024);         // K-major views
+            const uint64_t dKQm = desc_sw128(sKQ, 16384, 1024);      // MN-major view of K
+            const uint64_t dVm = desc_sw128(sV, 8192, 1024);
+            const uint64_t dS = desc_sw128(sS, 16, 1024), dW = desc_sw128(sW, 16, 1024);
+            const uint64_t dU = desc_sw128(sU, 16, 1024), dTP = desc_sw128(sTP, 16, 1024);
+            const uint64_t dTPP = desc_sw128(sTPP, 16, 1024), dPH = desc_sw128(sPH, 16, 1024);
             auto issue_p1 = [&](int n) {
-                const uint32_t base = sKQ + (n & 1) * 32768;
+                const uint32_t base = (n & 1) * 32768;
                 for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t a = base + (ks >> 2) * 16384 + (ks & 3) * 32;
-                    mma_bf16_ss(tm + TM_C12, desc_sw128(a, 16, 1024), desc_sw128(a, 16, 1024), id_p1, ks > 0);
+                    const uint64_t a = dKQk + ((base + (ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
+                    mma_bf16_ss(tm + TM_C12, a, a, id_p1, ks > 0);
                 }
             };
             bool ok = mbar_wait(bar_addr(sm, B_FULL_KQ), 0, lim, abort_flag);
@@ -315,55 +347,56 @@ gdn_prefill_tc_kernel(const __grid_constant__ TcParams p) {
             }
             for (int n = 0; ok && n < nchunks; ++n) {
                 const int s = n & 1;
-                const uint32_t kq = sKQ + s * 32768;
+                const uint32_t kq = s * 32768;   // stage offset inside the KQ buffer
                 if (!(ok = mbar_wait(bar_addr(sm, B_TREADY), n & 1, lim, abort_flag))) { fail(22); break; }
-                if (!(ok = mbar_wait(bar_addr(sm, B_FULL_V), n & 1, lim, abort_flag))) { fail(23); break; }
                 tc_fence_after();
-                // p2: W^T = K^T T'^T   (A = K tile, MN-major; B = T' K-major)
+                // p2: W^T = K^T T'^T into the U^T columns (A = K tile MN-major; B = T')
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(tm + TM_C12, desc_sw128(kq + ks * 2048, 16384, 1024),
-                                desc_sw128(sTP + ks * 32, 16, 1024), id_p2, ks > 0);
-                // p3: U^T = V^T T''^T
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(tm + TM_C3, desc_sw128(sV + ks * 2048, 8192, 1024),
-                                desc_sw128(sTPP + ks * 32, 16, 1024), id_p2, ks > 0);
-                mma_commit(bar_addr(sm, B_P23));
-                mma_commit(bar_addr(sm, B_EMPTY_V));
-                if (!(ok = mbar_wait(bar_addr(sm, B_WREADY), n & 1, lim, abort_flag))) { fail(24); break; }
-                if (!(ok = mbar_wait(bar_addr(sm, B_SREADY), n & 1, lim, abort_flag))) { fail(25); break; }
-                tc_fence_after();
-                // a: U^T -= S W^T
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                    const uint32_t offw = (ks >> 2) * 8192 + (ks & 3) * 32;
-                    mma_bf16_ss(tm + TM_C3, desc_sw128(sS + off, 16, 1024),
-                                desc_sw128(sW + offw, 16, 1024), id_a, 1);
-                }
-                // c1: O1 = S Q^T  (B = Q rows of the KQ tile)
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                    mma_bf16_ss(tm + TM_C5 + s * 128, desc_sw128(sS + off, 16, 1024),
-                                desc_sw128(kq + off + 8192, 16, 1024), id_c1, ks > 0);
-                }
-                mma_commit(bar_addr(sm, B_A));
+                    mma_bf16_ss(tm + TM_C3, dKQm + ((kq + ks * 2048) >> 4), dTP + ((ks * 32) >> 4),
+                                id_p2, ks > 0);
+                mma_commit(bar_addr(sm, B_P2));
+                // p1 of the next chunk as early as possible: the prep group has
+                // already consumed this chunk's p1 output
                 if (n + 1 < nchunks) {
                     if (!(ok = mbar_wait(bar_addr(sm, B_FULL_KQ + ((n + 1) & 1)), ((n + 1) >> 1) & 1, lim, abort_flag))) { fail(26); break; }
                     tc_fence_after();
                     issue_p1(n + 1);
                     mma_commit(bar_addr(sm, B_P1));
                 }
+                if (!(ok = mbar_wait(bar_addr(sm, B_WREADY), n & 1, lim, abort_flag))) { fail(24); break; }
+                if (!(ok = mbar_wait(bar_addr(sm, B_FULL_V), n & 1, lim, abort_flag))) { fail(23); break; }
+                tc_fence_after();
+                // p3: U^T = V^T T''^T (overwrites the extracted W^T)
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ss(tm + TM_C3, dVm + ((ks * 2048) >> 4), dTPP + ((ks * 32) >> 4), id_p2,
+                                ks > 0);
+                mma_commit(bar_addr(sm, B_P3));
+                mma_commit(bar_addr(sm, B_EMPTY_V));
+                if (!(ok = mbar_wait(bar_addr(sm, B_SREADY), n & 1, lim, abort_flag))) { fail(25); break; }
+                tc_fence_after();
+                // a: U^T -= S W^T
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                    const uint32_t offw = (ks >> 2) * 8192 + (ks & 3) * 32;
+                    mma_bf16_ss(tm + TM_C3, dS + (off >> 4), dW + (offw >> 4), id_a, 1);
+                }
+                mma_commit(bar_addr(sm, B_A));
+                // c1: O1 = S Q^T  (B = Q rows of the KQ tile); off the state chain
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                    mma_bf16_ss(tm + TM_C5 + s * 128, dS + (off >> 4), dKQk + ((kq + off + 8192) >> 4),
+                                id_c1, ks > 0);
+                }
                 if (!(ok = mbar_wait(bar_addr(sm, B_UREADY), n & 1, lim, abort_flag))) { fail(27); break; }
                 tc_fence_after();
-                // b: S += (D o U)^T K   (A = U tile K-major; B = K tile MN-major)
+                // b: S += U^T K   (A = U tile K-major; B = K tile MN-major)
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(tm + TM_C4, desc_sw128(sU + ks * 32, 16, 1024),
-                                desc_sw128(kq + ks * 2048, 16384, 1024), id_b, 1);
+                    mma_bf16_ss(tm + TM_C4, dU + ((ks * 32) >> 4), dKQm + ((kq + ks * 2048) >> 4), id_b, 1);
                 mma_commit(bar_addr(sm, B_B));
-                // c2: O2 = (D o U)^T Phat^T
-                const uint32_t ph = sPH + s * 8192;
+                // c2: O2 = U^T Phat^T
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(tm + TM_C6 + s * 128, desc_sw128(sU + ks * 32, 16, 1024),
-                                desc_sw128(ph + ks * 32, 16, 1024), id_c1, ks > 0);
+                    mma_bf16_ss(tm + TM_C6 + s * 128, dU + ((ks * 32) >> 4),
+                                dPH + ((s * 8192 + ks * 32) >> 4), id_c1, ks > 0);
                 mma_commit(bar_addr(sm, B_C));
                 mma_commit(bar_addr(sm, B_EMPTY_KQ + s));
             }
@@ -383,17 +416,21 @@ gdn_prefill_tc_kernel(const __grid_constant__ TcParams p) {
         float *Tf = reinterpret_cast<float *>(sm + OFF_TF);
         float *mm = reinterpret_cast<float *>(sm + OFF_MM) + pw * 256;
         const uint32_t lane_off = static_cast<uint32_t>(pw * 32) << 16;
+        GateRegs gr{0.f, 0.f, 0.f, 0.f};
+        if (pw == 0) gr = load_gates(p.g, p.beta, bos, eos, 0, nchunks, h, H, lane);
         for (int n = 0; n < nchunks; ++n) {
             const int s = n & 1;
-            const int64_t t0 = bos + (int64_t)n * C;
-            const int len = (int)((eos - t0) < C ? (eos - t0) : C);
             if (named_bar_any(1, 128, *abort_flag != 0)) break;
             if (pw == 0) {
-                float G0, G1, b0, b1;
-                chunk_gates(p.g, p.beta, t0, len, h, H, lane, G0, G1, b0, b1);
-                sc->G[lane] = G0; sc->G[lane + 32] = G1;
+                float G0, G1;
+                scan_gates(gr, lane, G0, G1);
+                const float b0 = gr.b0, b1 = gr.b1;
+                gr = load_gates(p.g, p.beta, bos, eos, n + 1, nchunks, h, H, lane);
+                const float GC = __shfl_sync(0xffffffffu, G1, 31);
+                sc->inv[lane] = expf(-G0); sc->inv[lane + 32] = expf(-G1);
                 sc->beta[lane] = b0; sc->beta[lane + 32] = b1;
-                sc->gam[lane] = expf(G0); sc->gam[lane + 32] = expf(G1);
+                sc->bg[lane] = b0 * expf(G0); sc->bg[lane + 32] = b1 * expf(G1);
+                sc->Dd[lane] = expf(GC - G0); sc->Dd[lane + 32] = expf(GC - G1);
             }
             named_bar_sync(1, 128);
             // A (strictly lower, decayed, beta-scaled) and Phat from p1
@@ -406,11 +443,19 @@ gdn_prefill_tc_kernel(const __grid_constant__ TcParams p) {
                 tmem_ld32(tm + lane_off + TM_C12, x0);
                 tmem_ld32(tm + lane_off + TM_C12 + 32, x1);
                 if (pt < 64) {
+                    // A[r][i] = beta_r exp(G_r - G_i) k_r.k_i = (beta_r gamma_r) exp(-G_i) KK[r][i]
                     const int r = pt;
-                    const float br = sc->beta[r], Gr = sc->G[r];
+                    const float bgr = sc->bg[r];
 #pragma unroll
-                    for (int i = 0; i < 64; ++i)
-                        Af[r * AP + i] = (i < r) ? br * expf(Gr - sc->G[i]) * x[i] : 0.f;
+                    for (int i = 0; i < 64; i += 4) {
+                        const float4 iv = *reinterpret_cast<const float4 *>(&sc->inv[i]);
+                        float4 a;
+                        a.x = (i < r) ? bgr * iv.x * x[i] : 0.f;
+                        a.y = (i + 1 < r) ? bgr * iv.y * x[i + 1] : 0.f;
+                        a.z = (i + 2 < r) ? bgr * iv.z * x[i + 2] : 0.f;
+                        a.w = (i + 3 < r) ? bgr * iv.w * x[i + 3] : 0.f;
+                        *reinterpret_cast<float4 *>(&Af[r * AP + i]) = a;
+                    }
                 } else {
                     const int r = pt - 64;
                     const uint32_t row = smem_u32(sm + OFF_PH + s * 8192);
@@ -436,10 +481,10 @@ gdn_prefill_tc_kernel(const __grid_constant__ TcParams p) {
                 float x[16];
 #pragma unroll
                 for (int r = 0; r < 16; ++r) {
-                    float acc = (r == c) ? 1.f : 0.f;
+                    float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int i = 0; i < r; ++i) acc = fmaf(-Ab[r * AP + i], x[i], acc);
-                    x[r] = acc;
+                    for (int i = 0; i < r; ++i) ps[i & 3] = fmaf(Ab[r * AP + i], x[i], ps[i & 3]);
+                    x[r] = ((r == c) ? 1.f : 0.f) - ((ps[0] + ps[1]) + (ps[2] + ps[3]));
                 }
 #pragma unroll
                 for (int r = 0; r < 16; ++r) Tf[(16 * b + r) * AP + 16 * b + c] = x[r];
@@ -460,34 +505,38 @@ gdn_prefill_tc_kernel(const __grid_constant__ TcParams p) {
             named_bar_sync(1, 128);
             if (pw == 0) solve_block(Af, Tf, mm, 3, 0, lane);
             named_bar_sync(1, 128);
-            // T' = T diag(beta gamma) and T'' = T diag(beta), bf16, K-major rows t
+            // T'' of the previous chunk may still be feeding its p3
+            if (n > 0 && !mbar_wait(bar_addr(sm, B_P3), (n - 1) & 1, lim, abort_flag)) fail(33);
+            // T' = diag(D) T diag(beta gamma), T'' = diag(D) T diag(beta), bf16, K-major rows t
             {
                 const int which = pt >> 6, r = pt & 63;
                 const uint32_t row = smem_u32(sm + (which ? OFF_TPP : OFF_TP));
+                const float *colscale = which ? sc->beta : sc->bg;
+                const float dr = sc->Dd[r];
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i0 = 8 * c + 2 * e;
-                        const float s0 = which ? sc->beta[i0] : sc->beta[i0] * sc->gam[i0];
-                        const float s1 = which ? sc->beta[i0 + 1] : sc->beta[i0 + 1] * sc->gam[i0 + 1];
-                        w[e] = pack_bf16(Tf[r * AP + i0] * s0, Tf[r * AP + i0 + 1] * s1);
-                    }
-                    st_shared_v4(row + sw128_chunk(r, c), w[0], w[1], w[2], w[3]);
+                    const float4 t0v = *reinterpret_cast<const float4 *>(&Tf[r * AP + 8 * c]);
+                    const float4 t1v = *reinterpret_cast<const float4 *>(&Tf[r * AP + 8 * c + 4]);
+                    const float4 s0v = *reinterpret_cast<const float4 *>(&colscale[8 * c]);
+                    const float4 s1v = *reinterpret_cast<const float4 *>(&colscale[8 * c + 4]);
+                    st_shared_v4(row + sw128_chunk(r, c),
+                                 pack_bf16(dr * t0v.x * s0v.x, dr * t0v.y * s0v.y),
+                                 pack_bf16(dr * t0v.z * s0v.z, dr * t0v.w * s0v.w),
+                                 pack_bf16(dr * t1v.x * s1v.x, dr * t1v.y * s1v.y),
+                                 pack_bf16(dr * t1v.z * s1v.z, dr * t1v.w * s1v.w));
                 }
             }
             fence_proxy_async_smem();
             mbar_arrive(bar_addr(sm, B_TREADY));
-            // W from p2's W^T (TMEM lane = d_k index, column = t)
-            if (!mbar_wait(bar_addr(sm, B_P23), n & 1, lim, abort_flag)) fail(32);
+            // W from p2's W^T (TMEM lane = d_k index, column = t), in the U^T columns
+            if (!mbar_wait(bar_addr(sm, B_P2), n & 1, lim, abort_flag)) fail(32);
             tc_fence_after();
             {
                 float x[32];
                 uint8_t *wt = sm + OFF_W + (pt >> 6) * 8192;
                 const int col = pt & 63;
                 for (int half = 0; half < 2; ++half) {
-                    tmem_ld32(tm + lane_off + TM_C12 + 32 * half, x);
+                    tmem_ld32(tm + lane_off + TM_C3 + 32 * half, x);
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
                         *reinterpret_cast<__nv_bfloat16 *>(wt + sw128_offset(32 * half + i, col)) =
@@ -503,12 +552,16 @@ gdn_prefill_tc_kernel(const __grid_constant__ TcParams p) {
         const int dv = tid;   // TMEM lane and state row
         const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
         ChainScalars *scb = reinterpret_cast<ChainScalars *>(sm + OFF_SCE);
+        GateRegs gr{0.f, 0.f, 0.f, 0.f};
+        if (warp == 0) gr = load_gates(p.g, p.beta, bos, eos, 0, nchunks, h, H, lane);
+        // scalars of chunk m from the prefetched gates; prefetch chunk m+1's
         auto compute_scalars = [&](int m) {
             if (warp == 0) {
                 const int64_t t0 = bos + (int64_t)m * C;
                 const int len = (int)((eos - t0) < C ? (eos - t0) : C);
-                float G0, G1, b0, b1;
-                chunk_gates(p.g, p.beta, t0, len, h, H, lane, G0, G1, b0, b1);
+                float G0, G1;
+                scan_gates(gr, lane, G0, G1);
+                gr = load_gates(p.g, p.beta, bos, eos, m + 1, nchunks, h, H, lane);
                 const float GC = __shfl_sync(0xffffffffu, G1, 31);
                 ChainScalars &cs = scb[m % 3];
                 cs.Dd[lane] = expf(GC - G0); cs.Dd[lane + 32] = expf(GC - G1);
@@ -554,7 +607,7 @@ gdn_prefill_tc_kernel(const __grid_constant__ TcParams p) {
             // ring of three: warp 0 may write chunk n+1's scalars while a
             // slower warp still reads chunk n-1's in its output epilogue
             const ChainScalars &cs = scb[n % 3];
-            // U epilogue: (D o U)^T -> U tile (row dv, 64 t)
+            // U epilogue: the D-scaled residual U^T -> U tile (row dv, 64 t)
             if (!mbar_wait(bar_addr(sm, B_A), n & 1, lim, abort_flag)) fail(41);
             tc_fence_after();
             {
@@ -563,14 +616,10 @@ gdn_prefill_tc_kernel(const __grid_constant__ TcParams p) {
                 for (int half = 0; half < 2; ++half) {
                     tmem_ld32(tm + lane_off + TM_C3 + 32 * half, x);
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const int tb = 32 * half + 8 * q4;
+                    for (int q4 = 0; q4 < 4; ++q4)
                         st_shared_v4(row + sw128_chunk(dv, 4 * half + q4),
-                                     pack_bf16(cs.Dd[tb] * x[8 * q4], cs.Dd[tb + 1] * x[8 * q4 + 1]),
-                                     pack_bf16(cs.Dd[tb + 2] * x[8 * q4 + 2], cs.Dd[tb + 3] * x[8 * q4 + 3]),
-                                     pack_bf16(cs.Dd[tb + 4] * x[8 * q4 + 4], cs.Dd[tb + 5] * x[8 * q4 + 5]),
-                                     pack_bf16(cs.Dd[tb + 6] * x[8 * q4 + 6], cs.Dd[tb + 7] * x[8 * q4 + 7]));
-                    }
+                                     pack_bf16(x[8 * q4], x[8 * q4 + 1]), pack_bf16(x[8 * q4 + 2], x[8 * q4 + 3]),
+                                     pack_bf16(x[8 * q4 + 4], x[8 * q4 + 5]), pack_bf16(x[8 * q4 + 6], x[8 * q4 + 7]));
                 }
             }
             fence_proxy_async_smem();
@@ -584,14 +633,10 @@ gdn_prefill_tc_kernel(const __grid_constant__ TcParams p) {
             tc_fence_after();
             {
                 float x[32];
-                const float gnext = last ? 1.f : scb[(n + 1) % 3].gC;
                 for (int c0 = 0; c0 < D; c0 += 32) {
                     tmem_ld32(tm + lane_off + TM_C4 + c0, x);
                     if (!last) {
                         store_s_bf16(x, c0);
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) x[j] *= gnext;
-                        tmem_st32(tm + lane_off + TM_C4 + c0, x);
                     } else if (p.state_out) {
 #pragma unroll
                         for (int j = 0; j < 32; j += 4)
@@ -599,18 +644,29 @@ gdn_prefill_tc_kernel(const __grid_constant__ TcParams p) {
                                 make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
                     }
                 }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                if (!last) {
+                    // the next (a) may start now; rescale the fp32 state for the
+                    // next (b), which the MMA thread issues only after U_READY
+                    mbar_arrive(bar_addr(sm, B_SREADY));
+                    const float gnext = scb[(n + 1) % 3].gC;
+                    for (int c0 = 0; c0 < D; c0 += 32) {
+                        tmem_ld32(tm + lane_off + TM_C4 + c0, x);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) x[j] *= gnext;
+                        tmem_st32(tm + lane_off + TM_C4 + c0, x);
+                    }
+                    tc_fence_before();
+                }
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            if (!last) mbar_arrive(bar_addr(sm, B_SREADY));
             // O epilogue: o_t = gamma_t O1 + exp(G_t - G_C) O2
             if (!mbar_wait(bar_addr(sm, B_C), n & 1, lim, abort_flag)) fail(43);
             tc_fence_after();
             {
-                const int64_t t0 = bos + (int64_t)n * C;
-                const int len = cs.len;
-                __nv_bfloat16 *o = p.out + ((size_t)t0 * H + h) * D + dv;
-                const size_t stride = (size_t)H * D;
+                // stage the [64 t][128 dv] bf16 tile in the U buffer (free once
+                // c2 has completed), then write whole 16-byte pieces of rows
+                __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_U);
                 float a[32], b[32];
                 for (int half = 0; half < 2; ++half) {
                     tmem_ld32(tm + lane_off + TM_C5 + s * 128 + 32 * half, a);
@@ -618,12 +674,24 @@ gdn_prefill_tc_kernel(const __grid_constant__ TcParams p) {
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int t = 32 * half + j;
-                        if (t < len)
-                            o[(size_t)t * stride] = __float2bfloat16_rn(fmaf(cs.gam[t], a[j], cs.invD[t] * b[j]));
+                        stage[t * D + dv] = __float2bfloat16_rn(fmaf(cs.gam[t], a[j], cs.invD[t] * b[j]));
                     }
                 }
+                tc_fence_before();
+                named_bar_sync(2, 128);
+                const int64_t t0 = bos + (int64_t)n * C;
+                const int len = cs.len;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int idx = k * 128 + dv;          // 1024 pieces of 16 bytes
+                    const int t = idx >> 4, piece = idx & 15;
+                    if (t < len) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(stage + t * D + piece * 8);
+                        *reinterpret_cast<uint4 *>(p.out + ((size_t)(t0 + t) * H + h) * D + piece * 8) = v;
+                    }
+                }
+                named_bar_sync(2, 128);   // the U buffer is rewritten by the next U epilogue
             }
-            tc_fence_before();
         }
     }
 
