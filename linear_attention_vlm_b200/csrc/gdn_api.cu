@@ -30,7 +30,6 @@ bool use_tc(int64_t total_tokens, int dk, int dtype) {
     return dtype == GDN_BF16 && dk == 128 && total_tokens > 0;
 }
 
-constexpr size_t kStatusBytes = 256;       // device status word(s) at the start of the workspace
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s bound on any in-kernel wait
 
 // Common validation of gdn_prefill's arguments (without workspace).
@@ -78,7 +77,9 @@ size_t gdn_prefill_workspace_size(int num_seqs, int64_t total_tokens, int H, int
     if (num_seqs < 1 || H < 1 || total_tokens < 0) return 0;
     if (chunk != gdn::kChunk || !shape_supported(dk, dv)) return 0;
     if (dtype != GDN_F32 && dtype != GDN_BF16) return 0;
-    return use_tc(total_tokens, dk, dtype) ? kStatusBytes : 0;
+    return use_tc(total_tokens, dk, dtype)
+               ? gdn::tc_workspace_bytes(num_seqs, total_tokens, H, /*varlen=*/true)
+               : 0;
 }
 
 int gdn_prefill_kernel_count(int num_seqs, int64_t total_tokens, int H, int dk, int dv,
@@ -86,7 +87,9 @@ int gdn_prefill_kernel_count(int num_seqs, int64_t total_tokens, int H, int dk, 
     if (num_seqs < 1 || H < 1 || total_tokens < 0) return 0;
     if (chunk != gdn::kChunk || !shape_supported(dk, dv)) return 0;
     if (dtype != GDN_F32 && dtype != GDN_BF16) return 0;
-    return 1;
+    // the workspace query cannot see whether cu_seqlens will be passed, so the
+    // count here assumes the packed (varlen) form; uniform batches launch one less
+    return use_tc(total_tokens, dk, dtype) ? gdn::tc_kernel_count(true) : 1;
 }
 
 int gdn_prefill(const void *q, const void *k, const void *v, const float *g, const float *beta,
@@ -105,8 +108,8 @@ int gdn_prefill(const void *q, const void *k, const void *v, const float *g, con
         int *err = static_cast<int *>(workspace);
         cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), s);
         if (e != cudaSuccess) return cuda_fail(e);
-        gdn::TcLaunch L{q, k, v, g, beta, state_in, out, state_out, cu_seqlens, nullptr,
-                        uniform_len, total_tokens, num_seqs, H, err, kWaitLimitNs};
+        gdn::TcLaunch L{q, k, v, g, beta, state_in, out, state_out, cu_seqlens, uniform_len,
+                        total_tokens, num_seqs, H, workspace, err, kWaitLimitNs};
         e = gdn::launch_prefill_tc(L, s);
         return e == cudaSuccess ? GDN_OK : cuda_fail(e);
     }

@@ -1,36 +1,34 @@
-// Fused chunkwise Gated DeltaNet prefill on the sm_100a tensor cores.
+// Chunkwise Gated DeltaNet prefill on the sm_100a tensor cores, as two
+// kernels: a fully parallel chunk-prep kernel and a sequential chain kernel.
 //
-// One CTA owns one (sequence, head) and walks its chunks of C = 64 tokens
-// with the fp32 d_v x d_k state held in tensor memory.  Per chunk (G =
-// cumsum of g inside the chunk, gamma = exp(G), D_t = exp(G_C - G_t)):
+// Chunk algebra (chunk of C = 64 tokens, start state S, G = cumsum of g inside
+// the chunk, gamma = exp(G), D_t = exp(G_C - G_t)):
 //
-//   p1   [K;Q] K^T                     -> KK^T (rows 0-63), QK^T (rows 64-127)
-//   prep A = strict_lower(beta_r exp(G_r - G_i) k_r.k_i);  T = (I + A)^-1
-//        T' = diag(D) T diag(beta gamma),  T'' = diag(D) T diag(beta),
-//        Phat = tril(Q K^T)
-//   p2   W^T  = K^T T'^T               (W  = D o T diag(beta gamma) K)
-//   p3   U^T  = V^T T''^T              (Ut = D o T diag(beta) V)
-//   a    U^T -= S W^T                  (U  = D o (Ut - W S^T): the D-scaled residual)
-//   c1   O1   = S Q^T
-//   b    S   += U^T K                  (S was pre-scaled by gamma_C)
-//   c2   O2   = U^T Phat^T
-//   out  o_t  = gamma_t O1[:,t] + exp(G_t - G_C) O2[:,t]
+//   A    = strict_lower(beta_r exp(G_r - G_i) k_r.k_i),   T = (I + A)^-1
+//   T'   = diag(D) T diag(beta gamma),   T'' = diag(D) T diag(beta)
+//   W    = T' K,   Phat = tril(Q K^T)
+//   U^T  = V^T T''^T - S W^T           (the D-scaled delta residual)
+//   S   <- gamma_C S + U^T K
+//   o_t  = gamma_t (S Q^T)[:,t] + exp(G_t - G_C) (U^T Phat^T)[:,t]
 //
-// which is the token recurrence S_t = a_t S_{t-1}(I - b_t k_t k_t^T) + b_t v_t
-// k_t^T, o_t = S_t q_t unrolled over the chunk (the exp(G_t - G_C) factor
-// undoes the D factor folded into the shared D-scaled residual operand).  All seven
-// products are M = 128 tcgen05 MMAs (bf16 operands in 128-byte-swizzled
-// shared memory, fp32 accumulators in TMEM); K, Q, V tiles arrive by TMA.
+// which is the token recurrence S_t = a_t S_{t-1}(I - b_t k_t k_t^T) +
+// b_t v_t k_t^T, o_t = S_t q_t unrolled over the chunk.
 //
-// Warp roles (320 threads):
-//   warps 0-3  chain: U / S / O epilogues (thread i <-> TMEM lane i = row i)
-//   warps 4-7  prep:  gates, A and Phat from p1, triangular solve, T', T'', W
-//   warp  8    MMA issue (one thread) and TMEM allocation
-//   warp  9    TMA producer (one thread)
-// The prep of chunk n+1 overlaps the state chain of chunk n.
+// gdn_chunk_prep_kernel: one CTA per (chunk, head), all chunks at once.
+//   TMA brings K and Q; p1 = [K;Q] K^T on tcgen05 (TMEM); four warps form A
+//   and Phat, invert I + A (16x16 diagonal blocks by substitution, the
+//   off-diagonal blocks with tf32 mma.sync), scale T' and T''; p2 = K^T T'^T
+//   on tcgen05 gives W^T, which is transposed into W.  W, T'' and Phat are
+//   written to the workspace in the 128-byte-swizzled layout the chain
+//   kernel's MMAs read, so it copies them with one bulk copy per chunk.
+// gdn_chunk_chain_kernel: one CTA per (sequence, head), fp32 state in TMEM:
+//   p3 U^T = V^T T''^T, (a) U^T -= S W^T, (b) S += U^T K, c1 S Q^T,
+//   c2 U^T Phat^T -- five M = 128 tcgen05 MMAs per chunk -- with a
+//   four-warp epilogue group (residual, state, output), one MMA thread and
+//   one TMA thread.  The state never leaves the SM between chunks.
 //
 // Tokens past the end of a sequence inside its last chunk get g = 0 and
-// beta = 0, which zeroes their rows of W and Ut and keeps the state
+// beta = 0, which zeroes their rows of W and T'' and keeps the state
 // untouched; their outputs are not stored.
 #include <string.h>
 
@@ -45,62 +43,49 @@ using namespace sm100;
 
 constexpr int C = 64;
 constexpr int D = 128;
-constexpr int kThreads = 320;
 constexpr int AP = 68;   // fp32 row pitch of the solve matrices
 
-// shared memory map (offsets from a 1024-byte aligned base)
-constexpr uint32_t OFF_KQ = 0;                         // [2 stages][2 kb][128 rows][128 B]
-constexpr uint32_t OFF_V = OFF_KQ + 2 * 32768;         // [2 kb][64 rows][128 B]
-constexpr uint32_t OFF_S = OFF_V + 16384;              // S bf16 [2 kb][128 rows dv][128 B]
-constexpr uint32_t OFF_W = OFF_S + 32768;              // W bf16 [2 kb][64 rows t][128 B]
-constexpr uint32_t OFF_U = OFF_W + 16384;              // U^T bf16 [128 rows dv][128 B]; output staging
-constexpr uint32_t OFF_TP = OFF_U + 16384;             // T'  bf16 [64 rows t][128 B]
-constexpr uint32_t OFF_TPP = OFF_TP + 8192;            // T'' bf16 [64][128 B]
-constexpr uint32_t OFF_PH = OFF_TPP + 8192;            // Phat bf16 [2 bufs][64][128 B]
-constexpr uint32_t OFF_AF = OFF_PH + 16384;            // A fp32 [64][AP]
-constexpr uint32_t OFF_TF = OFF_AF + 64 * AP * 4;      // T fp32 [64][AP]
-constexpr uint32_t OFF_SCP = OFF_TF + 64 * AP * 4;     // prep scalars: G log2(e), beta, beta gamma, D
-constexpr uint32_t OFF_SCE = OFF_SCP + 1024;           // chain scalars [3 bufs]: Dd, gam, invD [64], gC, len
-constexpr uint32_t OFF_MM = OFF_SCE + 3072;            // solve scratch: 4 warps x 16x16 fp32
-constexpr uint32_t OFF_BAR = OFF_MM + 4096;            // mbarriers, TMEM base, abort flag
-constexpr uint32_t SMEM_USED = OFF_BAR + 256;
-constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;      // + alignment slack
+// ------------------------------------------------------------ prep kernel layout
+constexpr int kPrepThreads = 160;                      // warps 0-3 prep, warp 4 control
+constexpr uint32_t P_KQ = 0;                           // [2 kb][128 rows: K 0-63, Q 64-127][128 B]
+constexpr uint32_t P_TP = P_KQ + 32768;                // T'  bf16 [64 t][128 B]
+constexpr uint32_t P_TPP = P_TP + 8192;                // T'' bf16 [64 t][128 B]
+constexpr uint32_t P_PH = P_TPP + 8192;                // Phat bf16 [64 t][128 B]
+constexpr uint32_t P_AF = P_PH + 8192;                 // A fp32 [64][AP]; later W staging [2 kb][64][128 B]
+constexpr uint32_t P_TF = P_AF + 64 * AP * 4;          // T fp32 [64][AP]
+constexpr uint32_t P_SC = P_TF + 64 * AP * 4;          // PrepScalars
+constexpr uint32_t P_MM = P_SC + 1024;                 // solve scratch, 4 warps x 16x16 fp32
+constexpr uint32_t P_BAR = P_MM + 4096;                // mbarriers + TMEM base
+constexpr uint32_t P_ALLOC = P_BAR + 64 + 1024;        // + alignment slack
+static_assert(64 * AP * 4 >= 16384, "W staging fits in the A buffer");
+constexpr uint32_t P_TM_COLS = 128;                    // p1 output at 0, p2 output at 64
+enum { PB_FULL = 0, PB_P1 = 1, PB_TREADY = 2, PB_P2 = 3, PB_FIN = 4, PB_NUM = 5 };
 
-// TMEM columns
-constexpr uint32_t TM_C12 = 0;     // p1 output (64 cols)
-constexpr uint32_t TM_C3 = 64;     // W^T from p2, then the U^T accumulator (64)
-constexpr uint32_t TM_C4 = 128;    // state S (128)
-constexpr uint32_t TM_C5 = 256;    // O1 [2 bufs] at 256, 384 (64 each)
-constexpr uint32_t TM_C6 = 320;    // O2 [2 bufs] at 320, 448
+// ------------------------------------------------------------ chain kernel layout
+constexpr int kChainThreads = 192;                     // warps 0-3 chain, 4 MMA, 5 TMA
+constexpr uint32_t C_STAGE = 81920;                    // per stage: KQ, V, W, T'', Phat
+constexpr uint32_t CS_KQ = 0, CS_V = 32768, CS_W = 49152, CS_TPP = 65536, CS_PH = 73728;
+constexpr uint32_t C_S = 2 * C_STAGE;                  // S bf16 [2 kb][128 dv][128 B]
+constexpr uint32_t C_U = C_S + 32768;                  // U^T bf16 [128 dv][128 B]; output staging
+constexpr uint32_t C_SCE = C_U + 16384;                // ChainScalars x 3
+constexpr uint32_t C_BAR = C_SCE + 3072;               // mbarriers + TMEM base + abort flag
+constexpr uint32_t C_ALLOC = C_BAR + 256 + 1024;
+static_assert(CS_PH + 8192 == C_STAGE, "stage layout");
+// TMEM columns of the chain kernel
+constexpr uint32_t TM_U = 64;      // U^T accumulator (64)
+constexpr uint32_t TM_S = 128;     // state S (128)
+constexpr uint32_t TM_O1 = 256;    // S Q^T [2 bufs] at 256, 384 (64 each)
+constexpr uint32_t TM_O2 = 320;    // U^T Phat^T [2 bufs] at 320, 448
 constexpr uint32_t TM_COLS = 512;
-
-// barrier indices
-enum {
-    B_FULL_KQ = 0,   // +stage
-    B_EMPTY_KQ = 2,  // +stage
-    B_FULL_V = 4,
-    B_EMPTY_V = 5,
-    B_P1 = 6,
-    B_P2 = 7,
-    B_A = 8,
-    B_B = 9,
-    B_C = 10,
-    B_TREADY = 11,
-    B_WREADY = 12,
-    B_SREADY = 13,
-    B_UREADY = 14,
-    B_FIN = 15,
-    B_P3 = 16,
-    NUM_BARS = 17
-};
+enum { CB_FULL = 0, CB_EMPTY = 2, CB_A = 4, CB_B = 5, CB_C = 6, CB_SREADY = 7, CB_UREADY = 8,
+       CB_FIN = 9, CB_NUM = 10 };
 
 struct ChainScalars {   // per chunk, chain group
-    float Dd[C];        // exp(G_C - G_t)
     float gam[C];       // exp(G_t)
     float invD[C];      // exp(G_t - G_C)
     float gC;           // exp(G_C)
     int len;
-    int pad[62];
+    int pad[126];
 };
 static_assert(sizeof(ChainScalars) == 1024, "scalar block size");
 
@@ -112,9 +97,46 @@ struct PrepScalars {
 };
 static_assert(sizeof(PrepScalars) == 1024, "scalar block size");
 
+struct PrepParams {
+    CUtensorMap map_q, map_k;
+    const float *g, *beta;
+    const int32_t *cu_seqlens;
+    const int32_t *chunk_off;    // varlen: first global chunk of each sequence, [N+1]
+    int64_t uniform_len;
+    int cps;                     // uniform: chunks per sequence
+    int num_seqs, H;
+    uint8_t *tiles;
+    int *err;
+    uint64_t timeout_ns;
+};
 
-__device__ __forceinline__ uint32_t bar_addr(uint8_t *sm, int i) {
-    return smem_u32(sm + OFF_BAR + 8 * i);
+struct ChainParams {
+    CUtensorMap map_q, map_k, map_v;
+    const float *g, *beta, *state_in;
+    float *state_out;
+    __nv_bfloat16 *out;
+    const int32_t *cu_seqlens;
+    const int32_t *chunk_off;
+    int64_t uniform_len;
+    int cps;
+    int H;
+    const uint8_t *tiles;
+    int *err;
+    uint64_t timeout_ns;
+};
+
+__device__ __forceinline__ uint8_t *aligned_smem(uint8_t *raw) {
+    // align by pointer arithmetic on the __shared__ array so that the
+    // compiler keeps shared-space (LDS/STS) addressing
+    return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
+
+// 1-D bulk copy global -> shared, completion as transaction bytes on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+        : "memory");
 }
 
 // Raw gates of one chunk held by one warp (lane l owns rows l and l+32),
@@ -224,43 +246,311 @@ __device__ __forceinline__ void solve_block(const float *Af, float *Tf, float *s
     __syncwarp();
 }
 
-// ---------------------------------------------------------------- kernel
 
-__global__ void __launch_bounds__(kThreads, 1)
-gdn_prefill_tc_kernel(const __grid_constant__ TcParams p) {
+// ---------------------------------------------------------------- chunk offsets
+
+// chunk_off[n] = sum_{m<n} ceil(L_m / 64) for n = 0..N (one block).
+__global__ void __launch_bounds__(1024)
+gdn_chunk_offsets_kernel(const int32_t *__restrict__ cu, int N, int32_t *__restrict__ chunk_off) {
+    __shared__ int32_t warp_sums[32];
+    __shared__ int32_t carry;
+    if (threadIdx.x == 0) carry = 0;
+    __syncthreads();
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    for (int base = 0; base < N; base += 1024) {
+        const int n = base + (int)threadIdx.x;
+        const int32_t c = n < N ? (cu[n + 1] - cu[n] + C - 1) / C : 0;
+        int32_t x = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) warp_sums[wid] = x;
+        __syncthreads();
+        if (wid == 0) {
+            int32_t w = warp_sums[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int32_t y = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += y;
+            }
+            warp_sums[lane] = w;   // inclusive over warps
+        }
+        __syncthreads();
+        const int32_t incl = x + (wid > 0 ? warp_sums[wid - 1] : 0) + carry;
+        if (n < N) chunk_off[n + 1] = incl;
+        if (base == 0 && threadIdx.x == 0) chunk_off[0] = 0;
+        __syncthreads();
+        if (threadIdx.x == 1023) carry = incl;
+        __syncthreads();
+    }
+    if (N == 0 && threadIdx.x == 0) chunk_off[0] = 0;
+}
+
+// ---------------------------------------------------------------- prep kernel
+
+__global__ void __launch_bounds__(kPrepThreads, 2)
+gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
     extern __shared__ uint8_t smraw[];
-    // align to 1024 B by pointer arithmetic on the __shared__ array itself, so
-    // that the compiler keeps shared-space (LDS/STS) addressing for `sm`
-    uint8_t *sm = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);
-    uint32_t *tmem_base_ptr = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 8 * NUM_BARS);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_BAR + 8 * NUM_BARS + 4);
+    uint8_t *sm = aligned_smem(smraw);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = p.H, h = blockIdx.y;
+    const int gc = blockIdx.x;
 
-    const int tid = threadIdx.x;
-    const int warp = tid >> 5, lane = tid & 31;
+    // which sequence and which of its chunks this CTA prepares
+    int nseq;
+    int64_t j;
+    if (p.chunk_off) {
+        if (gc >= p.chunk_off[p.num_seqs]) return;          // uniform across the CTA
+        int lo = 0, hi = p.num_seqs - 1;                     // last n with chunk_off[n] <= gc
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (p.chunk_off[mid] <= gc) lo = mid; else hi = mid - 1;
+        }
+        nseq = lo;
+        j = gc - p.chunk_off[lo];
+    } else {
+        nseq = gc / p.cps;
+        j = gc % p.cps;
+    }
+    int64_t bos, eos;
+    SeqBounds{p.cu_seqlens, p.uniform_len}.get(nseq, bos, eos);
+    const int64_t t0 = bos + j * C;
+    const int len = (eos - t0) < C ? (int)(eos - t0) : C;
+
+    uint32_t *tmem_base_ptr = reinterpret_cast<uint32_t *>(sm + P_BAR + 8 * PB_NUM);
+    auto bar = [&](int i) { return smem_u32(sm + P_BAR + 8 * i); };
+    if (tid == 0) {
+        mbar_init(bar(PB_FULL), 1);
+        mbar_init(bar(PB_P1), 1);
+        mbar_init(bar(PB_TREADY), 128);
+        mbar_init(bar(PB_P2), 1);
+        mbar_init(bar(PB_FIN), 1);
+        fence_mbar_init();
+    }
+    if (warp == 4) {
+        tmem_alloc(smem_u32(tmem_base_ptr), P_TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tmem_base_ptr;
+    const uint64_t lim = p.timeout_ns;
+    const int no_abort = 0;   // CTA-local failures end each wait by its own bound
+
+    if (warp == 4) {
+        if (lane == 0) {
+            const int z = (int)t0;
+            mbar_arrive_expect_tx(bar(PB_FULL), 32768);
+            for (int kb = 0; kb < 2; ++kb) {
+                const uint32_t dst = smem_u32(sm + P_KQ + kb * 16384);
+                tma_load_3d(dst, &p.map_k, kb * 64, h, z, bar(PB_FULL));
+                tma_load_3d(dst + 8192, &p.map_q, kb * 64, h, z, bar(PB_FULL));
+            }
+            bool ok = mbar_wait(bar(PB_FULL), 0, lim, &no_abort);
+            const uint64_t dKQk = desc_sw128(smem_u32(sm + P_KQ), 16, 1024);
+            const uint64_t dKQm = desc_sw128(smem_u32(sm + P_KQ), 16384, 1024);
+            const uint64_t dTP = desc_sw128(smem_u32(sm + P_TP), 16, 1024);
+            if (ok) {
+                tc_fence_after();
+                // p1: [K;Q] K^T -> columns 0..63
+                const uint32_t id_p1 = idesc_bf16(128, 64, false, false);
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint64_t a = dKQk + (((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
+                    mma_bf16_ss(tm, a, a, id_p1, ks > 0);
+                }
+                mma_commit(bar(PB_P1));
+                ok = mbar_wait(bar(PB_TREADY), 0, lim, &no_abort);
+            }
+            if (ok) {
+                tc_fence_after();
+                // p2: W^T = K^T T'^T -> columns 64..127 (A = K tile MN-major)
+                const uint32_t id_p2 = idesc_bf16(128, 64, true, false);
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ss(tm + 64, dKQm + ((ks * 2048) >> 4), dTP + ((ks * 32) >> 4), id_p2, ks > 0);
+                mma_commit(bar(PB_P2));
+            }
+            if (!ok && p.err) atomicCAS(p.err, 0, 51);
+            mma_commit(bar(PB_FIN));
+            mbar_wait(bar(PB_FIN), 0, lim, &no_abort);
+            mbar_wait(bar(PB_FULL), 0, lim, &no_abort);   // no TMA copy still landing at exit
+        }
+    } else {
+        // ------------------------------------------------------------ prep warps
+        const int pt = tid, pw = warp;
+        PrepScalars *sc = reinterpret_cast<PrepScalars *>(sm + P_SC);
+        float *Af = reinterpret_cast<float *>(sm + P_AF);
+        float *Tf = reinterpret_cast<float *>(sm + P_TF);
+        float *mm = reinterpret_cast<float *>(sm + P_MM) + pw * 256;
+        const uint32_t lane_off = static_cast<uint32_t>(pw * 32) << 16;
+        if (pw == 0) {
+            const GateRegs gr = load_gates(p.g, p.beta, bos, eos, (int)j, (int)j + 1, h, H, lane);
+            float G0, G1;
+            scan_gates(gr, lane, G0, G1);
+            const float GC = __shfl_sync(0xffffffffu, G1, 31);
+            sc->inv[lane] = expf(-G0); sc->inv[lane + 32] = expf(-G1);
+            sc->beta[lane] = gr.b0; sc->beta[lane + 32] = gr.b1;
+            sc->bg[lane] = gr.b0 * expf(G0); sc->bg[lane + 32] = gr.b1 * expf(G1);
+            sc->Dd[lane] = expf(GC - G0); sc->Dd[lane + 32] = expf(GC - G1);
+        }
+        named_bar_sync(1, 128);
+        bool ok = mbar_wait(bar(PB_P1), 0, lim, &no_abort);
+        tc_fence_after();
+        {
+            float x[64];
+            float (&x0)[32] = *reinterpret_cast<float (*)[32]>(&x[0]);
+            float (&x1)[32] = *reinterpret_cast<float (*)[32]>(&x[32]);
+            tmem_ld32(tm + lane_off, x0);
+            tmem_ld32(tm + lane_off + 32, x1);
+            if (pt < 64) {
+                // A[r][i] = beta_r exp(G_r - G_i) k_r.k_i = (beta_r gamma_r) exp(-G_i) KK[r][i]
+                const int r = pt;
+                const float bgr = sc->bg[r];
+#pragma unroll
+                for (int i = 0; i < 64; i += 4) {
+                    const float4 iv = *reinterpret_cast<const float4 *>(&sc->inv[i]);
+                    float4 a;
+                    a.x = (i < r) ? bgr * iv.x * x[i] : 0.f;
+                    a.y = (i + 1 < r) ? bgr * iv.y * x[i + 1] : 0.f;
+                    a.z = (i + 2 < r) ? bgr * iv.z * x[i + 2] : 0.f;
+                    a.w = (i + 3 < r) ? bgr * iv.w * x[i + 3] : 0.f;
+                    *reinterpret_cast<float4 *>(&Af[r * AP + i]) = a;
+                }
+            } else {
+                const int r = pt - 64;
+                const uint32_t row = smem_u32(sm + P_PH);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int i0 = 8 * c + 2 * e;
+                        w[e] = pack_bf16(i0 <= r ? x[i0] : 0.f, i0 + 1 <= r ? x[i0 + 1] : 0.f);
+                    }
+                    st_shared_v4(row + sw128_chunk(r, c), w[0], w[1], w[2], w[3]);
+                }
+            }
+        }
+        tc_fence_before();
+        named_bar_sync(1, 128);
+        // T = (I + A)^-1: 16x16 diagonal blocks by forward substitution ...
+        if (pt < 64) {
+            const int b = pt >> 4, c = pt & 15;
+            const float *Ab = Af + (16 * b) * AP + 16 * b;
+            float x[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                float ps[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int i = 0; i < r; ++i) ps[i & 3] = fmaf(Ab[r * AP + i], x[i], ps[i & 3]);
+                x[r] = ((r == c) ? 1.f : 0.f) - ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) Tf[(16 * b + r) * AP + 16 * b + c] = x[r];
+        } else {
+            for (int e = pt - 64; e < 6 * 256; e += 64) {   // zero the blocks above the diagonal
+                const int blk = e >> 8, w = e & 255;
+                const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+                const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+                Tf[(16 * bi + (w >> 4)) * AP + 16 * bj + (w & 15)] = 0.f;
+            }
+        }
+        named_bar_sync(1, 128);
+        // ... then the off-diagonal blocks, one band at a time
+        if (pw < 3) solve_block(Af, Tf, mm, pw + 1, pw, lane);
+        named_bar_sync(1, 128);
+        if (pw < 2) solve_block(Af, Tf, mm, pw + 2, pw, lane);
+        named_bar_sync(1, 128);
+        if (pw == 0) solve_block(Af, Tf, mm, 3, 0, lane);
+        named_bar_sync(1, 128);
+        // T' = diag(D) T diag(beta gamma), T'' = diag(D) T diag(beta): bf16, K-major rows t
+        {
+            const int which = pt >> 6, r = pt & 63;
+            const uint32_t row = smem_u32(sm + (which ? P_TPP : P_TP));
+            const float *colscale = which ? sc->beta : sc->bg;
+            const float dr = sc->Dd[r];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const float4 t0v = *reinterpret_cast<const float4 *>(&Tf[r * AP + 8 * c]);
+                const float4 t1v = *reinterpret_cast<const float4 *>(&Tf[r * AP + 8 * c + 4]);
+                const float4 s0v = *reinterpret_cast<const float4 *>(&colscale[8 * c]);
+                const float4 s1v = *reinterpret_cast<const float4 *>(&colscale[8 * c + 4]);
+                st_shared_v4(row + sw128_chunk(r, c), pack_bf16(dr * t0v.x * s0v.x, dr * t0v.y * s0v.y),
+                             pack_bf16(dr * t0v.z * s0v.z, dr * t0v.w * s0v.w),
+                             pack_bf16(dr * t1v.x * s1v.x, dr * t1v.y * s1v.y),
+                             pack_bf16(dr * t1v.z * s1v.z, dr * t1v.w * s1v.w));
+            }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bar(PB_TREADY));
+        // W from p2's W^T (TMEM lane = d_k index, column = t), staged over the A buffer
+        ok = mbar_wait(bar(PB_P2), 0, lim, &no_abort) && ok;
+        tc_fence_after();
+        {
+            float x[32];
+            uint8_t *wt = sm + P_AF + (pt >> 6) * 8192;
+            const int col = pt & 63;
+            for (int half = 0; half < 2; ++half) {
+                tmem_ld32(tm + lane_off + 64 + 32 * half, x);
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    *reinterpret_cast<__nv_bfloat16 *>(wt + sw128_offset(32 * half + i, col)) =
+                        __float2bfloat16_rn(x[i]);
+            }
+        }
+        tc_fence_before();
+        named_bar_sync(1, 128);
+        if (!ok && p.err && pt == 0) atomicCAS(p.err, 0, 52);
+        // W (16 KB), T'' (8 KB), Phat (8 KB) -> the workspace tile of (chunk, head)
+        uint8_t *dst = p.tiles + ((size_t)gc * H + h) * kTileBytes;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const int off = (k * 128 + pt) * 16;            // 0 .. 32 KB
+            const uint8_t *srcp = off < 16384 ? sm + P_AF + off : (off < 24576 ? sm + P_TPP + (off - 16384)
+                                                                                : sm + P_PH + (off - 24576));
+            *reinterpret_cast<uint4 *>(dst + off) = *reinterpret_cast<const uint4 *>(srcp);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 4) {
+        tc_fence_after();
+        tmem_dealloc(tm, P_TM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- chain kernel
+
+__global__ void __launch_bounds__(kChainThreads, 1)
+gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
+    extern __shared__ uint8_t smraw[];
+    uint8_t *sm = aligned_smem(smraw);
+    uint32_t *tmem_base_ptr = reinterpret_cast<uint32_t *>(sm + C_BAR + 8 * CB_NUM);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + C_BAR + 8 * CB_NUM + 4);
+    auto bar = [&](int i) { return smem_u32(sm + C_BAR + 8 * i); };
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.H;
-    // heads vary fastest; sequences are visited in the order given by p.order
-    const int unit = blockIdx.x;
-    const int nseq = p.order ? p.order[unit / H] : unit / H;
-    const int h = unit % H;
+    const int nseq = blockIdx.x / H, h = blockIdx.x % H;
     int64_t bos, eos;
     SeqBounds{p.cu_seqlens, p.uniform_len}.get(nseq, bos, eos);
     const int nchunks = (int)((eos - bos + C - 1) / C);
+    const int64_t gc0 = p.chunk_off ? (int64_t)p.chunk_off[nseq] : (int64_t)nseq * p.cps;
     const size_t state_off = ((size_t)nseq * H + h) * D * D;
 
     if (tid == 0) {
-        for (int i = 0; i < NUM_BARS; ++i) {
-            uint32_t cnt = 1;
-            if (i == B_TREADY || i == B_WREADY || i == B_SREADY || i == B_UREADY) cnt = 128;
-            mbar_init(bar_addr(sm, i), cnt);
-        }
+        for (int i = 0; i < CB_NUM; ++i)
+            mbar_init(bar(i), (i == CB_SREADY || i == CB_UREADY) ? 128 : 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 8) {
+    if (warp == 4) {
         tmem_alloc(smem_u32(tmem_base_ptr), TM_COLS);
         tmem_relinquish();
     }
-    if (warp == 9 && lane == 0) {
+    if (warp == 5 && lane == 0) {
         tma_prefetch_desc(&p.map_k);
         tma_prefetch_desc(&p.map_q);
         tma_prefetch_desc(&p.map_v);
@@ -270,7 +560,6 @@ gdn_prefill_tc_kernel(const __grid_constant__ TcParams p) {
     tc_fence_after();
     const uint32_t tm = *tmem_base_ptr;
     const uint64_t lim = p.timeout_ns;
-
     auto fail = [&](int code) {
         *abort_flag = 1;
         if (p.err) atomicCAS(p.err, 0, code);
@@ -280,278 +569,96 @@ gdn_prefill_tc_kernel(const __grid_constant__ TcParams p) {
         // empty sequence: the state passes through unchanged
         if (tid < 128 && p.state_out) {
             for (int j = 0; j < D; j += 4) {
-                float4 v = p.state_in ? *reinterpret_cast<const float4 *>(p.state_in + state_off + (size_t)tid * D + j)
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+                const float4 v = p.state_in ? *reinterpret_cast<const float4 *>(p.state_in + state_off + (size_t)tid * D + j)
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
                 *reinterpret_cast<float4 *>(p.state_out + state_off + (size_t)tid * D + j) = v;
             }
         }
-    } else if (warp == 9) {
-        // ------------------------------------------------------------ TMA producer
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ TMA / bulk producer
         if (lane == 0) {
-            int issued_kq[2] = {0, 0}, issued_v = 0;
+            int issued[2] = {0, 0};
             for (int n = 0; n < nchunks; ++n) {
                 const int s = n & 1;
+                const uint32_t st = smem_u32(sm + s * C_STAGE);
                 const int z = (int)(bos + (int64_t)n * C);
-                if (n >= 2 && !mbar_wait(bar_addr(sm, B_EMPTY_KQ + s), ((n - 2) >> 1) & 1, lim, abort_flag)) { fail(11); break; }
-                mbar_arrive_expect_tx(bar_addr(sm, B_FULL_KQ + s), 32768);
+                if (n >= 2 && !mbar_wait(bar(CB_EMPTY + s), ((n - 2) >> 1) & 1, lim, abort_flag)) { fail(61); break; }
+                const uint32_t full = bar(CB_FULL + s);
+                mbar_arrive_expect_tx(full, C_STAGE);
                 for (int kb = 0; kb < 2; ++kb) {
-                    const uint32_t dst = smem_u32(sm + OFF_KQ + s * 32768 + kb * 16384);
-                    tma_load_3d(dst, &p.map_k, kb * 64, h, z, bar_addr(sm, B_FULL_KQ + s));
-                    tma_load_3d(dst + 8192, &p.map_q, kb * 64, h, z, bar_addr(sm, B_FULL_KQ + s));
+                    tma_load_3d(st + CS_KQ + kb * 16384, &p.map_k, kb * 64, h, z, full);
+                    tma_load_3d(st + CS_KQ + kb * 16384 + 8192, &p.map_q, kb * 64, h, z, full);
+                    tma_load_3d(st + CS_V + kb * 8192, &p.map_v, kb * 64, h, z, full);
                 }
-                ++issued_kq[s];
-                if (n >= 1 && !mbar_wait(bar_addr(sm, B_EMPTY_V), (n - 1) & 1, lim, abort_flag)) { fail(12); break; }
-                mbar_arrive_expect_tx(bar_addr(sm, B_FULL_V), 16384);
-                for (int kb = 0; kb < 2; ++kb)
-                    tma_load_3d(smem_u32(sm + OFF_V + kb * 8192), &p.map_v, kb * 64, h, z, bar_addr(sm, B_FULL_V));
-                ++issued_v;
+                bulk_load(st + CS_W, p.tiles + ((size_t)(gc0 + n) * H + h) * kTileBytes, (uint32_t)kTileBytes, full);
+                ++issued[s];
             }
-            // no copy may still be landing in shared memory when the CTA exits
-            const int zero = 0;
+            const int zero = 0;   // no copy may still be landing in shared memory at exit
             for (int s = 0; s < 2; ++s)
-                if (issued_kq[s]) mbar_wait(bar_addr(sm, B_FULL_KQ + s), (issued_kq[s] - 1) & 1, lim, &zero);
-            if (issued_v) mbar_wait(bar_addr(sm, B_FULL_V), (issued_v - 1) & 1, lim, &zero);
+                if (issued[s]) mbar_wait(bar(CB_FULL + s), (issued[s] - 1) & 1, lim, &zero);
         }
-    } else if (warp == 8) {
+    } else if (warp == 4) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t id_p1 = idesc_bf16(128, 64, false, false);
-            const uint32_t id_p2 = idesc_bf16(128, 64, true, false);
+            const uint32_t id_n64 = idesc_bf16(128, 64, false, false);
+            const uint32_t id_p3 = idesc_bf16(128, 64, true, false);
             const uint32_t id_a = idesc_bf16(128, 64, false, false, true);
-            const uint32_t id_c1 = idesc_bf16(128, 64, false, false);
             const uint32_t id_b = idesc_bf16(128, 128, false, true);
-            const uint32_t sKQ = smem_u32(sm + OFF_KQ), sV = smem_u32(sm + OFF_V);  // tile bases
-            const uint32_t sS = smem_u32(sm + OFF_S), sW = smem_u32(sm + OFF_W);
-            const uint32_t sU = smem_u32(sm + OFF_U), sTP = smem_u32(sm + OFF_TP);
-            const uint32_t sTPP = smem_u32(sm + OFF_TPP), sPH = smem_u32(sm + OFF_PH);
-            // descriptors are built once; a byte offset `o` inside a tile adds o >> 4
-            const uint64_t dKQk = desc_sw128(sKQ, 16, 1024);         // K-major views
-            const uint64_t dKQm = desc_sw128(sKQ, 16384, 1024);      // MN-major view of K
-            const uint64_t dVm = desc_sw128(sV, 8192, 1024);
-            const uint64_t dS = desc_sw128(sS, 16, 1024), dW = desc_sw128(sW, 16, 1024);
-            const uint64_t dU = desc_sw128(sU, 16, 1024), dTP = desc_sw128(sTP, 16, 1024);
-            const uint64_t dTPP = desc_sw128(sTPP, 16, 1024), dPH = desc_sw128(sPH, 16, 1024);
-            auto issue_p1 = [&](int n) {
-                const uint32_t base = (n & 1) * 32768;
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint64_t a = dKQk + ((base + (ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
-                    mma_bf16_ss(tm + TM_C12, a, a, id_p1, ks > 0);
-                }
-            };
-            bool ok = mbar_wait(bar_addr(sm, B_FULL_KQ), 0, lim, abort_flag);
-            if (!ok) fail(21);
-            else {
-                tc_fence_after();
-                issue_p1(0);
-                mma_commit(bar_addr(sm, B_P1));
-            }
+            // descriptors are built once; a byte offset o inside a tile adds o >> 4
+            const uint64_t dSTk = desc_sw128(smem_u32(sm), 16, 1024);      // K-major views of stage data
+            const uint64_t dSTm = desc_sw128(smem_u32(sm), 16384, 1024);   // MN-major view of K
+            const uint64_t dVm = desc_sw128(smem_u32(sm), 8192, 1024);     // MN-major view of V
+            const uint64_t dS = desc_sw128(smem_u32(sm + C_S), 16, 1024);
+            const uint64_t dU = desc_sw128(smem_u32(sm + C_U), 16, 1024);
+            bool ok = true;
             for (int n = 0; ok && n < nchunks; ++n) {
                 const int s = n & 1;
-                const uint32_t kq = s * 32768;   // stage offset inside the KQ buffer
-                if (!(ok = mbar_wait(bar_addr(sm, B_TREADY), n & 1, lim, abort_flag))) { fail(22); break; }
+                const uint32_t st = s * C_STAGE;
+                if (!(ok = mbar_wait(bar(CB_FULL + s), (n >> 1) & 1, lim, abort_flag))) { fail(62); break; }
                 tc_fence_after();
-                // p2: W^T = K^T T'^T into the U^T columns (A = K tile MN-major; B = T')
+                // p3: U^T = V^T T''^T (the previous residual was consumed: U_READY(n-1))
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(tm + TM_C3, dKQm + ((kq + ks * 2048) >> 4), dTP + ((ks * 32) >> 4),
-                                id_p2, ks > 0);
-                mma_commit(bar_addr(sm, B_P2));
-                // p1 of the next chunk as early as possible: the prep group has
-                // already consumed this chunk's p1 output
-                if (n + 1 < nchunks) {
-                    if (!(ok = mbar_wait(bar_addr(sm, B_FULL_KQ + ((n + 1) & 1)), ((n + 1) >> 1) & 1, lim, abort_flag))) { fail(26); break; }
-                    tc_fence_after();
-                    issue_p1(n + 1);
-                    mma_commit(bar_addr(sm, B_P1));
-                }
-                if (!(ok = mbar_wait(bar_addr(sm, B_WREADY), n & 1, lim, abort_flag))) { fail(24); break; }
-                if (!(ok = mbar_wait(bar_addr(sm, B_FULL_V), n & 1, lim, abort_flag))) { fail(23); break; }
-                tc_fence_after();
-                // p3: U^T = V^T T''^T (overwrites the extracted W^T)
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(tm + TM_C3, dVm + ((ks * 2048) >> 4), dTPP + ((ks * 32) >> 4), id_p2,
-                                ks > 0);
-                mma_commit(bar_addr(sm, B_P3));
-                mma_commit(bar_addr(sm, B_EMPTY_V));
-                if (!(ok = mbar_wait(bar_addr(sm, B_SREADY), n & 1, lim, abort_flag))) { fail(25); break; }
+                    mma_bf16_ss(tm + TM_U, dVm + ((st + CS_V + ks * 2048) >> 4),
+                                dSTk + ((st + CS_TPP + ks * 32) >> 4), id_p3, ks > 0);
+                if (!(ok = mbar_wait(bar(CB_SREADY), n & 1, lim, abort_flag))) { fail(63); break; }
                 tc_fence_after();
                 // a: U^T -= S W^T
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                    const uint32_t offw = (ks >> 2) * 8192 + (ks & 3) * 32;
-                    mma_bf16_ss(tm + TM_C3, dS + (off >> 4), dW + (offw >> 4), id_a, 1);
+                    const uint32_t offw = st + CS_W + (ks >> 2) * 8192 + (ks & 3) * 32;
+                    mma_bf16_ss(tm + TM_U, dS + (off >> 4), dSTk + (offw >> 4), id_a, 1);
                 }
-                mma_commit(bar_addr(sm, B_A));
-                // c1: O1 = S Q^T  (B = Q rows of the KQ tile); off the state chain
+                mma_commit(bar(CB_A));
+                // c1: O1 = S Q^T (off the state chain)
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                    mma_bf16_ss(tm + TM_C5 + s * 128, dS + (off >> 4), dKQk + ((kq + off + 8192) >> 4),
-                                id_c1, ks > 0);
+                    mma_bf16_ss(tm + TM_O1 + s * 128, dS + (off >> 4),
+                                dSTk + ((st + CS_KQ + off + 8192) >> 4), id_n64, ks > 0);
                 }
-                if (!(ok = mbar_wait(bar_addr(sm, B_UREADY), n & 1, lim, abort_flag))) { fail(27); break; }
+                if (!(ok = mbar_wait(bar(CB_UREADY), n & 1, lim, abort_flag))) { fail(64); break; }
                 tc_fence_after();
                 // b: S += U^T K   (A = U tile K-major; B = K tile MN-major)
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(tm + TM_C4, dU + ((ks * 32) >> 4), dKQm + ((kq + ks * 2048) >> 4), id_b, 1);
-                mma_commit(bar_addr(sm, B_B));
+                    mma_bf16_ss(tm + TM_S, dU + ((ks * 32) >> 4), dSTm + ((st + CS_KQ + ks * 2048) >> 4), id_b, 1);
+                mma_commit(bar(CB_B));
                 // c2: O2 = U^T Phat^T
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(tm + TM_C6 + s * 128, dU + ((ks * 32) >> 4),
-                                dPH + ((s * 8192 + ks * 32) >> 4), id_c1, ks > 0);
-                mma_commit(bar_addr(sm, B_C));
-                mma_commit(bar_addr(sm, B_EMPTY_KQ + s));
+                    mma_bf16_ss(tm + TM_O2 + s * 128, dU + ((ks * 32) >> 4),
+                                dSTk + ((st + CS_PH + ks * 32) >> 4), id_n64, ks > 0);
+                mma_commit(bar(CB_C));
+                mma_commit(bar(CB_EMPTY + s));
             }
-            // drain: every issued MMA completes before TMEM is released
-            mma_commit(bar_addr(sm, B_FIN));
-            if (!mbar_wait(bar_addr(sm, B_FIN), 0, lim, abort_flag)) {
-                // one more bounded wait that ignores the abort flag
+            mma_commit(bar(CB_FIN));   // every issued MMA completes before TMEM is released
+            if (!mbar_wait(bar(CB_FIN), 0, lim, abort_flag)) {
                 const int zero = 0;
-                mbar_wait(bar_addr(sm, B_FIN), 0, lim, &zero);
+                mbar_wait(bar(CB_FIN), 0, lim, &zero);
             }
-        }
-    } else if (warp >= 4) {
-        // ------------------------------------------------------------ prep group
-        const int pt = tid - 128, pw = warp - 4;
-        PrepScalars *sc = reinterpret_cast<PrepScalars *>(sm + OFF_SCP);
-        float *Af = reinterpret_cast<float *>(sm + OFF_AF);
-        float *Tf = reinterpret_cast<float *>(sm + OFF_TF);
-        float *mm = reinterpret_cast<float *>(sm + OFF_MM) + pw * 256;
-        const uint32_t lane_off = static_cast<uint32_t>(pw * 32) << 16;
-        GateRegs gr{0.f, 0.f, 0.f, 0.f};
-        if (pw == 0) gr = load_gates(p.g, p.beta, bos, eos, 0, nchunks, h, H, lane);
-        for (int n = 0; n < nchunks; ++n) {
-            const int s = n & 1;
-            if (named_bar_any(1, 128, *abort_flag != 0)) break;
-            if (pw == 0) {
-                float G0, G1;
-                scan_gates(gr, lane, G0, G1);
-                const float b0 = gr.b0, b1 = gr.b1;
-                gr = load_gates(p.g, p.beta, bos, eos, n + 1, nchunks, h, H, lane);
-                const float GC = __shfl_sync(0xffffffffu, G1, 31);
-                sc->inv[lane] = expf(-G0); sc->inv[lane + 32] = expf(-G1);
-                sc->beta[lane] = b0; sc->beta[lane + 32] = b1;
-                sc->bg[lane] = b0 * expf(G0); sc->bg[lane + 32] = b1 * expf(G1);
-                sc->Dd[lane] = expf(GC - G0); sc->Dd[lane + 32] = expf(GC - G1);
-            }
-            named_bar_sync(1, 128);
-            // A (strictly lower, decayed, beta-scaled) and Phat from p1
-            if (!mbar_wait(bar_addr(sm, B_P1), n & 1, lim, abort_flag)) fail(31);
-            tc_fence_after();
-            {
-                float x[64];
-                float (&x0)[32] = *reinterpret_cast<float (*)[32]>(&x[0]);
-                float (&x1)[32] = *reinterpret_cast<float (*)[32]>(&x[32]);
-                tmem_ld32(tm + lane_off + TM_C12, x0);
-                tmem_ld32(tm + lane_off + TM_C12 + 32, x1);
-                if (pt < 64) {
-                    // A[r][i] = beta_r exp(G_r - G_i) k_r.k_i = (beta_r gamma_r) exp(-G_i) KK[r][i]
-                    const int r = pt;
-                    const float bgr = sc->bg[r];
-#pragma unroll
-                    for (int i = 0; i < 64; i += 4) {
-                        const float4 iv = *reinterpret_cast<const float4 *>(&sc->inv[i]);
-                        float4 a;
-                        a.x = (i < r) ? bgr * iv.x * x[i] : 0.f;
-                        a.y = (i + 1 < r) ? bgr * iv.y * x[i + 1] : 0.f;
-                        a.z = (i + 2 < r) ? bgr * iv.z * x[i + 2] : 0.f;
-                        a.w = (i + 3 < r) ? bgr * iv.w * x[i + 3] : 0.f;
-                        *reinterpret_cast<float4 *>(&Af[r * AP + i]) = a;
-                    }
-                } else {
-                    const int r = pt - 64;
-                    const uint32_t row = smem_u32(sm + OFF_PH + s * 8192);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int i0 = 8 * c + 2 * e;
-                            w[e] = pack_bf16(i0 <= r ? x[i0] : 0.f, i0 + 1 <= r ? x[i0 + 1] : 0.f);
-                        }
-                        st_shared_v4(row + sw128_chunk(r, c), w[0], w[1], w[2], w[3]);
-                    }
-                }
-            }
-            tc_fence_before();
-            fence_proxy_async_smem();
-            named_bar_sync(1, 128);
-            // T = (I + A)^-1: 16x16 diagonal blocks by forward substitution ...
-            if (pt < 64) {
-                const int b = pt >> 4, c = pt & 15;
-                const float *Ab = Af + (16 * b) * AP + 16 * b;
-                float x[16];
-#pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    float ps[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int i = 0; i < r; ++i) ps[i & 3] = fmaf(Ab[r * AP + i], x[i], ps[i & 3]);
-                    x[r] = ((r == c) ? 1.f : 0.f) - ((ps[0] + ps[1]) + (ps[2] + ps[3]));
-                }
-#pragma unroll
-                for (int r = 0; r < 16; ++r) Tf[(16 * b + r) * AP + 16 * b + c] = x[r];
-            } else {
-                // zero the blocks above the diagonal
-                for (int e = pt - 64; e < 6 * 256; e += 64) {
-                    const int blk = e >> 8, w = e & 255;
-                    const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-                    const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-                    Tf[(16 * bi + (w >> 4)) * AP + 16 * bj + (w & 15)] = 0.f;
-                }
-            }
-            named_bar_sync(1, 128);
-            // ... then the off-diagonal blocks, one band at a time
-            if (pw < 3) solve_block(Af, Tf, mm, pw + 1, pw, lane);
-            named_bar_sync(1, 128);
-            if (pw < 2) solve_block(Af, Tf, mm, pw + 2, pw, lane);
-            named_bar_sync(1, 128);
-            if (pw == 0) solve_block(Af, Tf, mm, 3, 0, lane);
-            named_bar_sync(1, 128);
-            // T'' of the previous chunk may still be feeding its p3
-            if (n > 0 && !mbar_wait(bar_addr(sm, B_P3), (n - 1) & 1, lim, abort_flag)) fail(33);
-            // T' = diag(D) T diag(beta gamma), T'' = diag(D) T diag(beta), bf16, K-major rows t
-            {
-                const int which = pt >> 6, r = pt & 63;
-                const uint32_t row = smem_u32(sm + (which ? OFF_TPP : OFF_TP));
-                const float *colscale = which ? sc->beta : sc->bg;
-                const float dr = sc->Dd[r];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const float4 t0v = *reinterpret_cast<const float4 *>(&Tf[r * AP + 8 * c]);
-                    const float4 t1v = *reinterpret_cast<const float4 *>(&Tf[r * AP + 8 * c + 4]);
-                    const float4 s0v = *reinterpret_cast<const float4 *>(&colscale[8 * c]);
-                    const float4 s1v = *reinterpret_cast<const float4 *>(&colscale[8 * c + 4]);
-                    st_shared_v4(row + sw128_chunk(r, c),
-                                 pack_bf16(dr * t0v.x * s0v.x, dr * t0v.y * s0v.y),
-                                 pack_bf16(dr * t0v.z * s0v.z, dr * t0v.w * s0v.w),
-                                 pack_bf16(dr * t1v.x * s1v.x, dr * t1v.y * s1v.y),
-                                 pack_bf16(dr * t1v.z * s1v.z, dr * t1v.w * s1v.w));
-                }
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(bar_addr(sm, B_TREADY));
-            // W from p2's W^T (TMEM lane = d_k index, column = t), in the U^T columns
-            if (!mbar_wait(bar_addr(sm, B_P2), n & 1, lim, abort_flag)) fail(32);
-            tc_fence_after();
-            {
-                float x[32];
-                uint8_t *wt = sm + OFF_W + (pt >> 6) * 8192;
-                const int col = pt & 63;
-                for (int half = 0; half < 2; ++half) {
-                    tmem_ld32(tm + lane_off + TM_C3 + 32 * half, x);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        *reinterpret_cast<__nv_bfloat16 *>(wt + sw128_offset(32 * half + i, col)) =
-                            __float2bfloat16_rn(x[i]);
-                }
-            }
-            tc_fence_before();
-            fence_proxy_async_smem();
-            mbar_arrive(bar_addr(sm, B_WREADY));
         }
     } else {
         // ------------------------------------------------------------ chain group
         const int dv = tid;   // TMEM lane and state row
         const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-        ChainScalars *scb = reinterpret_cast<ChainScalars *>(sm + OFF_SCE);
+        ChainScalars *scb = reinterpret_cast<ChainScalars *>(sm + C_SCE);
         GateRegs gr{0.f, 0.f, 0.f, 0.f};
         if (warp == 0) gr = load_gates(p.g, p.beta, bos, eos, 0, nchunks, h, H, lane);
         // scalars of chunk m from the prefetched gates; prefetch chunk m+1's
@@ -564,15 +671,14 @@ gdn_prefill_tc_kernel(const __grid_constant__ TcParams p) {
                 gr = load_gates(p.g, p.beta, bos, eos, m + 1, nchunks, h, H, lane);
                 const float GC = __shfl_sync(0xffffffffu, G1, 31);
                 ChainScalars &cs = scb[m % 3];
-                cs.Dd[lane] = expf(GC - G0); cs.Dd[lane + 32] = expf(GC - G1);
                 cs.gam[lane] = expf(G0); cs.gam[lane + 32] = expf(G1);
                 cs.invD[lane] = expf(G0 - GC); cs.invD[lane + 32] = expf(G1 - GC);
                 if (lane == 0) { cs.gC = expf(GC); cs.len = len; }
             }
         };
-        // write S (fp32 row dv, 32 columns starting at c0) as bf16 into the A tile
+        // write S (fp32 row dv, 32 columns from c0) as bf16 into the A tile
         auto store_s_bf16 = [&](const float (&x)[32], int c0) {
-            const uint32_t base = smem_u32(sm + OFF_S + (c0 >> 6) * 16384);
+            const uint32_t base = smem_u32(sm + C_S + (c0 >> 6) * 16384);
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
                 const int chunk = ((c0 & 63) >> 3) + q4;
@@ -589,52 +695,52 @@ gdn_prefill_tc_kernel(const __grid_constant__ TcParams p) {
             for (int c0 = 0; c0 < D; c0 += 32) {
 #pragma unroll
                 for (int j = 0; j < 32; j += 4) {
-                    float4 v = p.state_in ? *reinterpret_cast<const float4 *>(p.state_in + state_off + (size_t)dv * D + c0 + j)
-                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                    const float4 v = p.state_in ? *reinterpret_cast<const float4 *>(p.state_in + state_off + (size_t)dv * D + c0 + j)
+                                                : make_float4(0.f, 0.f, 0.f, 0.f);
                     x[j] = v.x; x[j + 1] = v.y; x[j + 2] = v.z; x[j + 3] = v.w;
                 }
                 store_s_bf16(x, c0);
 #pragma unroll
                 for (int j = 0; j < 32; ++j) x[j] *= gC0;
-                tmem_st32(tm + lane_off + TM_C4 + c0, x);
+                tmem_st32(tm + lane_off + TM_S + c0, x);
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(bar_addr(sm, B_SREADY));
+            mbar_arrive(bar(CB_SREADY));
         }
         for (int n = 0; n < nchunks; ++n) {
             const int s = n & 1;
-            // ring of three: warp 0 may write chunk n+1's scalars while a
-            // slower warp still reads chunk n-1's in its output epilogue
+            // ring of three: warp 0 may write chunk n+1's scalars while a slower
+            // warp still reads chunk n-1's in its output epilogue
             const ChainScalars &cs = scb[n % 3];
-            // U epilogue: the D-scaled residual U^T -> U tile (row dv, 64 t)
-            if (!mbar_wait(bar_addr(sm, B_A), n & 1, lim, abort_flag)) fail(41);
+            // residual epilogue: U^T (fp32, lane dv, 64 t) -> bf16 U tile
+            if (!mbar_wait(bar(CB_A), n & 1, lim, abort_flag)) fail(71);
             tc_fence_after();
             {
-                const uint32_t row = smem_u32(sm + OFF_U);
+                const uint32_t row = smem_u32(sm + C_U);
                 float x[32];
                 for (int half = 0; half < 2; ++half) {
-                    tmem_ld32(tm + lane_off + TM_C3 + 32 * half, x);
+                    tmem_ld32(tm + lane_off + TM_U + 32 * half, x);
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4)
-                        st_shared_v4(row + sw128_chunk(dv, 4 * half + q4),
-                                     pack_bf16(x[8 * q4], x[8 * q4 + 1]), pack_bf16(x[8 * q4 + 2], x[8 * q4 + 3]),
-                                     pack_bf16(x[8 * q4 + 4], x[8 * q4 + 5]), pack_bf16(x[8 * q4 + 6], x[8 * q4 + 7]));
+                        st_shared_v4(row + sw128_chunk(dv, 4 * half + q4), pack_bf16(x[8 * q4], x[8 * q4 + 1]),
+                                     pack_bf16(x[8 * q4 + 2], x[8 * q4 + 3]), pack_bf16(x[8 * q4 + 4], x[8 * q4 + 5]),
+                                     pack_bf16(x[8 * q4 + 6], x[8 * q4 + 7]));
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(bar_addr(sm, B_UREADY));
+            mbar_arrive(bar(CB_UREADY));
             const bool last = (n + 1 == nchunks);
             if (!last) compute_scalars(n + 1);
             if (named_bar_any(2, 128, *abort_flag != 0)) break;
-            // S epilogue
-            if (!mbar_wait(bar_addr(sm, B_B), n & 1, lim, abort_flag)) fail(42);
+            // state epilogue: publish the bf16 copy for the next (a), then rescale
+            if (!mbar_wait(bar(CB_B), n & 1, lim, abort_flag)) fail(72);
             tc_fence_after();
             {
                 float x[32];
                 for (int c0 = 0; c0 < D; c0 += 32) {
-                    tmem_ld32(tm + lane_off + TM_C4 + c0, x);
+                    tmem_ld32(tm + lane_off + TM_S + c0, x);
                     if (!last) {
                         store_s_bf16(x, c0);
                     } else if (p.state_out) {
@@ -647,30 +753,30 @@ gdn_prefill_tc_kernel(const __grid_constant__ TcParams p) {
                 fence_proxy_async_smem();
                 tc_fence_before();
                 if (!last) {
-                    // the next (a) may start now; rescale the fp32 state for the
+                    // the next (a) may start now; the fp32 state is rescaled for the
                     // next (b), which the MMA thread issues only after U_READY
-                    mbar_arrive(bar_addr(sm, B_SREADY));
+                    mbar_arrive(bar(CB_SREADY));
                     const float gnext = scb[(n + 1) % 3].gC;
                     for (int c0 = 0; c0 < D; c0 += 32) {
-                        tmem_ld32(tm + lane_off + TM_C4 + c0, x);
+                        tmem_ld32(tm + lane_off + TM_S + c0, x);
 #pragma unroll
                         for (int j = 0; j < 32; ++j) x[j] *= gnext;
-                        tmem_st32(tm + lane_off + TM_C4 + c0, x);
+                        tmem_st32(tm + lane_off + TM_S + c0, x);
                     }
                     tc_fence_before();
                 }
             }
-            // O epilogue: o_t = gamma_t O1 + exp(G_t - G_C) O2
-            if (!mbar_wait(bar_addr(sm, B_C), n & 1, lim, abort_flag)) fail(43);
+            // output epilogue: o_t = gamma_t O1 + exp(G_t - G_C) O2
+            if (!mbar_wait(bar(CB_C), n & 1, lim, abort_flag)) fail(73);
             tc_fence_after();
             {
                 // stage the [64 t][128 dv] bf16 tile in the U buffer (free once
                 // c2 has completed), then write whole 16-byte pieces of rows
-                __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_U);
+                __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(sm + C_U);
                 float a[32], b[32];
                 for (int half = 0; half < 2; ++half) {
-                    tmem_ld32(tm + lane_off + TM_C5 + s * 128 + 32 * half, a);
-                    tmem_ld32(tm + lane_off + TM_C6 + s * 128 + 32 * half, b);
+                    tmem_ld32(tm + lane_off + TM_O1 + s * 128 + 32 * half, a);
+                    tmem_ld32(tm + lane_off + TM_O2 + s * 128 + 32 * half, b);
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int t = 32 * half + j;
@@ -690,14 +796,14 @@ gdn_prefill_tc_kernel(const __grid_constant__ TcParams p) {
                         *reinterpret_cast<uint4 *>(p.out + ((size_t)(t0 + t) * H + h) * D + piece * 8) = v;
                     }
                 }
-                named_bar_sync(2, 128);   // the U buffer is rewritten by the next U epilogue
+                named_bar_sync(2, 128);   // the U buffer is rewritten by the next residual epilogue
             }
         }
     }
 
     // ---------------------------------------------------------------- teardown
     __syncthreads();
-    if (warp == 8) {
+    if (warp == 4) {
         tc_fence_after();
         tmem_dealloc(tm, TM_COLS);
     }
@@ -735,39 +841,76 @@ bool make_token_map(CUtensorMap *m, const void *base, int64_t T, int H) {
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t chunk_off_bytes(int num_seqs) { return align_up(4 * (size_t)(num_seqs + 1), 1024); }
+
+bool set_smem_attrs() {
+    static bool done[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    if (dev >= 0 && dev < 64 && done[dev]) return true;
+    if (cudaFuncSetAttribute(gdn_chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)P_ALLOC) != cudaSuccess)
+        return false;
+    if (cudaFuncSetAttribute(gdn_chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)C_ALLOC) != cudaSuccess)
+        return false;
+    if (dev >= 0 && dev < 64) done[dev] = true;
+    return true;
+}
+
 }  // namespace
 
-size_t prefill_tc_smem_bytes() { return SMEM_ALLOC; }
+size_t tc_workspace_bytes(int num_seqs, int64_t total_tokens, int H, bool varlen) {
+    return 1024 + chunk_off_bytes(num_seqs) +
+           (size_t)tc_chunk_bound(num_seqs, total_tokens, varlen) * (size_t)H * kTileBytes;
+}
+
+int tc_kernel_count(bool varlen) { return varlen ? 3 : 2; }
 
 cudaError_t launch_prefill_tc(const TcLaunch &L, cudaStream_t stream) {
-    TcParams p;
-    memset(&p, 0, sizeof(p));
-    if (!make_token_map(&p.map_q, L.q, L.total_tokens, L.H) ||
-        !make_token_map(&p.map_k, L.k, L.total_tokens, L.H) ||
-        !make_token_map(&p.map_v, L.v, L.total_tokens, L.H))
+    const bool varlen = L.cu_seqlens != nullptr;
+    uint8_t *ws = static_cast<uint8_t *>(L.workspace);
+    int32_t *chunk_off = varlen ? reinterpret_cast<int32_t *>(ws + 1024) : nullptr;
+    uint8_t *tiles = ws + 1024 + chunk_off_bytes(L.num_seqs);
+    const int cps = varlen ? 0 : (int)((L.uniform_len + C - 1) / C);
+    const int64_t bound = tc_chunk_bound(L.num_seqs, L.total_tokens, varlen);
+    if (bound <= 0) return cudaSuccess;
+    if (bound > 0x7fffffff || L.H > 65535) return cudaErrorInvalidValue;
+
+    PrepParams pp;
+    ChainParams cp;
+    memset(&pp, 0, sizeof(pp));
+    memset(&cp, 0, sizeof(cp));
+    if (!make_token_map(&pp.map_q, L.q, L.total_tokens, L.H) ||
+        !make_token_map(&pp.map_k, L.k, L.total_tokens, L.H) ||
+        !make_token_map(&cp.map_v, L.v, L.total_tokens, L.H))
         return cudaErrorInvalidValue;
-    p.g = L.g;
-    p.beta = L.beta;
-    p.state_in = L.state_in;
-    p.state_out = L.state_out;
-    p.out = static_cast<__nv_bfloat16 *>(L.out);
-    p.cu_seqlens = L.cu_seqlens;
-    p.uniform_len = L.uniform_len;
-    p.order = L.order;
-    p.H = L.H;
-    p.err = L.err;
-    p.timeout_ns = L.timeout_ns;
-    static bool attr_done[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gdn_prefill_tc_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_done[dev] = true;
-    }
-    const unsigned grid = (unsigned)L.num_seqs * (unsigned)L.H;
-    gdn_prefill_tc_kernel<<<grid, kThreads, SMEM_ALLOC, stream>>>(p);
+    cp.map_q = pp.map_q;
+    cp.map_k = pp.map_k;
+    pp.g = cp.g = L.g;
+    pp.beta = cp.beta = L.beta;
+    pp.cu_seqlens = cp.cu_seqlens = L.cu_seqlens;
+    pp.chunk_off = cp.chunk_off = chunk_off;
+    pp.uniform_len = cp.uniform_len = L.uniform_len;
+    pp.cps = cp.cps = cps;
+    pp.num_seqs = L.num_seqs;
+    pp.H = cp.H = L.H;
+    pp.tiles = tiles;
+    cp.tiles = tiles;
+    pp.err = cp.err = L.err;
+    pp.timeout_ns = cp.timeout_ns = L.timeout_ns;
+    cp.state_in = L.state_in;
+    cp.state_out = L.state_out;
+    cp.out = static_cast<__nv_bfloat16 *>(L.out);
+
+    if (!set_smem_attrs()) return cudaGetLastError() != cudaSuccess ? cudaGetLastError() : cudaErrorUnknown;
+    if (varlen) gdn_chunk_offsets_kernel<<<1, 1024, 0, stream>>>(L.cu_seqlens, L.num_seqs, chunk_off);
+    dim3 pgrid((unsigned)bound, (unsigned)L.H);
+    gdn_chunk_prep_kernel<<<pgrid, kPrepThreads, P_ALLOC, stream>>>(pp);
+    gdn_chunk_chain_kernel<<<(unsigned)L.num_seqs * (unsigned)L.H, kChainThreads, C_ALLOC, stream>>>(cp);
     return cudaGetLastError();
 }
 
