@@ -6,10 +6,10 @@
 //
 //   A    = strict_lower(beta_r exp(G_r - G_i) k_r.k_i),   T = (I + A)^-1
 //   T'   = diag(D) T diag(beta gamma),   T'' = diag(D) T diag(beta)
-//   W    = T' K,   Phat = tril(Q K^T)
+//   W    = T' K,   Qg = diag(gamma) Q,   Pt = diag(exp(G_t - G_C)) tril(Q K^T)
 //   U^T  = V^T T''^T - S W^T           (the D-scaled delta residual)
 //   S   <- gamma_C S + U^T K
-//   o_t  = gamma_t (S Q^T)[:,t] + exp(G_t - G_C) (U^T Phat^T)[:,t]
+//   O^T  = S Qg^T + U^T Pt^T           (o_t = S_t q_t for every token of the chunk)
 //
 // which is the token recurrence S_t = a_t S_{t-1}(I - b_t k_t k_t^T) +
 // b_t v_t k_t^T, o_t = S_t q_t unrolled over the chunk.
@@ -18,14 +18,16 @@
 //   TMA brings K and Q; p1 = [K;Q] K^T on tcgen05 (TMEM); four warps form A
 //   and Phat, invert I + A (16x16 diagonal blocks by substitution, the
 //   off-diagonal blocks with tf32 mma.sync), scale T' and T''; p2 = K^T T'^T
-//   on tcgen05 gives W^T, which is transposed into W.  W, T'' and Phat are
+//   on tcgen05 gives W^T, which is transposed into W.  W, Qg, T'' and Pt are
 //   written to the workspace in the 128-byte-swizzled layout the chain
 //   kernel's MMAs read, so it copies them with one bulk copy per chunk.
 // gdn_chunk_chain_kernel: one CTA per (sequence, head), fp32 state in TMEM:
-//   p3 U^T = V^T T''^T, (a) U^T -= S W^T, (b) S += U^T K, c1 S Q^T,
-//   c2 U^T Phat^T -- five M = 128 tcgen05 MMAs per chunk -- with a
-//   four-warp epilogue group (residual, state, output), one MMA thread and
-//   one TMA thread.  The state never leaves the SM between chunks.
+//   p3 U^T = V^T T''^T, (a) U^T -= S W^T, (b) S += U^T K, c1 O^T = S Qg^T,
+//   c2 O^T += U^T Pt^T -- five M = 128 tcgen05 MMAs per chunk, the S and U^T
+//   operands read from TMEM -- with a four-warp state group (residual and
+//   state epilogues, the serial chain), a four-warp output group (output
+//   epilogue, off the chain), one MMA thread and one TMA thread.  The state
+//   never leaves the SM between chunks.
 //
 // Tokens past the end of a sequence inside its last chunk get g = 0 and
 // beta = 0, which zeroes their rows of W and T'' and keeps the state
@@ -50,11 +52,11 @@ constexpr int kPrepThreads = 160;                      // warps 0-3 prep, warp 4
 constexpr uint32_t P_KQ = 0;                           // [2 kb][128 rows: K 0-63, Q 64-127][128 B]
 constexpr uint32_t P_TP = P_KQ + 32768;                // T'  bf16 [64 t][128 B]
 constexpr uint32_t P_TPP = P_TP + 8192;                // T'' bf16 [64 t][128 B]
-constexpr uint32_t P_PH = P_TPP + 8192;                // Phat bf16 [64 t][128 B]
+constexpr uint32_t P_PH = P_TPP + 8192;                // Pt bf16 [64 t][128 B]
 constexpr uint32_t P_AF = P_PH + 8192;                 // A fp32 [64][AP]; later W staging [2 kb][64][128 B]
 constexpr uint32_t P_TF = P_AF + 64 * AP * 4;          // T fp32 [64][AP]
 constexpr uint32_t P_SC = P_TF + 64 * AP * 4;          // PrepScalars
-constexpr uint32_t P_MM = P_SC + 1024;                 // solve scratch, 4 warps x 16x16 fp32
+constexpr uint32_t P_MM = P_SC + 2048;                 // solve scratch, 4 warps x 16x16 fp32
 constexpr uint32_t P_BAR = P_MM + 4096;                // mbarriers + TMEM base
 constexpr uint32_t P_ALLOC = P_BAR + 64 + 1024;        // + alignment slack
 static_assert(64 * AP * 4 >= 16384, "W staging fits in the A buffer");
@@ -62,30 +64,32 @@ constexpr uint32_t P_TM_COLS = 128;                    // p1 output at 0, p2 out
 enum { PB_FULL = 0, PB_P1 = 1, PB_TREADY = 2, PB_P2 = 3, PB_FIN = 4, PB_NUM = 5 };
 
 // ------------------------------------------------------------ chain kernel layout
-constexpr int kChainThreads = 192;                     // warps 0-3 chain, 4 MMA, 5 TMA
-constexpr uint32_t C_STAGE = 81920;                    // per stage: KQ, V, W, T'', Phat
-constexpr uint32_t CS_KQ = 0, CS_V = 32768, CS_W = 49152, CS_TPP = 65536, CS_PH = 73728;
-constexpr uint32_t C_S = 2 * C_STAGE;                  // S bf16 [2 kb][128 dv][128 B]
-constexpr uint32_t C_U = C_S + 32768;                  // U^T bf16 [128 dv][128 B]; output staging
-constexpr uint32_t C_SCE = C_U + 16384;                // ChainScalars x 3
+constexpr int kChainThreads = 320;                     // warps 0-3 chain, 4-7 output, 8 MMA, 9 TMA
+constexpr uint32_t C_STAGE = 81920;                    // per stage: K, V, W, Qg, T'', Pt
+constexpr uint32_t CS_K = 0, CS_V = 16384, CS_W = 32768, CS_QG = 49152, CS_TPP = 65536, CS_PT = 73728;
+constexpr uint32_t C_U = 2 * C_STAGE;                  // output staging [64 t][128 dv] bf16
+constexpr uint32_t C_SCE = C_U + 16384;                // ChainScalars x 3 (state group)
 constexpr uint32_t C_BAR = C_SCE + 3072;               // mbarriers + TMEM base + abort flag
 constexpr uint32_t C_ALLOC = C_BAR + 256 + 1024;
-static_assert(CS_PH + 8192 == C_STAGE, "stage layout");
-// TMEM columns of the chain kernel
-constexpr uint32_t TM_U = 64;      // U^T accumulator (64)
+static_assert(CS_PT + 8192 == C_STAGE && C_STAGE - CS_W == kTileBytes, "stage layout");
+// TMEM columns of the chain kernel.  The MMA A operands produced by the chain
+// itself (bf16 S and bf16 U^T) stay in TMEM: shared-memory bandwidth, not the
+// tensor core, bounds these small-N MMAs, so only B is read from shared memory.
+constexpr uint32_t TM_SBF = 0;     // S bf16, two per column (64)
+constexpr uint32_t TM_U = 64;      // U^T accumulator (64); then U^T bf16 in its first 32
 constexpr uint32_t TM_S = 128;     // state S (128)
-constexpr uint32_t TM_O1 = 256;    // S Q^T [2 bufs] at 256, 384 (64 each)
-constexpr uint32_t TM_O2 = 320;    // U^T Phat^T [2 bufs] at 320, 448
+constexpr uint32_t TM_O = 256;     // O^T [2 bufs] at 256, 320 (64 each)
 constexpr uint32_t TM_COLS = 512;
-enum { CB_FULL = 0, CB_EMPTY = 2, CB_A = 4, CB_B = 5, CB_C = 6, CB_SREADY = 7, CB_UREADY = 8,
-       CB_FIN = 9, CB_NUM = 10 };
+// Barriers that a role may complete twice before its consumer waits once are
+// per buffer (FULL/EMPTY per stage, C/OFREE per output buffer) and waited with
+// the parity of the buffer's use count, so that no phase can be skipped.
+enum { CB_FULL = 0, CB_EMPTY = 2, CB_A = 4, CB_B = 5, CB_C = 6, CB_SREADY = 8, CB_UREADY = 9,
+       CB_FIN = 10, CB_OFREE = 11, CB_NUM = 13 };
 
-struct ChainScalars {   // per chunk, chain group
-    float gam[C];       // exp(G_t)
-    float invD[C];      // exp(G_t - G_C)
+struct ChainScalars {   // per chunk, state group
     float gC;           // exp(G_C)
     int len;
-    int pad[126];
+    int pad[254];
 };
 static_assert(sizeof(ChainScalars) == 1024, "scalar block size");
 
@@ -94,8 +98,11 @@ struct PrepScalars {
     float beta[C];
     float bg[C];        // beta * gamma
     float Dd[C];        // exp(G_C - G_t)
+    float gam[C];       // exp(G_t)
+    float invD[C];      // exp(G_t - G_C)
+    float pad[2 * C];
 };
-static_assert(sizeof(PrepScalars) == 1024, "scalar block size");
+static_assert(sizeof(PrepScalars) == 2048, "scalar block size");
 
 struct PrepParams {
     CUtensorMap map_q, map_k;
@@ -111,7 +118,7 @@ struct PrepParams {
 };
 
 struct ChainParams {
-    CUtensorMap map_q, map_k, map_v;
+    CUtensorMap map_k, map_v;
     const float *g, *beta, *state_in;
     float *state_out;
     __nv_bfloat16 *out;
@@ -394,6 +401,8 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
             sc->beta[lane] = gr.b0; sc->beta[lane + 32] = gr.b1;
             sc->bg[lane] = gr.b0 * expf(G0); sc->bg[lane + 32] = gr.b1 * expf(G1);
             sc->Dd[lane] = expf(GC - G0); sc->Dd[lane + 32] = expf(GC - G1);
+            sc->gam[lane] = expf(G0); sc->gam[lane + 32] = expf(G1);
+            sc->invD[lane] = expf(G0 - GC); sc->invD[lane + 32] = expf(G1 - GC);
         }
         named_bar_sync(1, 128);
         bool ok = mbar_wait(bar(PB_P1), 0, lim, &no_abort);
@@ -419,7 +428,9 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
                     *reinterpret_cast<float4 *>(&Af[r * AP + i]) = a;
                 }
             } else {
+                // Pt[r][i] = exp(G_r - G_C) q_r.k_i for i <= r
                 const int r = pt - 64;
+                const float sr = sc->invD[r];
                 const uint32_t row = smem_u32(sm + P_PH);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
@@ -427,9 +438,27 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int i0 = 8 * c + 2 * e;
-                        w[e] = pack_bf16(i0 <= r ? x[i0] : 0.f, i0 + 1 <= r ? x[i0 + 1] : 0.f);
+                        w[e] = pack_bf16(i0 <= r ? sr * x[i0] : 0.f, i0 + 1 <= r ? sr * x[i0 + 1] : 0.f);
                     }
                     st_shared_v4(row + sw128_chunk(r, c), w[0], w[1], w[2], w[3]);
+                }
+                // Qg = diag(gamma) Q, in place over the Q rows of the KQ tile
+                // (p1, their only tensor-core reader here, has completed)
+                const float gr = sc->gam[r];
+#pragma unroll
+                for (int kb = 0; kb < 2; ++kb) {
+                    uint4 *qrow = reinterpret_cast<uint4 *>(sm + P_KQ + kb * 16384 + (64 + r) * 128);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint4 v = qrow[c];
+                        __nv_bfloat162 *hv = reinterpret_cast<__nv_bfloat162 *>(&v);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __bfloat1622float2(hv[e]);
+                            hv[e] = __floats2bfloat162_rn(gr * f.x, gr * f.y);
+                        }
+                        qrow[c] = v;   // a whole 16-byte chunk: the swizzle is untouched
+                    }
                 }
             }
         }
@@ -503,13 +532,16 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
         tc_fence_before();
         named_bar_sync(1, 128);
         if (!ok && p.err && pt == 0) atomicCAS(p.err, 0, 52);
-        // W (16 KB), T'' (8 KB), Phat (8 KB) -> the workspace tile of (chunk, head)
+        // W (16 KB), Qg (16 KB), T'' (8 KB), Pt (8 KB) -> the workspace tile of (chunk, head)
         uint8_t *dst = p.tiles + ((size_t)gc * H + h) * kTileBytes;
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const int off = (k * 128 + pt) * 16;            // 0 .. 32 KB
-            const uint8_t *srcp = off < 16384 ? sm + P_AF + off : (off < 24576 ? sm + P_TPP + (off - 16384)
-                                                                                : sm + P_PH + (off - 24576));
+        for (int k = 0; k < 24; ++k) {
+            const int off = (k * 128 + pt) * 16;            // 0 .. 48 KB
+            const uint8_t *srcp;
+            if (off < 16384) srcp = sm + P_AF + off;                                        // W
+            else if (off < 32768) srcp = sm + P_KQ + ((off - 16384) >> 13) * 16384 + 8192 + ((off - 16384) & 8191);  // Qg
+            else if (off < 40960) srcp = sm + P_TPP + (off - 32768);                        // T''
+            else srcp = sm + P_PH + (off - 40960);                                          // Pt
             *reinterpret_cast<uint4 *>(dst + off) = *reinterpret_cast<const uint4 *>(srcp);
         }
     }
@@ -542,17 +574,16 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
 
     if (tid == 0) {
         for (int i = 0; i < CB_NUM; ++i)
-            mbar_init(bar(i), (i == CB_SREADY || i == CB_UREADY) ? 128 : 1);
+            mbar_init(bar(i), (i == CB_SREADY || i == CB_UREADY || i >= CB_OFREE) ? 128 : 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 4) {
+    if (warp == 8) {
         tmem_alloc(smem_u32(tmem_base_ptr), TM_COLS);
         tmem_relinquish();
     }
-    if (warp == 5 && lane == 0) {
+    if (warp == 9 && lane == 0) {
         tma_prefetch_desc(&p.map_k);
-        tma_prefetch_desc(&p.map_q);
         tma_prefetch_desc(&p.map_v);
     }
     tc_fence_before();
@@ -574,7 +605,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                 *reinterpret_cast<float4 *>(p.state_out + state_off + (size_t)tid * D + j) = v;
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ------------------------------------------------------------ TMA / bulk producer
         if (lane == 0) {
             int issued[2] = {0, 0};
@@ -586,8 +617,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                 const uint32_t full = bar(CB_FULL + s);
                 mbar_arrive_expect_tx(full, C_STAGE);
                 for (int kb = 0; kb < 2; ++kb) {
-                    tma_load_3d(st + CS_KQ + kb * 16384, &p.map_k, kb * 64, h, z, full);
-                    tma_load_3d(st + CS_KQ + kb * 16384 + 8192, &p.map_q, kb * 64, h, z, full);
+                    tma_load_3d(st + CS_K + kb * 8192, &p.map_k, kb * 64, h, z, full);
                     tma_load_3d(st + CS_V + kb * 8192, &p.map_v, kb * 64, h, z, full);
                 }
                 bulk_load(st + CS_W, p.tiles + ((size_t)(gc0 + n) * H + h) * kTileBytes, (uint32_t)kTileBytes, full);
@@ -597,7 +627,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
             for (int s = 0; s < 2; ++s)
                 if (issued[s]) mbar_wait(bar(CB_FULL + s), (issued[s] - 1) & 1, lim, &zero);
         }
-    } else if (warp == 4) {
+    } else if (warp == 8) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t id_n64 = idesc_bf16(128, 64, false, false);
@@ -606,10 +636,8 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
             const uint32_t id_b = idesc_bf16(128, 128, false, true);
             // descriptors are built once; a byte offset o inside a tile adds o >> 4
             const uint64_t dSTk = desc_sw128(smem_u32(sm), 16, 1024);      // K-major views of stage data
-            const uint64_t dSTm = desc_sw128(smem_u32(sm), 16384, 1024);   // MN-major view of K
+            const uint64_t dSTm = desc_sw128(smem_u32(sm), 8192, 1024);    // MN-major view of K
             const uint64_t dVm = desc_sw128(smem_u32(sm), 8192, 1024);     // MN-major view of V
-            const uint64_t dS = desc_sw128(smem_u32(sm + C_S), 16, 1024);
-            const uint64_t dU = desc_sw128(smem_u32(sm + C_U), 16, 1024);
             bool ok = true;
             for (int n = 0; ok && n < nchunks; ++n) {
                 const int s = n & 1;
@@ -624,28 +652,29 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                 tc_fence_after();
                 // a: U^T -= S W^T
                 for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
                     const uint32_t offw = st + CS_W + (ks >> 2) * 8192 + (ks & 3) * 32;
-                    mma_bf16_ss(tm + TM_U, dS + (off >> 4), dSTk + (offw >> 4), id_a, 1);
+                    mma_bf16_ts(tm + TM_U, tm + TM_SBF + 8 * ks, dSTk + (offw >> 4), id_a, 1);
                 }
                 mma_commit(bar(CB_A));
-                // c1: O1 = S Q^T (off the state chain)
+                // the output group has read this buffer pair for chunk n-2
+                if (n >= 2 && !(ok = mbar_wait(bar(CB_OFREE + s), ((n - 2) >> 1) & 1, lim, abort_flag))) { fail(65); break; }
+                tc_fence_after();
+                // c1: O^T = S Qg^T (off the state chain)
                 for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                    mma_bf16_ss(tm + TM_O1 + s * 128, dS + (off >> 4),
-                                dSTk + ((st + CS_KQ + off + 8192) >> 4), id_n64, ks > 0);
+                    const uint32_t off = st + CS_QG + (ks >> 2) * 8192 + (ks & 3) * 32;
+                    mma_bf16_ts(tm + TM_O + s * 64, tm + TM_SBF + 8 * ks, dSTk + (off >> 4), id_n64, ks > 0);
                 }
                 if (!(ok = mbar_wait(bar(CB_UREADY), n & 1, lim, abort_flag))) { fail(64); break; }
                 tc_fence_after();
-                // b: S += U^T K   (A = U tile K-major; B = K tile MN-major)
+                // b: S += U^T K   (A = U^T bf16 in TMEM; B = K tile MN-major)
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(tm + TM_S, dU + ((ks * 32) >> 4), dSTm + ((st + CS_KQ + ks * 2048) >> 4), id_b, 1);
+                    mma_bf16_ts(tm + TM_S, tm + TM_U + 8 * ks, dSTm + ((st + CS_K + ks * 2048) >> 4), id_b, 1);
                 mma_commit(bar(CB_B));
-                // c2: O2 = U^T Phat^T
+                // c2: O^T += U^T Pt^T
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(tm + TM_O2 + s * 128, dU + ((ks * 32) >> 4),
-                                dSTk + ((st + CS_PH + ks * 32) >> 4), id_n64, ks > 0);
-                mma_commit(bar(CB_C));
+                    mma_bf16_ts(tm + TM_O + s * 64, tm + TM_U + 8 * ks, dSTk + ((st + CS_PT + ks * 32) >> 4),
+                                id_n64, 1);
+                mma_commit(bar(CB_C + s));
                 mma_commit(bar(CB_EMPTY + s));
             }
             mma_commit(bar(CB_FIN));   // every issued MMA completes before TMEM is released
@@ -654,8 +683,8 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                 mbar_wait(bar(CB_FIN), 0, lim, &zero);
             }
         }
-    } else {
-        // ------------------------------------------------------------ chain group
+    } else if (warp < 4) {
+        // ------------------------------------------------------------ state group
         const int dv = tid;   // TMEM lane and state row
         const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
         ChainScalars *scb = reinterpret_cast<ChainScalars *>(sm + C_SCE);
@@ -671,64 +700,53 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                 gr = load_gates(p.g, p.beta, bos, eos, m + 1, nchunks, h, H, lane);
                 const float GC = __shfl_sync(0xffffffffu, G1, 31);
                 ChainScalars &cs = scb[m % 3];
-                cs.gam[lane] = expf(G0); cs.gam[lane + 32] = expf(G1);
-                cs.invD[lane] = expf(G0 - GC); cs.invD[lane + 32] = expf(G1 - GC);
                 if (lane == 0) { cs.gC = expf(GC); cs.len = len; }
             }
         };
-        // write S (fp32 row dv, 32 columns from c0) as bf16 into the A tile
-        auto store_s_bf16 = [&](const float (&x)[32], int c0) {
-            const uint32_t base = smem_u32(sm + C_S + (c0 >> 6) * 16384);
+        // write 64 fp32 values of this lane's row as 32 packed bf16 columns
+        auto st_bf16_cols = [&](uint32_t col, const float (&x0)[32], const float (&x1)[32]) {
+            uint32_t pk[32];
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                const int chunk = ((c0 & 63) >> 3) + q4;
-                st_shared_v4(base + sw128_chunk(dv, chunk), pack_bf16(x[8 * q4], x[8 * q4 + 1]),
-                             pack_bf16(x[8 * q4 + 2], x[8 * q4 + 3]), pack_bf16(x[8 * q4 + 4], x[8 * q4 + 5]),
-                             pack_bf16(x[8 * q4 + 6], x[8 * q4 + 7]));
+            for (int j = 0; j < 16; ++j) {
+                pk[j] = pack_bf16(x0[2 * j], x0[2 * j + 1]);
+                pk[16 + j] = pack_bf16(x1[2 * j], x1[2 * j + 1]);
             }
+            tmem_st32u(tm + lane_off + col, pk);
         };
         compute_scalars(0);
         named_bar_sync(2, 128);
         {
             const float gC0 = scb[0].gC;
-            float x[32];
-            for (int c0 = 0; c0 < D; c0 += 32) {
+            float x0[32], x1[32];
+            for (int c0 = 0; c0 < D; c0 += 64) {
 #pragma unroll
                 for (int j = 0; j < 32; j += 4) {
-                    const float4 v = p.state_in ? *reinterpret_cast<const float4 *>(p.state_in + state_off + (size_t)dv * D + c0 + j)
-                                                : make_float4(0.f, 0.f, 0.f, 0.f);
-                    x[j] = v.x; x[j + 1] = v.y; x[j + 2] = v.z; x[j + 3] = v.w;
+                    const float *src = p.state_in + state_off + (size_t)dv * D + c0 + j;
+                    const float4 a = p.state_in ? *reinterpret_cast<const float4 *>(src) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    const float4 b = p.state_in ? *reinterpret_cast<const float4 *>(src + 32) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    x0[j] = a.x; x0[j + 1] = a.y; x0[j + 2] = a.z; x0[j + 3] = a.w;
+                    x1[j] = b.x; x1[j + 1] = b.y; x1[j + 2] = b.z; x1[j + 3] = b.w;
                 }
-                store_s_bf16(x, c0);
+                st_bf16_cols(TM_SBF + c0 / 2, x0, x1);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) x[j] *= gC0;
-                tmem_st32(tm + lane_off + TM_S + c0, x);
+                for (int j = 0; j < 32; ++j) { x0[j] *= gC0; x1[j] *= gC0; }
+                tmem_st32(tm + lane_off + TM_S + c0, x0);
+                tmem_st32(tm + lane_off + TM_S + c0 + 32, x1);
             }
-            fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(bar(CB_SREADY));
         }
         for (int n = 0; n < nchunks; ++n) {
             const int s = n & 1;
-            // ring of three: warp 0 may write chunk n+1's scalars while a slower
-            // warp still reads chunk n-1's in its output epilogue
-            const ChainScalars &cs = scb[n % 3];
-            // residual epilogue: U^T (fp32, lane dv, 64 t) -> bf16 U tile
+            // residual epilogue: U^T (fp32, lane dv, 64 t) -> bf16 in its own first 32 columns
             if (!mbar_wait(bar(CB_A), n & 1, lim, abort_flag)) fail(71);
             tc_fence_after();
             {
-                const uint32_t row = smem_u32(sm + C_U);
-                float x[32];
-                for (int half = 0; half < 2; ++half) {
-                    tmem_ld32(tm + lane_off + TM_U + 32 * half, x);
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4)
-                        st_shared_v4(row + sw128_chunk(dv, 4 * half + q4), pack_bf16(x[8 * q4], x[8 * q4 + 1]),
-                                     pack_bf16(x[8 * q4 + 2], x[8 * q4 + 3]), pack_bf16(x[8 * q4 + 4], x[8 * q4 + 5]),
-                                     pack_bf16(x[8 * q4 + 6], x[8 * q4 + 7]));
-                }
+                float x0[32], x1[32];
+                tmem_ld32(tm + lane_off + TM_U, x0);
+                tmem_ld32(tm + lane_off + TM_U + 32, x1);
+                st_bf16_cols(TM_U, x0, x1);
             }
-            fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(bar(CB_UREADY));
             const bool last = (n + 1 == nchunks);
@@ -738,19 +756,21 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
             if (!mbar_wait(bar(CB_B), n & 1, lim, abort_flag)) fail(72);
             tc_fence_after();
             {
-                float x[32];
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    tmem_ld32(tm + lane_off + TM_S + c0, x);
+                float x0[32], x1[32];
+                for (int c0 = 0; c0 < D; c0 += 64) {
+                    tmem_ld32(tm + lane_off + TM_S + c0, x0);
+                    tmem_ld32(tm + lane_off + TM_S + c0 + 32, x1);
                     if (!last) {
-                        store_s_bf16(x, c0);
+                        st_bf16_cols(TM_SBF + c0 / 2, x0, x1);
                     } else if (p.state_out) {
+                        float *dst = p.state_out + state_off + (size_t)dv * D + c0;
 #pragma unroll
-                        for (int j = 0; j < 32; j += 4)
-                            *reinterpret_cast<float4 *>(p.state_out + state_off + (size_t)dv * D + c0 + j) =
-                                make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
+                        for (int j = 0; j < 32; j += 4) {
+                            *reinterpret_cast<float4 *>(dst + j) = make_float4(x0[j], x0[j + 1], x0[j + 2], x0[j + 3]);
+                            *reinterpret_cast<float4 *>(dst + 32 + j) = make_float4(x1[j], x1[j + 1], x1[j + 2], x1[j + 3]);
+                        }
                     }
                 }
-                fence_proxy_async_smem();
                 tc_fence_before();
                 if (!last) {
                     // the next (a) may start now; the fp32 state is rescaled for the
@@ -758,52 +778,56 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                     mbar_arrive(bar(CB_SREADY));
                     const float gnext = scb[(n + 1) % 3].gC;
                     for (int c0 = 0; c0 < D; c0 += 32) {
-                        tmem_ld32(tm + lane_off + TM_S + c0, x);
+                        tmem_ld32(tm + lane_off + TM_S + c0, x0);
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) x[j] *= gnext;
-                        tmem_st32(tm + lane_off + TM_S + c0, x);
+                        for (int j = 0; j < 32; ++j) x0[j] *= gnext;
+                        tmem_st32(tm + lane_off + TM_S + c0, x0);
                     }
                     tc_fence_before();
                 }
             }
-            // output epilogue: o_t = gamma_t O1 + exp(G_t - G_C) O2
-            if (!mbar_wait(bar(CB_C), n & 1, lim, abort_flag)) fail(73);
+        }
+    } else {
+        // ------------------------------------------------------------ output group
+        // O^T (lane dv, 64 t) -> bf16 rows of out; off the state chain
+        const int dv = tid - 128;   // TMEM lane
+        const uint32_t lane_off = static_cast<uint32_t>((warp - 4) * 32) << 16;
+        __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(sm + C_U);
+        for (int n = 0; n < nchunks; ++n) {
+            const int s = n & 1;
+            // all four warps are done with chunk n-1's staging buffer
+            if (named_bar_any(3, 128, *abort_flag != 0)) break;
+            if (!mbar_wait(bar(CB_C + s), (n >> 1) & 1, lim, abort_flag)) fail(73);
             tc_fence_after();
-            {
-                // stage the [64 t][128 dv] bf16 tile in the U buffer (free once
-                // c2 has completed), then write whole 16-byte pieces of rows
-                __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(sm + C_U);
-                float a[32], b[32];
-                for (int half = 0; half < 2; ++half) {
-                    tmem_ld32(tm + lane_off + TM_O1 + s * 128 + 32 * half, a);
-                    tmem_ld32(tm + lane_off + TM_O2 + s * 128 + 32 * half, b);
+            float a[32], b[32];
+            tmem_ld32(tm + lane_off + TM_O + s * 64, a);
+            tmem_ld32(tm + lane_off + TM_O + s * 64 + 32, b);
+            tc_fence_before();
+            mbar_arrive(bar(CB_OFREE + s));   // the MMA thread may reuse this buffer
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int t = 32 * half + j;
-                        stage[t * D + dv] = __float2bfloat16_rn(fmaf(cs.gam[t], a[j], cs.invD[t] * b[j]));
-                    }
-                }
-                tc_fence_before();
-                named_bar_sync(2, 128);
-                const int64_t t0 = bos + (int64_t)n * C;
-                const int len = cs.len;
+            for (int j = 0; j < 32; ++j) {
+                stage[j * D + dv] = __float2bfloat16_rn(a[j]);
+                stage[(32 + j) * D + dv] = __float2bfloat16_rn(b[j]);
+            }
+            named_bar_sync(3, 128);
+            // whole 16-byte pieces of the [64 t][128 dv] tile, rows t < len
+            const int64_t t0 = bos + (int64_t)n * C;
+            const int len = (int)((eos - t0) < C ? (eos - t0) : C);
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const int idx = k * 128 + dv;          // 1024 pieces of 16 bytes
-                    const int t = idx >> 4, piece = idx & 15;
-                    if (t < len) {
-                        const uint4 v = *reinterpret_cast<const uint4 *>(stage + t * D + piece * 8);
-                        *reinterpret_cast<uint4 *>(p.out + ((size_t)(t0 + t) * H + h) * D + piece * 8) = v;
-                    }
+            for (int k = 0; k < 8; ++k) {
+                const int idx = k * 128 + dv;          // 1024 pieces of 16 bytes
+                const int t = idx >> 4, piece = idx & 15;
+                if (t < len) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(stage + t * D + piece * 8);
+                    *reinterpret_cast<uint4 *>(p.out + ((size_t)(t0 + t) * H + h) * D + piece * 8) = v;
                 }
-                named_bar_sync(2, 128);   // the U buffer is rewritten by the next residual epilogue
             }
         }
     }
 
     // ---------------------------------------------------------------- teardown
     __syncthreads();
-    if (warp == 4) {
+    if (warp == 8) {
         tc_fence_after();
         tmem_dealloc(tm, TM_COLS);
     }
@@ -888,7 +912,6 @@ cudaError_t launch_prefill_tc(const TcLaunch &L, cudaStream_t stream) {
         !make_token_map(&pp.map_k, L.k, L.total_tokens, L.H) ||
         !make_token_map(&cp.map_v, L.v, L.total_tokens, L.H))
         return cudaErrorInvalidValue;
-    cp.map_q = pp.map_q;
     cp.map_k = pp.map_k;
     pp.g = cp.g = L.g;
     pp.beta = cp.beta = L.beta;

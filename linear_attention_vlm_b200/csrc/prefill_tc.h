@@ -10,9 +10,10 @@
 namespace gdn {
 
 // Bytes of per-chunk factors the prep kernel hands to the chain kernel for
-// one (chunk, head): W (64 x 128 bf16), T'' (64 x 64 bf16), Phat (64 x 64 bf16),
-// each already in the 128-byte-swizzled shared-memory layout of the MMAs.
-constexpr size_t kTileBytes = 32768;
+// one (chunk, head): W (64 x 128 bf16), diag(gamma) Q (64 x 128 bf16),
+// T'' (64 x 64 bf16) and the scaled QK^T triangle (64 x 64 bf16), each already
+// in the 128-byte-swizzled shared-memory layout of the MMAs.
+constexpr size_t kTileBytes = 49152;
 
 struct TcLaunch {
     const void *q, *k, *v;
