@@ -133,6 +133,36 @@ int gdn_decode_step(const void *q, const void *k, const void *v,
 int gdn_prefill_kernel_count(int num_seqs, int64_t total_tokens, int H, int dk, int dv,
                              int chunk, int dtype);
 
+/*
+ * gdn_prefill_noalloc -- gdn_prefill for callers that cannot allocate device
+ * memory (for instance a serving loop that reserves all of its device memory
+ * at start-up and forbids any later cudaMalloc, or a host that cannot pass the
+ * library a workspace pointer).  The InfiniteVL pages have no counterpart: it
+ * changes only where the scratch lives, not what is computed.
+ *
+ * Arguments, layouts, results and status codes are those of gdn_prefill,
+ * without the workspace pair.  The scratch is one array of
+ * GDN_NOALLOC_SCRATCH_BYTES compiled into libgdn.so, which every GPU that
+ * loads the library holds until the process exits.  Requests whose
+ * gdn_prefill_workspace_size() exceeds it return GDN_ERR_WORKSPACE before
+ * anything is enqueued (16 MiB covers, e.g., 16 heads x 1024 tokens in one
+ * sequence); shapes that need no workspace are not limited.
+ *
+ * The function calls no cudaMalloc, cudaFree or other allocating routine.  The
+ * first call on a device looks the array's device address up (with that
+ * device current) and caches it; make that first call before any stream
+ * capture.  Every call on a device shares the one array: calls whose work
+ * overlaps on the GPU (different streams, or other host threads) race on it
+ * and must be serialised by the caller.  Each call clears what has to start
+ * at zero, so stale contents from an earlier call are harmless.
+ */
+#define GDN_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+int gdn_prefill_noalloc(const void *q, const void *k, const void *v, const float *g,
+                        const float *beta, const float *state_in, void *out,
+                        float *state_out, const int32_t *cu_seqlens, int num_seqs,
+                        int64_t total_tokens, int H, int dk, int dv, int chunk,
+                        int dtype, void *stream);
+
 /* Static, human-readable name of a gdn_status value. */
 const char *gdn_status_string(int status);
 

@@ -57,6 +57,8 @@ int check_prefill(const void *q, const void *k, const void *v, const float *g,
 
 }  // namespace
 
+int gdn::note_cuda_error(cudaError_t e) { return cuda_fail(e); }
+
 extern "C" {
 
 const char *gdn_status_string(int status) {

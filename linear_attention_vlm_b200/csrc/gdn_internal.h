@@ -33,6 +33,10 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(x);
 }
 
+// Records e as this host thread's last CUDA error (gdn_last_cuda_error) and
+// returns GDN_ERR_CUDA.
+int note_cuda_error(cudaError_t e);
+
 // Launchers (return cudaError_t of the launch).
 cudaError_t launch_decode(int dtype, int dk, const void *q, const void *k, const void *v,
                           const float *g, const float *beta, const float *state_in,

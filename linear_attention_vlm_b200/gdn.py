@@ -52,6 +52,9 @@ def _load():
     lib.gdn_prefill.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, vp, i32, i64, i32, i32, i32,
                                 i32, i32, vp, sz, vp]
     lib.gdn_prefill.restype = i32
+    lib.gdn_prefill_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, vp, i32, i64, i32, i32,
+                                        i32, i32, i32, vp]
+    lib.gdn_prefill_noalloc.restype = i32
     lib.gdn_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i32, i32, i32, i32, i32, vp]
     lib.gdn_decode_step.restype = i32
     lib.gdn_status_string.argtypes = [i32]
@@ -156,6 +159,42 @@ def gdn_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tens
                              chunk, dt, _ptr(workspace), ws_bytes, _stream(dev))
     if st != GDN_OK:
         raise GdnError(st, "gdn_prefill")
+    return out, state_out
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def gdn_prefill_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                        beta: torch.Tensor, state_in: Optional[torch.Tensor] = None,
+                        cu_seqlens: Optional[torch.Tensor] = None, *,
+                        num_seqs: Optional[int] = None, out: Optional[torch.Tensor] = None,
+                        state_out: Optional[torch.Tensor] = None, chunk: int = CHUNK,
+                        want_state: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """gdn_prefill without a workspace: the library's fixed scratch array
+    (NOALLOC_SCRATCH_BYTES per device) is used instead.  For callers that
+    cannot allocate device memory; concurrent calls on one device race."""
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("gdn_prefill_noalloc needs CUDA tensors")
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32 or cu_seqlens.device != dev:
+            raise ValueError("cu_seqlens must be int32 on the same device")
+        N = cu_seqlens.numel() - 1
+    else:
+        N = 1 if num_seqs is None else int(num_seqs)
+    if out is None:
+        out = torch.empty((T, H, dv), dtype=q.dtype, device=dev)
+    if state_out is None and want_state:
+        state_out = torch.empty((N, H, dv, dk), dtype=torch.float32, device=dev)
+    st = _load().gdn_prefill_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                     _ptr(state_in), _ptr(out), _ptr(state_out),
+                                     _ptr(cu_seqlens), N, T, H, dk, dv, chunk,
+                                     _dtype_code(q.dtype), _stream(dev))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_prefill_noalloc")
     return out, state_out
 
 
