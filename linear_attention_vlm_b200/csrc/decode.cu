@@ -10,52 +10,54 @@
 // same threads (in-place updates are safe).  The kernel is HBM-bound: 2 d_k
 // d_v 4 bytes of state traffic against ~6 d_k d_v flops.
 //
-// Layout: one CTA of 4 warps per (sequence, head).  A row of 128 fp32 is
-// split over LPR = d_k / 16 lanes (16 floats = four 128-bit loads each), so a
-// warp covers 32 / LPR rows per pass; UNR passes are issued before any is
-// consumed so that every thread keeps UNR x 64 bytes of loads in flight.
+// Layout: one CTA of NW warps per (sequence, head).  A row of d_k fp32 is
+// split over LPR = d_k / 16 lanes, 16 floats each, held as four 16-byte
+// pieces.  With COAL the lanes of a row take consecutive 16-byte pieces, so
+// each load instruction of a row covers whole 128-byte lines; otherwise a
+// lane owns 64 contiguous bytes.  UNR passes (of 32 / LPR rows per warp) are
+// loaded before any is consumed, so each thread keeps UNR x 64 bytes of loads
+// in flight.
 #include "gdn_internal.h"
 
 namespace gdn {
 namespace {
 
-template <typename T>
-__device__ __forceinline__ void load16(const T *p, float (&x)[16]);
+// column of the e-th float (e = 4 i + j) that lane `seg` owns
+template <int LPR, bool COAL>
+__device__ __forceinline__ int col_of(int seg, int i) {
+    return COAL ? (i * LPR + seg) * 4 : seg * 16 + 4 * i;
+}
+
+template <typename T, int LPR, bool COAL>
+__device__ __forceinline__ void load_vec(const T *p, int seg, float (&x)[16]);
 
 template <>
-__device__ __forceinline__ void load16<float>(const float *p, float (&x)[16]) {
-    const float4 *p4 = reinterpret_cast<const float4 *>(p);
+__device__ __forceinline__ void load_vec<float, 8, true>(const float *p, int seg, float (&x)[16]) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        float4 t = __ldg(p4 + i);
+        const float4 t = __ldg(reinterpret_cast<const float4 *>(p + col_of<8, true>(seg, i)));
         x[4 * i] = t.x; x[4 * i + 1] = t.y; x[4 * i + 2] = t.z; x[4 * i + 3] = t.w;
     }
 }
 
-template <>
-__device__ __forceinline__ void load16<__nv_bfloat16>(const __nv_bfloat16 *p, float (&x)[16]) {
-    const uint4 *p4 = reinterpret_cast<const uint4 *>(p);
+template <typename T, int LPR, bool COAL>
+__device__ __forceinline__ void load_vec(const T *p, int seg, float (&x)[16]) {
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        uint4 t = __ldg(p4 + i);
-        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&t);
+    for (int i = 0; i < 4; ++i) {
+        const int c = col_of<LPR, COAL>(seg, i);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            float2 f = __bfloat1622float2(h[j]);
-            x[8 * i + 2 * j] = f.x;
-            x[8 * i + 2 * j + 1] = f.y;
-        }
+        for (int j = 0; j < 4; ++j) x[4 * i + j] = to_f32(p[c + j]);
     }
 }
 
-template <typename T, int D, int UNR>
-__global__ void __launch_bounds__(128)
+template <typename T, int D, int UNR, int NW, bool COAL>
+__global__ void __launch_bounds__(NW * 32)
 gdn_decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                   const float *__restrict__ g, const float *__restrict__ beta,
                   const float *state_in, float *state_out, T *__restrict__ out) {
     constexpr int LPR = D / 16;           // lanes per row
     constexpr int RPW = 32 / LPR;         // rows per warp per pass
-    constexpr int RPP = RPW * 4;          // rows per CTA per pass
+    constexpr int RPP = RPW * NW;         // rows per CTA per pass
     constexpr int PASSES = D / RPP;
     static_assert(PASSES % UNR == 0, "UNR must divide the pass count");
 
@@ -64,8 +66,8 @@ gdn_decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
     const int seg = lane % LPR, rloc = lane / LPR;
 
     float kr[16], qr[16];
-    load16<T>(k + (size_t)bh * D + seg * 16, kr);
-    load16<T>(q + (size_t)bh * D + seg * 16, qr);
+    load_vec<T, LPR, COAL>(k + (size_t)bh * D, seg, kr);
+    load_vec<T, LPR, COAL>(q + (size_t)bh * D, seg, qr);
     float kq = 0.f;
 #pragma unroll
     for (int j = 0; j < 16; ++j) kq = fmaf(kr[j], qr[j], kq);
@@ -75,8 +77,8 @@ gdn_decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
     const float b = __ldg(beta + bh);
 
     const size_t sbase = (size_t)bh * D * D;
-    const float4 *Sin = reinterpret_cast<const float4 *>(state_in + sbase);
-    float4 *Sout = reinterpret_cast<float4 *>(state_out + sbase);
+    const float *Sin = state_in + sbase;
+    float *Sout = state_out + sbase;
 
 #pragma unroll 1
     for (int p0 = 0; p0 < PASSES; p0 += UNR) {
@@ -85,9 +87,9 @@ gdn_decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
 #pragma unroll
         for (int u = 0; u < UNR; ++u) {
             const int row = (p0 + u) * RPP + warp * RPW + rloc;
-            const float4 *src = Sin + ((size_t)row * D + seg * 16) / 4;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) s[u][i] = src[i];
+            for (int i = 0; i < 4; ++i)
+                s[u][i] = *reinterpret_cast<const float4 *>(Sin + (size_t)row * D + col_of<LPR, COAL>(seg, i));
             vr[u] = to_f32(v[(size_t)bh * D + row]);
         }
 #pragma unroll
@@ -111,7 +113,6 @@ gdn_decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
                 sq += __shfl_xor_sync(0xffffffffu, sq, o);
             }
             const float uu = b * (vr[u] - a * sk);
-            float4 *dst = Sout + ((size_t)row * D + seg * 16) / 4;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 float4 t;
@@ -119,37 +120,62 @@ gdn_decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
                 t.y = fmaf(a, s[u][i].y, uu * kr[4 * i + 1]);
                 t.z = fmaf(a, s[u][i].z, uu * kr[4 * i + 2]);
                 t.w = fmaf(a, s[u][i].w, uu * kr[4 * i + 3]);
-                dst[i] = t;
+                *reinterpret_cast<float4 *>(Sout + (size_t)row * D + col_of<LPR, COAL>(seg, i)) = t;
             }
             if (seg == 0) out[(size_t)bh * D + row] = from_f32<T>(fmaf(a, sq, uu * kq));
         }
     }
 }
 
-template <typename T, int D>
-cudaError_t launch_decode_t(const void *q, const void *k, const void *v, const float *g,
-                            const float *beta, const float *state_in, float *state_out,
-                            void *out, int B, int H, cudaStream_t stream) {
-    constexpr int UNR = (D == 128) ? 4 : 2;
+}  // namespace
+
+// Variant selector, also used by the tuning harness: unr in {1,2,4,8}
+// (dividing the pass count), nw in {4,8}, coal in {0,1}.
+template <typename T, int D, int UNR, int NW, bool COAL>
+static cudaError_t launch_decode_v(const void *q, const void *k, const void *v, const float *g,
+                                   const float *beta, const float *state_in, float *state_out,
+                                   void *out, int B, int H, cudaStream_t stream) {
     const unsigned grid = (unsigned)B * (unsigned)H;
-    gdn_decode_kernel<T, D, UNR><<<grid, 128, 0, stream>>>(
+    gdn_decode_kernel<T, D, UNR, NW, COAL><<<grid, NW * 32, 0, stream>>>(
         static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), g, beta,
         state_in, state_out, static_cast<T *>(out));
     return cudaGetLastError();
 }
 
-}  // namespace
+cudaError_t launch_decode_variant(int variant, int dtype, int dk, const void *q, const void *k,
+                                  const void *v, const float *g, const float *beta,
+                                  const float *state_in, float *state_out, void *out, int B, int H,
+                                  cudaStream_t stream) {
+#define GDN_DEC(T, D, U, W, C) \
+    return launch_decode_v<T, D, U, W, C>(q, k, v, g, beta, state_in, state_out, out, B, H, stream)
+    if (dtype == 1 && dk == 128) {
+        switch (variant) {
+            case 0: GDN_DEC(__nv_bfloat16, 128, 4, 4, false);
+            case 1: GDN_DEC(__nv_bfloat16, 128, 4, 4, true);
+            case 2: GDN_DEC(__nv_bfloat16, 128, 2, 4, true);
+            case 3: GDN_DEC(__nv_bfloat16, 128, 2, 8, true);
+            case 4: GDN_DEC(__nv_bfloat16, 128, 4, 8, true);
+            case 5: GDN_DEC(__nv_bfloat16, 128, 1, 8, true);
+            case 6: GDN_DEC(__nv_bfloat16, 128, 8, 4, true);
+            default: break;
+        }
+    }
+    // defaults, from a sweep on B200 (64 x 16 heads, L2 flushed): coalesced
+    // 128-byte row pieces, 8 warps, 4 passes in flight
+    if (dtype == 0) {
+        if (dk == 128) GDN_DEC(float, 128, 4, 8, true);
+        GDN_DEC(float, 64, 2, 4, true);
+    }
+    if (dk == 128) GDN_DEC(__nv_bfloat16, 128, 4, 8, true);
+    GDN_DEC(__nv_bfloat16, 64, 2, 4, true);
+#undef GDN_DEC
+}
 
 cudaError_t launch_decode(int dtype, int dk, const void *q, const void *k, const void *v,
                           const float *g, const float *beta, const float *state_in,
                           float *state_out, void *out, int B, int H, cudaStream_t stream) {
-    if (dtype == 0) {
-        return dk == 128 ? launch_decode_t<float, 128>(q, k, v, g, beta, state_in, state_out, out, B, H, stream)
-                         : launch_decode_t<float, 64>(q, k, v, g, beta, state_in, state_out, out, B, H, stream);
-    }
-    return dk == 128
-               ? launch_decode_t<__nv_bfloat16, 128>(q, k, v, g, beta, state_in, state_out, out, B, H, stream)
-               : launch_decode_t<__nv_bfloat16, 64>(q, k, v, g, beta, state_in, state_out, out, B, H, stream);
+    return launch_decode_variant(-1, dtype, dk, q, k, v, g, beta, state_in, state_out, out, B, H,
+                                 stream);
 }
 
 }  // namespace gdn
