@@ -196,7 +196,7 @@ def run_native(args):
     st_out = torch.empty((1, H, dv, dk), dtype=torch.float32, device=dev)
     ws_bytes = gdn.gdn_prefill_workspace_size(1, T, H, dk, dv, w.chunk, w.dtype)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
-    launches_per_prefill = gdn.gdn_prefill_kernel_count(1, T, H, dk, dv, w.chunk, w.dtype)
+    launches_per_prefill = gdn.gdn_prefill_kernel_count(1, T, H, dk, dv, w.chunk, w.dtype, packed=False)
 
     def prefill_once():
         gdn.gdn_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], None, None, out=out,

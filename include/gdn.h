@@ -126,12 +126,14 @@ int gdn_decode_step(const void *q, const void *k, const void *v,
                     int dtype, void *stream);
 
 /*
- * Number of kernel launches gdn_prefill makes for these sizes (0 for
- * arguments it would reject).  Pure host arithmetic; lets callers account
- * for the library's launches inside a CUDA graph or a timed region.
+ * Number of kernel launches gdn_prefill makes for these sizes on the current
+ * device (0 for arguments it would reject); `packed` is nonzero when
+ * cu_seqlens will be passed.  Host-side only (it may query the device's SM
+ * count); lets callers account for the library's launches inside a CUDA graph
+ * or a timed region.
  */
 int gdn_prefill_kernel_count(int num_seqs, int64_t total_tokens, int H, int dk, int dv,
-                             int chunk, int dtype);
+                             int chunk, int dtype, int packed);
 
 /*
  * gdn_prefill_noalloc -- gdn_prefill for callers that cannot allocate device

@@ -85,13 +85,13 @@ size_t gdn_prefill_workspace_size(int num_seqs, int64_t total_tokens, int H, int
 }
 
 int gdn_prefill_kernel_count(int num_seqs, int64_t total_tokens, int H, int dk, int dv,
-                             int chunk, int dtype) {
+                             int chunk, int dtype, int packed) {
     if (num_seqs < 1 || H < 1 || total_tokens < 0) return 0;
     if (chunk != gdn::kChunk || !shape_supported(dk, dv)) return 0;
     if (dtype != GDN_F32 && dtype != GDN_BF16) return 0;
-    // the workspace query cannot see whether cu_seqlens will be passed, so the
-    // count here assumes the packed (varlen) form; uniform batches launch one less
-    return use_tc(total_tokens, dk, dtype) ? gdn::tc_kernel_count(true) : 1;
+    return use_tc(total_tokens, dk, dtype)
+               ? gdn::tc_kernel_count(num_seqs, total_tokens, H, packed != 0)
+               : 1;
 }
 
 int gdn_prefill(const void *q, const void *k, const void *v, const float *g, const float *beta,

@@ -45,31 +45,46 @@ using namespace sm100;
 
 constexpr int C = 64;
 constexpr int D = 128;
-constexpr int AP = 68;   // fp32 row pitch of the solve matrices
-
 // ------------------------------------------------------------ prep kernel layout
-constexpr int kPrepThreads = 160;                      // warps 0-3 prep, warp 4 control
+// 128 threads and ~56 KB of shared memory per CTA, so that four chunks are in
+// flight per SM.  Thread 0 also issues the TMA copies and the two MMAs.
+constexpr int kPrepThreads = 128;
 constexpr uint32_t P_KQ = 0;                           // [2 kb][128 rows: K 0-63, Q 64-127][128 B]
 constexpr uint32_t P_TP = P_KQ + 32768;                // T'  bf16 [64 t][128 B]
-constexpr uint32_t P_TPP = P_TP + 8192;                // T'' bf16 [64 t][128 B]
-constexpr uint32_t P_PH = P_TPP + 8192;                // Pt bf16 [64 t][128 B]
-constexpr uint32_t P_AF = P_PH + 8192;                 // A fp32 [64][AP]; later W staging [2 kb][64][128 B]
-constexpr uint32_t P_TF = P_AF + 64 * AP * 4;          // T fp32 [64][AP]
-constexpr uint32_t P_SC = P_TF + 64 * AP * 4;          // PrepScalars
-constexpr uint32_t P_MM = P_SC + 2048;                 // solve scratch, 4 warps x 16x16 fp32
-constexpr uint32_t P_BAR = P_MM + 4096;                // mbarriers + TMEM base
-constexpr uint32_t P_ALLOC = P_BAR + 64 + 1024;        // + alignment slack
-static_assert(64 * AP * 4 >= 16384, "W staging fits in the A buffer");
-constexpr uint32_t P_TM_COLS = 128;                    // p1 output at 0, p2 output at 64
-enum { PB_FULL = 0, PB_P1 = 1, PB_TREADY = 2, PB_P2 = 3, PB_FIN = 4, PB_NUM = 5 };
+constexpr uint32_t P_TPP = P_TP + 8192;                // T'' bf16 [64 t][128 B] (p2 reads [T'; T''] as one A)
+constexpr uint32_t P_SC = P_TPP + 8192;                // PrepScalars
+constexpr uint32_t P_MM = P_SC + 1536;                 // solve scratch, 4 warps x 16 x 20 fp32
+constexpr uint32_t P_BAR = P_MM + 4 * 16 * 20 * 4;     // mbarriers + TMEM base
+constexpr uint32_t P_ALLOC = P_BAR + 64 + 1008;        // + alignment slack
+constexpr uint32_t P_TM_COLS = 128;                    // p1 output at 0..63, then p2 output at 0..127
+enum { PB_FULL = 0, PB_P1 = 1, PB_P2 = 2, PB_NUM = 3 };
+// The lower block triangles of A and T = (I + A)^-1, as ten 16x16 fp32 blocks
+// each (block (i, j), j <= i, at index i (i + 1) / 2 + j).  A lives over the
+// T'/T'' buffers (written only after the solve), T over the Q rows of the KQ
+// tile (dead once Qg is out): five blocks in each 8 KB half.
+constexpr int AB_P = 20, TB_P = 24;                    // row pitches: conflict-free mma fragment loads
+constexpr uint32_t P_AB = P_TP;
+constexpr uint32_t AB_BYTES = 16 * AB_P * 4, TB_BYTES = 16 * TB_P * 4;
+static_assert(10 * AB_BYTES <= 16384 && 5 * TB_BYTES <= 8192, "block triangles fit");
+static_assert(4 * (P_ALLOC + 1024) <= 233472, "four prep CTAs per SM");
+
+__device__ __forceinline__ int tri_blk(int i, int j) { return i * (i + 1) / 2 + j; }
+__device__ __forceinline__ float *a_blk(uint8_t *sm, int i, int j) {
+    return reinterpret_cast<float *>(sm + P_AB + tri_blk(i, j) * AB_BYTES);
+}
+__device__ __forceinline__ float *t_blk(uint8_t *sm, int i, int j) {
+    const int b = tri_blk(i, j);
+    return reinterpret_cast<float *>(sm + P_KQ + (b < 5 ? 8192 + b * TB_BYTES : 24576 + (b - 5) * TB_BYTES));
+}
 
 // ------------------------------------------------------------ chain kernel layout
 constexpr int kChainThreads = 320;                     // warps 0-3 chain, 4-7 output, 8 MMA, 9 TMA
 constexpr uint32_t C_STAGE = 81920;                    // per stage: K, V, W, Qg, T'', Pt
 constexpr uint32_t CS_K = 0, CS_V = 16384, CS_W = 32768, CS_QG = 49152, CS_TPP = 65536, CS_PT = 73728;
 constexpr uint32_t C_U = 2 * C_STAGE;                  // output staging [64 t][128 dv] bf16
-constexpr uint32_t C_SCE = C_U + 16384;                // ChainScalars x 3 (state group)
-constexpr uint32_t C_BAR = C_SCE + 3072;               // mbarriers + TMEM base + abort flag
+constexpr uint32_t C_SCE = C_U + 16384;                // ChainScalars x 3 (state chain)
+constexpr uint32_t C_SCX = C_SCE + 3072;               // ChainScalars x 3 (identity chain)
+constexpr uint32_t C_BAR = C_SCX + 3072;               // mbarriers + TMEM base + abort flag
 constexpr uint32_t C_ALLOC = C_BAR + 256 + 1024;
 static_assert(CS_PT + 8192 == C_STAGE && C_STAGE - CS_W == kTileBytes, "stage layout");
 // TMEM columns of the chain kernel.  The MMA A operands produced by the chain
@@ -79,12 +94,14 @@ constexpr uint32_t TM_SBF = 0;     // S bf16, two per column (64)
 constexpr uint32_t TM_U = 64;      // U^T accumulator (64); then U^T bf16 in its first 32
 constexpr uint32_t TM_S = 128;     // state S (128)
 constexpr uint32_t TM_O = 256;     // O^T [2 bufs] at 256, 320 (64 each)
+constexpr uint32_t TM_X = 256;     // identity chain (transition ranges): its S bf16, U^T, S at +0, +64, +128
 constexpr uint32_t TM_COLS = 512;
 // Barriers that a role may complete twice before its consumer waits once are
 // per buffer (FULL/EMPTY per stage, C/OFREE per output buffer) and waited with
 // the parity of the buffer's use count, so that no phase can be skipped.
 enum { CB_FULL = 0, CB_EMPTY = 2, CB_A = 4, CB_B = 5, CB_C = 6, CB_SREADY = 8, CB_UREADY = 9,
-       CB_FIN = 10, CB_OFREE = 11, CB_NUM = 13 };
+       CB_FIN = 10, CB_OFREE = 11, CB_A2 = 13, CB_B2 = 14, CB_SREADY2 = 15, CB_UREADY2 = 16,
+       CB_NUM = 17 };
 
 struct ChainScalars {   // per chunk, state group
     float gC;           // exp(G_C)
@@ -100,9 +117,8 @@ struct PrepScalars {
     float Dd[C];        // exp(G_C - G_t)
     float gam[C];       // exp(G_t)
     float invD[C];      // exp(G_t - G_C)
-    float pad[2 * C];
 };
-static_assert(sizeof(PrepScalars) == 2048, "scalar block size");
+static_assert(sizeof(PrepScalars) == 1536, "scalar block size");
 
 struct PrepParams {
     CUtensorMap map_q, map_k;
@@ -127,7 +143,10 @@ struct ChainParams {
     int64_t uniform_len;
     int cps;
     int H;
+    int nseg, seg_len;           // chunk ranges per sequence, chunks per range
     const uint8_t *tiles;
+    const float *seg_start;      // start states of ranges 1.. [N][H][nseg-1][D][D]
+    float *trans_r, *trans_m;    // transitions of ranges 0..nseg-2, same layout
     int *err;
     uint64_t timeout_ns;
 };
@@ -226,29 +245,27 @@ __device__ __forceinline__ void mma16(float (&acc)[2][4], const float *X, int px
 // Off-diagonal block (i, j) of T = (I + A)^-1 (16x16 blocks):
 //   T_ij = -T_ii * sum_{k=j}^{i-1} A_ik T_kj
 // computed by one warp with tf32 tensor-core MMAs.
-__device__ __forceinline__ void solve_block(const float *Af, float *Tf, float *scratch, int i, int j,
-                                            int lane) {
+__device__ __forceinline__ void solve_block(uint8_t *sm, float *scratch, int i, int j, int lane) {
     float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    for (int k = j; k < i; ++k)
-        mma16(acc, Af + (16 * i) * AP + 16 * k, AP, Tf + (16 * k) * AP + 16 * j, AP, lane);
+    for (int k = j; k < i; ++k) mma16(acc, a_blk(sm, i, k), AB_P, t_blk(sm, k, j), TB_P, lane);
     const int g = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
-        scratch[g * 16 + 8 * nt + 2 * t] = acc[nt][0];
-        scratch[g * 16 + 8 * nt + 2 * t + 1] = acc[nt][1];
-        scratch[(g + 8) * 16 + 8 * nt + 2 * t] = acc[nt][2];
-        scratch[(g + 8) * 16 + 8 * nt + 2 * t + 1] = acc[nt][3];
+        scratch[g * 20 + 8 * nt + 2 * t] = acc[nt][0];
+        scratch[g * 20 + 8 * nt + 2 * t + 1] = acc[nt][1];
+        scratch[(g + 8) * 20 + 8 * nt + 2 * t] = acc[nt][2];
+        scratch[(g + 8) * 20 + 8 * nt + 2 * t + 1] = acc[nt][3];
     }
     __syncwarp();
     float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    mma16(acc2, Tf + (16 * i) * AP + 16 * i, AP, scratch, 16, lane);
-    float *dst = Tf + (16 * i) * AP + 16 * j;
+    mma16(acc2, t_blk(sm, i, i), TB_P, scratch, 20, lane);
+    float *dst = t_blk(sm, i, j);
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
-        dst[g * AP + 8 * nt + 2 * t] = -acc2[nt][0];
-        dst[g * AP + 8 * nt + 2 * t + 1] = -acc2[nt][1];
-        dst[(g + 8) * AP + 8 * nt + 2 * t] = -acc2[nt][2];
-        dst[(g + 8) * AP + 8 * nt + 2 * t + 1] = -acc2[nt][3];
+        dst[g * TB_P + 8 * nt + 2 * t] = -acc2[nt][0];
+        dst[g * TB_P + 8 * nt + 2 * t + 1] = -acc2[nt][1];
+        dst[(g + 8) * TB_P + 8 * nt + 2 * t] = -acc2[nt][2];
+        dst[(g + 8) * TB_P + 8 * nt + 2 * t + 1] = -acc2[nt][3];
     }
     __syncwarp();
 }
@@ -297,7 +314,7 @@ gdn_chunk_offsets_kernel(const int32_t *__restrict__ cu, int N, int32_t *__restr
 
 // ---------------------------------------------------------------- prep kernel
 
-__global__ void __launch_bounds__(kPrepThreads, 2)
+__global__ void __launch_bounds__(kPrepThreads, 4)
 gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = aligned_smem(smraw);
@@ -324,19 +341,17 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
     int64_t bos, eos;
     SeqBounds{p.cu_seqlens, p.uniform_len}.get(nseq, bos, eos);
     const int64_t t0 = bos + j * C;
-    const int len = (eos - t0) < C ? (int)(eos - t0) : C;
 
     uint32_t *tmem_base_ptr = reinterpret_cast<uint32_t *>(sm + P_BAR + 8 * PB_NUM);
     auto bar = [&](int i) { return smem_u32(sm + P_BAR + 8 * i); };
     if (tid == 0) {
         mbar_init(bar(PB_FULL), 1);
         mbar_init(bar(PB_P1), 1);
-        mbar_init(bar(PB_TREADY), 128);
         mbar_init(bar(PB_P2), 1);
-        mbar_init(bar(PB_FIN), 1);
         fence_mbar_init();
     }
-    if (warp == 4) {
+    __syncwarp();
+    if (warp == 0) {
         tmem_alloc(smem_u32(tmem_base_ptr), P_TM_COLS);
         tmem_relinquish();
     }
@@ -346,215 +361,220 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
     const uint32_t tm = *tmem_base_ptr;
     const uint64_t lim = p.timeout_ns;
     const int no_abort = 0;   // CTA-local failures end each wait by its own bound
+    bool ok = true;
+    PrepScalars *sc = reinterpret_cast<PrepScalars *>(sm + P_SC);
+    uint8_t *tile = p.tiles + ((size_t)gc * H + h) * kTileBytes;   // [W 16K][Qg 16K][T'' 8K][Pt 8K]
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
 
-    if (warp == 4) {
-        if (lane == 0) {
-            const int z = (int)t0;
-            mbar_arrive_expect_tx(bar(PB_FULL), 32768);
-            for (int kb = 0; kb < 2; ++kb) {
-                const uint32_t dst = smem_u32(sm + P_KQ + kb * 16384);
-                tma_load_3d(dst, &p.map_k, kb * 64, h, z, bar(PB_FULL));
-                tma_load_3d(dst + 8192, &p.map_q, kb * 64, h, z, bar(PB_FULL));
-            }
-            bool ok = mbar_wait(bar(PB_FULL), 0, lim, &no_abort);
+    if (tid == 0) {
+        // K, Q -> shared memory; p1 = [K; Q] K^T -> TMEM columns 0..63
+        const int z = (int)t0;
+        mbar_arrive_expect_tx(bar(PB_FULL), 32768);
+        for (int kb = 0; kb < 2; ++kb) {
+            const uint32_t dst = smem_u32(sm + P_KQ + kb * 16384);
+            tma_load_3d(dst, &p.map_k, kb * 64, h, z, bar(PB_FULL));
+            tma_load_3d(dst + 8192, &p.map_q, kb * 64, h, z, bar(PB_FULL));
+        }
+        ok = mbar_wait(bar(PB_FULL), 0, lim, &no_abort);
+        if (ok) {
+            tc_fence_after();
             const uint64_t dKQk = desc_sw128(smem_u32(sm + P_KQ), 16, 1024);
-            const uint64_t dKQm = desc_sw128(smem_u32(sm + P_KQ), 16384, 1024);
-            const uint64_t dTP = desc_sw128(smem_u32(sm + P_TP), 16, 1024);
-            if (ok) {
-                tc_fence_after();
-                // p1: [K;Q] K^T -> columns 0..63
-                const uint32_t id_p1 = idesc_bf16(128, 64, false, false);
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint64_t a = dKQk + (((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
-                    mma_bf16_ss(tm, a, a, id_p1, ks > 0);
-                }
-                mma_commit(bar(PB_P1));
-                ok = mbar_wait(bar(PB_TREADY), 0, lim, &no_abort);
+            const uint32_t id_p1 = idesc_bf16(128, 64, false, false);
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t a = dKQk + (((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
+                mma_bf16_ss(tm, a, a, id_p1, ks > 0);
             }
-            if (ok) {
-                tc_fence_after();
-                // p2: W^T = K^T T'^T -> columns 64..127 (A = K tile MN-major)
-                const uint32_t id_p2 = idesc_bf16(128, 64, true, false);
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(tm + 64, dKQm + ((ks * 2048) >> 4), dTP + ((ks * 32) >> 4), id_p2, ks > 0);
-                mma_commit(bar(PB_P2));
-            }
-            if (!ok && p.err) atomicCAS(p.err, 0, 51);
-            mma_commit(bar(PB_FIN));
-            mbar_wait(bar(PB_FIN), 0, lim, &no_abort);
-            mbar_wait(bar(PB_FULL), 0, lim, &no_abort);   // no TMA copy still landing at exit
         }
-    } else {
-        // ------------------------------------------------------------ prep warps
-        const int pt = tid, pw = warp;
-        PrepScalars *sc = reinterpret_cast<PrepScalars *>(sm + P_SC);
-        float *Af = reinterpret_cast<float *>(sm + P_AF);
-        float *Tf = reinterpret_cast<float *>(sm + P_TF);
-        float *mm = reinterpret_cast<float *>(sm + P_MM) + pw * 256;
-        const uint32_t lane_off = static_cast<uint32_t>(pw * 32) << 16;
-        if (pw == 0) {
-            const GateRegs gr = load_gates(p.g, p.beta, bos, eos, (int)j, (int)j + 1, h, H, lane);
-            float G0, G1;
-            scan_gates(gr, lane, G0, G1);
-            const float GC = __shfl_sync(0xffffffffu, G1, 31);
-            sc->inv[lane] = expf(-G0); sc->inv[lane + 32] = expf(-G1);
-            sc->beta[lane] = gr.b0; sc->beta[lane + 32] = gr.b1;
-            sc->bg[lane] = gr.b0 * expf(G0); sc->bg[lane + 32] = gr.b1 * expf(G1);
-            sc->Dd[lane] = expf(GC - G0); sc->Dd[lane + 32] = expf(GC - G1);
-            sc->gam[lane] = expf(G0); sc->gam[lane + 32] = expf(G1);
-            sc->invD[lane] = expf(G0 - GC); sc->invD[lane + 32] = expf(G1 - GC);
-        }
-        named_bar_sync(1, 128);
-        bool ok = mbar_wait(bar(PB_P1), 0, lim, &no_abort);
-        tc_fence_after();
-        {
-            float x[64];
-            float (&x0)[32] = *reinterpret_cast<float (*)[32]>(&x[0]);
-            float (&x1)[32] = *reinterpret_cast<float (*)[32]>(&x[32]);
-            tmem_ld32(tm + lane_off, x0);
-            tmem_ld32(tm + lane_off + 32, x1);
-            if (pt < 64) {
-                // A[r][i] = beta_r exp(G_r - G_i) k_r.k_i = (beta_r gamma_r) exp(-G_i) KK[r][i]
-                const int r = pt;
-                const float bgr = sc->bg[r];
+        mma_commit(bar(PB_P1));   // also on failure, so that no thread waits out its bound
+    } else if (warp == 1) {
+        const GateRegs gr = load_gates(p.g, p.beta, bos, eos, (int)j, (int)j + 1, h, H, lane);
+        float G0, G1;
+        scan_gates(gr, lane, G0, G1);
+        const float GC = __shfl_sync(0xffffffffu, G1, 31);
+        sc->inv[lane] = expf(-G0); sc->inv[lane + 32] = expf(-G1);
+        sc->beta[lane] = gr.b0; sc->beta[lane + 32] = gr.b1;
+        sc->bg[lane] = gr.b0 * expf(G0); sc->bg[lane + 32] = gr.b1 * expf(G1);
+        sc->Dd[lane] = expf(GC - G0); sc->Dd[lane + 32] = expf(GC - G1);
+        sc->gam[lane] = expf(G0); sc->gam[lane + 32] = expf(G1);
+        sc->invD[lane] = expf(G0 - GC); sc->invD[lane + 32] = expf(G1 - GC);
+    }
+    __syncwarp();
+    __syncthreads();
+    ok = mbar_wait(bar(PB_P1), 0, lim, &no_abort) && ok;
+    tc_fence_after();
+    {
+        float x[64];
+        float (&x0)[32] = *reinterpret_cast<float (*)[32]>(&x[0]);
+        float (&x1)[32] = *reinterpret_cast<float (*)[32]>(&x[32]);
+        tmem_ld32(tm + lane_off, x0);
+        tmem_ld32(tm + lane_off + 32, x1);
+        if (tid < 64) {
+            // A[r][i] = beta_r exp(G_r - G_i) k_r.k_i = (beta_r gamma_r) exp(-G_i) KK[r][i], i < r
+            const int r = tid, rb = r >> 4;
+            const float bgr = sc->bg[r];
 #pragma unroll
-                for (int i = 0; i < 64; i += 4) {
+            for (int jb = 0; jb < 4; ++jb) {
+                if (jb > rb) break;
+                float *dst = a_blk(sm, rb, jb) + (r & 15) * AB_P;
+#pragma unroll
+                for (int c = 0; c < 16; c += 4) {
+                    const int i = 16 * jb + c;
                     const float4 iv = *reinterpret_cast<const float4 *>(&sc->inv[i]);
                     float4 a;
                     a.x = (i < r) ? bgr * iv.x * x[i] : 0.f;
                     a.y = (i + 1 < r) ? bgr * iv.y * x[i + 1] : 0.f;
                     a.z = (i + 2 < r) ? bgr * iv.z * x[i + 2] : 0.f;
                     a.w = (i + 3 < r) ? bgr * iv.w * x[i + 3] : 0.f;
-                    *reinterpret_cast<float4 *>(&Af[r * AP + i]) = a;
-                }
-            } else {
-                // Pt[r][i] = exp(G_r - G_C) q_r.k_i for i <= r
-                const int r = pt - 64;
-                const float sr = sc->invD[r];
-                const uint32_t row = smem_u32(sm + P_PH);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i0 = 8 * c + 2 * e;
-                        w[e] = pack_bf16(i0 <= r ? sr * x[i0] : 0.f, i0 + 1 <= r ? sr * x[i0 + 1] : 0.f);
-                    }
-                    st_shared_v4(row + sw128_chunk(r, c), w[0], w[1], w[2], w[3]);
-                }
-                // Qg = diag(gamma) Q, in place over the Q rows of the KQ tile
-                // (p1, their only tensor-core reader here, has completed)
-                const float gr = sc->gam[r];
-#pragma unroll
-                for (int kb = 0; kb < 2; ++kb) {
-                    uint4 *qrow = reinterpret_cast<uint4 *>(sm + P_KQ + kb * 16384 + (64 + r) * 128);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        uint4 v = qrow[c];
-                        __nv_bfloat162 *hv = reinterpret_cast<__nv_bfloat162 *>(&v);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 f = __bfloat1622float2(hv[e]);
-                            hv[e] = __floats2bfloat162_rn(gr * f.x, gr * f.y);
-                        }
-                        qrow[c] = v;   // a whole 16-byte chunk: the swizzle is untouched
-                    }
+                    *reinterpret_cast<float4 *>(dst + c) = a;
                 }
             }
-        }
-        tc_fence_before();
-        named_bar_sync(1, 128);
-        // T = (I + A)^-1: 16x16 diagonal blocks by forward substitution ...
-        if (pt < 64) {
-            const int b = pt >> 4, c = pt & 15;
-            const float *Ab = Af + (16 * b) * AP + 16 * b;
-            float x[16];
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float ps[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int i = 0; i < r; ++i) ps[i & 3] = fmaf(Ab[r * AP + i], x[i], ps[i & 3]);
-                x[r] = ((r == c) ? 1.f : 0.f) - ((ps[0] + ps[1]) + (ps[2] + ps[3]));
-            }
-#pragma unroll
-            for (int r = 0; r < 16; ++r) Tf[(16 * b + r) * AP + 16 * b + c] = x[r];
         } else {
-            for (int e = pt - 64; e < 6 * 256; e += 64) {   // zero the blocks above the diagonal
-                const int blk = e >> 8, w = e & 255;
-                const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-                const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-                Tf[(16 * bi + (w >> 4)) * AP + 16 * bj + (w & 15)] = 0.f;
-            }
-        }
-        named_bar_sync(1, 128);
-        // ... then the off-diagonal blocks, one band at a time
-        if (pw < 3) solve_block(Af, Tf, mm, pw + 1, pw, lane);
-        named_bar_sync(1, 128);
-        if (pw < 2) solve_block(Af, Tf, mm, pw + 2, pw, lane);
-        named_bar_sync(1, 128);
-        if (pw == 0) solve_block(Af, Tf, mm, 3, 0, lane);
-        named_bar_sync(1, 128);
-        // T' = diag(D) T diag(beta gamma), T'' = diag(D) T diag(beta): bf16, K-major rows t
-        {
-            const int which = pt >> 6, r = pt & 63;
-            const uint32_t row = smem_u32(sm + (which ? P_TPP : P_TP));
-            const float *colscale = which ? sc->beta : sc->bg;
-            const float dr = sc->Dd[r];
+            // Pt[r][i] = exp(G_r - G_C) q_r.k_i for i <= r, straight to the tile
+            const int r = tid - 64;
+            const float sr = sc->invD[r];
+            uint8_t *pt_row = tile + 40960;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-                const float4 t0v = *reinterpret_cast<const float4 *>(&Tf[r * AP + 8 * c]);
-                const float4 t1v = *reinterpret_cast<const float4 *>(&Tf[r * AP + 8 * c + 4]);
-                const float4 s0v = *reinterpret_cast<const float4 *>(&colscale[8 * c]);
-                const float4 s1v = *reinterpret_cast<const float4 *>(&colscale[8 * c + 4]);
-                st_shared_v4(row + sw128_chunk(r, c), pack_bf16(dr * t0v.x * s0v.x, dr * t0v.y * s0v.y),
-                             pack_bf16(dr * t0v.z * s0v.z, dr * t0v.w * s0v.w),
-                             pack_bf16(dr * t1v.x * s1v.x, dr * t1v.y * s1v.y),
-                             pack_bf16(dr * t1v.z * s1v.z, dr * t1v.w * s1v.w));
-            }
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(bar(PB_TREADY));
-        // W from p2's W^T (TMEM lane = d_k index, column = t), staged over the A buffer
-        ok = mbar_wait(bar(PB_P2), 0, lim, &no_abort) && ok;
-        tc_fence_after();
-        {
-            float x[32];
-            uint8_t *wt = sm + P_AF + (pt >> 6) * 8192;
-            const int col = pt & 63;
-            for (int half = 0; half < 2; ++half) {
-                tmem_ld32(tm + lane_off + 64 + 32 * half, x);
+                uint32_t w[4];
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    *reinterpret_cast<__nv_bfloat16 *>(wt + sw128_offset(32 * half + i, col)) =
-                        __float2bfloat16_rn(x[i]);
+                for (int e = 0; e < 4; ++e) {
+                    const int i0 = 8 * c + 2 * e;
+                    w[e] = pack_bf16(i0 <= r ? sr * x[i0] : 0.f, i0 + 1 <= r ? sr * x[i0 + 1] : 0.f);
+                }
+                *reinterpret_cast<uint4 *>(pt_row + sw128_chunk(r, c)) = make_uint4(w[0], w[1], w[2], w[3]);
             }
-        }
-        tc_fence_before();
-        named_bar_sync(1, 128);
-        if (!ok && p.err && pt == 0) atomicCAS(p.err, 0, 52);
-        // W (16 KB), Qg (16 KB), T'' (8 KB), Pt (8 KB) -> the workspace tile of (chunk, head)
-        uint8_t *dst = p.tiles + ((size_t)gc * H + h) * kTileBytes;
+            // Qg = diag(gamma) Q: each 16-byte chunk keeps its swizzled position
+            const float gr = sc->gam[r];
 #pragma unroll
-        for (int k = 0; k < 24; ++k) {
-            const int off = (k * 128 + pt) * 16;            // 0 .. 48 KB
-            const uint8_t *srcp;
-            if (off < 16384) srcp = sm + P_AF + off;                                        // W
-            else if (off < 32768) srcp = sm + P_KQ + ((off - 16384) >> 13) * 16384 + 8192 + ((off - 16384) & 8191);  // Qg
-            else if (off < 40960) srcp = sm + P_TPP + (off - 32768);                        // T''
-            else srcp = sm + P_PH + (off - 40960);                                          // Pt
-            *reinterpret_cast<uint4 *>(dst + off) = *reinterpret_cast<const uint4 *>(srcp);
+            for (int kb = 0; kb < 2; ++kb) {
+                const uint4 *qrow = reinterpret_cast<const uint4 *>(sm + P_KQ + kb * 16384 + (64 + r) * 128);
+                uint4 *grow = reinterpret_cast<uint4 *>(tile + 16384 + kb * 8192 + r * 128);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint4 v = qrow[c];
+                    __nv_bfloat162 *hv = reinterpret_cast<__nv_bfloat162 *>(&v);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(hv[e]);
+                        hv[e] = __floats2bfloat162_rn(gr * f.x, gr * f.y);
+                    }
+                    grow[c] = v;
+                }
+            }
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 4) {
+    // T = (I + A)^-1: 16x16 diagonal blocks by forward substitution ...
+    if (tid < 64) {
+        const int b = tid >> 4, c = tid & 15;
+        const float *Ab = a_blk(sm, b, b);
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int i = 0; i < r; ++i) ps[i & 3] = fmaf(Ab[r * AB_P + i], x[i], ps[i & 3]);
+            x[r] = ((r == c) ? 1.f : 0.f) - ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+        }
+        float *Tb = t_blk(sm, b, b);
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Tb[r * TB_P + c] = x[r];
+    }
+    __syncthreads();
+    // ... then the off-diagonal blocks, one band at a time
+    float *mm = reinterpret_cast<float *>(sm + P_MM) + warp * 320;
+    if (warp < 3) solve_block(sm, mm, warp + 1, warp, lane);
+    __syncthreads();
+    if (warp < 2) solve_block(sm, mm, warp + 2, warp, lane);
+    __syncthreads();
+    if (warp == 0) solve_block(sm, mm, 3, 0, lane);
+    __syncthreads();
+    // T' = diag(D) T diag(beta gamma), T'' = diag(D) T diag(beta): bf16, K-major rows t;
+    // T'' also goes to the tile
+    {
+        const int which = tid >> 6, r = tid & 63, rb = r >> 4;
+        const uint32_t row = smem_u32(sm + (which ? P_TPP : P_TP));
+        const float *colscale = which ? sc->beta : sc->bg;
+        const float dr = sc->Dd[r];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint32_t w0 = 0u, w1 = 0u, w2 = 0u, w3 = 0u;
+            if ((c >> 1) <= rb) {
+                const float *tr = t_blk(sm, rb, c >> 1) + (r & 15) * TB_P + 8 * (c & 1);
+                const float4 t0v = *reinterpret_cast<const float4 *>(tr);
+                const float4 t1v = *reinterpret_cast<const float4 *>(tr + 4);
+                const float4 s0v = *reinterpret_cast<const float4 *>(&colscale[8 * c]);
+                const float4 s1v = *reinterpret_cast<const float4 *>(&colscale[8 * c + 4]);
+                w0 = pack_bf16(dr * t0v.x * s0v.x, dr * t0v.y * s0v.y);
+                w1 = pack_bf16(dr * t0v.z * s0v.z, dr * t0v.w * s0v.w);
+                w2 = pack_bf16(dr * t1v.x * s1v.x, dr * t1v.y * s1v.y);
+                w3 = pack_bf16(dr * t1v.z * s1v.z, dr * t1v.w * s1v.w);
+            }
+            st_shared_v4(row + sw128_chunk(r, c), w0, w1, w2, w3);
+            if (which)
+                *reinterpret_cast<uint4 *>(tile + 32768 + sw128_chunk(r, c)) = make_uint4(w0, w1, w2, w3);
+        }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+        // p2: [T'; T''] K -> TMEM columns 0..127; lanes 0..63 are W = T' K
+        // (A K-major, B = the K tile MN-major)
+        tc_fence_after();
+        const uint64_t dTP = desc_sw128(smem_u32(sm + P_TP), 16, 1024);
+        const uint64_t dKm = desc_sw128(smem_u32(sm + P_KQ), 16384, 1024);
+        const uint32_t id_p2 = idesc_bf16(128, 128, false, true);
+        for (int ks = 0; ks < 4; ++ks)
+            mma_bf16_ss(tm, dTP + ((ks * 32) >> 4), dKm + ((ks * 2048) >> 4), id_p2, ks > 0);
+        mma_commit(bar(PB_P2));
+    }
+    __syncwarp();
+    if (warp < 2) {
+        // W rows t = tid -> the tile, [2 kb][64 t][128 B] swizzled
+        ok = mbar_wait(bar(PB_P2), 0, lim, &no_abort) && ok;
+        tc_fence_after();
+        const int t = tid;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            float x[32];
+            tmem_ld32(tm + lane_off + 32 * q4, x);
+            uint8_t *wrow = tile + (q4 >> 1) * 8192;
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const float *e = x + 8 * c4;
+                *reinterpret_cast<uint4 *>(wrow + sw128_chunk(t, (q4 & 1) * 4 + c4)) =
+                    make_uint4(pack_bf16(e[0], e[1]), pack_bf16(e[2], e[3]), pack_bf16(e[4], e[5]),
+                               pack_bf16(e[6], e[7]));
+            }
+        }
+    }
+    if (!ok && p.err) atomicCAS(p.err, 0, 52);
+    if (tid == 0) mbar_wait(bar(PB_FULL), 0, lim, &no_abort);   // no TMA copy still landing at exit
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tm, P_TM_COLS);
     }
 }
 
 // ---------------------------------------------------------------- chain kernel
+//
+// A CTA walks one range of chunks of one (sequence, head).
+//   MODE_OUT:   from a known start state (state_in for a sequence's first
+//               range, a combined state for the others); writes the outputs
+//               and, for the last range, the final state.
+//   MODE_TRANS: the range's affine transition S_end = S_start M + R.  Chain R
+//               starts from zero with the values, chain X from the identity
+//               without them; they run side by side, one state warpgroup
+//               each, and R and M = X_end go to the workspace.
+// With one range per sequence (nseg = 1) MODE_OUT is the whole prefill.
 
+enum { MODE_OUT = 0, MODE_TRANS = 1 };
+
+template <int MODE>
 __global__ void __launch_bounds__(kChainThreads, 1)
 gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
     extern __shared__ uint8_t smraw[];
@@ -565,16 +585,25 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.H;
-    const int nseq = blockIdx.x / H, h = blockIdx.x % H;
+    const int per = MODE == MODE_OUT ? p.nseg : p.nseg - 1;      // ranges per (sequence, head)
+    const int nseq = blockIdx.x / (H * per), h = (blockIdx.x / per) % H, seg = blockIdx.x % per;
     int64_t bos, eos;
     SeqBounds{p.cu_seqlens, p.uniform_len}.get(nseq, bos, eos);
     const int nchunks = (int)((eos - bos + C - 1) / C);
-    const int64_t gc0 = p.chunk_off ? (int64_t)p.chunk_off[nseq] : (int64_t)nseq * p.cps;
+    const int cb = seg * p.seg_len;                                 // first chunk of the range
+    const int ce = min(nchunks, cb + p.seg_len);
+    const int nloc = ce > cb ? ce - cb : 0;
+    const int64_t gc0 = (p.chunk_off ? (int64_t)p.chunk_off[nseq] : (int64_t)nseq * p.cps) + cb;
     const size_t state_off = ((size_t)nseq * H + h) * D * D;
+    const size_t unit_off = (((size_t)nseq * H + h) * (p.nseg - 1) + (seg - (MODE == MODE_OUT ? 1 : 0))) * D * D;
+    const float *start = MODE == MODE_TRANS ? nullptr
+                         : (seg == 0 ? p.state_in : p.seg_start + unit_off);
+    float *finish = MODE == MODE_TRANS ? nullptr : (seg == p.nseg - 1 ? p.state_out : nullptr);
 
     if (tid == 0) {
         for (int i = 0; i < CB_NUM; ++i)
-            mbar_init(bar(i), (i == CB_SREADY || i == CB_UREADY || i >= CB_OFREE) ? 128 : 1);
+            mbar_init(bar(i), (i == CB_SREADY || i == CB_UREADY || i == CB_SREADY2 || i == CB_UREADY2 ||
+                               i == CB_OFREE || i == CB_OFREE + 1) ? 128 : 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -596,23 +625,32 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
         if (p.err) atomicCAS(p.err, 0, code);
     };
 
-    if (nchunks == 0) {
-        // empty sequence: the state passes through unchanged
-        if (tid < 128 && p.state_out) {
+    if (nloc == 0) {
+        // empty range: the state passes through (MODE_OUT); an empty transition
+        // is R = 0, M = I (MODE_TRANS)
+        if (tid < 128) {
             for (int j = 0; j < D; j += 4) {
-                const float4 v = p.state_in ? *reinterpret_cast<const float4 *>(p.state_in + state_off + (size_t)tid * D + j)
-                                            : make_float4(0.f, 0.f, 0.f, 0.f);
-                *reinterpret_cast<float4 *>(p.state_out + state_off + (size_t)tid * D + j) = v;
+                if (MODE == MODE_OUT && finish) {
+                    const float4 v = start ? *reinterpret_cast<const float4 *>(start + (seg == 0 ? state_off : 0) + (size_t)tid * D + j)
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+                    *reinterpret_cast<float4 *>(finish + state_off + (size_t)tid * D + j) = v;
+                }
+                if (MODE == MODE_TRANS) {
+                    *reinterpret_cast<float4 *>(p.trans_r + unit_off + (size_t)tid * D + j) = make_float4(0.f, 0.f, 0.f, 0.f);
+                    float4 e = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (tid >= j && tid < j + 4) (&e.x)[tid - j] = 1.f;
+                    *reinterpret_cast<float4 *>(p.trans_m + unit_off + (size_t)tid * D + j) = e;
+                }
             }
         }
     } else if (warp == 9) {
         // ------------------------------------------------------------ TMA / bulk producer
         if (lane == 0) {
             int issued[2] = {0, 0};
-            for (int n = 0; n < nchunks; ++n) {
+            for (int n = 0; n < nloc; ++n) {
                 const int s = n & 1;
                 const uint32_t st = smem_u32(sm + s * C_STAGE);
-                const int z = (int)(bos + (int64_t)n * C);
+                const int z = (int)(bos + (int64_t)(cb + n) * C);
                 if (n >= 2 && !mbar_wait(bar(CB_EMPTY + s), ((n - 2) >> 1) & 1, lim, abort_flag)) { fail(61); break; }
                 const uint32_t full = bar(CB_FULL + s);
                 mbar_arrive_expect_tx(full, C_STAGE);
@@ -636,46 +674,69 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
             const uint32_t id_b = idesc_bf16(128, 128, false, true);
             // descriptors are built once; a byte offset o inside a tile adds o >> 4
             const uint64_t dSTk = desc_sw128(smem_u32(sm), 16, 1024);      // K-major views of stage data
-            const uint64_t dSTm = desc_sw128(smem_u32(sm), 8192, 1024);    // MN-major view of K
-            const uint64_t dVm = desc_sw128(smem_u32(sm), 8192, 1024);     // MN-major view of V
+            const uint64_t dSTm = desc_sw128(smem_u32(sm), 8192, 1024);    // MN-major views of K and V
             bool ok = true;
-            for (int n = 0; ok && n < nchunks; ++n) {
+            // (a): U^T (+)= -S W^T for the chain whose tensor memory starts at `base`
+            auto issue_a = [&](uint32_t base, uint32_t st, uint32_t accumulate_first) {
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t offw = st + CS_W + (ks >> 2) * 8192 + (ks & 3) * 32;
+                    mma_bf16_ts(tm + base + TM_U, tm + base + TM_SBF + 8 * ks, dSTk + (offw >> 4), id_a,
+                                ks > 0 ? 1u : accumulate_first);
+                }
+            };
+            // (b): S += U^T K  (A = U^T bf16 in TMEM; B = K tile MN-major)
+            auto issue_b = [&](uint32_t base, uint32_t st) {
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ts(tm + base + TM_S, tm + base + TM_U + 8 * ks,
+                                dSTm + ((st + CS_K + ks * 2048) >> 4), id_b, 1);
+            };
+            for (int n = 0; ok && n < nloc; ++n) {
                 const int s = n & 1;
                 const uint32_t st = s * C_STAGE;
                 if (!(ok = mbar_wait(bar(CB_FULL + s), (n >> 1) & 1, lim, abort_flag))) { fail(62); break; }
                 tc_fence_after();
                 // p3: U^T = V^T T''^T (the previous residual was consumed: U_READY(n-1))
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(tm + TM_U, dVm + ((st + CS_V + ks * 2048) >> 4),
+                    mma_bf16_ss(tm + TM_U, dSTm + ((st + CS_V + ks * 2048) >> 4),
                                 dSTk + ((st + CS_TPP + ks * 32) >> 4), id_p3, ks > 0);
                 if (!(ok = mbar_wait(bar(CB_SREADY), n & 1, lim, abort_flag))) { fail(63); break; }
                 tc_fence_after();
-                // a: U^T -= S W^T
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t offw = st + CS_W + (ks >> 2) * 8192 + (ks & 3) * 32;
-                    mma_bf16_ts(tm + TM_U, tm + TM_SBF + 8 * ks, dSTk + (offw >> 4), id_a, 1);
-                }
+                issue_a(0, st, 1);
                 mma_commit(bar(CB_A));
-                // the output group has read this buffer pair for chunk n-2
-                if (n >= 2 && !(ok = mbar_wait(bar(CB_OFREE + s), ((n - 2) >> 1) & 1, lim, abort_flag))) { fail(65); break; }
-                tc_fence_after();
-                // c1: O^T = S Qg^T (off the state chain)
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t off = st + CS_QG + (ks >> 2) * 8192 + (ks & 3) * 32;
-                    mma_bf16_ts(tm + TM_O + s * 64, tm + TM_SBF + 8 * ks, dSTk + (off >> 4), id_n64, ks > 0);
+                if (MODE == MODE_TRANS) {
+                    if (!(ok = mbar_wait(bar(CB_SREADY2), n & 1, lim, abort_flag))) { fail(66); break; }
+                    tc_fence_after();
+                    issue_a(TM_X, st, 0);   // U_X^T = -X W^T (no values)
+                    mma_commit(bar(CB_A2));
+                    if (!(ok = mbar_wait(bar(CB_UREADY), n & 1, lim, abort_flag))) { fail(64); break; }
+                    tc_fence_after();
+                    issue_b(0, st);
+                    mma_commit(bar(CB_B));
+                    if (!(ok = mbar_wait(bar(CB_UREADY2), n & 1, lim, abort_flag))) { fail(67); break; }
+                    tc_fence_after();
+                    issue_b(TM_X, st);
+                    mma_commit(bar(CB_B2));
+                    mma_commit(bar(CB_EMPTY + s));
+                } else {
+                    // the output group has read this buffer pair for chunk n-2
+                    if (n >= 2 && !(ok = mbar_wait(bar(CB_OFREE + s), ((n - 2) >> 1) & 1, lim, abort_flag))) { fail(65); break; }
+                    tc_fence_after();
+                    // c1: O^T = S Qg^T (off the state chain)
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t off = st + CS_QG + (ks >> 2) * 8192 + (ks & 3) * 32;
+                        mma_bf16_ts(tm + TM_O + s * 64, tm + TM_SBF + 8 * ks, dSTk + (off >> 4), id_n64, ks > 0);
+                    }
+                    if (!(ok = mbar_wait(bar(CB_UREADY), n & 1, lim, abort_flag))) { fail(64); break; }
+                    tc_fence_after();
+                    issue_b(0, st);
+                    mma_commit(bar(CB_B));
+                    // c2: O^T += U^T Pt^T
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16_ts(tm + TM_O + s * 64, tm + TM_U + 8 * ks, dSTk + ((st + CS_PT + ks * 32) >> 4),
+                                    id_n64, 1);
+                    mma_commit(bar(CB_C + s));
+                    mma_commit(bar(CB_EMPTY + s));
                 }
-                if (!(ok = mbar_wait(bar(CB_UREADY), n & 1, lim, abort_flag))) { fail(64); break; }
-                tc_fence_after();
-                // b: S += U^T K   (A = U^T bf16 in TMEM; B = K tile MN-major)
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ts(tm + TM_S, tm + TM_U + 8 * ks, dSTm + ((st + CS_K + ks * 2048) >> 4), id_b, 1);
-                mma_commit(bar(CB_B));
-                // c2: O^T += U^T Pt^T
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ts(tm + TM_O + s * 64, tm + TM_U + 8 * ks, dSTk + ((st + CS_PT + ks * 32) >> 4),
-                                id_n64, 1);
-                mma_commit(bar(CB_C + s));
-                mma_commit(bar(CB_EMPTY + s));
             }
             mma_commit(bar(CB_FIN));   // every issued MMA completes before TMEM is released
             if (!mbar_wait(bar(CB_FIN), 0, lim, abort_flag)) {
@@ -683,24 +744,28 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                 mbar_wait(bar(CB_FIN), 0, lim, &zero);
             }
         }
-    } else if (warp < 4) {
-        // ------------------------------------------------------------ state group
-        const int dv = tid;   // TMEM lane and state row
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-        ChainScalars *scb = reinterpret_cast<ChainScalars *>(sm + C_SCE);
+    } else if (warp < 4 || MODE == MODE_TRANS) {
+        // ------------------------------------------------------------ state group(s)
+        // warps 0-3: the state chain (R in MODE_TRANS); warps 4-7 in MODE_TRANS: chain X
+        const bool xchain = warp >= 4;
+        const int wg = warp & 3;
+        const int dv = tid & 127;   // TMEM lane and state row
+        const uint32_t lane_off = static_cast<uint32_t>(wg * 32) << 16;
+        const uint32_t base = xchain ? TM_X : 0;
+        const int bA = xchain ? CB_A2 : CB_A, bB = xchain ? CB_B2 : CB_B;
+        const int bS = xchain ? CB_SREADY2 : CB_SREADY, bU = xchain ? CB_UREADY2 : CB_UREADY;
+        const int nb = xchain ? 3 : 2;    // named barrier of this group
+        ChainScalars *scb = reinterpret_cast<ChainScalars *>(sm + (xchain ? C_SCX : C_SCE));
         GateRegs gr{0.f, 0.f, 0.f, 0.f};
-        if (warp == 0) gr = load_gates(p.g, p.beta, bos, eos, 0, nchunks, h, H, lane);
-        // scalars of chunk m from the prefetched gates; prefetch chunk m+1's
+        if (wg == 0) gr = load_gates(p.g, p.beta, bos, eos, cb, ce, h, H, lane);
+        // scalars of local chunk m from the prefetched gates; prefetch chunk m+1's
         auto compute_scalars = [&](int m) {
-            if (warp == 0) {
-                const int64_t t0 = bos + (int64_t)m * C;
-                const int len = (int)((eos - t0) < C ? (eos - t0) : C);
+            if (wg == 0) {
                 float G0, G1;
                 scan_gates(gr, lane, G0, G1);
-                gr = load_gates(p.g, p.beta, bos, eos, m + 1, nchunks, h, H, lane);
+                gr = load_gates(p.g, p.beta, bos, eos, cb + m + 1, ce, h, H, lane);
                 const float GC = __shfl_sync(0xffffffffu, G1, 31);
-                ChainScalars &cs = scb[m % 3];
-                if (lane == 0) { cs.gC = expf(GC); cs.len = len; }
+                if (lane == 0) scb[m % 3].gC = expf(GC);
             }
         };
         // write 64 fp32 values of this lane's row as 32 packed bf16 columns
@@ -711,59 +776,71 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                 pk[j] = pack_bf16(x0[2 * j], x0[2 * j + 1]);
                 pk[16 + j] = pack_bf16(x1[2 * j], x1[2 * j + 1]);
             }
-            tmem_st32u(tm + lane_off + col, pk);
+            tmem_st32u(tm + lane_off + base + col, pk);
         };
         compute_scalars(0);
-        named_bar_sync(2, 128);
+        named_bar_sync(nb, 128);
         {
+            // start state: given (MODE_OUT), zero (chain R) or the identity (chain X)
             const float gC0 = scb[0].gC;
             float x0[32], x1[32];
             for (int c0 = 0; c0 < D; c0 += 64) {
 #pragma unroll
                 for (int j = 0; j < 32; j += 4) {
-                    const float *src = p.state_in + state_off + (size_t)dv * D + c0 + j;
-                    const float4 a = p.state_in ? *reinterpret_cast<const float4 *>(src) : make_float4(0.f, 0.f, 0.f, 0.f);
-                    const float4 b = p.state_in ? *reinterpret_cast<const float4 *>(src + 32) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+                    if (start) {
+                        const float *src = start + (seg == 0 ? state_off : 0) + (size_t)dv * D + c0 + j;
+                        a = *reinterpret_cast<const float4 *>(src);
+                        b = *reinterpret_cast<const float4 *>(src + 32);
+                    }
                     x0[j] = a.x; x0[j + 1] = a.y; x0[j + 2] = a.z; x0[j + 3] = a.w;
                     x1[j] = b.x; x1[j + 1] = b.y; x1[j + 2] = b.z; x1[j + 3] = b.w;
+                }
+                if (xchain) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        x0[j] = (dv == c0 + j) ? 1.f : 0.f;
+                        x1[j] = (dv == c0 + 32 + j) ? 1.f : 0.f;
+                    }
                 }
                 st_bf16_cols(TM_SBF + c0 / 2, x0, x1);
 #pragma unroll
                 for (int j = 0; j < 32; ++j) { x0[j] *= gC0; x1[j] *= gC0; }
-                tmem_st32(tm + lane_off + TM_S + c0, x0);
-                tmem_st32(tm + lane_off + TM_S + c0 + 32, x1);
+                tmem_st32(tm + lane_off + base + TM_S + c0, x0);
+                tmem_st32(tm + lane_off + base + TM_S + c0 + 32, x1);
             }
             tc_fence_before();
-            mbar_arrive(bar(CB_SREADY));
+            mbar_arrive(bar(bS));
         }
-        for (int n = 0; n < nchunks; ++n) {
-            const int s = n & 1;
+        float *dest = MODE == MODE_TRANS ? (xchain ? p.trans_m : p.trans_r) + unit_off
+                                         : (finish ? finish + state_off : nullptr);
+        for (int n = 0; n < nloc; ++n) {
             // residual epilogue: U^T (fp32, lane dv, 64 t) -> bf16 in its own first 32 columns
-            if (!mbar_wait(bar(CB_A), n & 1, lim, abort_flag)) fail(71);
+            if (!mbar_wait(bar(bA), n & 1, lim, abort_flag)) fail(71);
             tc_fence_after();
             {
                 float x0[32], x1[32];
-                tmem_ld32(tm + lane_off + TM_U, x0);
-                tmem_ld32(tm + lane_off + TM_U + 32, x1);
+                tmem_ld32(tm + lane_off + base + TM_U, x0);
+                tmem_ld32(tm + lane_off + base + TM_U + 32, x1);
                 st_bf16_cols(TM_U, x0, x1);
             }
             tc_fence_before();
-            mbar_arrive(bar(CB_UREADY));
-            const bool last = (n + 1 == nchunks);
+            mbar_arrive(bar(bU));
+            const bool last = (n + 1 == nloc);
             if (!last) compute_scalars(n + 1);
-            if (named_bar_any(2, 128, *abort_flag != 0)) break;
+            if (named_bar_any(nb, 128, *abort_flag != 0)) break;
             // state epilogue: publish the bf16 copy for the next (a), then rescale
-            if (!mbar_wait(bar(CB_B), n & 1, lim, abort_flag)) fail(72);
+            if (!mbar_wait(bar(bB), n & 1, lim, abort_flag)) fail(72);
             tc_fence_after();
             {
                 float x0[32], x1[32];
                 for (int c0 = 0; c0 < D; c0 += 64) {
-                    tmem_ld32(tm + lane_off + TM_S + c0, x0);
-                    tmem_ld32(tm + lane_off + TM_S + c0 + 32, x1);
+                    tmem_ld32(tm + lane_off + base + TM_S + c0, x0);
+                    tmem_ld32(tm + lane_off + base + TM_S + c0 + 32, x1);
                     if (!last) {
                         st_bf16_cols(TM_SBF + c0 / 2, x0, x1);
-                    } else if (p.state_out) {
-                        float *dst = p.state_out + state_off + (size_t)dv * D + c0;
+                    } else if (dest) {
+                        float *dst = dest + (size_t)dv * D + c0;
 #pragma unroll
                         for (int j = 0; j < 32; j += 4) {
                             *reinterpret_cast<float4 *>(dst + j) = make_float4(x0[j], x0[j + 1], x0[j + 2], x0[j + 3]);
@@ -775,25 +852,25 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                 if (!last) {
                     // the next (a) may start now; the fp32 state is rescaled for the
                     // next (b), which the MMA thread issues only after U_READY
-                    mbar_arrive(bar(CB_SREADY));
+                    mbar_arrive(bar(bS));
                     const float gnext = scb[(n + 1) % 3].gC;
                     for (int c0 = 0; c0 < D; c0 += 32) {
-                        tmem_ld32(tm + lane_off + TM_S + c0, x0);
+                        tmem_ld32(tm + lane_off + base + TM_S + c0, x0);
 #pragma unroll
                         for (int j = 0; j < 32; ++j) x0[j] *= gnext;
-                        tmem_st32(tm + lane_off + TM_S + c0, x0);
+                        tmem_st32(tm + lane_off + base + TM_S + c0, x0);
                     }
                     tc_fence_before();
                 }
             }
         }
     } else {
-        // ------------------------------------------------------------ output group
+        // ------------------------------------------------------------ output group (MODE_OUT)
         // O^T (lane dv, 64 t) -> bf16 rows of out; off the state chain
         const int dv = tid - 128;   // TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>((warp - 4) * 32) << 16;
         __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(sm + C_U);
-        for (int n = 0; n < nchunks; ++n) {
+        for (int n = 0; n < nloc; ++n) {
             const int s = n & 1;
             // all four warps are done with chunk n-1's staging buffer
             if (named_bar_any(3, 128, *abort_flag != 0)) break;
@@ -811,7 +888,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
             }
             named_bar_sync(3, 128);
             // whole 16-byte pieces of the [64 t][128 dv] tile, rows t < len
-            const int64_t t0 = bos + (int64_t)n * C;
+            const int64_t t0 = bos + (int64_t)(cb + n) * C;
             const int len = (int)((eos - t0) < C ? (eos - t0) : C);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
@@ -830,6 +907,102 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
     if (warp == 8) {
         tc_fence_after();
         tmem_dealloc(tm, TM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- segment combine
+//
+// Start state of every range after the first: S_{j+1} = S_j M_j + R_j,
+// sequentially over the ranges of one (sequence, head).  Rows of S are
+// independent, so a CTA owns 16 of them (grid (N*H, 8), four warps, 32 output
+// columns each).  The products run on tf32 mma.sync with the 3xTF32 split
+// (x = hi + lo, hi*hi + hi*lo + lo*hi), which keeps them at fp32 accuracy.
+// M_{j+1} streams into the other half of a double buffer (cp.async) while
+// step j computes.
+constexpr int kCombRows = 16;
+constexpr int kCombMP = 136, kCombSP = 132;   // row pitches: conflict-free fragment loads
+constexpr size_t kCombSmem = (size_t)(2 * D * kCombMP + kCombRows * kCombSP) * sizeof(float);
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)),
+                 "l"(reinterpret_cast<uint64_t>(src))
+                 : "memory");
+}
+
+__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo) {
+    hi = tf32(x);
+    lo = tf32(x - __uint_as_float(hi));
+}
+
+__global__ void __launch_bounds__(128)
+gdn_scan_combine_kernel(const float *__restrict__ state_in, const float *__restrict__ trans_r,
+                        const float *__restrict__ trans_m, float *__restrict__ seg_start, int nseg) {
+    extern __shared__ float smf[];
+    float *Ms = smf;                          // M_j [k][n], two buffers
+    float *Ss = Ms + 2 * D * kCombMP;         // S rows [16][D]
+    const int nh = blockIdx.x, r0 = blockIdx.y * kCombRows;
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31, g = lane >> 2, q = lane & 3;
+    auto stage = [&](int j) {
+        const float *src = trans_m + ((size_t)nh * (nseg - 1) + j) * D * D;
+        float *dst = Ms + (j & 1) * D * kCombMP;
+        for (int i = t; i < D * D / 4; i += 128) cp_async16(dst + (i >> 5) * kCombMP + 4 * (i & 31), src + 4 * i);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    if (nseg > 1) stage(0);
+    for (int i = t; i < kCombRows * D; i += 128)
+        Ss[(i >> 7) * kCombSP + (i & 127)] =
+            state_in ? state_in[(size_t)nh * D * D + (size_t)(r0 + (i >> 7)) * D + (i & 127)] : 0.f;
+    for (int j = 0; j + 1 < nseg; ++j) {
+        const size_t u = ((size_t)nh * (nseg - 1) + j) * D * D;
+        const float *rrow0 = trans_r + u + (size_t)(r0 + g) * D, *rrow1 = rrow0 + 8 * D;
+        float acc[4][4], accx[4][4];   // hi*hi terms; the two cross terms (seeded with R_j)
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            const int col = 32 * warp + 8 * nt + 2 * q;
+            const float2 a = *reinterpret_cast<const float2 *>(rrow0 + col);
+            const float2 b = *reinterpret_cast<const float2 *>(rrow1 + col);
+            accx[nt][0] = a.x; accx[nt][1] = a.y; accx[nt][2] = b.x; accx[nt][3] = b.y;
+            acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+        }
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        __syncthreads();   // M_j landed for every thread; S_j rows are written
+        if (j + 2 < nseg) stage(j + 1);
+        const float *M = Ms + (j & 1) * D * kCombMP;
+#pragma unroll 2
+        for (int ks = 0; ks < D / 8; ++ks) {
+            const int k0 = 8 * ks;
+            uint32_t ah[4], al[4];
+            split_tf32(Ss[g * kCombSP + k0 + q], ah[0], al[0]);
+            split_tf32(Ss[(g + 8) * kCombSP + k0 + q], ah[1], al[1]);
+            split_tf32(Ss[g * kCombSP + k0 + q + 4], ah[2], al[2]);
+            split_tf32(Ss[(g + 8) * kCombSP + k0 + q + 4], ah[3], al[3]);
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                const int n = 32 * warp + 8 * nt + g;
+                uint32_t bh0, bl0, bh1, bl1;
+                split_tf32(M[(k0 + q) * kCombMP + n], bh0, bl0);
+                split_tf32(M[(k0 + q + 4) * kCombMP + n], bh1, bl1);
+                mma_tf32(accx[nt], al[0], al[1], al[2], al[3], bh0, bh1);
+                mma_tf32(accx[nt], ah[0], ah[1], ah[2], ah[3], bl0, bl1);
+                mma_tf32(acc[nt], ah[0], ah[1], ah[2], ah[3], bh0, bh1);
+            }
+        }
+        float *o0 = seg_start + u + (size_t)(r0 + g) * D, *o1 = o0 + 8 * D;
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[nt][e] += accx[nt][e];
+            const int col = 32 * warp + 8 * nt + 2 * q;
+            *reinterpret_cast<float2 *>(o0 + col) = make_float2(acc[nt][0], acc[nt][1]);
+            *reinterpret_cast<float2 *>(o1 + col) = make_float2(acc[nt][2], acc[nt][3]);
+        }
+        __syncthreads();   // every warp has read S_j
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            const int col = 32 * warp + 8 * nt + 2 * q;
+            *reinterpret_cast<float2 *>(Ss + g * kCombSP + col) = make_float2(acc[nt][0], acc[nt][1]);
+            *reinterpret_cast<float2 *>(Ss + (g + 8) * kCombSP + col) = make_float2(acc[nt][2], acc[nt][3]);
+        }
     }
 }
 
@@ -870,29 +1043,55 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 size_t chunk_off_bytes(int num_seqs) { return align_up(4 * (size_t)(num_seqs + 1), 1024); }
 
+// bytes of one of the three range-state arrays (R, M, start states)
+size_t scan_array_bytes(int num_seqs, int H, int nseg) {
+    return (size_t)num_seqs * H * (size_t)(nseg > 1 ? nseg - 1 : 0) * D * D * sizeof(float);
+}
+
 bool set_smem_attrs() {
     static bool done[64] = {false};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
     if (dev >= 0 && dev < 64 && done[dev]) return true;
     if (cudaFuncSetAttribute(gdn_chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)P_ALLOC) != cudaSuccess)
-        return false;
-    if (cudaFuncSetAttribute(gdn_chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)C_ALLOC) != cudaSuccess)
+                             (int)P_ALLOC) != cudaSuccess ||
+        cudaFuncSetAttribute(gdn_chunk_prep_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             100) != cudaSuccess ||
+        cudaFuncSetAttribute(gdn_chunk_chain_kernel<MODE_OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)C_ALLOC) != cudaSuccess ||
+        cudaFuncSetAttribute(gdn_chunk_chain_kernel<MODE_TRANS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)C_ALLOC) != cudaSuccess ||
+        cudaFuncSetAttribute(gdn_scan_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kCombSmem) != cudaSuccess)
         return false;
     if (dev >= 0 && dev < 64) done[dev] = true;
     return true;
 }
 
+// SM count of the current device, capped at the reference count the
+// workspace is sized for (host query only).
+int scan_sm_count() {
+    int dev = 0, sms = kScanRefSMs;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms < kScanRefSMs ? sms : kScanRefSMs;
+}
+
 }  // namespace
 
 size_t tc_workspace_bytes(int num_seqs, int64_t total_tokens, int H, bool varlen) {
+    // range states are sized for an unpacked call on the reference SM count;
+    // packed (varlen) calls run one range per sequence and leave them unused
+    const int nseg = tc_scan_segments(num_seqs, total_tokens, H, false, kScanRefSMs);
     return 1024 + chunk_off_bytes(num_seqs) +
-           (size_t)tc_chunk_bound(num_seqs, total_tokens, varlen) * (size_t)H * kTileBytes;
+           (size_t)tc_chunk_bound(num_seqs, total_tokens, varlen) * (size_t)H * kTileBytes +
+           3 * scan_array_bytes(num_seqs, H, nseg);
 }
 
-int tc_kernel_count(bool varlen) { return varlen ? 3 : 2; }
+int tc_kernel_count(int num_seqs, int64_t total_tokens, int H, bool varlen) {
+    if (varlen) return 3;
+    return tc_scan_segments(num_seqs, total_tokens, H, false, scan_sm_count()) > 1 ? 4 : 2;
+}
 
 cudaError_t launch_prefill_tc(const TcLaunch &L, cudaStream_t stream) {
     const bool varlen = L.cu_seqlens != nullptr;
@@ -903,6 +1102,12 @@ cudaError_t launch_prefill_tc(const TcLaunch &L, cudaStream_t stream) {
     const int64_t bound = tc_chunk_bound(L.num_seqs, L.total_tokens, varlen);
     if (bound <= 0) return cudaSuccess;
     if (bound > 0x7fffffff || L.H > 65535) return cudaErrorInvalidValue;
+    // sequence-parallel ranges for few long sequences (never more than the
+    // workspace was sized for: the SM count is capped at the reference count)
+    const int nseg = tc_scan_segments(L.num_seqs, L.total_tokens, L.H, varlen, scan_sm_count());
+    const int seg_len = nseg > 1 ? (cps + nseg - 1) / nseg : 0x3fffffff;
+    float *scan_base = reinterpret_cast<float *>(tiles + (size_t)bound * L.H * kTileBytes);
+    const size_t scan_elems = scan_array_bytes(L.num_seqs, L.H, nseg) / sizeof(float);
 
     PrepParams pp;
     ChainParams cp;
@@ -928,12 +1133,24 @@ cudaError_t launch_prefill_tc(const TcLaunch &L, cudaStream_t stream) {
     cp.state_in = L.state_in;
     cp.state_out = L.state_out;
     cp.out = static_cast<__nv_bfloat16 *>(L.out);
+    cp.nseg = nseg;
+    cp.seg_len = seg_len;
+    cp.trans_r = scan_base;
+    cp.trans_m = scan_base + scan_elems;
+    cp.seg_start = scan_base + 2 * scan_elems;
 
     if (!set_smem_attrs()) return cudaGetLastError() != cudaSuccess ? cudaGetLastError() : cudaErrorUnknown;
     if (varlen) gdn_chunk_offsets_kernel<<<1, 1024, 0, stream>>>(L.cu_seqlens, L.num_seqs, chunk_off);
     dim3 pgrid((unsigned)bound, (unsigned)L.H);
     gdn_chunk_prep_kernel<<<pgrid, kPrepThreads, P_ALLOC, stream>>>(pp);
-    gdn_chunk_chain_kernel<<<(unsigned)L.num_seqs * (unsigned)L.H, kChainThreads, C_ALLOC, stream>>>(cp);
+    const unsigned units = (unsigned)L.num_seqs * (unsigned)L.H;
+    if (nseg > 1) {
+        gdn_chunk_chain_kernel<MODE_TRANS><<<units * (nseg - 1), kChainThreads, C_ALLOC, stream>>>(cp);
+        dim3 cgrid(units, D / kCombRows);
+        gdn_scan_combine_kernel<<<cgrid, 128, kCombSmem, stream>>>(L.state_in, cp.trans_r, cp.trans_m,
+                                                                  scan_base + 2 * scan_elems, nseg);
+    }
+    gdn_chunk_chain_kernel<MODE_OUT><<<units * nseg, kChainThreads, C_ALLOC, stream>>>(cp);
     return cudaGetLastError();
 }
 

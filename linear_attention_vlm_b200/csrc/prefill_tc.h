@@ -33,10 +33,31 @@ inline int64_t tc_chunk_bound(int num_seqs, int64_t total_tokens, bool varlen) {
     return varlen ? (total_tokens + 63) / 64 + num_seqs : num_seqs * ((total_tokens / num_seqs + 63) / 64);
 }
 
-// Workspace layout: [status 256 B][chunk offsets, 4 (N+1) B, padded to 1 KiB]
-// [tiles: chunk_bound * H * kTileBytes].
+// Sequence-parallel ranges: a batch of few long unpacked sequences is split
+// into nseg ranges of chunks per sequence so that about one CTA per SM works
+// on it (see the chain kernel); 1 means one range per sequence.
+constexpr int kScanMaxSegs = 16;     // ranges per sequence at most
+constexpr int kScanMinChunks = 8;    // chunks per range at least
+constexpr int kScanRefSMs = 148;     // SM count the workspace is sized for (B200)
+
+inline int tc_scan_segments(int num_seqs, int64_t total_tokens, int H, bool varlen, int sm_count) {
+    if (varlen || num_seqs < 1 || H < 1 || total_tokens <= 0) return 1;
+    const int64_t units = (int64_t)num_seqs * H;
+    if (2 * units > sm_count) return 1;
+    const int64_t cps = (total_tokens / num_seqs + 63) / 64;
+    int64_t nseg = sm_count / units;
+    if (nseg > kScanMaxSegs) nseg = kScanMaxSegs;
+    if (nseg > cps / kScanMinChunks) nseg = cps / kScanMinChunks;
+    if (nseg < 2) return 1;
+    const int64_t len = (cps + nseg - 1) / nseg;
+    return (int)((cps + len - 1) / len);    // no empty trailing range
+}
+
+// Workspace layout: [status 1 KiB][chunk offsets, 4 (N+1) B, padded to 1 KiB]
+// [tiles: chunk_bound * H * kTileBytes][range transitions R, M and range start
+// states: 3 x N * H * (nseg - 1) * 64 KiB].
 size_t tc_workspace_bytes(int num_seqs, int64_t total_tokens, int H, bool varlen);
-int tc_kernel_count(bool varlen);
+int tc_kernel_count(int num_seqs, int64_t total_tokens, int H, bool varlen);
 cudaError_t launch_prefill_tc(const TcLaunch &L, cudaStream_t stream);
 
 }  // namespace gdn

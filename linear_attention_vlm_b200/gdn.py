@@ -47,7 +47,7 @@ def _load():
     i32, i64 = ctypes.c_int, ctypes.c_int64
     lib.gdn_prefill_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32, i32]
     lib.gdn_prefill_workspace_size.restype = sz
-    lib.gdn_prefill_kernel_count.argtypes = [i32, i64, i32, i32, i32, i32, i32]
+    lib.gdn_prefill_kernel_count.argtypes = [i32, i64, i32, i32, i32, i32, i32, i32]
     lib.gdn_prefill_kernel_count.restype = i32
     lib.gdn_prefill.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, vp, i32, i64, i32, i32, i32,
                                 i32, i32, vp, sz, vp]
@@ -108,9 +108,10 @@ def gdn_prefill_workspace_size(num_seqs: int, total_tokens: int, H: int, dk: int
 
 
 def gdn_prefill_kernel_count(num_seqs: int, total_tokens: int, H: int, dk: int, dv: int,
-                             chunk: int = CHUNK, dtype: torch.dtype = torch.bfloat16) -> int:
+                             chunk: int = CHUNK, dtype: torch.dtype = torch.bfloat16,
+                             packed: bool = False) -> int:
     return int(_load().gdn_prefill_kernel_count(num_seqs, total_tokens, H, dk, dv, chunk,
-                                                _dtype_code(dtype)))
+                                                _dtype_code(dtype), int(packed)))
 
 
 def gdn_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
