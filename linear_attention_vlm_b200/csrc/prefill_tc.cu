@@ -64,7 +64,13 @@ enum { PB_FULL = 0, PB_P1 = 1, PB_P2 = 2, PB_NUM = 3 };
 // tile (dead once Qg is out): five blocks in each 8 KB half.
 constexpr int AB_P = 20, TB_P = 24;                    // row pitches: conflict-free mma fragment loads
 constexpr uint32_t P_AB = P_TP;
-constexpr uint32_t AB_BYTES = 16 * AB_P * 4, TB_BYTES = 16 * TB_P * 4;
+// A blocks sit 1296 B apart (324 words, 4 banks of skew) so that the two
+// diagonal blocks one warp reads during the substitution fall in different banks
+// T blocks sit 1568 B apart (8 banks of skew), so that the blocks of one
+// block-row, read side by side when T' and T'' are formed, use different banks
+constexpr uint32_t AB_BYTES = 1296, TB_BYTES = 1568;
+static_assert(AB_BYTES >= 16 * AB_P * 4 && AB_BYTES % 16 == 0, "A block stride");
+static_assert(TB_BYTES >= 16 * TB_P * 4 && TB_BYTES % 16 == 0, "T block stride");
 static_assert(10 * AB_BYTES <= 16384 && 5 * TB_BYTES <= 8192, "block triangles fit");
 static_assert(4 * (P_ALLOC + 1024) <= 233472, "four prep CTAs per SM");
 
@@ -146,7 +152,9 @@ struct ChainParams {
     int nseg, seg_len;           // chunk ranges per sequence, chunks per range
     const uint8_t *tiles;
     const float *seg_start;      // start states of ranges 1.. [N][H][nseg-1][D][D]
-    float *trans_r, *trans_m;    // transitions of ranges 0..nseg-2, same layout
+    float *trans_r, *trans_m;    // transitions R, M of ranges 0..nseg-2, same layout
+    int wait_tiles;              // the prep kernel may still run: wait before reading tiles
+    int wait_start;              // the combine may still run: wait before reading seg_start
     int *err;
     uint64_t timeout_ns;
 };
@@ -163,6 +171,19 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
         : "memory");
+}
+
+// 1-D bulk copy shared -> global (bulk async-group completion).
+__device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 ::"l"(reinterpret_cast<uint64_t>(dst)), "r"(src), "r"(bytes)
+                 : "memory");
+}
+
+// Commit this thread's bulk stores and wait until they have read shared memory.
+__device__ __forceinline__ void bulk_commit_wait_read() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
 // Raw gates of one chunk held by one warp (lane l owns rows l and l+32),
@@ -242,32 +263,50 @@ __device__ __forceinline__ void mma16(float (&acc)[2][4], const float *X, int px
     }
 }
 
-// Off-diagonal block (i, j) of T = (I + A)^-1 (16x16 blocks):
-//   T_ij = -T_ii * sum_{k=j}^{i-1} A_ik T_kj
-// computed by one warp with tf32 tensor-core MMAs.
-__device__ __forceinline__ void solve_block(uint8_t *sm, float *scratch, int i, int j, int lane) {
-    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    for (int k = j; k < i; ++k) mma16(acc, a_blk(sm, i, k), AB_P, t_blk(sm, k, j), TB_P, lane);
+// Store a 16x16 mma accumulator pair (columns 0-7, 8-15) as fp32 rows of
+// pitch `pitch`, negated if `neg`.
+__device__ __forceinline__ void store16(float *dst, int pitch, const float (&acc)[2][4], bool neg, int lane) {
     const int g = lane >> 2, t = lane & 3;
+    const float sg = neg ? -1.f : 1.f;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
-        scratch[g * 20 + 8 * nt + 2 * t] = acc[nt][0];
-        scratch[g * 20 + 8 * nt + 2 * t + 1] = acc[nt][1];
-        scratch[(g + 8) * 20 + 8 * nt + 2 * t] = acc[nt][2];
-        scratch[(g + 8) * 20 + 8 * nt + 2 * t + 1] = acc[nt][3];
+        *reinterpret_cast<float2 *>(dst + g * pitch + 8 * nt + 2 * t) = make_float2(sg * acc[nt][0], sg * acc[nt][1]);
+        *reinterpret_cast<float2 *>(dst + (g + 8) * pitch + 8 * nt + 2 * t) = make_float2(sg * acc[nt][2], sg * acc[nt][3]);
     }
+}
+
+// Off-diagonal blocks of T = (I + A)^-1 from the diagonal ones (16x16 blocks
+// b = 0..3), by the 2x2 block-inverse rule applied twice:
+//   level 1:  T_10 = -T_11 A_10 T_00,  T_32 = -T_33 A_32 T_22
+//   level 2:  X = A_[23][01] T_[01][01]  (the four blocks X_ij, i = 2,3, j = 0,1)
+//             T_[23][01] = -T_[23][23] X
+// Warp w does its share of each level; the caller separates the levels with
+// CTA barriers.  tf32 tensor-core MMAs, fp32 accumulation.
+__device__ __forceinline__ void merge_level1(uint8_t *sm, float *scratch, int w, int lane) {
+    const int i = 2 * w + 1, j = 2 * w;   // (1, 0) for warp 0, (3, 2) for warp 1
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    mma16(acc, a_blk(sm, i, j), AB_P, t_blk(sm, j, j), TB_P, lane);
+    store16(scratch, 20, acc, false, lane);
     __syncwarp();
     float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     mma16(acc2, t_blk(sm, i, i), TB_P, scratch, 20, lane);
-    float *dst = t_blk(sm, i, j);
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-        dst[g * TB_P + 8 * nt + 2 * t] = -acc2[nt][0];
-        dst[g * TB_P + 8 * nt + 2 * t + 1] = -acc2[nt][1];
-        dst[(g + 8) * TB_P + 8 * nt + 2 * t] = -acc2[nt][2];
-        dst[(g + 8) * TB_P + 8 * nt + 2 * t + 1] = -acc2[nt][3];
-    }
-    __syncwarp();
+    store16(t_blk(sm, i, j), TB_P, acc2, true, lane);
+}
+
+// X_ij = sum_{k=j}^{1} A_ik T_kj for (i, j) = (2 + (w >> 1), w & 1), into scratch
+__device__ __forceinline__ void merge_level2a(uint8_t *sm, float *scratch, int w, int lane) {
+    const int i = 2 + (w >> 1), j = w & 1;
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    for (int k = j; k < 2; ++k) mma16(acc, a_blk(sm, i, k), AB_P, t_blk(sm, k, j), TB_P, lane);
+    store16(scratch, 20, acc, false, lane);
+}
+
+// T_ij = -sum_{k=2}^{i} T_ik X_kj; X_kj is in the scratch of warp 2 (k - 2) + j
+__device__ __forceinline__ void merge_level2b(uint8_t *sm, float *scratch0, int w, int lane) {
+    const int i = 2 + (w >> 1), j = w & 1;
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    for (int k = 2; k <= i; ++k) mma16(acc, t_blk(sm, i, k), TB_P, scratch0 + (2 * (k - 2) + j) * 320, 20, lane);
+    store16(t_blk(sm, i, j), TB_P, acc, true, lane);
 }
 
 
@@ -321,6 +360,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.H, h = blockIdx.y;
     const int gc = blockIdx.x;
+    grid_dep_launch();   // the next kernel may stage its prologue while this grid drains
 
     // which sequence and which of its chunks this CTA prepares
     int nseq;
@@ -349,6 +389,14 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
         mbar_init(bar(PB_P1), 1);
         mbar_init(bar(PB_P2), 1);
         fence_mbar_init();
+        // K, Q -> shared memory, in flight during the TMEM allocation
+        const int z = (int)t0;
+        mbar_arrive_expect_tx(bar(PB_FULL), 32768);
+        for (int kb = 0; kb < 2; ++kb) {
+            const uint32_t dst = smem_u32(sm + P_KQ + kb * 16384);
+            tma_load_3d(dst, &p.map_k, kb * 64, h, z, bar(PB_FULL));
+            tma_load_3d(dst + 8192, &p.map_q, kb * 64, h, z, bar(PB_FULL));
+        }
     }
     __syncwarp();
     if (warp == 0) {
@@ -365,16 +413,10 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
     PrepScalars *sc = reinterpret_cast<PrepScalars *>(sm + P_SC);
     uint8_t *tile = p.tiles + ((size_t)gc * H + h) * kTileBytes;   // [W 16K][Qg 16K][T'' 8K][Pt 8K]
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    float *mm = reinterpret_cast<float *>(sm + P_MM);          // 4 warps x 16 x 20 fp32
 
     if (tid == 0) {
-        // K, Q -> shared memory; p1 = [K; Q] K^T -> TMEM columns 0..63
-        const int z = (int)t0;
-        mbar_arrive_expect_tx(bar(PB_FULL), 32768);
-        for (int kb = 0; kb < 2; ++kb) {
-            const uint32_t dst = smem_u32(sm + P_KQ + kb * 16384);
-            tma_load_3d(dst, &p.map_k, kb * 64, h, z, bar(PB_FULL));
-            tma_load_3d(dst + 8192, &p.map_q, kb * 64, h, z, bar(PB_FULL));
-        }
+        // p1 = [K; Q] K^T -> TMEM columns 0..63
         ok = mbar_wait(bar(PB_FULL), 0, lim, &no_abort);
         if (ok) {
             tc_fence_after();
@@ -399,13 +441,32 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
         sc->invD[lane] = expf(G0 - GC); sc->invD[lane + 32] = expf(G1 - GC);
     }
     __syncwarp();
-    __syncthreads();
-    ok = mbar_wait(bar(PB_P1), 0, lim, &no_abort) && ok;
-    tc_fence_after();
+    __syncthreads();   // gates scanned; K and Q landed (thread 0 waited for them)
+    float x[64];       // this lane's row of p1
     {
-        float x[64];
         float (&x0)[32] = *reinterpret_cast<float (*)[32]>(&x[0]);
         float (&x1)[32] = *reinterpret_cast<float (*)[32]>(&x[32]);
+        if (tid >= 64) {
+            // Qg = diag(gamma) Q straight to the tile, read while p1 runs.  The
+            // swizzled bytes keep their positions; consecutive threads take
+            // consecutive 16-byte pieces, so every warp writes 512 contiguous bytes.
+            ok = mbar_wait(bar(PB_FULL), 0, lim, &no_abort);   // complete: makes the TMA data visible here
+#pragma unroll 4
+            for (int k = 0; k < 16; ++k) {
+                const int q = (tid - 64) + 64 * k, kb = q >> 9, r = (q >> 3) & 63, pc = q & 7;
+                const float gr = sc->gam[r];
+                uint4 v = *reinterpret_cast<const uint4 *>(sm + P_KQ + kb * 16384 + 8192 + r * 128 + pc * 16);
+                __nv_bfloat162 *hv = reinterpret_cast<__nv_bfloat162 *>(&v);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(hv[e]);
+                    hv[e] = __floats2bfloat162_rn(gr * f.x, gr * f.y);
+                }
+                *reinterpret_cast<uint4 *>(tile + 16384 + kb * 8192 + r * 128 + pc * 16) = v;
+            }
+        }
+        ok = mbar_wait(bar(PB_P1), 0, lim, &no_abort) && ok;
+        tc_fence_after();
         tmem_ld32(tm + lane_off, x0);
         tmem_ld32(tm + lane_off + 32, x1);
         if (tid < 64) {
@@ -428,100 +489,68 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
                     *reinterpret_cast<float4 *>(dst + c) = a;
                 }
             }
-        } else {
-            // Pt[r][i] = exp(G_r - G_C) q_r.k_i for i <= r, straight to the tile
-            const int r = tid - 64;
-            const float sr = sc->invD[r];
-            uint8_t *pt_row = tile + 40960;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint32_t w[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int i0 = 8 * c + 2 * e;
-                    w[e] = pack_bf16(i0 <= r ? sr * x[i0] : 0.f, i0 + 1 <= r ? sr * x[i0 + 1] : 0.f);
-                }
-                *reinterpret_cast<uint4 *>(pt_row + sw128_chunk(r, c)) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-            // Qg = diag(gamma) Q: each 16-byte chunk keeps its swizzled position
-            const float gr = sc->gam[r];
-#pragma unroll
-            for (int kb = 0; kb < 2; ++kb) {
-                const uint4 *qrow = reinterpret_cast<const uint4 *>(sm + P_KQ + kb * 16384 + (64 + r) * 128);
-                uint4 *grow = reinterpret_cast<uint4 *>(tile + 16384 + kb * 8192 + r * 128);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint4 v = qrow[c];
-                    __nv_bfloat162 *hv = reinterpret_cast<__nv_bfloat162 *>(&v);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(hv[e]);
-                        hv[e] = __floats2bfloat162_rn(gr * f.x, gr * f.y);
-                    }
-                    grow[c] = v;
-                }
-            }
         }
     }
     tc_fence_before();
-    __syncthreads();
-    // T = (I + A)^-1: 16x16 diagonal blocks by forward substitution ...
+    __syncthreads();   // A complete; Q no longer read (T goes over it)
     if (tid < 64) {
+        // T = (I + A)^-1: 16x16 diagonal blocks by forward substitution
         const int b = tid >> 4, c = tid & 15;
         const float *Ab = a_blk(sm, b, b);
-        float x[16];
+        float y[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
             float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < r; ++i) ps[i & 3] = fmaf(Ab[r * AB_P + i], x[i], ps[i & 3]);
-            x[r] = ((r == c) ? 1.f : 0.f) - ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+            for (int i = 0; i < r; ++i) ps[i & 3] = fmaf(Ab[r * AB_P + i], y[i], ps[i & 3]);
+            y[r] = ((r == c) ? 1.f : 0.f) - ((ps[0] + ps[1]) + (ps[2] + ps[3]));
         }
         float *Tb = t_blk(sm, b, b);
 #pragma unroll
-        for (int r = 0; r < 16; ++r) Tb[r * TB_P + c] = x[r];
+        for (int r = 0; r < 16; ++r) Tb[r * TB_P + c] = y[r];
     }
     __syncthreads();
-    // ... then the off-diagonal blocks, one band at a time
-    float *mm = reinterpret_cast<float *>(sm + P_MM) + warp * 320;
-    if (warp < 3) solve_block(sm, mm, warp + 1, warp, lane);
+    if (warp < 2) merge_level1(sm, mm + warp * 320, warp, lane);
     __syncthreads();
-    if (warp < 2) solve_block(sm, mm, warp + 2, warp, lane);
+    merge_level2a(sm, mm + warp * 320, warp, lane);
     __syncthreads();
-    if (warp == 0) solve_block(sm, mm, 3, 0, lane);
+    merge_level2b(sm, mm, warp, lane);
     __syncthreads();
-    // T' = diag(D) T diag(beta gamma), T'' = diag(D) T diag(beta): bf16, K-major rows t;
-    // T'' also goes to the tile
-    {
-        const int which = tid >> 6, r = tid & 63, rb = r >> 4;
-        const uint32_t row = smem_u32(sm + (which ? P_TPP : P_TP));
-        const float *colscale = which ? sc->beta : sc->bg;
-        const float dr = sc->Dd[r];
+    // T' = diag(D) T diag(beta gamma) into both row halves of the p2 A tile;
+    // T'' = diag(D) T diag(beta) straight to the tile.  Thread tid takes the
+    // 16-byte pieces tid + 128 k (row q / 8, physical chunk q % 8), so that
+    // every warp writes 512 contiguous bytes.
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            uint32_t w0 = 0u, w1 = 0u, w2 = 0u, w3 = 0u;
-            if ((c >> 1) <= rb) {
-                const float *tr = t_blk(sm, rb, c >> 1) + (r & 15) * TB_P + 8 * (c & 1);
-                const float4 t0v = *reinterpret_cast<const float4 *>(tr);
-                const float4 t1v = *reinterpret_cast<const float4 *>(tr + 4);
-                const float4 s0v = *reinterpret_cast<const float4 *>(&colscale[8 * c]);
-                const float4 s1v = *reinterpret_cast<const float4 *>(&colscale[8 * c + 4]);
-                w0 = pack_bf16(dr * t0v.x * s0v.x, dr * t0v.y * s0v.y);
-                w1 = pack_bf16(dr * t0v.z * s0v.z, dr * t0v.w * s0v.w);
-                w2 = pack_bf16(dr * t1v.x * s1v.x, dr * t1v.y * s1v.y);
-                w3 = pack_bf16(dr * t1v.z * s1v.z, dr * t1v.w * s1v.w);
-            }
-            st_shared_v4(row + sw128_chunk(r, c), w0, w1, w2, w3);
-            if (which)
-                *reinterpret_cast<uint4 *>(tile + 32768 + sw128_chunk(r, c)) = make_uint4(w0, w1, w2, w3);
+    for (int k = 0; k < 4; ++k) {
+        const int q = tid + 128 * k, r = q >> 3, pc = q & 7, c = pc ^ (r & 7), rb = r >> 4;
+        const float dr = sc->Dd[r];
+        uint32_t a0 = 0u, a1 = 0u, a2 = 0u, a3 = 0u, b0 = 0u, b1 = 0u, b2 = 0u, b3 = 0u;
+        if ((c >> 1) <= rb) {
+            const float *tr = t_blk(sm, rb, c >> 1) + (r & 15) * TB_P + 8 * (c & 1);
+            const float4 t0v = *reinterpret_cast<const float4 *>(tr);
+            const float4 t1v = *reinterpret_cast<const float4 *>(tr + 4);
+            const float4 g0 = *reinterpret_cast<const float4 *>(&sc->bg[8 * c]);
+            const float4 g1 = *reinterpret_cast<const float4 *>(&sc->bg[8 * c + 4]);
+            const float4 e0 = *reinterpret_cast<const float4 *>(&sc->beta[8 * c]);
+            const float4 e1 = *reinterpret_cast<const float4 *>(&sc->beta[8 * c + 4]);
+            const float4 u0 = make_float4(dr * t0v.x, dr * t0v.y, dr * t0v.z, dr * t0v.w);
+            const float4 u1 = make_float4(dr * t1v.x, dr * t1v.y, dr * t1v.z, dr * t1v.w);
+            a0 = pack_bf16(u0.x * g0.x, u0.y * g0.y); a1 = pack_bf16(u0.z * g0.z, u0.w * g0.w);
+            a2 = pack_bf16(u1.x * g1.x, u1.y * g1.y); a3 = pack_bf16(u1.z * g1.z, u1.w * g1.w);
+            b0 = pack_bf16(u0.x * e0.x, u0.y * e0.y); b1 = pack_bf16(u0.z * e0.z, u0.w * e0.w);
+            b2 = pack_bf16(u1.x * e1.x, u1.y * e1.y); b3 = pack_bf16(u1.z * e1.z, u1.w * e1.w);
         }
+        const uint32_t off = r * 128 + pc * 16;
+        st_shared_v4(smem_u32(sm + P_TP + off), a0, a1, a2, a3);
+        st_shared_v4(smem_u32(sm + P_TP + 8192 + off), a0, a1, a2, a3);
+        *reinterpret_cast<uint4 *>(tile + 32768 + off) = make_uint4(b0, b1, b2, b3);
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     if (tid == 0) {
-        // p2: [T'; T''] K -> TMEM columns 0..127; lanes 0..63 are W = T' K
-        // (A K-major, B = the K tile MN-major)
+        // p2: [T'; T'] K -> TMEM columns 0..127: W = T' K in lanes 0..63 and
+        // again in lanes 64..127 (A K-major, B = the K tile MN-major)
         tc_fence_after();
         const uint64_t dTP = desc_sw128(smem_u32(sm + P_TP), 16, 1024);
         const uint64_t dKm = desc_sw128(smem_u32(sm + P_KQ), 16384, 1024);
@@ -531,24 +560,48 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
         mma_commit(bar(PB_P2));
     }
     __syncwarp();
-    if (warp < 2) {
-        // W rows t = tid -> the tile, [2 kb][64 t][128 B] swizzled
+    if (tid >= 64) {
+        // Pt[r][i] = exp(G_r - G_C) q_r.k_i for i <= r, from this lane's p1 row,
+        // staged over the Q rows (T, which lived there, is dead)
+        const int r = tid - 64;
+        const float sr = sc->invD[r];
+        const uint32_t pt_s = smem_u32(sm + P_KQ + 8192);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i0 = 8 * c + 2 * e;
+                w[e] = pack_bf16(i0 <= r ? sr * x[i0] : 0.f, i0 + 1 <= r ? sr * x[i0 + 1] : 0.f);
+            }
+            st_shared_v4(pt_s + sw128_chunk(r, c), w[0], w[1], w[2], w[3]);
+        }
+    }
+    {
+        // W row t staged over the T' tile (p2, its last reader, has completed):
+        // warps 0-1 stage d_k 0..63 (kb 0), warps 2-3 d_k 64..127 (kb 1)
         ok = mbar_wait(bar(PB_P2), 0, lim, &no_abort) && ok;
         tc_fence_after();
-        const int t = tid;
+        const int t = tid & 63, kb = tid >> 6;
+        const uint32_t w_s = smem_u32(sm + P_TP + kb * 8192);
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-            float x[32];
-            tmem_ld32(tm + lane_off + 32 * q4, x);
-            uint8_t *wrow = tile + (q4 >> 1) * 8192;
+        for (int h2 = 0; h2 < 2; ++h2) {
+            float y[32];
+            tmem_ld32(tm + lane_off + 64 * kb + 32 * h2, y);
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) {
-                const float *e = x + 8 * c4;
-                *reinterpret_cast<uint4 *>(wrow + sw128_chunk(t, (q4 & 1) * 4 + c4)) =
-                    make_uint4(pack_bf16(e[0], e[1]), pack_bf16(e[2], e[3]), pack_bf16(e[4], e[5]),
-                               pack_bf16(e[6], e[7]));
+                const float *e = y + 8 * c4;
+                st_shared_v4(w_s + sw128_chunk(t, 4 * h2 + c4), pack_bf16(e[0], e[1]), pack_bf16(e[2], e[3]),
+                             pack_bf16(e[4], e[5]), pack_bf16(e[6], e[7]));
             }
         }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+        bulk_store(tile, smem_u32(sm + P_TP), 16384);                // W
+        bulk_store(tile + 40960, smem_u32(sm + P_KQ + 8192), 8192);  // Pt
+        bulk_commit_wait_read();
     }
     if (!ok && p.err) atomicCAS(p.err, 0, 52);
     if (tid == 0) mbar_wait(bar(PB_FULL), 0, lim, &no_abort);   // no TMA copy still landing at exit
@@ -585,8 +638,12 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.H;
-    const int per = MODE == MODE_OUT ? p.nseg : p.nseg - 1;      // ranges per (sequence, head)
-    const int nseq = blockIdx.x / (H * per), h = (blockIdx.x / per) % H, seg = blockIdx.x % per;
+    if (MODE == MODE_TRANS) grid_dep_launch();   // the combine may stage its prologue early
+    // ranges per (sequence, head); CTAs are ordered range-major, so that the
+    // first ranges (which need no combined start state) are scheduled first
+    const int per = MODE == MODE_OUT ? p.nseg : p.nseg - 1;
+    const int nunits = (int)(gridDim.x / per);
+    const int seg = blockIdx.x / nunits, nseq = (blockIdx.x % nunits) / H, h = blockIdx.x % H;
     int64_t bos, eos;
     SeqBounds{p.cu_seqlens, p.uniform_len}.get(nseq, bos, eos);
     const int nchunks = (int)((eos - bos + C - 1) / C);
@@ -595,9 +652,9 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
     const int nloc = ce > cb ? ce - cb : 0;
     const int64_t gc0 = (p.chunk_off ? (int64_t)p.chunk_off[nseq] : (int64_t)nseq * p.cps) + cb;
     const size_t state_off = ((size_t)nseq * H + h) * D * D;
-    const size_t unit_off = (((size_t)nseq * H + h) * (p.nseg - 1) + (seg - (MODE == MODE_OUT ? 1 : 0))) * D * D;
+    const size_t unit = ((size_t)nseq * H + h) * (p.nseg - 1) + (seg - (MODE == MODE_OUT ? 1 : 0));
     const float *start = MODE == MODE_TRANS ? nullptr
-                         : (seg == 0 ? p.state_in : p.seg_start + unit_off);
+                         : (seg == 0 ? p.state_in : p.seg_start + unit * D * D);
     float *finish = MODE == MODE_TRANS ? nullptr : (seg == p.nseg - 1 ? p.state_out : nullptr);
 
     if (tid == 0) {
@@ -636,10 +693,10 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                     *reinterpret_cast<float4 *>(finish + state_off + (size_t)tid * D + j) = v;
                 }
                 if (MODE == MODE_TRANS) {
-                    *reinterpret_cast<float4 *>(p.trans_r + unit_off + (size_t)tid * D + j) = make_float4(0.f, 0.f, 0.f, 0.f);
+                    *reinterpret_cast<float4 *>(p.trans_r + unit * D * D + (size_t)tid * D + j) = make_float4(0.f, 0.f, 0.f, 0.f);
                     float4 e = make_float4(0.f, 0.f, 0.f, 0.f);
                     if (tid >= j && tid < j + 4) (&e.x)[tid - j] = 1.f;
-                    *reinterpret_cast<float4 *>(p.trans_m + unit_off + (size_t)tid * D + j) = e;
+                    *reinterpret_cast<float4 *>(p.trans_m + unit * D * D + (size_t)tid * D + j) = e;
                 }
             }
         }
@@ -653,12 +710,20 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                 const int z = (int)(bos + (int64_t)(cb + n) * C);
                 if (n >= 2 && !mbar_wait(bar(CB_EMPTY + s), ((n - 2) >> 1) & 1, lim, abort_flag)) { fail(61); break; }
                 const uint32_t full = bar(CB_FULL + s);
-                mbar_arrive_expect_tx(full, C_STAGE);
+                const uint8_t *tile = p.tiles + ((size_t)(gc0 + n) * H + h) * kTileBytes;
+                // a transition range reads W and T'' only
+                mbar_arrive_expect_tx(full, MODE == MODE_TRANS ? C_STAGE - 24576 : C_STAGE);
                 for (int kb = 0; kb < 2; ++kb) {
                     tma_load_3d(st + CS_K + kb * 8192, &p.map_k, kb * 64, h, z, full);
                     tma_load_3d(st + CS_V + kb * 8192, &p.map_v, kb * 64, h, z, full);
                 }
-                bulk_load(st + CS_W, p.tiles + ((size_t)(gc0 + n) * H + h) * kTileBytes, (uint32_t)kTileBytes, full);
+                if (n == 0 && p.wait_tiles) grid_dep_wait();   // tiles come from the prep kernel
+                if (MODE == MODE_TRANS) {
+                    bulk_load(st + CS_W, tile, 16384, full);
+                    bulk_load(st + CS_TPP, tile + (CS_TPP - CS_W), 8192, full);
+                } else {
+                    bulk_load(st + CS_W, tile, (uint32_t)kTileBytes, full);
+                }
                 ++issued[s];
             }
             const int zero = 0;   // no copy may still be landing in shared memory at exit
@@ -779,6 +844,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
             tmem_st32u(tm + lane_off + base + col, pk);
         };
         compute_scalars(0);
+        if (MODE == MODE_OUT && seg > 0 && p.wait_start) grid_dep_wait();   // start state from the combine
         named_bar_sync(nb, 128);
         {
             // start state: given (MODE_OUT), zero (chain R) or the identity (chain X)
@@ -812,7 +878,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
             tc_fence_before();
             mbar_arrive(bar(bS));
         }
-        float *dest = MODE == MODE_TRANS ? (xchain ? p.trans_m : p.trans_r) + unit_off
+        float *dest = MODE == MODE_TRANS ? (xchain ? p.trans_m : p.trans_r) + unit * D * D
                                          : (finish ? finish + state_off : nullptr);
         for (int n = 0; n < nloc; ++n) {
             // residual epilogue: U^T (fp32, lane dv, 64 t) -> bf16 in its own first 32 columns
@@ -903,6 +969,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
     }
 
     // ---------------------------------------------------------------- teardown
+    if (p.wait_tiles) grid_dep_wait();   // (also for an empty range: completion implies the prep's)
     __syncthreads();
     if (warp == 8) {
         tc_fence_after();
@@ -914,14 +981,18 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
 //
 // Start state of every range after the first: S_{j+1} = S_j M_j + R_j,
 // sequentially over the ranges of one (sequence, head).  Rows of S are
-// independent, so a CTA owns 16 of them (grid (N*H, 8), four warps, 32 output
-// columns each).  The products run on tf32 mma.sync with the 3xTF32 split
-// (x = hi + lo, hi*hi + hi*lo + lo*hi), which keeps them at fp32 accuracy.
-// M_{j+1} streams into the other half of a double buffer (cp.async) while
-// step j computes.
+// independent, so a CTA owns 16 of them: grid (N*H, 8), eight warps.  Warp w
+// multiplies the k-slice [32 (w/2), +32) of S_j against column half w%2 of
+// M_j; the four k-slice partials meet in shared memory, where R_j is added.
+// The products run on bf16 mma.sync with each fp32 operand split in two
+// (x = hi + lo, both bf16; S M ~= S_hi M_hi + S_hi M_lo + S_lo M_hi), which
+// keeps about 16 mantissa bits; accumulation is fp32.  M_{j+1} streams into
+// the other half of a double buffer (cp.async) while step j computes.
 constexpr int kCombRows = 16;
-constexpr int kCombMP = 136, kCombSP = 132;   // row pitches: conflict-free fragment loads
-constexpr size_t kCombSmem = (size_t)(2 * D * kCombMP + kCombRows * kCombSP) * sizeof(float);
+constexpr int kCombThreads = 256;
+constexpr int kCombMP = 132, kCombSP = 136, kCombPP = 132;   // row pitches: conflict-free fragments
+constexpr size_t kCombSmem =
+    (size_t)(2 * D * kCombMP + kCombRows * kCombSP + 4 * kCombRows * kCombPP) * sizeof(float);
 
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)),
@@ -929,79 +1000,105 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
                  : "memory");
 }
 
-__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo) {
-    hi = tf32(x);
-    lo = tf32(x - __uint_as_float(hi));
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__global__ void __launch_bounds__(128)
+// (x, y) -> packed bf16 hi = rn(x, y) and lo = rn(x - hi_x, y - hi_y)
+__device__ __forceinline__ void split2(float x, float y, uint32_t &hi, uint32_t &lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+    const float2 hf = __bfloat1622float2(h);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    lo = pack_bf16(x - hf.x, y - hf.y);
+}
+
+__global__ void __launch_bounds__(kCombThreads, 1)
 gdn_scan_combine_kernel(const float *__restrict__ state_in, const float *__restrict__ trans_r,
-                        const float *__restrict__ trans_m, float *__restrict__ seg_start, int nseg) {
+                        const float *__restrict__ trans_m, float *__restrict__ seg_start, int nseg,
+                        int *err, uint64_t timeout_ns) {
+    (void)err;
+    (void)timeout_ns;
     extern __shared__ float smf[];
-    float *Ms = smf;                          // M_j [k][n], two buffers
-    float *Ss = Ms + 2 * D * kCombMP;         // S rows [16][D]
+    float *Ms = smf;                              // M_j [k][n], two buffers
+    float *Ss = Ms + 2 * D * kCombMP;             // S_j rows [16][D]
+    float *Ps = Ss + kCombRows * kCombSP;         // k-slice partials [4][16][D]
     const int nh = blockIdx.x, r0 = blockIdx.y * kCombRows;
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31, g = lane >> 2, q = lane & 3;
+    const int kg = warp >> 1, ch = warp & 1;
+    grid_dep_wait();     // the transitions come from the previous kernel
+    grid_dep_launch();   // the output pass may launch; its first ranges do not need this grid
     auto stage = [&](int j) {
         const float *src = trans_m + ((size_t)nh * (nseg - 1) + j) * D * D;
         float *dst = Ms + (j & 1) * D * kCombMP;
-        for (int i = t; i < D * D / 4; i += 128) cp_async16(dst + (i >> 5) * kCombMP + 4 * (i & 31), src + 4 * i);
+        for (int i = t; i < D * D / 4; i += kCombThreads)
+            cp_async16(dst + (i >> 5) * kCombMP + 4 * (i & 31), src + 4 * i);
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
     if (nseg > 1) stage(0);
-    for (int i = t; i < kCombRows * D; i += 128)
+    for (int i = t; i < kCombRows * D; i += kCombThreads)
         Ss[(i >> 7) * kCombSP + (i & 127)] =
             state_in ? state_in[(size_t)nh * D * D + (size_t)(r0 + (i >> 7)) * D + (i & 127)] : 0.f;
     for (int j = 0; j + 1 < nseg; ++j) {
-        const size_t u = ((size_t)nh * (nseg - 1) + j) * D * D;
-        const float *rrow0 = trans_r + u + (size_t)(r0 + g) * D, *rrow1 = rrow0 + 8 * D;
-        float acc[4][4], accx[4][4];   // hi*hi terms; the two cross terms (seeded with R_j)
+        const size_t u = ((size_t)nh * (nseg - 1) + j) * D * D + (size_t)r0 * D;   // rows r0.. of step j
+        float rv[kCombRows * D / kCombThreads];
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-            const int col = 32 * warp + 8 * nt + 2 * q;
-            const float2 a = *reinterpret_cast<const float2 *>(rrow0 + col);
-            const float2 b = *reinterpret_cast<const float2 *>(rrow1 + col);
-            accx[nt][0] = a.x; accx[nt][1] = a.y; accx[nt][2] = b.x; accx[nt][3] = b.y;
-            acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-        }
+        for (int i = 0; i < kCombRows * D / kCombThreads; ++i) rv[i] = trans_r[u + t + kCombThreads * i];
+        float acc[8][4], accx[8][4];   // hi*hi terms; the two cross terms
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[nt][e] = accx[nt][e] = 0.f;
         asm volatile("cp.async.wait_group 0;" ::: "memory");
         __syncthreads();   // M_j landed for every thread; S_j rows are written
         if (j + 2 < nseg) stage(j + 1);
         const float *M = Ms + (j & 1) * D * kCombMP;
-#pragma unroll 2
-        for (int ks = 0; ks < D / 8; ++ks) {
-            const int k0 = 8 * ks;
-            uint32_t ah[4], al[4];
-            split_tf32(Ss[g * kCombSP + k0 + q], ah[0], al[0]);
-            split_tf32(Ss[(g + 8) * kCombSP + k0 + q], ah[1], al[1]);
-            split_tf32(Ss[g * kCombSP + k0 + q + 4], ah[2], al[2]);
-            split_tf32(Ss[(g + 8) * kCombSP + k0 + q + 4], ah[3], al[3]);
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                const int n = 32 * warp + 8 * nt + g;
+        for (int ks = 0; ks < 2; ++ks) {
+            const int k0 = 32 * kg + 16 * ks;
+            uint32_t ah[4], al[4];
+            const float2 s00 = *reinterpret_cast<const float2 *>(Ss + g * kCombSP + k0 + 2 * q);
+            const float2 s10 = *reinterpret_cast<const float2 *>(Ss + (g + 8) * kCombSP + k0 + 2 * q);
+            const float2 s01 = *reinterpret_cast<const float2 *>(Ss + g * kCombSP + k0 + 2 * q + 8);
+            const float2 s11 = *reinterpret_cast<const float2 *>(Ss + (g + 8) * kCombSP + k0 + 2 * q + 8);
+            split2(s00.x, s00.y, ah[0], al[0]);
+            split2(s10.x, s10.y, ah[1], al[1]);
+            split2(s01.x, s01.y, ah[2], al[2]);
+            split2(s11.x, s11.y, ah[3], al[3]);
+            const float *m0 = M + (k0 + 2 * q) * kCombMP, *m8 = m0 + 8 * kCombMP;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                const int n = 64 * ch + 8 * nt + g;
                 uint32_t bh0, bl0, bh1, bl1;
-                split_tf32(M[(k0 + q) * kCombMP + n], bh0, bl0);
-                split_tf32(M[(k0 + q + 4) * kCombMP + n], bh1, bl1);
-                mma_tf32(accx[nt], al[0], al[1], al[2], al[3], bh0, bh1);
-                mma_tf32(accx[nt], ah[0], ah[1], ah[2], ah[3], bl0, bl1);
-                mma_tf32(acc[nt], ah[0], ah[1], ah[2], ah[3], bh0, bh1);
+                split2(m0[n], m0[kCombMP + n], bh0, bl0);
+                split2(m8[n], m8[kCombMP + n], bh1, bl1);
+                mma_bf16_16816(accx[nt], al[0], al[1], al[2], al[3], bh0, bh1);
+                mma_bf16_16816(accx[nt], ah[0], ah[1], ah[2], ah[3], bl0, bl1);
+                mma_bf16_16816(acc[nt], ah[0], ah[1], ah[2], ah[3], bh0, bh1);
             }
         }
-        float *o0 = seg_start + u + (size_t)(r0 + g) * D, *o1 = o0 + 8 * D;
+        float *P = Ps + kg * kCombRows * kCombPP;
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[nt][e] += accx[nt][e];
-            const int col = 32 * warp + 8 * nt + 2 * q;
-            *reinterpret_cast<float2 *>(o0 + col) = make_float2(acc[nt][0], acc[nt][1]);
-            *reinterpret_cast<float2 *>(o1 + col) = make_float2(acc[nt][2], acc[nt][3]);
+        for (int nt = 0; nt < 8; ++nt) {
+            const int col = 64 * ch + 8 * nt + 2 * q;
+            *reinterpret_cast<float2 *>(P + g * kCombPP + col) =
+                make_float2(acc[nt][0] + accx[nt][0], acc[nt][1] + accx[nt][1]);
+            *reinterpret_cast<float2 *>(P + (g + 8) * kCombPP + col) =
+                make_float2(acc[nt][2] + accx[nt][2], acc[nt][3] + accx[nt][3]);
         }
-        __syncthreads();   // every warp has read S_j
+        __syncthreads();   // partials complete; every warp has read S_j
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-            const int col = 32 * warp + 8 * nt + 2 * q;
-            *reinterpret_cast<float2 *>(Ss + g * kCombSP + col) = make_float2(acc[nt][0], acc[nt][1]);
-            *reinterpret_cast<float2 *>(Ss + (g + 8) * kCombSP + col) = make_float2(acc[nt][2], acc[nt][3]);
+        for (int i = 0; i < kCombRows * D / kCombThreads; ++i) {
+            const int e = t + kCombThreads * i, row = e >> 7, col = e & 127;
+            float v = rv[i];
+#pragma unroll
+            for (int s = 0; s < 4; ++s) v += Ps[(s * kCombRows + row) * kCombPP + col];
+            seg_start[u + e] = v;
+            Ss[row * kCombSP + col] = v;
         }
     }
 }
@@ -1043,9 +1140,26 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 size_t chunk_off_bytes(int num_seqs) { return align_up(4 * (size_t)(num_seqs + 1), 1024); }
 
-// bytes of one of the three range-state arrays (R, M, start states)
-size_t scan_array_bytes(int num_seqs, int H, int nseg) {
-    return (size_t)num_seqs * H * (size_t)(nseg > 1 ? nseg - 1 : 0) * D * D * sizeof(float);
+// units of the range-transition arrays (R, M, start states)
+size_t scan_units(int num_seqs, int H, int nseg) {
+    return (size_t)num_seqs * H * (size_t)(nseg > 1 ? nseg - 1 : 0);
+}
+
+// Launch with programmatic stream serialization (see launch_prefill_tc).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 bool set_smem_attrs() {
@@ -1085,7 +1199,7 @@ size_t tc_workspace_bytes(int num_seqs, int64_t total_tokens, int H, bool varlen
     const int nseg = tc_scan_segments(num_seqs, total_tokens, H, false, kScanRefSMs);
     return 1024 + chunk_off_bytes(num_seqs) +
            (size_t)tc_chunk_bound(num_seqs, total_tokens, varlen) * (size_t)H * kTileBytes +
-           3 * scan_array_bytes(num_seqs, H, nseg);
+           3 * scan_units(num_seqs, H, nseg) * D * D * sizeof(float);
 }
 
 int tc_kernel_count(int num_seqs, int64_t total_tokens, int H, bool varlen) {
@@ -1106,8 +1220,8 @@ cudaError_t launch_prefill_tc(const TcLaunch &L, cudaStream_t stream) {
     // workspace was sized for: the SM count is capped at the reference count)
     const int nseg = tc_scan_segments(L.num_seqs, L.total_tokens, L.H, varlen, scan_sm_count());
     const int seg_len = nseg > 1 ? (cps + nseg - 1) / nseg : 0x3fffffff;
-    float *scan_base = reinterpret_cast<float *>(tiles + (size_t)bound * L.H * kTileBytes);
-    const size_t scan_elems = scan_array_bytes(L.num_seqs, L.H, nseg) / sizeof(float);
+    uint8_t *scan_base = tiles + (size_t)bound * L.H * kTileBytes;
+    const size_t su = scan_units(L.num_seqs, L.H, nseg);
 
     PrepParams pp;
     ChainParams cp;
@@ -1135,22 +1249,37 @@ cudaError_t launch_prefill_tc(const TcLaunch &L, cudaStream_t stream) {
     cp.out = static_cast<__nv_bfloat16 *>(L.out);
     cp.nseg = nseg;
     cp.seg_len = seg_len;
-    cp.trans_r = scan_base;
-    cp.trans_m = scan_base + scan_elems;
-    cp.seg_start = scan_base + 2 * scan_elems;
+    cp.trans_r = reinterpret_cast<float *>(scan_base);
+    cp.trans_m = cp.trans_r + su * D * D;
+    cp.seg_start = cp.trans_m + su * D * D;
 
     if (!set_smem_attrs()) return cudaGetLastError() != cudaSuccess ? cudaGetLastError() : cudaErrorUnknown;
     if (varlen) gdn_chunk_offsets_kernel<<<1, 1024, 0, stream>>>(L.cu_seqlens, L.num_seqs, chunk_off);
     dim3 pgrid((unsigned)bound, (unsigned)L.H);
     gdn_chunk_prep_kernel<<<pgrid, kPrepThreads, P_ALLOC, stream>>>(pp);
     const unsigned units = (unsigned)L.num_seqs * (unsigned)L.H;
+    // TRANS, the combine and OUT are launched with programmatic stream
+    // serialization: each may start its prologue while the previous kernel
+    // drains, and waits (griddepcontrol.wait) before it reads that kernel's
+    // results.
     if (nseg > 1) {
-        gdn_chunk_chain_kernel<MODE_TRANS><<<units * (nseg - 1), kChainThreads, C_ALLOC, stream>>>(cp);
-        dim3 cgrid(units, D / kCombRows);
-        gdn_scan_combine_kernel<<<cgrid, 128, kCombSmem, stream>>>(L.state_in, cp.trans_r, cp.trans_m,
-                                                                  scan_base + 2 * scan_elems, nseg);
+        ChainParams ct = cp;
+        ct.wait_tiles = 1;
+        ct.wait_start = 0;
+        cudaError_t e = launch_pdl(gdn_chunk_chain_kernel<MODE_TRANS>, dim3(units * (nseg - 1)), dim3(kChainThreads),
+                                   C_ALLOC, stream, ct);
+        if (e != cudaSuccess) return e;
+        e = launch_pdl(gdn_scan_combine_kernel, dim3(units, D / kCombRows), dim3(kCombThreads), kCombSmem, stream,
+                       L.state_in, static_cast<const float *>(cp.trans_r), static_cast<const float *>(cp.trans_m),
+                       const_cast<float *>(cp.seg_start), nseg, L.err, L.timeout_ns);
+        if (e != cudaSuccess) return e;
     }
-    gdn_chunk_chain_kernel<MODE_OUT><<<units * nseg, kChainThreads, C_ALLOC, stream>>>(cp);
+    ChainParams co = cp;
+    co.wait_tiles = nseg > 1 ? 0 : 1;   // after the combine, the prep kernel has completed
+    co.wait_start = nseg > 1 ? 1 : 0;
+    const cudaError_t e = launch_pdl(gdn_chunk_chain_kernel<MODE_OUT>, dim3(units * nseg), dim3(kChainThreads),
+                                     C_ALLOC, stream, co);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

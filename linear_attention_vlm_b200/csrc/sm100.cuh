@@ -102,6 +102,17 @@ __device__ __forceinline__ bool named_bar_any(int id, int nthreads, bool pred) {
     return r != 0;
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+
+// Block until the grids this one depends on (launched before it in the
+// stream) have completed and their memory is visible; a no-op when the
+// kernel was launched without programmatic stream serialization.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Allow the next grid in the stream to be scheduled once every CTA of this
+// grid has issued this (or exited).
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *m) {
