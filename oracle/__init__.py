@@ -126,3 +126,8 @@ def decode_step(q, k, v, g, beta, state) -> Tuple[np.ndarray, np.ndarray]:
     if rc != 0:
         raise RuntimeError("gdn_oracle_decode failed (%d)" % rc)
     return out, s
+
+
+# Steps around the recurrence inside one layer (plain numpy, fp64).
+from .layer_ops import (ACT_NONE, ACT_SILU, GATE_SIGMOID, GATE_SILU,  # noqa: E402,F401
+                        log_sigmoid, output_gate, preprocess, sigmoid)
