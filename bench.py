@@ -214,6 +214,17 @@ def run_native(args):
         t = toks[i % len(toks)]
         gdn.gdn_decode_step(t["q"], t["k"], t["v"], t["g"], t["beta"], S, S, out=dout)
 
+    # ---- layer steps around the recurrence, on the prefill shapes
+    lx = {k: v.to(dev) for k, v in W.layer_inputs(T, H, dk, w.dtype, seed=rank).items()}
+    gate_out = torch.empty_like(lx["z"])
+
+    def preprocess_once():
+        gdn.gdn_preprocess(lx["xq"], lx["xk"], lx["xv"], lx["conv_w"], lx["a"], lx["b"], None, None,
+                           activation=gdn.ACT_SILU, want_state=False)
+
+    def gate_once():
+        gdn.gdn_output_gate(out, lx["z"], lx["norm_w"], gate=gdn.GATE_SIGMOID, out=gate_out)
+
     # ---- e2e buffers (pinned host, fresh device copies each step)
     pin = {k: v.pin_memory() for k, v in host.items() if isinstance(v, torch.Tensor) and k != "cu_seqlens"}
     out_h = torch.empty((T, H, dv), dtype=w.dtype).pin_memory()
@@ -235,6 +246,8 @@ def run_native(args):
         prefill_once()
         decode_once(i)
         e2e_once()
+        preprocess_once()
+        gate_once()
     torch.cuda.synchronize()
 
     def timed(fn, steps, do_flush=True):
@@ -259,10 +272,17 @@ def run_native(args):
         ms_prefill = timed(lambda i: prefill_once(), K)
         ms_decode = timed(decode_once, K)
         ms_e2e = timed(lambda i: e2e_once(), max(3, K // 10), do_flush=False)
+        ms_pre = timed(lambda i: preprocess_once(), K)
+        ms_gate = timed(lambda i: gate_once(), K)
         wall = time.time() - t_wall0
     ms_prefill = max_over_ranks(ms_prefill, world)
     ms_decode = max_over_ranks(ms_decode, world)
     ms_e2e = max_over_ranks(ms_e2e, world)
+    ms_pre = max_over_ranks(ms_pre, world)
+    ms_gate = max_over_ranks(ms_gate, world)
+    el = 2 if w.dtype == torch.bfloat16 else 4
+    pre_bytes = 6 * T * H * dk * el + 4 * T * H * 4 + 3 * H * dk * 16    # x in, q/k/v out, a/b in, g/beta out, taps
+    gate_bytes = 3 * T * H * dv * el + dv * 4                             # o, z in, y out, norm weight
 
     tokens = T * world
     value = aggregate_throughput(T, world, ms_prefill)
@@ -304,9 +324,21 @@ def run_native(args):
                                 "achieved": d_gbs, "peak": hbm, "unit": "GB/s",
                                 "frac": d_gbs / hbm, "traffic": None,
                                 "algorithmic_bytes": dbytes}},
+        "preprocess": {"metric": "pre-processing tokens/s (conv4 + SiLU + q/k L2 norm + gates), prefill shapes",
+                       "value": aggregate_throughput(T, world, ms_pre), "unit": "tokens/s", "ms_per_step": ms_pre,
+                       "roofline": {"kernel": "gdn_preprocess_kernel", "bound": "hbm",
+                                    "achieved": pre_bytes / (ms_pre * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                                    "frac": pre_bytes / (ms_pre * 1e-3) / 1e9 / hbm, "traffic": None,
+                                    "algorithmic_bytes": pre_bytes}},
+        "output_gate": {"metric": "output gate tokens/s (RMS norm + sigmoid gate), prefill shapes",
+                        "value": aggregate_throughput(T, world, ms_gate), "unit": "tokens/s", "ms_per_step": ms_gate,
+                        "roofline": {"kernel": "gdn_output_gate_kernel", "bound": "hbm",
+                                     "achieved": gate_bytes / (ms_gate * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                                     "frac": gate_bytes / (ms_gate * 1e-3) / 1e9 / hbm, "traffic": None,
+                                     "algorithmic_bytes": gate_bytes}},
         "e2e": {"value": aggregate_throughput(T, world, ms_e2e), "unit": "tokens/s",
                 "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": K * launches_per_prefill + K + max(3, K // 10) * launches_per_prefill,
+        "gpu_launches": K * launches_per_prefill + K + max(3, K // 10) * launches_per_prefill + 2 * K,
         "clocks": clk.summary(),
         "timed_wall_s": wall,
     }

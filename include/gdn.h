@@ -172,6 +172,68 @@ const char *gdn_status_string(int status);
  * library ("" if none).  Valid until the next call on this thread. */
 const char *gdn_last_cuda_error(void);
 
+/* ------------------------------------------------------------------ layer steps around the recurrence
+ *
+ * The explainer page (InfiniteVL, "Step 2: Process tokens with Hybrid
+ * Blocks") gives every Gated DeltaNet layer a 1-D convolution of window 4 and
+ * an output gate, and fixes nothing else about them.  These two entry points
+ * take the plainest reading: the convolution is causal and depthwise over the
+ * q, k and v channels (restarted at each sequence start), q and k are then
+ * L2-normalised, beta = sigmoid(b) and g = log(sigmoid(a)); the output gate is
+ * y = n(o) * act(z).  Conventions are those above (device pointers, 16-byte
+ * alignment, asynchronous, no allocation).
+ */
+
+typedef enum gdn_activation { GDN_ACT_NONE = 0, GDN_ACT_SILU = 1 } gdn_activation;
+typedef enum gdn_gate { GDN_GATE_SIGMOID = 0, GDN_GATE_SILU = 1 } gdn_gate;
+
+/*
+ * From a layer's raw projections to gdn_prefill's inputs, per (token, head):
+ *
+ *   y_X[t] = act( sum_{i=0..3} conv_w[X][h][c][i] * x_X[t - 3 + i] )
+ *            for X = q, k, v; positions before a sequence's first token come
+ *            from conv_state_in (slot j = position start - 3 + j), or are 0
+ *   q = y_q / sqrt(sum_c y_q^2 + eps),   k likewise,   v = y_v
+ *   g = log(sigmoid(a)) = -softplus(-a),   beta = sigmoid(b)
+ *
+ *   xq, xk, xv     [total_tokens, H, d]  dtype  raw projections
+ *   conv_w         [3, H, d, 4]          fp32   (q, k, v; tap 3 = current token)
+ *   a_logit, b_logit [total_tokens, H]   fp32
+ *   conv_state_in  [num_seqs, 3, 3, H, d] dtype (slot, tensor, head, channel),
+ *                  or NULL for zeros
+ *   q, k, v        [total_tokens, H, d]  dtype (written)
+ *   g, beta        [total_tokens, H]     fp32  (written)
+ *   conv_state_out [num_seqs, 3, 3, H, d] dtype (written: the raw inputs at the
+ *                  last three positions of each sequence, older ones from
+ *                  conv_state_in when a sequence is shorter), or NULL; it may
+ *                  equal conv_state_in (in-place update)
+ *   cu_seqlens     as in gdn_prefill (NULL: num_seqs equal sequences)
+ *   activation     GDN_ACT_NONE or GDN_ACT_SILU (applied after the convolution)
+ *   eps            in [0, 1]
+ *
+ * With cu_seqlens = [0, 1, ..., B] this is the per-token step of decoding.
+ * Supported: d in {64, 128}, dtype GDN_F32 or GDN_BF16.  Outputs may not
+ * overlap inputs or each other (GDN_ERR_INVALID_ARG).
+ */
+int gdn_preprocess(const void *xq, const void *xk, const void *xv, const float *conv_w,
+                   const float *a_logit, const float *b_logit, const void *conv_state_in, void *q,
+                   void *k, void *v, float *g, float *beta, void *conv_state_out,
+                   const int32_t *cu_seqlens, int num_seqs, int64_t total_tokens, int H, int d,
+                   int activation, float eps, int dtype, void *stream);
+
+/*
+ * Output gate over rows of d_v values (rows = tokens x heads):
+ *
+ *   n = o                                        if norm_w is NULL
+ *   n = o / sqrt(mean_c o^2 + eps) * norm_w[c]   otherwise (RMS norm per row)
+ *   y = n * sigmoid(z)   (GDN_GATE_SIGMOID)   or   n * z * sigmoid(z)   (GDN_GATE_SILU)
+ *
+ *   o, z, y   [rows, dv] dtype;  norm_w [dv] fp32 or NULL.
+ * y may equal o (in place); no other overlap.  Supported: dv in {64, 128}.
+ */
+int gdn_output_gate(const void *o, const void *z, const float *norm_w, void *y, int64_t rows, int dv,
+                    int gate, float eps, int dtype, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,11 +1,15 @@
 """B200-native Gated DeltaNet hot path (InfiniteVL's linear token mixer).
 
-Chunkwise prefill with a carried fp32 state and a bandwidth-bound decode step,
-written as CUDA kernels for sm_100a behind the C ABI in ``include/gdn.h``.
+Chunkwise prefill with a carried fp32 state, a bandwidth-bound decode step and
+the layer steps around them (short convolution / norms / gates before, the
+output gate after), written as CUDA kernels for sm_100a behind the C ABI in
+``include/gdn.h``.
 This package is the thin Python binding of that library.
 """
-from .gdn import (CHUNK, GDN_BF16, GDN_F32, GdnError, declared_symbols, gdn_decode_step,
-                  gdn_prefill, gdn_prefill_kernel_count, gdn_prefill_noalloc, gdn_prefill_workspace_size, library, status_string)
+from .gdn import (ACT_NONE, ACT_SILU, CHUNK, GATE_SIGMOID, GATE_SILU, GDN_BF16, GDN_F32, GdnError,
+                  declared_symbols, gdn_decode_step, gdn_output_gate, gdn_prefill, gdn_prefill_kernel_count,
+                  gdn_prefill_noalloc, gdn_prefill_workspace_size, gdn_preprocess, library, status_string)
 
-__all__ = ["CHUNK", "GDN_BF16", "GDN_F32", "GdnError", "declared_symbols", "gdn_decode_step",
-           "gdn_prefill", "gdn_prefill_kernel_count", "gdn_prefill_noalloc", "gdn_prefill_workspace_size", "library", "status_string"]
+__all__ = ["ACT_NONE", "ACT_SILU", "CHUNK", "GATE_SIGMOID", "GATE_SILU", "GDN_BF16", "GDN_F32", "GdnError",
+           "declared_symbols", "gdn_decode_step", "gdn_output_gate", "gdn_prefill", "gdn_prefill_kernel_count",
+           "gdn_prefill_noalloc", "gdn_prefill_workspace_size", "gdn_preprocess", "library", "status_string"]

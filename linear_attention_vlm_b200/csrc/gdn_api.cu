@@ -55,6 +55,13 @@ int check_prefill(const void *q, const void *k, const void *v, const float *g,
     return GDN_OK;
 }
 
+// true if [a, a + na) and [b, b + nb) share a byte
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    if (!a || !b || na == 0 || nb == 0) return false;
+    const char *x = static_cast<const char *>(a), *y = static_cast<const char *>(b);
+    return x < y + nb && y < x + na;
+}
+
 }  // namespace
 
 int gdn::note_cuda_error(cudaError_t e) { return cuda_fail(e); }
@@ -139,6 +146,82 @@ int gdn_decode_step(const void *q, const void *k, const void *v, const float *g,
     }
     cudaError_t e = gdn::launch_decode(dtype, dk, q, k, v, g, beta, state_in, state_out, out, B,
                                        H, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e);
+}
+
+int gdn_preprocess(const void *xq, const void *xk, const void *xv, const float *conv_w,
+                   const float *a_logit, const float *b_logit, const void *conv_state_in, void *q,
+                   void *k, void *v, float *g, float *beta, void *conv_state_out,
+                   const int32_t *cu_seqlens, int num_seqs, int64_t total_tokens, int H, int d,
+                   int activation, float eps, int dtype, void *stream) {
+    if (num_seqs < 1 || H < 1 || total_tokens < 0) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (activation != GDN_ACT_NONE && activation != GDN_ACT_SILU) return GDN_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || eps > 1.f) return GDN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return GDN_ERR_UNSUPPORTED;
+    if ((int64_t)num_seqs * 3 * 3 * H * d > (int64_t)INT32_MAX) return GDN_ERR_INVALID_ARG;
+    if (total_tokens > (int64_t)INT32_MAX * 32) return GDN_ERR_INVALID_ARG;
+    if (!cu_seqlens && total_tokens % num_seqs != 0) return GDN_ERR_INVALID_ARG;
+    if (total_tokens > 0 && (!xq || !xk || !xv || !conv_w || !a_logit || !b_logit || !q || !k || !v || !g || !beta))
+        return GDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {xq, xk, xv, conv_w, a_logit, b_logit, conv_state_in, q, k, v, g, beta, conv_state_out,
+                          cu_seqlens};
+    for (const void *p : ptrs)
+        if (p && misaligned(p)) return GDN_ERR_INVALID_ARG;
+    const size_t es = dtype == GDN_BF16 ? 2 : 4;
+    const size_t tens = (size_t)total_tokens * H * d * es, gates = (size_t)total_tokens * H * 4;
+    const size_t st = (size_t)num_seqs * 9 * H * d * es;
+    // no output may overlap an input; the convolution state may be updated in place
+    const void *outs[] = {q, k, v, g, beta};
+    const size_t out_n[] = {tens, tens, tens, gates, gates};
+    const void *ins[] = {xq, xk, xv, a_logit, b_logit, conv_state_in, conv_w};
+    const size_t in_n[] = {tens, tens, tens, gates, gates, st, (size_t)3 * H * d * 16};
+    for (int i = 0; i < 5; ++i) {
+        for (int j = 0; j < 7; ++j)
+            if (overlaps(outs[i], out_n[i], ins[j], in_n[j])) return GDN_ERR_INVALID_ARG;
+        if (overlaps(outs[i], out_n[i], conv_state_out, st)) return GDN_ERR_INVALID_ARG;
+        for (int j = i + 1; j < 5; ++j)
+            if (overlaps(outs[i], out_n[i], outs[j], out_n[j])) return GDN_ERR_INVALID_ARG;
+    }
+    for (int j = 0; j < 7; ++j)
+        if (j != 5 && overlaps(conv_state_out, st, ins[j], in_n[j])) return GDN_ERR_INVALID_ARG;
+    if (conv_state_out && conv_state_in && conv_state_out != conv_state_in && overlaps(conv_state_out, st, conv_state_in, st))
+        return GDN_ERR_INVALID_ARG;
+    if (total_tokens == 0 && !conv_state_out) return GDN_OK;
+    gdn::PreprocessArgs A;
+    A.xq = xq; A.xk = xk; A.xv = xv;
+    A.conv_w = conv_w; A.a_logit = a_logit; A.b_logit = b_logit;
+    A.cs_in = conv_state_in;
+    A.q = q; A.k = k; A.v = v; A.g = g; A.beta = beta;
+    A.cs_out = conv_state_out;
+    A.cu_seqlens = cu_seqlens;
+    A.num_seqs = num_seqs;
+    A.total_tokens = total_tokens;
+    A.H = H; A.d = d; A.activation = activation; A.dtype = dtype;
+    A.eps = eps;
+    const cudaError_t e = gdn::launch_preprocess(A, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e);
+}
+
+int gdn_output_gate(const void *o, const void *z, const float *norm_w, void *y, int64_t rows, int dv,
+                    int gate, float eps, int dtype, void *stream) {
+    if (rows < 0) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (gate != GDN_GATE_SIGMOID && gate != GDN_GATE_SILU) return GDN_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || eps > 1.f) return GDN_ERR_INVALID_ARG;
+    if (dv != 64 && dv != 128) return GDN_ERR_UNSUPPORTED;
+    if (rows == 0) return GDN_OK;
+    if (rows > (int64_t)INT32_MAX * 8) return GDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {o, z, y};
+    for (const void *p : ptrs)
+        if (!p || misaligned(p)) return GDN_ERR_INVALID_ARG;
+    if (norm_w && misaligned(norm_w)) return GDN_ERR_INVALID_ARG;
+    const size_t n = (size_t)rows * dv * (dtype == GDN_BF16 ? 2 : 4);
+    // y may equal o (in place); no other overlap
+    if (y != o && overlaps(y, n, o, n)) return GDN_ERR_INVALID_ARG;
+    if (overlaps(y, n, z, n) || overlaps(y, n, norm_w, (size_t)dv * 4)) return GDN_ERR_INVALID_ARG;
+    const cudaError_t e = gdn::launch_output_gate(dtype, dv, o, z, norm_w, y, rows, gate, eps,
+                                                  static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GDN_OK : cuda_fail(e);
 }
 

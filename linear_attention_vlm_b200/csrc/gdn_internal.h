@@ -48,4 +48,23 @@ cudaError_t launch_prefill_simt(int dtype, int dk, const void *q, const void *k,
                                 const int32_t *cu_seqlens, int64_t uniform_len,
                                 int num_seqs, int H, cudaStream_t stream);
 
+// Layer steps around the recurrence (layer_ops.cu).
+struct PreprocessArgs {
+    const void *xq, *xk, *xv;          // raw projections [T, H, d], dtype
+    const float *conv_w;               // [3, H, d, 4]
+    const float *a_logit, *b_logit;    // [T, H]
+    const void *cs_in;                 // [N, 3, 3, H, d] dtype, or null (zeros)
+    void *q, *k, *v;                   // [T, H, d] dtype (written)
+    float *g, *beta;                   // [T, H] (written)
+    void *cs_out;                      // [N, 3, 3, H, d] dtype, or null
+    const int32_t *cu_seqlens;         // [N+1] or null (N equal sequences)
+    int num_seqs;
+    int64_t total_tokens;
+    int H, d, activation, dtype;
+    float eps;
+};
+cudaError_t launch_preprocess(const PreprocessArgs &A, cudaStream_t stream);
+cudaError_t launch_output_gate(int dtype, int dv, const void *o, const void *z, const float *norm_w, void *y,
+                               int64_t rows, int gate, float eps, cudaStream_t stream);
+
 }  // namespace gdn

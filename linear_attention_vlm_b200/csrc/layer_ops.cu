@@ -1,0 +1,343 @@
+// The layer steps around the Gated DeltaNet recurrence (explainer page,
+// "Step 2: Process tokens with Hybrid Blocks": every Gated DeltaNet layer
+// has a 1-D convolution of window 4 and an output gate).
+//
+// gdn_preprocess_kernel: per (token, head), from the raw projections
+//   y_X = act( sum_{i=0..3} w_X[c][i] x_X[t - 3 + i] )     X in {q, k, v},
+//         causal, depthwise, restarted at each sequence start (earlier
+//         positions come from the carried convolution state, else zero)
+//   q = y_q / sqrt(|y_q|^2 + eps),  k likewise,  v = y_v
+//   g = log(sigmoid(a)),  beta = sigmoid(b)
+// A CTA stages the raw inputs of 64 tokens (+3 before them) of one head in
+// shared memory, so every input is read from HBM once with all loads in
+// flight together; lanes own d/32 consecutive channels, and the L2 norms are
+// warp reductions.
+// gdn_conv_state_kernel writes the convolution state after each sequence
+// (the raw inputs at its last three positions); it runs after the main
+// kernel, so the state may be updated in place.
+// gdn_output_gate_kernel: y = n(o) * act(z) per (token, head), n the identity
+// or an RMS norm over d_v with per-channel weights, act sigmoid or SiLU; one
+// warp per (token, head).
+// All three are HBM-bound streaming kernels.
+#include "gdn_internal.h"
+
+namespace gdn {
+namespace {
+
+template <typename T, int CPL>
+__device__ __forceinline__ void load_ch(const T *p, float (&x)[CPL]) {
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) x[j] = to_f32(p[j]);
+}
+
+template <>
+__device__ __forceinline__ void load_ch<__nv_bfloat16, 4>(const __nv_bfloat16 *p, float (&x)[4]) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+}
+
+template <>
+__device__ __forceinline__ void load_ch<float, 4>(const float *p, float (&x)[4]) {
+    const float4 u = *reinterpret_cast<const float4 *>(p);
+    x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
+}
+
+template <typename T, int CPL>
+__device__ __forceinline__ void store_ch(T *p, const float (&x)[CPL]) {
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) p[j] = from_f32<T>(x[j]);
+}
+
+template <>
+__device__ __forceinline__ void store_ch<__nv_bfloat16, 4>(__nv_bfloat16 *p, const float (&x)[4]) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(x[0], x[1]);
+    const __nv_bfloat162 b = __floats2bfloat162_rn(x[2], x[3]);
+    uint2 u;
+    u.x = *reinterpret_cast<const uint32_t *>(&a);
+    u.y = *reinterpret_cast<const uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(p) = u;
+}
+
+template <>
+__device__ __forceinline__ void store_ch<float, 4>(float *p, const float (&x)[4]) {
+    *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
+}
+
+__device__ __forceinline__ float warp_sum(float s) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    return s;
+}
+
+// sigmoid and SiLU with the fast exponential and a correctly rounded
+// reciprocal (relative error ~1e-6, far below the bf16 storage step)
+__device__ __forceinline__ float sigmoid_f(float x) { return __frcp_rn(1.f + __expf(-x)); }
+__device__ __forceinline__ float silu_f(float x) { return x * __frcp_rn(1.f + __expf(-x)); }
+
+// log(sigmoid(x)) = min(x, 0) - log1p(exp(-|x|)), without overflow
+__device__ __forceinline__ float log_sigmoid_f(float x) { return fminf(x, 0.f) - log1pf(expf(-fabsf(x))); }
+
+// Sequence n containing token t: the last n with bos(n) <= t (empty sequences
+// share their start with the next one and are skipped that way).
+__device__ __forceinline__ int seq_of(const SeqBounds &sb, int N, int64_t t) {
+    if (!sb.cu) return (int)(t / sb.uniform_len);
+    int lo = 0, hi = N - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (sb.cu[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+constexpr int kPreTokensPerWarp = 8;
+constexpr int kPreWarps = 8;
+constexpr int kPreTokens = kPreTokensPerWarp * kPreWarps;   // tokens per CTA
+constexpr int kPreWin = kPreTokens + 3;                      // staged positions
+
+template <typename T, int D>
+constexpr size_t preprocess_smem() {
+    return (size_t)3 * kPreWin * D * sizeof(T) + (size_t)3 * D * 4 * sizeof(float);
+}
+
+template <typename T>
+__device__ __forceinline__ const T *pick3(int X, const T *a, const T *b, const T *c) {
+    return X == 0 ? a : (X == 1 ? b : c);
+}
+
+// One CTA per (64 tokens, head).  The raw inputs of positions t0-3 .. t0+63
+// and the head's convolution weights are staged in shared memory with 16-byte
+// loads (all in flight at once); then warp w computes tokens t0+8w .. +7, each
+// lane d/32 consecutive channels.
+template <typename T, int D>
+__global__ void __launch_bounds__(kPreWarps * 32)
+gdn_preprocess_kernel(const T *__restrict__ xq, const T *__restrict__ xk, const T *__restrict__ xv,
+                      const float *__restrict__ conv_w, const float *__restrict__ a_logit,
+                      const float *__restrict__ b_logit, const T *__restrict__ cs_in,
+                      T *__restrict__ q, T *__restrict__ k, T *__restrict__ v, float *__restrict__ g,
+                      float *__restrict__ beta, SeqBounds sb, int N, int64_t T_total, int H, int act,
+                      float eps) {
+    constexpr int CPL = D / 32;
+    constexpr int VEC = 16 / (int)sizeof(T), PIECES = D / VEC;
+    extern __shared__ __align__(16) uint8_t smraw[];
+    T *xs = reinterpret_cast<T *>(smraw);                                   // [3][kPreWin][D]
+    float *ws = reinterpret_cast<float *>(smraw + (size_t)3 * kPreWin * D * sizeof(T));   // [3][D][4]
+    const int h = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t0 = (int64_t)blockIdx.x * kPreTokens;
+    const size_t row = (size_t)H * D;   // elements per token of one tensor
+
+    for (int i = threadIdx.x; i < 3 * kPreWin * PIECES; i += blockDim.x) {
+        const int X = i / (kPreWin * PIECES), rem = i % (kPreWin * PIECES), r = rem / PIECES, pc = rem % PIECES;
+        const int64_t p = t0 - 3 + r;
+        if (p >= 0 && p < T_total)
+            *reinterpret_cast<uint4 *>(xs + ((size_t)X * kPreWin + r) * D + pc * VEC) =
+                *reinterpret_cast<const uint4 *>(pick3(X, xq, xk, xv) + (size_t)p * row + (size_t)h * D + pc * VEC);
+    }
+    for (int i = threadIdx.x; i < 3 * D; i += blockDim.x) {
+        const int X = i / D, c = i % D;
+        *reinterpret_cast<float4 *>(ws + 4 * i) =
+            *reinterpret_cast<const float4 *>(conv_w + (((size_t)X * H + h) * D + c) * 4);
+    }
+    __syncthreads();
+
+    const int64_t tb = t0 + warp * kPreTokensPerWarp;
+    if (tb >= T_total) return;
+    const int nt = (int)(tb + kPreTokensPerWarp < T_total ? kPreTokensPerWarp : T_total - tb);
+    const int c0 = lane * CPL;
+    float w[3][CPL][4];   // this lane's taps, held for all of its tokens
+#pragma unroll
+    for (int X = 0; X < 3; ++X)
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) {
+            const float4 t4 = *reinterpret_cast<const float4 *>(ws + (X * D + c0 + j) * 4);
+            w[X][j][0] = t4.x; w[X][j][1] = t4.y; w[X][j][2] = t4.z; w[X][j][3] = t4.w;
+        }
+    int n = seq_of(sb, N, tb);
+    int64_t bos, eos;
+    sb.get(n, bos, eos);
+    for (int it = 0; it < nt; ++it) {
+        const int64_t t = tb + it;
+        while (t >= eos) {   // the next non-empty sequence starts at t
+            ++n;
+            sb.get(n, bos, eos);
+        }
+        const int lr = (int)(t - t0);                                   // staged row of t is lr + 3
+        const int inseq = (int)(t - bos < 3 ? t - bos : 3);             // taps 3 - inseq .. 3 are in the sequence
+        float y[3][CPL];
+#pragma unroll
+        for (int X = 0; X < 3; ++X) {
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) y[X][j] = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float xv4[CPL];
+                if (inseq == 3 || i + inseq >= 3) {                     // warp-uniform
+                    load_ch<T, CPL>(xs + (X * kPreWin + lr + i) * D + c0, xv4);
+                } else if (cs_in) {
+                    load_ch<T, CPL>(cs_in + (((size_t)n * 3 + (i + inseq)) * 3 + X) * row + (size_t)h * D + c0, xv4);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < CPL; ++j) xv4[j] = 0.f;
+                }
+#pragma unroll
+                for (int j = 0; j < CPL; ++j) y[X][j] = fmaf(w[X][j][i], xv4[j], y[X][j]);
+            }
+            if (act) {
+#pragma unroll
+                for (int j = 0; j < CPL; ++j) y[X][j] = silu_f(y[X][j]);
+            }
+        }
+        float ss[2] = {0.f, 0.f};
+#pragma unroll
+        for (int X = 0; X < 2; ++X)
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) ss[X] = fmaf(y[X][j], y[X][j], ss[X]);
+#pragma unroll
+        for (int X = 0; X < 2; ++X) {
+            const float r = rsqrtf(warp_sum(ss[X]) + eps);
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) y[X][j] *= r;
+        }
+        const size_t o = (size_t)t * row + (size_t)h * D + c0;
+        store_ch<T, CPL>(q + o, y[0]);
+        store_ch<T, CPL>(k + o, y[1]);
+        store_ch<T, CPL>(v + o, y[2]);
+    }
+    if (lane < nt) {   // gates: one token per lane
+        const size_t i = (size_t)(tb + lane) * H + h;
+        g[i] = log_sigmoid_f(a_logit[i]);
+        beta[i] = sigmoid_f(b_logit[i]);
+    }
+}
+
+// state_out[n][s] = raw inputs at position eos - 3 + s (from the carried state
+// when that position precedes the sequence).  Each thread owns one
+// (tensor, head, channel) and reads all three values before writing any.
+template <typename T>
+__global__ void __launch_bounds__(256)
+gdn_conv_state_kernel(const T *__restrict__ xq, const T *__restrict__ xk, const T *__restrict__ xv,
+                      const T *cs_in, T *cs_out, SeqBounds sb, int H, int D) {
+    const int n = blockIdx.x;
+    int64_t bos, eos;
+    sb.get(n, bos, eos);
+    const int hd = H * D;
+    for (int i = blockIdx.y * blockDim.x + threadIdx.x; i < 3 * hd; i += gridDim.y * blockDim.x) {
+        const int X = i / hd, c = i % hd;
+        const T *x = pick3(X, xq, xk, xv);
+        T val[3];
+#pragma unroll
+        for (int s = 0; s < 3; ++s) {
+            const int64_t p = eos - 3 + s;
+            if (p >= bos) val[s] = x[(size_t)p * hd + c];
+            else if (cs_in) val[s] = cs_in[(((size_t)n * 3 + (p - bos + 3)) * 3 + X) * hd + c];
+            else val[s] = from_f32<T>(0.f);
+        }
+#pragma unroll
+        for (int s = 0; s < 3; ++s) cs_out[(((size_t)n * 3 + s) * 3 + X) * hd + c] = val[s];
+    }
+}
+
+constexpr int kGateWarps = 8;
+constexpr int kGateRowsPerWarp = 4;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kGateWarps * 32)
+gdn_output_gate_kernel(const T *__restrict__ o, const T *__restrict__ z, const float *__restrict__ norm_w,
+                       T *__restrict__ y, int64_t rows, int gate, float eps) {
+    constexpr int CPL = D / 32;
+    const int64_t r0 = ((int64_t)blockIdx.x * kGateWarps + (threadIdx.x >> 5)) * kGateRowsPerWarp;
+    if (r0 >= rows) return;
+    const int lane = threadIdx.x & 31, c0 = lane * CPL;
+    float wn[CPL];
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) wn[j] = norm_w ? norm_w[c0 + j] : 1.f;
+    // all rows' loads first, so that they are in flight together
+    float ov[kGateRowsPerWarp][CPL], zv[kGateRowsPerWarp][CPL];
+#pragma unroll
+    for (int rr = 0; rr < kGateRowsPerWarp; ++rr) {
+        const int64_t r = r0 + rr;
+        if (r < rows) {
+            load_ch<T, CPL>(o + (size_t)r * D + c0, ov[rr]);
+            load_ch<T, CPL>(z + (size_t)r * D + c0, zv[rr]);
+        }
+    }
+#pragma unroll
+    for (int rr = 0; rr < kGateRowsPerWarp; ++rr) {
+        const int64_t r = r0 + rr;
+        if (r >= rows) break;   // warp-uniform
+        float sc = 1.f;
+        if (norm_w) {
+            float ss = 0.f;
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) ss = fmaf(ov[rr][j], ov[rr][j], ss);
+            sc = rsqrtf(warp_sum(ss) * (1.f / D) + eps);
+        }
+        float res[CPL];
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) {
+            const float s = sigmoid_f(zv[rr][j]);
+            res[j] = ov[rr][j] * sc * wn[j] * (gate ? zv[rr][j] * s : s);
+        }
+        store_ch<T, CPL>(y + (size_t)r * D + c0, res);
+    }
+}
+
+template <typename T, int D>
+cudaError_t launch_preprocess_t(const PreprocessArgs &A, cudaStream_t stream) {
+    static bool attr_done[64] = {false};   // per device: the dynamic shared memory limit
+    int dev = 0;
+    cudaError_t ea = cudaGetDevice(&dev);
+    if (ea != cudaSuccess) return ea;
+    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
+        ea = cudaFuncSetAttribute(gdn_preprocess_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)preprocess_smem<T, D>());
+        if (ea != cudaSuccess) return ea;
+        if (dev >= 0 && dev < 64) attr_done[dev] = true;
+    }
+    const SeqBounds sb{A.cu_seqlens, A.cu_seqlens ? 0 : A.total_tokens / A.num_seqs};
+    cudaError_t e = cudaSuccess;
+    if (A.total_tokens > 0) {
+    const dim3 grid((unsigned)((A.total_tokens + kPreTokens - 1) / kPreTokens), (unsigned)A.H);
+    gdn_preprocess_kernel<T, D><<<grid, kPreWarps * 32, preprocess_smem<T, D>(), stream>>>(
+        static_cast<const T *>(A.xq), static_cast<const T *>(A.xk), static_cast<const T *>(A.xv), A.conv_w,
+        A.a_logit, A.b_logit, static_cast<const T *>(A.cs_in), static_cast<T *>(A.q), static_cast<T *>(A.k),
+        static_cast<T *>(A.v), A.g, A.beta, sb, A.num_seqs, A.total_tokens, A.H, A.activation, A.eps);
+    e = cudaGetLastError();
+    }
+    if (e != cudaSuccess || !A.cs_out) return e;
+    const int work = 3 * A.H * D;
+    const dim3 sgrid((unsigned)A.num_seqs, (unsigned)((work + 255) / 256));
+    gdn_conv_state_kernel<T><<<sgrid, 256, 0, stream>>>(
+        static_cast<const T *>(A.xq), static_cast<const T *>(A.xk), static_cast<const T *>(A.xv),
+        static_cast<const T *>(A.cs_in), static_cast<T *>(A.cs_out), sb, A.H, D);
+    return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_gate_t(const void *o, const void *z, const float *norm_w, void *y, int64_t rows, int gate,
+                          float eps, cudaStream_t stream) {
+    const int64_t per_cta = (int64_t)kGateWarps * kGateRowsPerWarp;
+    const unsigned grid = (unsigned)((rows + per_cta - 1) / per_cta);
+    gdn_output_gate_kernel<T, D><<<grid, kGateWarps * 32, 0, stream>>>(
+        static_cast<const T *>(o), static_cast<const T *>(z), norm_w, static_cast<T *>(y), rows, gate, eps);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_preprocess(const PreprocessArgs &A, cudaStream_t stream) {
+    if (A.dtype == 1) return A.d == 128 ? launch_preprocess_t<__nv_bfloat16, 128>(A, stream)
+                                        : launch_preprocess_t<__nv_bfloat16, 64>(A, stream);
+    return A.d == 128 ? launch_preprocess_t<float, 128>(A, stream) : launch_preprocess_t<float, 64>(A, stream);
+}
+
+cudaError_t launch_output_gate(int dtype, int dv, const void *o, const void *z, const float *norm_w, void *y,
+                               int64_t rows, int gate, float eps, cudaStream_t stream) {
+    if (dtype == 1) return dv == 128 ? launch_gate_t<__nv_bfloat16, 128>(o, z, norm_w, y, rows, gate, eps, stream)
+                                     : launch_gate_t<__nv_bfloat16, 64>(o, z, norm_w, y, rows, gate, eps, stream);
+    return dv == 128 ? launch_gate_t<float, 128>(o, z, norm_w, y, rows, gate, eps, stream)
+                     : launch_gate_t<float, 64>(o, z, norm_w, y, rows, gate, eps, stream);
+}
+
+}  // namespace gdn

@@ -21,6 +21,8 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "gdn.h")
 
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_WORKSPACE = 0, 1, 2, 3, 5
 GDN_F32, GDN_BF16 = 0, 1
+ACT_NONE, ACT_SILU = 0, 1
+GATE_SIGMOID, GATE_SILU = 0, 1
 CHUNK = 64
 
 _lib = None
@@ -57,6 +59,12 @@ def _load():
     lib.gdn_prefill_noalloc.restype = i32
     lib.gdn_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i32, i32, i32, i32, i32, vp]
     lib.gdn_decode_step.restype = i32
+    f32 = ctypes.c_float
+    lib.gdn_preprocess.argtypes = [vp, vp, vp, fp, fp, fp, vp, vp, vp, vp, fp, fp, vp, vp, i32, i64,
+                                   i32, i32, i32, f32, i32, vp]
+    lib.gdn_preprocess.restype = i32
+    lib.gdn_output_gate.argtypes = [vp, vp, fp, vp, i64, i32, i32, f32, i32, vp]
+    lib.gdn_output_gate.restype = i32
     lib.gdn_status_string.argtypes = [i32]
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_last_cuda_error.argtypes = []
@@ -227,3 +235,73 @@ def gdn_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.
     if st != GDN_OK:
         raise GdnError(st, "gdn_decode_step")
     return out, state_out
+
+
+def gdn_preprocess(xq: torch.Tensor, xk: torch.Tensor, xv: torch.Tensor, conv_w: torch.Tensor,
+                   a: torch.Tensor, b: torch.Tensor, conv_state_in: Optional[torch.Tensor] = None,
+                   cu_seqlens: Optional[torch.Tensor] = None, *, num_seqs: Optional[int] = None,
+                   activation: int = ACT_NONE, eps: float = 1e-6, conv_state_out: Optional[torch.Tensor] = None,
+                   want_state: bool = True):
+    """Raw projections -> gdn_prefill's inputs (include/gdn.h, gdn_preprocess).
+    xq, xk, xv [T, H, d]; conv_w [3, H, d, 4] fp32; a, b [T, H] fp32 logits;
+    conv_state_in [N, 3, 3, H, d] (dtype of x) or None.  Returns
+    (q, k, v, g, beta, conv_state_out); pass conv_state_out=conv_state_in to
+    update the convolution state in place."""
+    T, H, d = xq.shape
+    dev = xq.device
+    if dev.type != "cuda":
+        raise ValueError("gdn_preprocess needs CUDA tensors")
+    if xk.shape != (T, H, d) or xv.shape != (T, H, d):
+        raise ValueError("xq/xk/xv shapes disagree")
+    if xk.dtype != xq.dtype or xv.dtype != xq.dtype:
+        raise ValueError("xq, xk, xv must share a dtype")
+    if conv_w.shape != (3, H, d, 4) or conv_w.dtype != torch.float32:
+        raise ValueError("conv_w must be fp32 [3, H, d, 4]")
+    if a.shape != (T, H) or b.shape != (T, H) or a.dtype != torch.float32 or b.dtype != torch.float32:
+        raise ValueError("a and b must be fp32 [T, H]")
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32 or cu_seqlens.device != dev:
+            raise ValueError("cu_seqlens must be int32 on the same device")
+        N = cu_seqlens.numel() - 1
+    else:
+        N = 1 if num_seqs is None else int(num_seqs)
+    if conv_state_in is not None and (conv_state_in.shape != (N, 3, 3, H, d) or conv_state_in.dtype != xq.dtype):
+        raise ValueError("conv_state_in must be [N, 3, 3, H, d] in the dtype of x")
+    for t in (xk, xv, conv_w, a, b, conv_state_in, conv_state_out, cu_seqlens):
+        if t is not None and t.device != dev:
+            raise ValueError("all tensors must be on %s" % dev)
+    q, k, v = (torch.empty_like(xq) for _ in range(3))
+    g = torch.empty((T, H), dtype=torch.float32, device=dev)
+    beta = torch.empty_like(g)
+    if conv_state_out is None and want_state:
+        conv_state_out = torch.empty((N, 3, 3, H, d), dtype=xq.dtype, device=dev)
+    st = _load().gdn_preprocess(_ptr(xq), _ptr(xk), _ptr(xv), _ptr(conv_w), _ptr(a), _ptr(b),
+                                _ptr(conv_state_in), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                _ptr(conv_state_out), _ptr(cu_seqlens), N, T, H, d, int(activation),
+                                float(eps), _dtype_code(xq.dtype), _stream(dev))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_preprocess")
+    return q, k, v, g, beta, conv_state_out
+
+
+def gdn_output_gate(o: torch.Tensor, z: torch.Tensor, norm_w: Optional[torch.Tensor] = None, *,
+                    gate: int = GATE_SIGMOID, eps: float = 1e-6, out: Optional[torch.Tensor] = None):
+    """y = n(o) * act(z) over the last dimension (include/gdn.h,
+    gdn_output_gate).  o, z [..., dv] of one dtype; norm_w [dv] fp32 or None.
+    ``out`` may be ``o`` (in place)."""
+    dev = o.device
+    if dev.type != "cuda":
+        raise ValueError("gdn_output_gate needs CUDA tensors")
+    if z.shape != o.shape or z.dtype != o.dtype or z.device != dev:
+        raise ValueError("o and z must share shape, dtype and device")
+    dv = o.shape[-1]
+    if norm_w is not None and (norm_w.shape != (dv,) or norm_w.dtype != torch.float32 or norm_w.device != dev):
+        raise ValueError("norm_w must be fp32 [dv] on the same device")
+    if out is None:
+        out = torch.empty_like(o)
+    rows = o.numel() // dv if dv else 0
+    st = _load().gdn_output_gate(_ptr(o), _ptr(z), _ptr(norm_w), _ptr(out), rows, dv, int(gate), float(eps),
+                                 _dtype_code(o.dtype), _stream(dev))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_output_gate")
+    return out

@@ -90,3 +90,39 @@ def test_binding_refuses_cpu_tensors():
         gdn.gdn_prefill(x, x, x, s, s)
     with pytest.raises(ValueError):
         gdn.gdn_decode_step(x[:1], x[:1], x[:1], s[:1], s[:1], torch.zeros(1, 2, 64, 64))
+
+
+def _pre_raw(lib, **kw):
+    base = 1 << 20
+    args = dict(xq=base, xk=2 * base, xv=3 * base, w=4 * base, a=5 * base, b=6 * base, csi=None,
+                q=7 * base, k=8 * base, v=9 * base, g=10 * base, beta=11 * base, cso=None, cu=None,
+                N=1, T=64, H=2, d=64, act=0, eps=1e-6, dtype=1, stream=None)
+    args.update(kw)
+    return lib.gdn_preprocess(args["xq"], args["xk"], args["xv"], args["w"], args["a"], args["b"],
+                              args["csi"], args["q"], args["k"], args["v"], args["g"], args["beta"],
+                              args["cso"], args["cu"], args["N"], args["T"], args["H"], args["d"],
+                              args["act"], ctypes.c_float(args["eps"]), args["dtype"], args["stream"])
+
+
+def test_preprocess_rejects_bad_arguments(lib):
+    inv, uns = binding.GDN_ERR_INVALID_ARG, binding.GDN_ERR_UNSUPPORTED
+    assert _pre_raw(lib, xq=None) == inv
+    assert _pre_raw(lib, g=(11 << 20) + 4) == inv                 # misaligned
+    assert _pre_raw(lib, d=96) == uns
+    assert _pre_raw(lib, act=2) == inv
+    assert _pre_raw(lib, eps=-1.0) == inv
+    assert _pre_raw(lib, N=3, T=64) == inv                        # uniform split must be exact
+    assert _pre_raw(lib, q=1 << 20) == inv                        # output over an input
+    assert _pre_raw(lib, cso=(5 << 20) + 64) == inv               # state over an input
+    assert _pre_raw(lib, T=0) == binding.GDN_OK                   # nothing to do, nothing enqueued
+
+
+def test_output_gate_rejects_bad_arguments(lib):
+    inv = binding.GDN_ERR_INVALID_ARG
+    f = lambda o=1 << 20, z=2 << 20, w=None, y=3 << 20, rows=10, dv=64, gate=0, eps=1e-6, dt=1: \
+        lib.gdn_output_gate(o, z, w, y, rows, dv, gate, ctypes.c_float(eps), dt, None)
+    assert f(o=None) == inv
+    assert f(gate=5) == inv
+    assert f(dv=32) == binding.GDN_ERR_UNSUPPORTED
+    assert f(y=(2 << 20) + 16) == inv                            # y over z
+    assert f(rows=0) == binding.GDN_OK

@@ -220,3 +220,28 @@ def random_prefill(T_list: Sequence[int], H: int, dk: int, dv: int,
     return dict(q=_round(q, dtype), k=_round(k, dtype), v=_round(v, dtype),
                 g=torch.from_numpy(g), beta=torch.from_numpy(beta), state_in=state,
                 cu_seqlens=torch.from_numpy(cu.astype(np.int32)))
+
+
+def layer_inputs(T: int, H: int, d: int, dtype: torch.dtype = torch.bfloat16, seed: int = 0,
+                 num_seqs: int = 1, state: bool = False) -> Dict[str, torch.Tensor]:
+    """Raw inputs of the layer steps around the recurrence (pre-processing
+    and output gate), on the CPU: projections x_q, x_k, x_v ~ N(0, 1) and gate
+    input z ~ N(0, 4) in the storage dtype; convolution taps ~ N(0, 0.5^2),
+    gate logits a ~ N(3, 1) (alpha = sigmoid(a), mean g near -0.05, like the
+    tiny workload) and b ~ N(0, 1) (beta = sigmoid(b), like the prefill
+    workload) in fp32; the RMS-norm weight ~ U[0.5, 1.5]; optionally a
+    convolution state ~ N(0, 1) per sequence."""
+    rng = _rng(seed, 7)
+    out = {
+        "xq": _round(rng.standard_normal((T, H, d), dtype=np.float32), dtype),
+        "xk": _round(rng.standard_normal((T, H, d), dtype=np.float32), dtype),
+        "xv": _round(rng.standard_normal((T, H, d), dtype=np.float32), dtype),
+        "z": _round(2.0 * rng.standard_normal((T, H, d), dtype=np.float32), dtype),
+        "conv_w": torch.from_numpy((0.5 * rng.standard_normal((3, H, d, 4))).astype(np.float32)),
+        "a": torch.from_numpy((3.0 + rng.standard_normal((T, H))).astype(np.float32)),
+        "b": torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)),
+        "norm_w": torch.from_numpy(rng.uniform(0.5, 1.5, d).astype(np.float32)),
+    }
+    if state:
+        out["conv_state"] = _round(rng.standard_normal((num_seqs, 3, 3, H, d), dtype=np.float32), dtype)
+    return out
