@@ -225,6 +225,17 @@ def run_native(args):
     def gate_once():
         gdn.gdn_output_gate(out, lx["z"], lx["norm_w"], gate=gdn.GATE_SIGMOID, out=gate_out)
 
+    # ---- streaming session: one GDN layer step per video frame (~274 tokens per
+    # frame in the pages' streaming measurement), state carried, graph replay
+    FRAME = 274
+    P = W.layer_inputs(FRAME, H, dk, w.dtype, seed=rank)
+    sess = gdn.GdnSession(1, H, dk, FRAME, P["conv_w"].to(dev), P["norm_w"].to(dev), dtype=w.dtype,
+                          activation=gdn.ACT_SILU)
+    for name in ("xq", "xk", "xv", "a", "b", "z"):
+        getattr(sess, name)[:FRAME].copy_(P[name].to(dev))
+    frame_launches = 2 + gdn.gdn_prefill_kernel_count(1, FRAME, H, dk, dv, w.chunk, w.dtype) + 1
+    decode_launches = 2 + 1 + 1
+
     # ---- e2e buffers (pinned host, fresh device copies each step)
     pin = {k: v.pin_memory() for k, v in host.items() if isinstance(v, torch.Tensor) and k != "cu_seqlens"}
     out_h = torch.empty((T, H, dv), dtype=w.dtype).pin_memory()
@@ -248,6 +259,9 @@ def run_native(args):
         e2e_once()
         preprocess_once()
         gate_once()
+        sess.prefill(FRAME)
+        sess.prefill(FRAME, eager=True)
+        sess.decode()
     torch.cuda.synchronize()
 
     def timed(fn, steps, do_flush=True):
@@ -274,12 +288,18 @@ def run_native(args):
         ms_e2e = timed(lambda i: e2e_once(), max(3, K // 10), do_flush=False)
         ms_pre = timed(lambda i: preprocess_once(), K)
         ms_gate = timed(lambda i: gate_once(), K)
+        ms_frame_graph = timed(lambda i: sess.prefill(FRAME), K)
+        ms_frame_eager = timed(lambda i: sess.prefill(FRAME, eager=True), K)
+        ms_dec_graph = timed(lambda i: sess.decode(), K)
         wall = time.time() - t_wall0
     ms_prefill = max_over_ranks(ms_prefill, world)
     ms_decode = max_over_ranks(ms_decode, world)
     ms_e2e = max_over_ranks(ms_e2e, world)
     ms_pre = max_over_ranks(ms_pre, world)
     ms_gate = max_over_ranks(ms_gate, world)
+    ms_frame_graph = max_over_ranks(ms_frame_graph, world)
+    ms_frame_eager = max_over_ranks(ms_frame_eager, world)
+    ms_dec_graph = max_over_ranks(ms_dec_graph, world)
     el = 2 if w.dtype == torch.bfloat16 else 4
     pre_bytes = 6 * T * H * dk * el + 4 * T * H * 4 + 3 * H * dk * 16    # x in, q/k/v out, a/b in, g/beta out, taps
     gate_bytes = 3 * T * H * dv * el + dv * 4                             # o, z in, y out, norm weight
@@ -336,9 +356,17 @@ def run_native(args):
                                      "achieved": gate_bytes / (ms_gate * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
                                      "frac": gate_bytes / (ms_gate * 1e-3) / 1e9 / hbm, "traffic": None,
                                      "algorithmic_bytes": gate_bytes}},
+        "streaming": {"metric": "GDN layer frames/s: pre-processing + recurrence with carried state + "
+                                "output gate per %d-token frame x %d heads, CUDA-graph replay" % (FRAME, H),
+                      "value": 1e3 / ms_frame_graph * world, "unit": "frames/s",
+                      "ms_per_frame_graph": ms_frame_graph, "ms_per_frame_eager": ms_frame_eager,
+                      "kernels_per_frame": frame_launches,
+                      "decode_step_ms_graph": ms_dec_graph, "kernels_per_decode_step": decode_launches,
+                      "l2": "flushed before every frame"},
         "e2e": {"value": aggregate_throughput(T, world, ms_e2e), "unit": "tokens/s",
                 "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": K * launches_per_prefill + K + max(3, K // 10) * launches_per_prefill + 2 * K,
+        "gpu_launches": (K * launches_per_prefill + K + max(3, K // 10) * launches_per_prefill + 2 * K
+                         + 2 * K * frame_launches + K * decode_launches),
         "clocks": clk.summary(),
         "timed_wall_s": wall,
     }

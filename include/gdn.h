@@ -234,6 +234,71 @@ int gdn_preprocess(const void *xq, const void *xk, const void *xv, const float *
 int gdn_output_gate(const void *o, const void *z, const float *norm_w, void *y, int64_t rows, int dv,
                     int gate, float eps, int dtype, void *stream);
 
+/* ------------------------------------------------------------------ streaming session
+ *
+ * One Gated DeltaNet layer step over a constant-size memory, captured as a
+ * CUDA graph and replayed (InfiniteVL project page, "Advanced Usage: CUDA
+ * Graph Acceleration" and "Accelerated Streaming Inference": the fixed-size
+ * state lets the whole streaming-prefill computation, and the decode step,
+ * be captured once and replayed without launch overhead; a video is fed
+ * segment by segment while the state is carried).
+ *
+ * A step, for each of num_streams independent streams:
+ *   gdn_preprocess (convolution state carried in place) ->
+ *   gdn_prefill (tokens > 0; recurrent state carried in place) or
+ *   gdn_decode_step (one token) -> gdn_output_gate.
+ *
+ * The caller owns every buffer and keeps it in place for the session's
+ * lifetime (the graphs hold the addresses).  Sizes, with R = num_streams *
+ * seg_tokens rows:
+ *   xq, xk, xv, z, y, q, k, v, o   [R, H, d] dtype
+ *   a, b, g, beta                  [R, H] fp32
+ *   state                          [num_streams, H, d, d] fp32
+ *   conv_state                     [num_streams, 3, 3, H, d] dtype
+ *   conv_w [3, H, d, 4] fp32;  norm_w [d] fp32 or NULL (no RMS norm)
+ *   workspace                      gdn_session_workspace_size() bytes
+ * Per step the caller writes xq, xk, xv, a, b, z for `tokens` tokens of every
+ * stream, stream-major ([num_streams][tokens] at the start of each buffer),
+ * and reads y in the same layout; q, k, v, o, g, beta are scratch.  The
+ * decode step uses one row per stream.
+ *
+ * gdn_session_create allocates no device memory: it checks the buffers, runs
+ * the kernels' one-time per-device set-up and creates a capture stream.  The
+ * first step for a token count captures its graph (up to 8 counts are kept;
+ * capturing synchronises nothing); later steps only launch it on `stream`.
+ * Calls on one session are serialised by a host lock.  Steps share the
+ * buffers, so the caller orders them on the device (one stream, or events).
+ */
+typedef struct gdn_session gdn_session;
+
+typedef struct gdn_session_buffers_t {
+    void *xq, *xk, *xv;       /* raw projections of the next step (caller writes) */
+    float *a, *b;             /* gate logits of the next step (caller writes) */
+    void *z;                  /* output-gate input of the next step (caller writes) */
+    void *y;                  /* gated output of the last step (caller reads) */
+    void *q, *k, *v, *o;      /* scratch */
+    float *g, *beta;          /* scratch */
+    float *state;             /* recurrent state, carried */
+    void *conv_state;         /* convolution state, carried */
+    const float *conv_w;      /* convolution taps */
+    const float *norm_w;      /* RMS-norm weights, or NULL */
+    void *workspace;          /* prefill workspace */
+    size_t workspace_bytes;
+} gdn_session_buffers_t;
+
+size_t gdn_session_workspace_size(int num_streams, int H, int d, int seg_tokens, int dtype);
+int gdn_session_create(int num_streams, int H, int d, int seg_tokens, int dtype, int activation, int gate,
+                       float eps, const gdn_session_buffers_t *buffers, gdn_session **out);
+/* a step of `tokens` in [1, seg_tokens] per stream, as a graph replay */
+int gdn_session_prefill(gdn_session *s, int tokens, void *stream);
+/* one token per stream, as a graph replay */
+int gdn_session_decode(gdn_session *s, void *stream);
+/* the same step launched kernel by kernel, without a graph (tokens = 0: decode) */
+int gdn_session_step_eager(gdn_session *s, int tokens, void *stream);
+/* number of instantiated graphs */
+int gdn_session_graph_count(const gdn_session *s);
+void gdn_session_destroy(gdn_session *s);
+
 #ifdef __cplusplus
 }
 #endif

@@ -67,4 +67,9 @@ cudaError_t launch_preprocess(const PreprocessArgs &A, cudaStream_t stream);
 cudaError_t launch_output_gate(int dtype, int dv, const void *o, const void *z, const float *norm_w, void *y,
                                int64_t rows, int gate, float eps, cudaStream_t stream);
 
+// One-time per-device kernel attribute set-up (shared-memory limits), so that
+// later launches can be captured into CUDA graphs without it.
+cudaError_t prefill_tc_setup();
+cudaError_t layer_ops_setup(int dtype, int d);
+
 }  // namespace gdn

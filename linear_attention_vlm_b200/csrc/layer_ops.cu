@@ -71,10 +71,11 @@ __device__ __forceinline__ float warp_sum(float s) {
     return s;
 }
 
-// sigmoid and SiLU with the fast exponential and a correctly rounded
-// reciprocal (relative error ~1e-6, far below the bf16 storage step)
-__device__ __forceinline__ float sigmoid_f(float x) { return __frcp_rn(1.f + __expf(-x)); }
-__device__ __forceinline__ float silu_f(float x) { return x * __frcp_rn(1.f + __expf(-x)); }
+// sigmoid and SiLU with the fast exponential and division intrinsics
+// (relative error ~1e-6, far below the bf16 storage step; a huge exp(-x)
+// gives 0, the correct limit)
+__device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
+__device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.f + __expf(-x)); }
 
 // log(sigmoid(x)) = min(x, 0) - log1p(exp(-|x|)), without overflow
 __device__ __forceinline__ float log_sigmoid_f(float x) { return fminf(x, 0.f) - log1pf(expf(-fabsf(x))); }
@@ -99,6 +100,12 @@ constexpr int kPreWin = kPreTokens + 3;                      // staged positions
 template <typename T, int D>
 constexpr size_t preprocess_smem() {
     return (size_t)3 * kPreWin * D * sizeof(T) + (size_t)3 * D * 4 * sizeof(float);
+}
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(reinterpret_cast<uint64_t>(src))
+                 : "memory");
 }
 
 template <typename T>
@@ -127,18 +134,19 @@ gdn_preprocess_kernel(const T *__restrict__ xq, const T *__restrict__ xk, const 
     const int64_t t0 = (int64_t)blockIdx.x * kPreTokens;
     const size_t row = (size_t)H * D;   // elements per token of one tensor
 
+    // asynchronous 16-byte copies: every piece of the tile is in flight at once
     for (int i = threadIdx.x; i < 3 * kPreWin * PIECES; i += blockDim.x) {
         const int X = i / (kPreWin * PIECES), rem = i % (kPreWin * PIECES), r = rem / PIECES, pc = rem % PIECES;
         const int64_t p = t0 - 3 + r;
-        if (p >= 0 && p < T_total)
-            *reinterpret_cast<uint4 *>(xs + ((size_t)X * kPreWin + r) * D + pc * VEC) =
-                *reinterpret_cast<const uint4 *>(pick3(X, xq, xk, xv) + (size_t)p * row + (size_t)h * D + pc * VEC);
+        if (p >= 0 && p < T_total)   // other rows are never read
+            cp_async16(xs + ((size_t)X * kPreWin + r) * D + pc * VEC,
+                       pick3(X, xq, xk, xv) + (size_t)p * row + (size_t)h * D + pc * VEC);
     }
     for (int i = threadIdx.x; i < 3 * D; i += blockDim.x) {
         const int X = i / D, c = i % D;
-        *reinterpret_cast<float4 *>(ws + 4 * i) =
-            *reinterpret_cast<const float4 *>(conv_w + (((size_t)X * H + h) * D + c) * 4);
+        cp_async16(ws + 4 * i, conv_w + (((size_t)X * H + h) * D + c) * 4);
     }
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
     __syncthreads();
 
     const int64_t tb = t0 + warp * kPreTokensPerWarp;
@@ -156,6 +164,52 @@ gdn_preprocess_kernel(const T *__restrict__ xq, const T *__restrict__ xk, const 
     int n = seq_of(sb, N, tb);
     int64_t bos, eos;
     sb.get(n, bos, eos);
+    if (nt == kPreTokensPerWarp && tb - 3 >= bos && tb + kPreTokensPerWarp <= eos) {
+        // Fast path: all 8 tokens and their 3 predecessors lie in one sequence.
+        // One tensor at a time, the lane holds the 11 staged rows of its
+        // channels and forms the 8 outputs from them (each row read once).
+        const int lr0 = (int)(tb - t0);   // staged row of position tb - 3
+#pragma unroll
+        for (int X = 0; X < 3; ++X) {
+            float xr[kPreTokensPerWarp + 3][CPL];
+#pragma unroll
+            for (int r = 0; r < kPreTokensPerWarp + 3; ++r)
+                load_ch<T, CPL>(xs + (X * kPreWin + lr0 + r) * D + c0, xr[r]);
+            float yv[kPreTokensPerWarp][CPL];
+#pragma unroll
+            for (int u = 0; u < kPreTokensPerWarp; ++u)
+#pragma unroll
+                for (int j = 0; j < CPL; ++j) {
+                    float a = w[X][j][0] * xr[u][j];
+                    a = fmaf(w[X][j][1], xr[u + 1][j], a);
+                    a = fmaf(w[X][j][2], xr[u + 2][j], a);
+                    a = fmaf(w[X][j][3], xr[u + 3][j], a);
+                    yv[u][j] = act ? silu_f(a) : a;
+                }
+            if (X < 2) {   // L2 norm per token: 8 independent warp reductions
+                float ss[kPreTokensPerWarp];
+#pragma unroll
+                for (int u = 0; u < kPreTokensPerWarp; ++u) {
+                    ss[u] = 0.f;
+#pragma unroll
+                    for (int j = 0; j < CPL; ++j) ss[u] = fmaf(yv[u][j], yv[u][j], ss[u]);
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                    for (int u = 0; u < kPreTokensPerWarp; ++u) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], o);
+#pragma unroll
+                for (int u = 0; u < kPreTokensPerWarp; ++u) {
+                    const float rn = rsqrtf(ss[u] + eps);
+#pragma unroll
+                    for (int j = 0; j < CPL; ++j) yv[u][j] *= rn;
+                }
+            }
+            T *dst = (X == 0 ? q : (X == 1 ? k : v)) + (size_t)tb * row + (size_t)h * D + c0;
+#pragma unroll
+            for (int u = 0; u < kPreTokensPerWarp; ++u) store_ch<T, CPL>(dst + (size_t)u * row, yv[u]);
+        }
+    } else
     for (int it = 0; it < nt; ++it) {
         const int64_t t = tb + it;
         while (t >= eos) {   // the next non-empty sequence starts at t
@@ -169,19 +223,31 @@ gdn_preprocess_kernel(const T *__restrict__ xq, const T *__restrict__ xk, const 
         for (int X = 0; X < 3; ++X) {
 #pragma unroll
             for (int j = 0; j < CPL; ++j) y[X][j] = 0.f;
+            if (inseq == 3) {   // warp-uniform: every tap from the staged tile
+                const T *src = xs + (X * kPreWin + lr) * D + c0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float xv4[CPL];
-                if (inseq == 3 || i + inseq >= 3) {                     // warp-uniform
-                    load_ch<T, CPL>(xs + (X * kPreWin + lr + i) * D + c0, xv4);
-                } else if (cs_in) {
-                    load_ch<T, CPL>(cs_in + (((size_t)n * 3 + (i + inseq)) * 3 + X) * row + (size_t)h * D + c0, xv4);
-                } else {
+                for (int i = 0; i < 4; ++i) {
+                    float xv4[CPL];
+                    load_ch<T, CPL>(src + i * D, xv4);
 #pragma unroll
-                    for (int j = 0; j < CPL; ++j) xv4[j] = 0.f;
+                    for (int j = 0; j < CPL; ++j) y[X][j] = fmaf(w[X][j][i], xv4[j], y[X][j]);
                 }
+            } else {            // the first three tokens of a sequence
 #pragma unroll
-                for (int j = 0; j < CPL; ++j) y[X][j] = fmaf(w[X][j][i], xv4[j], y[X][j]);
+                for (int i = 0; i < 4; ++i) {
+                    float xv4[CPL];
+                    if (i + inseq >= 3) {
+                        load_ch<T, CPL>(xs + (X * kPreWin + lr + i) * D + c0, xv4);
+                    } else if (cs_in) {
+                        load_ch<T, CPL>(cs_in + (((size_t)n * 3 + (i + inseq)) * 3 + X) * row + (size_t)h * D + c0,
+                                        xv4);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < CPL; ++j) xv4[j] = 0.f;
+                    }
+#pragma unroll
+                    for (int j = 0; j < CPL; ++j) y[X][j] = fmaf(w[X][j][i], xv4[j], y[X][j]);
+                }
             }
             if (act) {
 #pragma unroll
@@ -283,9 +349,10 @@ gdn_output_gate_kernel(const T *__restrict__ o, const T *__restrict__ z, const f
     }
 }
 
+// One-time per device: the dynamic shared-memory limit of the kernel.
 template <typename T, int D>
-cudaError_t launch_preprocess_t(const PreprocessArgs &A, cudaStream_t stream) {
-    static bool attr_done[64] = {false};   // per device: the dynamic shared memory limit
+cudaError_t preprocess_attr() {
+    static bool attr_done[64] = {false};
     int dev = 0;
     cudaError_t ea = cudaGetDevice(&dev);
     if (ea != cudaSuccess) return ea;
@@ -295,6 +362,13 @@ cudaError_t launch_preprocess_t(const PreprocessArgs &A, cudaStream_t stream) {
         if (ea != cudaSuccess) return ea;
         if (dev >= 0 && dev < 64) attr_done[dev] = true;
     }
+    return cudaSuccess;
+}
+
+template <typename T, int D>
+cudaError_t launch_preprocess_t(const PreprocessArgs &A, cudaStream_t stream) {
+    const cudaError_t ea = preprocess_attr<T, D>();
+    if (ea != cudaSuccess) return ea;
     const SeqBounds sb{A.cu_seqlens, A.cu_seqlens ? 0 : A.total_tokens / A.num_seqs};
     cudaError_t e = cudaSuccess;
     if (A.total_tokens > 0) {
@@ -330,6 +404,11 @@ cudaError_t launch_preprocess(const PreprocessArgs &A, cudaStream_t stream) {
     if (A.dtype == 1) return A.d == 128 ? launch_preprocess_t<__nv_bfloat16, 128>(A, stream)
                                         : launch_preprocess_t<__nv_bfloat16, 64>(A, stream);
     return A.d == 128 ? launch_preprocess_t<float, 128>(A, stream) : launch_preprocess_t<float, 64>(A, stream);
+}
+
+cudaError_t layer_ops_setup(int dtype, int d) {
+    if (dtype == 1) return d == 128 ? preprocess_attr<__nv_bfloat16, 128>() : preprocess_attr<__nv_bfloat16, 64>();
+    return d == 128 ? preprocess_attr<float, 128>() : preprocess_attr<float, 64>();
 }
 
 cudaError_t launch_output_gate(int dtype, int dv, const void *o, const void *z, const float *norm_w, void *y,

@@ -1207,6 +1207,12 @@ int tc_kernel_count(int num_seqs, int64_t total_tokens, int H, bool varlen) {
     return tc_scan_segments(num_seqs, total_tokens, H, false, scan_sm_count()) > 1 ? 4 : 2;
 }
 
+cudaError_t prefill_tc_setup() {
+    if (set_smem_attrs()) return cudaSuccess;
+    const cudaError_t e = cudaGetLastError();
+    return e != cudaSuccess ? e : cudaErrorUnknown;
+}
+
 cudaError_t launch_prefill_tc(const TcLaunch &L, cudaStream_t stream) {
     const bool varlen = L.cu_seqlens != nullptr;
     uint8_t *ws = static_cast<uint8_t *>(L.workspace);

@@ -65,6 +65,20 @@ def _load():
     lib.gdn_preprocess.restype = i32
     lib.gdn_output_gate.argtypes = [vp, vp, fp, vp, i64, i32, i32, f32, i32, vp]
     lib.gdn_output_gate.restype = i32
+    lib.gdn_session_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+    lib.gdn_session_workspace_size.restype = sz
+    lib.gdn_session_create.argtypes = [i32, i32, i32, i32, i32, i32, i32, f32, vp, vp]
+    lib.gdn_session_create.restype = i32
+    lib.gdn_session_prefill.argtypes = [vp, i32, vp]
+    lib.gdn_session_prefill.restype = i32
+    lib.gdn_session_decode.argtypes = [vp, vp]
+    lib.gdn_session_decode.restype = i32
+    lib.gdn_session_step_eager.argtypes = [vp, i32, vp]
+    lib.gdn_session_step_eager.restype = i32
+    lib.gdn_session_graph_count.argtypes = [vp]
+    lib.gdn_session_graph_count.restype = i32
+    lib.gdn_session_destroy.argtypes = [vp]
+    lib.gdn_session_destroy.restype = None
     lib.gdn_status_string.argtypes = [i32]
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_last_cuda_error.argtypes = []
@@ -305,3 +319,95 @@ def gdn_output_gate(o: torch.Tensor, z: torch.Tensor, norm_w: Optional[torch.Ten
     if st != GDN_OK:
         raise GdnError(st, "gdn_output_gate")
     return out
+
+
+class _SessionBuffers(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("xq", "xk", "xv", "a", "b", "z", "y", "q", "k", "v", "o", "g",
+                                                "beta", "state", "conv_state", "conv_w", "norm_w", "workspace")] + \
+               [("workspace_bytes", ctypes.c_size_t)]
+
+
+class GdnSession:
+    """Streaming session (include/gdn.h, gdn_session_*): one layer step --
+    pre-processing, the recurrence with a carried state, the output gate --
+    over buffers allocated here once, captured as a CUDA graph per token
+    count and replayed.  Write the next step's inputs into ``xq, xk, xv, a,
+    b, z`` (``[num_streams * tokens, ...]`` at the start, stream-major), call
+    ``prefill(tokens)`` or ``decode()``, read ``y``.  ``feed`` does the copies."""
+
+    def __init__(self, num_streams: int, H: int, d: int, seg_tokens: int, conv_w: torch.Tensor,
+                 norm_w: Optional[torch.Tensor] = None, *, dtype: torch.dtype = torch.bfloat16,
+                 activation: int = ACT_NONE, gate: int = GATE_SIGMOID, eps: float = 1e-6, device=None):
+        dev = torch.device(device) if device is not None else conv_w.device
+        if dev.type != "cuda":
+            raise ValueError("GdnSession needs a CUDA device")
+        if conv_w.shape != (3, H, d, 4) or conv_w.dtype != torch.float32:
+            raise ValueError("conv_w must be fp32 [3, H, d, 4]")
+        self.B, self.H, self.d, self.seg, self.dtype = num_streams, H, d, seg_tokens, dtype
+        R = num_streams * seg_tokens
+        mk = lambda *shape, dt=dtype: torch.zeros(shape, dtype=dt, device=dev)
+        self.xq, self.xk, self.xv, self.z, self.y = (mk(R, H, d) for _ in range(5))
+        self.a, self.b = mk(R, H, dt=torch.float32), mk(R, H, dt=torch.float32)
+        self._scratch = [mk(R, H, d) for _ in range(4)] + [mk(R, H, dt=torch.float32) for _ in range(2)]
+        self.state = mk(num_streams, H, d, d, dt=torch.float32)
+        self.conv_state = mk(num_streams, 3, 3, H, d)
+        self.conv_w = conv_w.to(dev).contiguous().clone()
+        self.norm_w = None if norm_w is None else norm_w.to(dev, torch.float32).contiguous().clone()
+        lib = _load()
+        ws_bytes = int(lib.gdn_session_workspace_size(num_streams, H, d, seg_tokens, _dtype_code(dtype)))
+        self.workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+        q, k, v, o, g, beta = self._scratch
+        self._buf = _SessionBuffers(*(_ptr(t) for t in (self.xq, self.xk, self.xv, self.a, self.b, self.z, self.y,
+                                                         q, k, v, o, g, beta, self.state, self.conv_state,
+                                                         self.conv_w, self.norm_w, self.workspace)), ws_bytes)
+        self._h = ctypes.c_void_p()
+        st = lib.gdn_session_create(num_streams, H, d, seg_tokens, _dtype_code(dtype), int(activation), int(gate),
+                                    float(eps), ctypes.byref(self._buf), ctypes.byref(self._h))
+        if st != GDN_OK:
+            raise GdnError(st, "gdn_session_create")
+        self.device = dev
+
+    def prefill(self, tokens: Optional[int] = None, eager: bool = False) -> torch.Tensor:
+        tokens = self.seg if tokens is None else int(tokens)
+        lib = _load()
+        s = _stream(self.device)
+        st = lib.gdn_session_step_eager(self._h, tokens, s) if eager else lib.gdn_session_prefill(self._h, tokens, s)
+        if st != GDN_OK:
+            raise GdnError(st, "gdn_session_prefill")
+        return self.y[: self.B * tokens]
+
+    def decode(self, eager: bool = False) -> torch.Tensor:
+        lib = _load()
+        s = _stream(self.device)
+        st = lib.gdn_session_step_eager(self._h, 0, s) if eager else lib.gdn_session_decode(self._h, s)
+        if st != GDN_OK:
+            raise GdnError(st, "gdn_session_decode")
+        return self.y[: self.B]
+
+    def feed(self, xq, xk, xv, a, b, z, eager: bool = False) -> torch.Tensor:
+        """Copy one step's inputs ([num_streams * tokens, ...], stream-major;
+        tokens = 1 means a decode step) into the staging buffers and run it."""
+        n = xq.shape[0]
+        if n % self.B != 0:
+            raise ValueError("rows must be a multiple of num_streams")
+        for dst, src in ((self.xq, xq), (self.xk, xk), (self.xv, xv), (self.a, a), (self.b, b), (self.z, z)):
+            dst[:n].copy_(src, non_blocking=True)
+        return self.prefill(n // self.B, eager=eager)
+
+    def graph_count(self) -> int:
+        return int(_load().gdn_session_graph_count(self._h))
+
+    def reset(self) -> None:
+        self.state.zero_()
+        self.conv_state.zero_()
+
+    def close(self) -> None:
+        if getattr(self, "_h", None) is not None and self._h.value:
+            _load().gdn_session_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -126,3 +126,20 @@ def test_output_gate_rejects_bad_arguments(lib):
     assert f(dv=32) == binding.GDN_ERR_UNSUPPORTED
     assert f(y=(2 << 20) + 16) == inv                            # y over z
     assert f(rows=0) == binding.GDN_OK
+
+
+def test_session_create_rejects_bad_arguments(lib):
+    bufs = binding._SessionBuffers(*([1 << 20] * 18), 1 << 30)
+    h = ctypes.c_void_p()
+    f = lambda **kw: lib.gdn_session_create(kw.get("B", 1), kw.get("H", 2), kw.get("d", 64), kw.get("seg", 64),
+                                            kw.get("dtype", 1), kw.get("act", 0), kw.get("gate", 0),
+                                            ctypes.c_float(kw.get("eps", 1e-6)), ctypes.byref(kw.get("bufs", bufs)),
+                                            ctypes.byref(h))
+    assert f(d=96) == binding.GDN_ERR_UNSUPPORTED
+    assert f(B=0) == binding.GDN_ERR_INVALID_ARG
+    assert f(gate=3) == binding.GDN_ERR_INVALID_ARG
+    bad = binding._SessionBuffers(*([1 << 20] * 17 + [0]), 0)            # no workspace (bf16, d = 128 needs one)
+    assert f(bufs=bad, d=128) == binding.GDN_ERR_WORKSPACE
+    bad = binding._SessionBuffers(*([0] + [1 << 20] * 17), 1 << 30)        # a missing buffer
+    assert f(bufs=bad) == binding.GDN_ERR_INVALID_ARG
+    assert h.value is None
