@@ -85,14 +85,32 @@ __device__ __forceinline__ float *t_blk(uint8_t *sm, int i, int j) {
 
 // ------------------------------------------------------------ chain kernel layout
 constexpr int kChainThreads = 320;                     // warps 0-3 chain, 4-7 output, 8 MMA, 9 TMA
-constexpr uint32_t C_STAGE = 81920;                    // per stage: K, V, W, Qg, T'', Pt
-constexpr uint32_t CS_K = 0, CS_V = 16384, CS_W = 32768, CS_QG = 49152, CS_TPP = 65536, CS_PT = 73728;
-constexpr uint32_t C_U = 2 * C_STAGE;                  // output staging [64 t][128 dv] bf16
-constexpr uint32_t C_SCE = C_U + 16384;                // ChainScalars x 3 (state chain)
-constexpr uint32_t C_SCX = C_SCE + 3072;               // ChainScalars x 3 (identity chain)
-constexpr uint32_t C_BAR = C_SCX + 3072;               // mbarriers + TMEM base + abort flag
-constexpr uint32_t C_ALLOC = C_BAR + 256 + 1024;
-static_assert(CS_PT + 8192 == C_STAGE && C_STAGE - CS_W == kTileBytes, "stage layout");
+// Stages of the load pipeline.  An output range needs all of a chunk's data
+// (K, V and the 48 KB prep tile: two stages of 80 KB); a transition range
+// needs K, V, W and T'' only, and runs three stages of 56 KB so that a chunk's
+// loads are issued two chunks ahead.
+template <int MODE> struct ChainLayout;
+template <> struct ChainLayout<0> {   // MODE_OUT
+    static constexpr int NST = 2;
+    static constexpr uint32_t STAGE = 81920;
+    static constexpr uint32_t K = 0, V = 16384, W = 32768, QG = 49152, TPP = 65536, PT = 73728;
+};
+template <> struct ChainLayout<1> {   // MODE_TRANS
+    static constexpr int NST = 3;
+    static constexpr uint32_t STAGE = 57344;
+    static constexpr uint32_t K = 0, V = 16384, W = 32768, QG = 0, TPP = 49152, PT = 0;
+};
+static_assert(ChainLayout<0>::PT + 8192 == ChainLayout<0>::STAGE &&
+              ChainLayout<0>::STAGE - ChainLayout<0>::W == kTileBytes, "stage layout");
+static_assert(ChainLayout<1>::TPP + 8192 == ChainLayout<1>::STAGE, "stage layout");
+// After the stages: output staging [64 t][128 dv] bf16, ChainScalars x 3 per
+// chain, mbarriers + TMEM base + abort flag.
+template <int MODE> __host__ __device__ constexpr uint32_t c_u() { return ChainLayout<MODE>::NST * ChainLayout<MODE>::STAGE; }
+template <int MODE> __host__ __device__ constexpr uint32_t c_sce() { return c_u<MODE>() + 16384; }
+template <int MODE> __host__ __device__ constexpr uint32_t c_scx() { return c_sce<MODE>() + 3072; }
+template <int MODE> __host__ __device__ constexpr uint32_t c_bar() { return c_scx<MODE>() + 3072; }
+template <int MODE> __host__ __device__ constexpr uint32_t c_alloc() { return c_bar<MODE>() + 256 + 1024; }
+static_assert(c_alloc<0>() <= 232448 && c_alloc<1>() <= 232448, "chain kernel shared memory");
 // TMEM columns of the chain kernel.  The MMA A operands produced by the chain
 // itself (bf16 S and bf16 U^T) stay in TMEM: shared-memory bandwidth, not the
 // tensor core, bounds these small-N MMAs, so only B is read from shared memory.
@@ -105,9 +123,9 @@ constexpr uint32_t TM_COLS = 512;
 // Barriers that a role may complete twice before its consumer waits once are
 // per buffer (FULL/EMPTY per stage, C/OFREE per output buffer) and waited with
 // the parity of the buffer's use count, so that no phase can be skipped.
-enum { CB_FULL = 0, CB_EMPTY = 2, CB_A = 4, CB_B = 5, CB_C = 6, CB_SREADY = 8, CB_UREADY = 9,
-       CB_FIN = 10, CB_OFREE = 11, CB_A2 = 13, CB_B2 = 14, CB_SREADY2 = 15, CB_UREADY2 = 16,
-       CB_NUM = 17 };
+enum { CB_FULL = 0, CB_EMPTY = 3, CB_A = 6, CB_B = 7, CB_C = 8, CB_SREADY = 10, CB_UREADY = 11,
+       CB_FIN = 12, CB_OFREE = 13, CB_A2 = 15, CB_B2 = 16, CB_SREADY2 = 17, CB_UREADY2 = 18,
+       CB_NUM = 19 };   // FULL, EMPTY: one per stage (up to 3); C, OFREE: one per output buffer
 
 struct ChainScalars {   // per chunk, state group
     float gC;           // exp(G_C)
@@ -632,6 +650,9 @@ __global__ void __launch_bounds__(kChainThreads, 1)
 gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = aligned_smem(smraw);
+    using Lay = ChainLayout<MODE>;
+    constexpr int NST = Lay::NST;
+    constexpr uint32_t C_BAR = c_bar<MODE>();
     uint32_t *tmem_base_ptr = reinterpret_cast<uint32_t *>(sm + C_BAR + 8 * CB_NUM);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + C_BAR + 8 * CB_NUM + 4);
     auto bar = [&](int i) { return smem_u32(sm + C_BAR + 8 * i); };
@@ -703,31 +724,52 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
     } else if (warp == 9) {
         // ------------------------------------------------------------ TMA / bulk producer
         if (lane == 0) {
-            int issued[2] = {0, 0};
+            int issued[NST] = {};
+            // Pull chunk m's data into L2 while its stage is still in use, so
+            // that the copy into shared memory, once the stage frees up, is an
+            // L2 hit.
+            auto prefetch = [&](int m) {
+                if (m >= nloc) return;
+                const int zm = (int)(bos + (int64_t)(cb + m) * C);
+                for (int kb = 0; kb < 2; ++kb) {
+                    tma_prefetch_3d(&p.map_k, kb * 64, h, zm);
+                    tma_prefetch_3d(&p.map_v, kb * 64, h, zm);
+                }
+                const uint8_t *tm_ = p.tiles + ((size_t)(gc0 + m) * H + h) * kTileBytes;
+                if (MODE == MODE_TRANS) {
+                    bulk_prefetch_l2(tm_, 16384);
+                    bulk_prefetch_l2(tm_ + (ChainLayout<0>::TPP - ChainLayout<0>::W), 8192);
+                } else {
+                    bulk_prefetch_l2(tm_, (uint32_t)kTileBytes);
+                }
+            };
             for (int n = 0; n < nloc; ++n) {
-                const int s = n & 1;
-                const uint32_t st = smem_u32(sm + s * C_STAGE);
+                const int s = n % NST;
+                const uint32_t st = smem_u32(sm + s * Lay::STAGE);
                 const int z = (int)(bos + (int64_t)(cb + n) * C);
-                if (n >= 2 && !mbar_wait(bar(CB_EMPTY + s), ((n - 2) >> 1) & 1, lim, abort_flag)) { fail(61); break; }
+                if (n >= NST) {
+                    prefetch(n);   // (the tiles are complete: the wait below chunk 0's loads came first)
+                    if (!mbar_wait(bar(CB_EMPTY + s), ((n - NST) / NST) & 1, lim, abort_flag)) { fail(61); break; }
+                }
                 const uint32_t full = bar(CB_FULL + s);
                 const uint8_t *tile = p.tiles + ((size_t)(gc0 + n) * H + h) * kTileBytes;
                 // a transition range reads W and T'' only
-                mbar_arrive_expect_tx(full, MODE == MODE_TRANS ? C_STAGE - 24576 : C_STAGE);
+                mbar_arrive_expect_tx(full, Lay::STAGE);
                 for (int kb = 0; kb < 2; ++kb) {
-                    tma_load_3d(st + CS_K + kb * 8192, &p.map_k, kb * 64, h, z, full);
-                    tma_load_3d(st + CS_V + kb * 8192, &p.map_v, kb * 64, h, z, full);
+                    tma_load_3d(st + Lay::K + kb * 8192, &p.map_k, kb * 64, h, z, full);
+                    tma_load_3d(st + Lay::V + kb * 8192, &p.map_v, kb * 64, h, z, full);
                 }
                 if (n == 0 && p.wait_tiles) grid_dep_wait();   // tiles come from the prep kernel
-                if (MODE == MODE_TRANS) {
-                    bulk_load(st + CS_W, tile, 16384, full);
-                    bulk_load(st + CS_TPP, tile + (CS_TPP - CS_W), 8192, full);
+                if (MODE == MODE_TRANS) {   // W and T'' of the tile
+                    bulk_load(st + Lay::W, tile, 16384, full);
+                    bulk_load(st + Lay::TPP, tile + (ChainLayout<0>::TPP - ChainLayout<0>::W), 8192, full);
                 } else {
-                    bulk_load(st + CS_W, tile, (uint32_t)kTileBytes, full);
+                    bulk_load(st + Lay::W, tile, (uint32_t)kTileBytes, full);
                 }
                 ++issued[s];
             }
             const int zero = 0;   // no copy may still be landing in shared memory at exit
-            for (int s = 0; s < 2; ++s)
+            for (int s = 0; s < NST; ++s)
                 if (issued[s]) mbar_wait(bar(CB_FULL + s), (issued[s] - 1) & 1, lim, &zero);
         }
     } else if (warp == 8) {
@@ -744,7 +786,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
             // (a): U^T (+)= -S W^T for the chain whose tensor memory starts at `base`
             auto issue_a = [&](uint32_t base, uint32_t st, uint32_t accumulate_first) {
                 for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t offw = st + CS_W + (ks >> 2) * 8192 + (ks & 3) * 32;
+                    const uint32_t offw = st + Lay::W + (ks >> 2) * 8192 + (ks & 3) * 32;
                     mma_bf16_ts(tm + base + TM_U, tm + base + TM_SBF + 8 * ks, dSTk + (offw >> 4), id_a,
                                 ks > 0 ? 1u : accumulate_first);
                 }
@@ -753,17 +795,17 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
             auto issue_b = [&](uint32_t base, uint32_t st) {
                 for (int ks = 0; ks < 4; ++ks)
                     mma_bf16_ts(tm + base + TM_S, tm + base + TM_U + 8 * ks,
-                                dSTm + ((st + CS_K + ks * 2048) >> 4), id_b, 1);
+                                dSTm + ((st + Lay::K + ks * 2048) >> 4), id_b, 1);
             };
             for (int n = 0; ok && n < nloc; ++n) {
-                const int s = n & 1;
-                const uint32_t st = s * C_STAGE;
-                if (!(ok = mbar_wait(bar(CB_FULL + s), (n >> 1) & 1, lim, abort_flag))) { fail(62); break; }
+                const int s = n % NST, ob = n & 1;   // stage, output buffer
+                const uint32_t st = s * Lay::STAGE;
+                if (!(ok = mbar_wait(bar(CB_FULL + s), (n / NST) & 1, lim, abort_flag))) { fail(62); break; }
                 tc_fence_after();
                 // p3: U^T = V^T T''^T (the previous residual was consumed: U_READY(n-1))
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(tm + TM_U, dSTm + ((st + CS_V + ks * 2048) >> 4),
-                                dSTk + ((st + CS_TPP + ks * 32) >> 4), id_p3, ks > 0);
+                    mma_bf16_ss(tm + TM_U, dSTm + ((st + Lay::V + ks * 2048) >> 4),
+                                dSTk + ((st + Lay::TPP + ks * 32) >> 4), id_p3, ks > 0);
                 if (!(ok = mbar_wait(bar(CB_SREADY), n & 1, lim, abort_flag))) { fail(63); break; }
                 tc_fence_after();
                 issue_a(0, st, 1);
@@ -783,13 +825,13 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                     mma_commit(bar(CB_B2));
                     mma_commit(bar(CB_EMPTY + s));
                 } else {
-                    // the output group has read this buffer pair for chunk n-2
-                    if (n >= 2 && !(ok = mbar_wait(bar(CB_OFREE + s), ((n - 2) >> 1) & 1, lim, abort_flag))) { fail(65); break; }
+                    // the output group has read this output buffer for chunk n-2
+                    if (n >= 2 && !(ok = mbar_wait(bar(CB_OFREE + ob), ((n - 2) >> 1) & 1, lim, abort_flag))) { fail(65); break; }
                     tc_fence_after();
                     // c1: O^T = S Qg^T (off the state chain)
                     for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t off = st + CS_QG + (ks >> 2) * 8192 + (ks & 3) * 32;
-                        mma_bf16_ts(tm + TM_O + s * 64, tm + TM_SBF + 8 * ks, dSTk + (off >> 4), id_n64, ks > 0);
+                        const uint32_t off = st + Lay::QG + (ks >> 2) * 8192 + (ks & 3) * 32;
+                        mma_bf16_ts(tm + TM_O + ob * 64, tm + TM_SBF + 8 * ks, dSTk + (off >> 4), id_n64, ks > 0);
                     }
                     if (!(ok = mbar_wait(bar(CB_UREADY), n & 1, lim, abort_flag))) { fail(64); break; }
                     tc_fence_after();
@@ -797,9 +839,9 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                     mma_commit(bar(CB_B));
                     // c2: O^T += U^T Pt^T
                     for (int ks = 0; ks < 4; ++ks)
-                        mma_bf16_ts(tm + TM_O + s * 64, tm + TM_U + 8 * ks, dSTk + ((st + CS_PT + ks * 32) >> 4),
+                        mma_bf16_ts(tm + TM_O + ob * 64, tm + TM_U + 8 * ks, dSTk + ((st + Lay::PT + ks * 32) >> 4),
                                     id_n64, 1);
-                    mma_commit(bar(CB_C + s));
+                    mma_commit(bar(CB_C + ob));
                     mma_commit(bar(CB_EMPTY + s));
                 }
             }
@@ -820,7 +862,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
         const int bA = xchain ? CB_A2 : CB_A, bB = xchain ? CB_B2 : CB_B;
         const int bS = xchain ? CB_SREADY2 : CB_SREADY, bU = xchain ? CB_UREADY2 : CB_UREADY;
         const int nb = xchain ? 3 : 2;    // named barrier of this group
-        ChainScalars *scb = reinterpret_cast<ChainScalars *>(sm + (xchain ? C_SCX : C_SCE));
+        ChainScalars *scb = reinterpret_cast<ChainScalars *>(sm + (xchain ? c_scx<MODE>() : c_sce<MODE>()));
         GateRegs gr{0.f, 0.f, 0.f, 0.f};
         if (wg == 0) gr = load_gates(p.g, p.beta, bos, eos, cb, ce, h, H, lane);
         // scalars of local chunk m from the prefetched gates; prefetch chunk m+1's
@@ -935,7 +977,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
         // O^T (lane dv, 64 t) -> bf16 rows of out; off the state chain
         const int dv = tid - 128;   // TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>((warp - 4) * 32) << 16;
-        __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(sm + C_U);
+        __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(sm + c_u<MODE>());
         for (int n = 0; n < nloc; ++n) {
             const int s = n & 1;
             // all four warps are done with chunk n-1's staging buffer
@@ -1172,9 +1214,9 @@ bool set_smem_attrs() {
         cudaFuncSetAttribute(gdn_chunk_prep_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                              100) != cudaSuccess ||
         cudaFuncSetAttribute(gdn_chunk_chain_kernel<MODE_OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)C_ALLOC) != cudaSuccess ||
+                             (int)c_alloc<MODE_OUT>()) != cudaSuccess ||
         cudaFuncSetAttribute(gdn_chunk_chain_kernel<MODE_TRANS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)C_ALLOC) != cudaSuccess ||
+                             (int)c_alloc<MODE_TRANS>()) != cudaSuccess ||
         cudaFuncSetAttribute(gdn_scan_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kCombSmem) != cudaSuccess)
         return false;
@@ -1273,7 +1315,7 @@ cudaError_t launch_prefill_tc(const TcLaunch &L, cudaStream_t stream) {
         ct.wait_tiles = 1;
         ct.wait_start = 0;
         cudaError_t e = launch_pdl(gdn_chunk_chain_kernel<MODE_TRANS>, dim3(units * (nseg - 1)), dim3(kChainThreads),
-                                   C_ALLOC, stream, ct);
+                                   c_alloc<MODE_TRANS>(), stream, ct);
         if (e != cudaSuccess) return e;
         e = launch_pdl(gdn_scan_combine_kernel, dim3(units, D / kCombRows), dim3(kCombThreads), kCombSmem, stream,
                        L.state_in, static_cast<const float *>(cp.trans_r), static_cast<const float *>(cp.trans_m),
@@ -1284,7 +1326,7 @@ cudaError_t launch_prefill_tc(const TcLaunch &L, cudaStream_t stream) {
     co.wait_tiles = nseg > 1 ? 0 : 1;   // after the combine, the prep kernel has completed
     co.wait_start = nseg > 1 ? 1 : 0;
     const cudaError_t e = launch_pdl(gdn_chunk_chain_kernel<MODE_OUT>, dim3(units * nseg), dim3(kChainThreads),
-                                     C_ALLOC, stream, co);
+                                     c_alloc<MODE_OUT>(), stream, co);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
