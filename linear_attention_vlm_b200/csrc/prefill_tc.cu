@@ -920,8 +920,6 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
             tc_fence_before();
             mbar_arrive(bar(bS));
         }
-        float *dest = MODE == MODE_TRANS ? (xchain ? p.trans_m : p.trans_r) + unit * D * D
-                                         : (finish ? finish + state_off : nullptr);
         for (int n = 0; n < nloc; ++n) {
             // residual epilogue: U^T (fp32, lane dv, 64 t) -> bf16 in its own first 32 columns
             if (!mbar_wait(bar(bA), n & 1, lim, abort_flag)) fail(71);
@@ -947,14 +945,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                     tmem_ld32(tm + lane_off + base + TM_S + c0 + 32, x1);
                     if (!last) {
                         st_bf16_cols(TM_SBF + c0 / 2, x0, x1);
-                    } else if (dest) {
-                        float *dst = dest + (size_t)dv * D + c0;
-#pragma unroll
-                        for (int j = 0; j < 32; j += 4) {
-                            *reinterpret_cast<float4 *>(dst + j) = make_float4(x0[j], x0[j + 1], x0[j + 2], x0[j + 3]);
-                            *reinterpret_cast<float4 *>(dst + 32 + j) = make_float4(x1[j], x1[j + 1], x1[j + 2], x1[j + 3]);
-                        }
-                    }
+                    }   // the last state stays in TMEM; it leaves at teardown (coalesced)
                 }
                 tc_fence_before();
                 if (!last) {
@@ -1012,7 +1003,48 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
 
     // ---------------------------------------------------------------- teardown
     if (p.wait_tiles) grid_dep_wait();   // (also for an empty range: completion implies the prep's)
-    __syncthreads();
+    tc_fence_before();
+    __syncthreads();   // every MMA has completed (the MMA thread waited for them) and no copy is landing
+    // Final states (R and M of a transition range, state_out of a sequence's
+    // last output range) leave TMEM through shared memory, whose stages are
+    // idle now: each state warp writes its rows (padded pitch, conflict-free),
+    // then all threads store 16-byte pieces in row order.
+    if (nloc > 0 && *abort_flag == 0) {
+        constexpr int PITCH = D + 4;
+        const int nchains = MODE == MODE_TRANS ? 2 : 1;
+        for (int c = 0; c < nchains; ++c) {
+            float *dst = MODE == MODE_TRANS ? (c ? p.trans_m : p.trans_r) + unit * D * D
+                                            : (finish ? finish + state_off : nullptr);
+            if (!dst) break;   // uniform over the CTA
+            float *stg = reinterpret_cast<float *>(sm) + c * D * PITCH;
+            if ((warp >> 2) == c && warp < 8) {
+                tc_fence_after();
+                const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+                const int row = (warp & 3) * 32 + lane;
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    float x[32];
+                    tmem_ld32(tm + lane_off + (c ? TM_X : 0) + TM_S + c0, x);
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<float4 *>(stg + row * PITCH + c0 + j) = make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
+                }
+            }
+        }
+        __syncthreads();
+        for (int c = 0; c < nchains; ++c) {
+            float *dst = MODE == MODE_TRANS ? (c ? p.trans_m : p.trans_r) + unit * D * D
+                                            : (finish ? finish + state_off : nullptr);
+            if (!dst) break;
+            const float *stg = reinterpret_cast<const float *>(sm) + c * D * PITCH;
+            for (int i = threadIdx.x; i < D * D / 4; i += blockDim.x) {
+                const int row = i >> 5, c4 = i & 31;
+                *reinterpret_cast<float4 *>(dst + row * D + 4 * c4) =
+                    *reinterpret_cast<const float4 *>(stg + row * PITCH + 4 * c4);
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+    }
     if (warp == 8) {
         tc_fence_after();
         tmem_dealloc(tm, TM_COLS);
