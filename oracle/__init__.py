@@ -131,3 +131,7 @@ def decode_step(q, k, v, g, beta, state) -> Tuple[np.ndarray, np.ndarray]:
 # Steps around the recurrence inside one layer (plain numpy, fp64).
 from .layer_ops import (ACT_NONE, ACT_SILU, GATE_SIGMOID, GATE_SILU,  # noqa: E402,F401
                         log_sigmoid, output_gate, preprocess, sigmoid)
+
+# The hybrid block's other token mixer (plain numpy, fp64).
+from .attention import positions as rope_positions  # noqa: E402,F401
+from .attention import rope, swa_attention  # noqa: E402,F401
