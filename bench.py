@@ -71,6 +71,14 @@ def prefill_flops(T, H, d, C=64):
     return T * H * (5 * C * d + 6 * d * d + C * C / 3.0)
 
 
+def swa_attention_flops(T, Hq, d, window):
+    """2 d multiply-adds for q.k and 2 d for p v per (query, visible key,
+    head); one sequence of T tokens."""
+    w = min(window, T)
+    pairs = w * (w + 1) // 2 + (T - w) * w
+    return 4 * d * Hq * pairs
+
+
 def decode_bytes(B, H, dk, dv, elem=2):
     return B * H * (2 * dv * dk * 4 + (2 * dk + dv) * elem + 8 + dv * elem)
 
@@ -236,6 +244,21 @@ def run_native(args):
     frame_launches = 2 + gdn.gdn_prefill_kernel_count(1, FRAME, H, dk, dv, w.chunk, w.dtype) + 1
     decode_launches = 2 + 1 + 1
 
+    # ---- sliding-window attention layer of the hybrid block: RoPE on q and k,
+    # then causal attention over an 8K window with 16 query / 2 key-value heads
+    SWA_T = 32768
+    ax = {k: v.to(dev) for k, v in W.attention_inputs(SWA_T, seed=rank).items()}
+    swa_q, swa_k = torch.empty_like(ax["q"]), torch.empty_like(ax["k"])
+    swa_o = torch.empty_like(ax["q"])
+
+    def swa_attn_once():
+        gdn.gdn_swa_attention(swa_q, swa_k, ax["v"], window=W.SWA_WINDOW, out=swa_o)
+
+    def swa_layer_once():
+        gdn.gdn_rope(ax["q"], out=swa_q)
+        gdn.gdn_rope(ax["k"], out=swa_k)
+        swa_attn_once()
+
     # ---- e2e buffers (pinned host, fresh device copies each step)
     pin = {k: v.pin_memory() for k, v in host.items() if isinstance(v, torch.Tensor) and k != "cu_seqlens"}
     out_h = torch.empty((T, H, dv), dtype=w.dtype).pin_memory()
@@ -262,6 +285,7 @@ def run_native(args):
         sess.prefill(FRAME)
         sess.prefill(FRAME, eager=True)
         sess.decode()
+        swa_layer_once()
     torch.cuda.synchronize()
 
     def timed(fn, steps, do_flush=True):
@@ -291,6 +315,8 @@ def run_native(args):
         ms_frame_graph = timed(lambda i: sess.prefill(FRAME), K)
         ms_frame_eager = timed(lambda i: sess.prefill(FRAME, eager=True), K)
         ms_dec_graph = timed(lambda i: sess.decode(), K)
+        ms_swa_attn = timed(lambda i: swa_attn_once(), K)
+        ms_swa_layer = timed(lambda i: swa_layer_once(), K)
         wall = time.time() - t_wall0
     ms_prefill = max_over_ranks(ms_prefill, world)
     ms_decode = max_over_ranks(ms_decode, world)
@@ -300,6 +326,10 @@ def run_native(args):
     ms_frame_graph = max_over_ranks(ms_frame_graph, world)
     ms_frame_eager = max_over_ranks(ms_frame_eager, world)
     ms_dec_graph = max_over_ranks(ms_dec_graph, world)
+    ms_swa_attn = max_over_ranks(ms_swa_attn, world)
+    ms_swa_layer = max_over_ranks(ms_swa_layer, world)
+    swa_flops = swa_attention_flops(SWA_T, W.SWA_HQ, W.SWA_D, W.SWA_WINDOW)
+    swa_tf = swa_flops / (ms_swa_attn * 1e-3) / 1e12
     el = 2 if w.dtype == torch.bfloat16 else 4
     pre_bytes = 6 * T * H * dk * el + 4 * T * H * 4 + 3 * H * dk * 16    # x in, q/k/v out, a/b in, g/beta out, taps
     gate_bytes = 3 * T * H * dv * el + dv * 4                             # o, z in, y out, norm weight
@@ -363,10 +393,19 @@ def run_native(args):
                       "kernels_per_frame": frame_launches,
                       "decode_step_ms_graph": ms_dec_graph, "kernels_per_decode_step": decode_launches,
                       "l2": "flushed before every frame"},
+        "swa": {"metric": "sliding-window attention layer tokens/s (RoPE on q and k + attention), "
+                          "T=%d, window %d, %d query / %d key-value heads, d %d, bf16"
+                          % (SWA_T, W.SWA_WINDOW, W.SWA_HQ, W.SWA_HKV, W.SWA_D),
+                "value": aggregate_throughput(SWA_T, world, ms_swa_layer), "unit": "tokens/s",
+                "ms_per_step": ms_swa_layer, "attention_ms": ms_swa_attn,
+                "roofline": {"kernel": "swa_fwd_kernel", "bound": "tensor", "achieved": swa_tf,
+                             "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": swa_tf / pk["bf16_tflops"],
+                             "traffic": None, "algorithmic_flops": swa_flops},
+                "l2": "flushed before every step"},
         "e2e": {"value": aggregate_throughput(T, world, ms_e2e), "unit": "tokens/s",
                 "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": (K * launches_per_prefill + K + max(3, K // 10) * launches_per_prefill + 2 * K
-                         + 2 * K * frame_launches + K * decode_launches),
+                         + 2 * K * frame_launches + K * decode_launches + K + 3 * K),
         "clocks": clk.summary(),
         "timed_wall_s": wall,
     }

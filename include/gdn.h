@@ -234,6 +234,58 @@ int gdn_preprocess(const void *xq, const void *xk, const void *xv, const float *
 int gdn_output_gate(const void *o, const void *z, const float *norm_w, void *y, int64_t rows, int dv,
                     int gate, float eps, int dtype, void *stream);
 
+/* ------------------------------------------------------------------ sliding-window attention
+ *
+ * The hybrid block's other token mixer (InfiniteVL explainer page, "Step 2:
+ * Process tokens with Hybrid Blocks" and the "Sliding Window Attention"
+ * concept box): softmax attention restricted to a recent window of tokens
+ * (8K), with rotary positions and grouped-query heads (16 query heads, 2
+ * key/value heads).  Readings taken where the page is silent: the window
+ * counts tokens and includes the query token itself; RoPE is the rotate-half
+ * form at the token's position inside its sequence.
+ */
+
+/*
+ * Rotate-half RoPE over rows of d values (rows = tokens x heads):
+ *
+ *   p = (position of the token inside its sequence) + pos_offset
+ *   theta_i = base^(-2i/d),  a = p * theta_i,  for i < d/2:
+ *   out[i]       = x[i] cos a - x[i + d/2] sin a
+ *   out[i + d/2] = x[i + d/2] cos a + x[i] sin a
+ *
+ *   x, out       [total_tokens, H, d] dtype; out may equal x (in place), no
+ *                other overlap
+ *   cu_seqlens   as in gdn_prefill (NULL: num_seqs equal sequences)
+ *   pos_offset   >= 0, added to every position (a stream's tokens seen so far)
+ *   base         > 1 (10000 is the usual choice)
+ * The angle is reduced in double precision before the fp32 sine and cosine.
+ * Supported: d a multiple of 8 in [8, 256]; dtype GDN_F32 or GDN_BF16.
+ */
+int gdn_rope(const void *x, void *out, const int32_t *cu_seqlens, int num_seqs, int64_t total_tokens, int H, int d,
+             int pos_offset, float base, int dtype, void *stream);
+
+/*
+ * Causal sliding-window attention with grouped key/value heads, per sequence:
+ *
+ *   o[t, h] = sum_s softmax_s(scale * q[t, h] . k[s, h / (Hq / Hkv)]) v[s, h / (Hq / Hkv)]
+ *   over the keys s of t's sequence with t - window < s <= t
+ *
+ *   q        [total_tokens, Hq, d]   bf16 (already rotated)
+ *   k, v     [total_tokens, Hkv, d]  bf16 (k already rotated)
+ *   o        [total_tokens, Hq, d]   bf16 (written; may not overlap q, k, v)
+ *   cu_seqlens  as in gdn_prefill (NULL: num_seqs equal sequences)
+ *   window   >= 1 tokens;  scale > 0, or 0 for 1/sqrt(d)
+ *   status   device int32 or NULL: set to a nonzero code (left as is
+ *            otherwise; the caller clears it) when a wait inside the kernel
+ *            gave up after 2 s, in which case o is not valid
+ * Scores and the row sums are fp32; the probabilities enter the P V product
+ * as bf16.  Supported: dtype GDN_BF16, d = 128, Hq a multiple of Hkv,
+ * Hq <= 65535, total_tokens < 2^31 - 256.
+ */
+int gdn_swa_attention(const void *q, const void *k, const void *v, void *o, const int32_t *cu_seqlens,
+                      int num_seqs, int64_t total_tokens, int Hq, int Hkv, int d, int window, float scale,
+                      int dtype, int32_t *status, void *stream);
+
 /* ------------------------------------------------------------------ streaming session
  *
  * One Gated DeltaNet layer step over a constant-size memory, captured as a

@@ -2,6 +2,7 @@
 // workspace sizing and dispatch to the kernels.  No allocation, no device
 // synchronisation.
 #include <cuda_runtime.h>
+#include <math.h>
 #include <stdint.h>
 #include <stdio.h>
 #include <string.h>
@@ -222,6 +223,56 @@ int gdn_output_gate(const void *o, const void *z, const float *norm_w, void *y, 
     if (overlaps(y, n, z, n) || overlaps(y, n, norm_w, (size_t)dv * 4)) return GDN_ERR_INVALID_ARG;
     const cudaError_t e = gdn::launch_output_gate(dtype, dv, o, z, norm_w, y, rows, gate, eps,
                                                   static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e);
+}
+
+int gdn_rope(const void *x, void *out, const int32_t *cu_seqlens, int num_seqs, int64_t total_tokens, int H, int d,
+             int pos_offset, float base, int dtype, void *stream) {
+    if (num_seqs < 1 || H < 1 || total_tokens < 0 || pos_offset < 0) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (!(base > 1.f) || !(base < 3.0e38f)) return GDN_ERR_INVALID_ARG;
+    if (d < 8 || d > 256 || d % 8 != 0) return GDN_ERR_UNSUPPORTED;
+    if (total_tokens > (int64_t)INT32_MAX || total_tokens + pos_offset > (int64_t)INT32_MAX)
+        return GDN_ERR_INVALID_ARG;
+    if (!cu_seqlens && total_tokens % num_seqs != 0) return GDN_ERR_INVALID_ARG;
+    if (total_tokens == 0) return GDN_OK;
+    if (!x || !out || misaligned(x) || misaligned(out) || (cu_seqlens && misaligned(cu_seqlens)))
+        return GDN_ERR_INVALID_ARG;
+    const size_t n = (size_t)total_tokens * H * d * (dtype == GDN_BF16 ? 2 : 4);
+    if (out != x && overlaps(out, n, x, n)) return GDN_ERR_INVALID_ARG;   // in place, or apart
+    const cudaError_t e = gdn::launch_rope(dtype, x, out, cu_seqlens, num_seqs, total_tokens, H, d, pos_offset,
+                                           (double)base, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e);
+}
+
+int gdn_swa_attention(const void *q, const void *k, const void *v, void *o, const int32_t *cu_seqlens,
+                      int num_seqs, int64_t total_tokens, int Hq, int Hkv, int d, int window, float scale,
+                      int dtype, int32_t *status, void *stream) {
+    if (num_seqs < 1 || Hq < 1 || Hkv < 1 || total_tokens < 0 || window < 1) return GDN_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0 || Hq > 65535) return GDN_ERR_INVALID_ARG;
+    if (!(scale >= 0.f) || !(scale < 3.0e38f)) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_BF16 || d != 128) return GDN_ERR_UNSUPPORTED;
+    if (total_tokens > (int64_t)INT32_MAX - 256) return GDN_ERR_INVALID_ARG;
+    if (!cu_seqlens && total_tokens % num_seqs != 0) return GDN_ERR_INVALID_ARG;
+    if (total_tokens == 0) return GDN_OK;
+    const void *ptrs[] = {q, k, v, o};
+    for (const void *p : ptrs)
+        if (!p || misaligned(p)) return GDN_ERR_INVALID_ARG;
+    if ((cu_seqlens && misaligned(cu_seqlens)) || (reinterpret_cast<uintptr_t>(status) & 3u))
+        return GDN_ERR_INVALID_ARG;
+    const size_t nq = (size_t)total_tokens * Hq * d * 2, nkv = (size_t)total_tokens * Hkv * d * 2;
+    if (overlaps(o, nq, q, nq) || overlaps(o, nq, k, nkv) || overlaps(o, nq, v, nkv)) return GDN_ERR_INVALID_ARG;
+    gdn::SwaLaunch L;
+    L.q = q; L.k = k; L.v = v; L.o = o;
+    L.cu_seqlens = cu_seqlens;
+    L.num_seqs = num_seqs;
+    L.total_tokens = total_tokens;
+    L.Hq = Hq; L.Hkv = Hkv; L.window = window;
+    L.scale = scale > 0.f ? scale : 1.f / sqrtf((float)d);
+    L.err = status;
+    L.timeout_ns = kWaitLimitNs;
+    const cudaError_t e = gdn::launch_swa(L, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GDN_OK : cuda_fail(e);
 }
 

@@ -72,4 +72,21 @@ cudaError_t launch_output_gate(int dtype, int dv, const void *o, const void *z, 
 cudaError_t prefill_tc_setup();
 cudaError_t layer_ops_setup(int dtype, int d);
 
+// Sliding-window attention and RoPE (swa.cu).
+struct SwaLaunch {
+    const void *q, *k, *v;             // [T, Hq | Hkv | Hkv, 128] bf16
+    void *o;                           // [T, Hq, 128] bf16
+    const int32_t *cu_seqlens;         // [N+1] or null (N equal sequences)
+    int num_seqs;
+    int64_t total_tokens;
+    int Hq, Hkv, window;
+    float scale;
+    int *err;                          // device status word, or null
+    uint64_t timeout_ns;               // bound on every wait inside the kernel
+};
+cudaError_t launch_swa(const SwaLaunch &L, cudaStream_t stream);
+cudaError_t swa_setup();
+cudaError_t launch_rope(int dtype, const void *x, void *out, const int32_t *cu_seqlens, int num_seqs,
+                        int64_t total_tokens, int H, int d, int offset, double base, cudaStream_t stream);
+
 }  // namespace gdn

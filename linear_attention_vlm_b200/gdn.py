@@ -65,6 +65,10 @@ def _load():
     lib.gdn_preprocess.restype = i32
     lib.gdn_output_gate.argtypes = [vp, vp, fp, vp, i64, i32, i32, f32, i32, vp]
     lib.gdn_output_gate.restype = i32
+    lib.gdn_rope.argtypes = [vp, vp, vp, i32, i64, i32, i32, i32, f32, i32, vp]
+    lib.gdn_rope.restype = i32
+    lib.gdn_swa_attention.argtypes = [vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, f32, i32, vp, vp]
+    lib.gdn_swa_attention.restype = i32
     lib.gdn_session_workspace_size.argtypes = [i32, i32, i32, i32, i32]
     lib.gdn_session_workspace_size.restype = sz
     lib.gdn_session_create.argtypes = [i32, i32, i32, i32, i32, i32, i32, f32, vp, vp]
@@ -318,6 +322,65 @@ def gdn_output_gate(o: torch.Tensor, z: torch.Tensor, norm_w: Optional[torch.Ten
                                  _dtype_code(o.dtype), _stream(dev))
     if st != GDN_OK:
         raise GdnError(st, "gdn_output_gate")
+    return out
+
+
+def _seq_count(cu_seqlens: Optional[torch.Tensor], num_seqs: Optional[int], dev) -> int:
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32 or cu_seqlens.device != dev:
+            raise ValueError("cu_seqlens must be int32 on the same device")
+        return cu_seqlens.numel() - 1
+    return 1 if num_seqs is None else int(num_seqs)
+
+
+def gdn_rope(x: torch.Tensor, cu_seqlens: Optional[torch.Tensor] = None, *, num_seqs: Optional[int] = None,
+             offset: int = 0, base: float = 10000.0, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Rotate-half RoPE of x [T, H, d] at each token's position inside its
+    sequence plus ``offset`` (include/gdn.h, gdn_rope).  ``out`` may be ``x``."""
+    T, H, d = x.shape
+    dev = x.device
+    if dev.type != "cuda":
+        raise ValueError("gdn_rope needs CUDA tensors")
+    N = _seq_count(cu_seqlens, num_seqs, dev)
+    if out is None:
+        out = torch.empty_like(x)
+    elif out.shape != x.shape or out.dtype != x.dtype or out.device != dev:
+        raise ValueError("out must match x")
+    st = _load().gdn_rope(_ptr(x), _ptr(out), _ptr(cu_seqlens), N, T, H, d, int(offset), float(base),
+                          _dtype_code(x.dtype), _stream(dev))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_rope")
+    return out
+
+
+def gdn_swa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: Optional[torch.Tensor] = None,
+                      *, num_seqs: Optional[int] = None, window: int = 8192, scale: Optional[float] = None,
+                      out: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Causal sliding-window attention with grouped key/value heads
+    (include/gdn.h, gdn_swa_attention).  q [T, Hq, d], k, v [T, Hkv, d] bf16,
+    already rotated.  ``status`` (int32 [1] on the device, cleared by the
+    caller) receives a nonzero code if a wait inside the kernel gave up."""
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("gdn_swa_attention needs CUDA tensors")
+    if k.shape != (T, Hkv, d) or v.shape != (T, Hkv, d):
+        raise ValueError("k and v must be [T, Hkv, d]")
+    if k.dtype != q.dtype or v.dtype != q.dtype or k.device != dev or v.device != dev:
+        raise ValueError("q, k, v must share dtype and device")
+    N = _seq_count(cu_seqlens, num_seqs, dev)
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != q.dtype or out.device != dev:
+        raise ValueError("out must match q")
+    if status is not None and (status.dtype != torch.int32 or status.device != dev):
+        raise ValueError("status must be int32 on the same device")
+    st = _load().gdn_swa_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(cu_seqlens), N, T, Hq, Hkv, d,
+                                   int(window), 0.0 if scale is None else float(scale), _dtype_code(q.dtype),
+                                   _ptr(status), _stream(dev))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_swa_attention")
     return out
 
 

@@ -143,3 +143,40 @@ def test_session_create_rejects_bad_arguments(lib):
     bad = binding._SessionBuffers(*([0] + [1 << 20] * 17), 1 << 30)        # a missing buffer
     assert f(bufs=bad) == binding.GDN_ERR_INVALID_ARG
     assert h.value is None
+
+
+def test_rope_rejects_bad_arguments(lib):
+    inv, uns = binding.GDN_ERR_INVALID_ARG, binding.GDN_ERR_UNSUPPORTED
+    f = lambda x=1 << 20, out=2 << 20, cu=None, N=1, T=64, H=2, d=64, off=0, base=10000.0, dt=1: \
+        lib.gdn_rope(x, out, cu, N, T, H, d, off, ctypes.c_float(base), dt, None)
+    assert f(x=None) == inv
+    assert f(out=(2 << 20) + 8) == inv                            # misaligned
+    assert f(d=12) == uns
+    assert f(d=264) == uns
+    assert f(base=1.0) == inv
+    assert f(off=-1) == inv
+    assert f(dt=4) == inv
+    assert f(N=3, T=64) == inv                                    # uniform split must be exact
+    assert f(out=(1 << 20) + 64) == inv                           # partial overlap (in place is fine)
+    assert f(T=0) == binding.GDN_OK
+
+
+def test_swa_attention_rejects_bad_arguments(lib):
+    inv, uns = binding.GDN_ERR_INVALID_ARG, binding.GDN_ERR_UNSUPPORTED
+    base = 1 << 24
+
+    def f(q=base, k=2 * base, v=3 * base, o=4 * base, cu=None, N=1, T=256, Hq=4, Hkv=2, d=128, win=64,
+          scale=0.0, dt=1, status=None):
+        return lib.gdn_swa_attention(q, k, v, o, cu, N, T, Hq, Hkv, d, win, ctypes.c_float(scale), dt, status, None)
+    assert f(q=None) == inv
+    assert f(o=4 * base + 8) == inv                               # misaligned
+    assert f(d=64) == uns
+    assert f(dt=0) == uns                                         # fp32 attention is not built
+    assert f(dt=3) == inv
+    assert f(Hq=3, Hkv=2) == inv
+    assert f(win=0) == inv
+    assert f(scale=-1.0) == inv
+    assert f(N=3, T=256) == inv
+    assert f(o=base + 4096) == inv                                # output over q
+    assert f(status=4 * base + 2) == inv
+    assert f(T=0) == binding.GDN_OK

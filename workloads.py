@@ -245,3 +245,23 @@ def layer_inputs(T: int, H: int, d: int, dtype: torch.dtype = torch.bfloat16, se
     if state:
         out["conv_state"] = _round(rng.standard_normal((num_seqs, 3, 3, H, d), dtype=np.float32), dtype)
     return out
+
+
+# sliding-window attention layer of the hybrid block: 16 query heads, 2
+# key/value heads, window 8K tokens (InfiniteVL explainer page, "Step 2");
+# head dimension 128 as for the linear layers
+SWA_HQ, SWA_HKV, SWA_D, SWA_WINDOW = 16, 2, 128, 8192
+
+
+def attention_inputs(T: int, Hq: int = SWA_HQ, Hkv: int = SWA_HKV, d: int = SWA_D,
+                     dtype: torch.dtype = torch.bfloat16, seed: int = 0,
+                     q_scale: float = 1.0) -> Dict[str, torch.Tensor]:
+    """Inputs of the sliding-window attention layer, on the CPU: q ~
+    N(0, q_scale^2), k, v ~ N(0, 1), [T, H, d] in the storage dtype (scores
+    q.k / sqrt(d) then have standard deviation q_scale)."""
+    rng = _rng(seed, 8)
+    return {
+        "q": _round(q_scale * rng.standard_normal((T, Hq, d), dtype=np.float32), dtype),
+        "k": _round(rng.standard_normal((T, Hkv, d), dtype=np.float32), dtype),
+        "v": _round(rng.standard_normal((T, Hkv, d), dtype=np.float32), dtype),
+    }
