@@ -22,8 +22,10 @@
 // TMEM-resident A operand.  The running maximum m only moves (and O is
 // rescaled) when a block raises it by more than 8 (a factor 256), so
 // rescales are rare; P, the row sum and O all use the same m, so the final
-// O / sum is exact up to rounding.  S_{j+1} and P_{j-1} V_{j-1} run on the
-// tensor core while the softmax of block j runs.
+// O / sum is exact up to rounding.  A block is therefore read once: its
+// probabilities are formed against the current m while its maximum is
+// tracked, and formed again only when that maximum moves m.  S_{j+1} and
+// P_{j-1} V_{j-1} run on the tensor core while the softmax of block j runs.
 //
 // The key range of a CTA is [max(bos(t0), t0 - window + 1), t_last]; blocks
 // of that range that every row of the tile sees whole skip the mask.  Query
@@ -63,8 +65,8 @@ enum : int {
     BR_VEMPTY = BR_VFULL + kKVStages,
     BR_SFULL = BR_VEMPTY + kKVStages,   // + S buffer (2)
     BR_PREADY = BR_SFULL + 2,           // + P buffer (2)
-    BR_PVDONE = BR_PREADY + 2,
-    BR_FIN = BR_PVDONE + 1,
+    BR_PVDONE = BR_PREADY + 2,          // + P buffer (2): P V with that buffer completed
+    BR_FIN = BR_PVDONE + 2,
     BR_NUM = BR_FIN + 1
 };
 constexpr uint32_t SM_TMEM_SLOT = SM_BAR + 8 * BR_NUM;
@@ -148,6 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar(BR_PREADY + b), 128);
         }
         mbar_init(bar(BR_PVDONE), 1);
+        mbar_init(bar(BR_PVDONE + 1), 1);
         mbar_init(bar(BR_FIN), 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -226,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int ks = 0; ks < kBN / 16; ++ks)
                     mma_bf16_ts(tm + TM_O, tm + TM_P + b * (kBN / 2) + 8 * ks, dMN + ((vofs + ks * 2048) >> 4), id_o,
                                 (j > 0 || ks > 0) ? 1u : 0u);
-                mma_commit(bar(BR_PVDONE));
+                mma_commit(bar(BR_PVDONE + b));
                 mma_commit(bar(BR_VEMPTY + s));
                 if (j + 2 < nkb) ok = qk(j + 2);
             }
@@ -248,89 +251,116 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t span = static_cast<uint32_t>(hi_t - lo_t);
         const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
         const float c = p.c;
+        constexpr unsigned kAll = 0xffffffffu;
         float m = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < nkb; ++j) {
             const int b = j & 1, kb = kstart + j * kBN;
             const bool masked = !(kb + kBN - 1 <= t0 && kb >= lo_all);
             const int rel = kb - lo_t;   // key kb + i is visible iff (rel + i) in [0, span]
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(BR_SFULL + b), (j >> 1) & 1, lim, abort_flag));
+            ok = __all_sync(kAll, mbar_wait(bar(BR_SFULL + b), (j >> 1) & 1, lim, abort_flag));
             if (!ok) { fail(87); break; }
+            if (j >= 2) {   // P buffer b was last read by P_{j-2} V_{j-2}
+                ok = __all_sync(kAll, mbar_wait(bar(BR_PVDONE + b), ((j - 2) >> 1) & 1, lim, abort_flag));
+                if (!ok) { fail(88); break; }
+            }
             tc_fence_after();
             const uint32_t sa = tm + lane_off + TM_S + b * kBN;
-            // pass 1: row maximum of the visible scores
-            float mx = -INFINITY;
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                float v[32];
-                tmem_ld32(sa + 32 * c4, v);
-                if (masked) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (static_cast<uint32_t>(rel + 32 * c4 + i) <= span) mx = fmaxf(mx, v[i]);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) mx = fmaxf(mx, v[i]);
-                }
-            }
-            const float mb = mx * c;
+            const uint32_t pa = tm + lane_off + TM_P + b * (kBN / 2);
             float alpha = 1.f;
             bool rescale = false;
-            if (mb > m + kRescaleThreshold) {   // also taken when m is still -inf
-                if (m != -INFINITY) {
-                    alpha = exp2f(m - mb);
-                    rescale = true;
-                }
-                m = mb;
-            }
-            const float msub = (m == -INFINITY) ? 0.f : m;
-            // pass 2: probabilities, row sum, bf16 pairs for the tensor core
-            uint32_t pk[2][32];
-            float sum = 0.f;
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                float v[32];
-                tmem_ld32(sa + 32 * c4, v);
-#pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    float p0 = exp2f(fmaf(v[i], c, -msub));
-                    float p1 = exp2f(fmaf(v[i + 1], c, -msub));
-                    if (masked) {
-                        if (static_cast<uint32_t>(rel + 32 * c4 + i) > span) p0 = 0.f;
-                        if (static_cast<uint32_t>(rel + 32 * c4 + i + 1) > span) p1 = 0.f;
+            // move m up to mb when that raises it by more than the threshold
+            auto raise = [&](float mb) {
+                if (mb > m + kRescaleThreshold) {   // also taken when m is still -inf
+                    if (m != -INFINITY) {
+                        alpha *= ex2_approx(m - mb);
+                        rescale = true;
                     }
-                    sum += p0 + p1;
-                    pk[c4 >> 1][(c4 & 1) * 16 + (i >> 1)] = pack_bf16(p0, p1);
+                    m = mb;
                 }
+            };
+            if (__any_sync(kAll, m == -INFINITY)) {
+                // a row without a maximum yet: find this block's first
+                float mx = -INFINITY;
+#pragma unroll 1
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    float v[32];
+                    tmem_ld32(sa + 32 * c4, v);
+                    float a[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (!masked || static_cast<uint32_t>(rel + 32 * c4 + i) <= span) a[i & 3] = fmaxf(a[i & 3], v[i]);
+                    mx = fmaxf(mx, fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])));
+                }
+                raise(mx * c);
+            }
+            // probabilities against the current maximum, written to P chunk by
+            // chunk; rerun (rarely) when this block raises the maximum too far
+            float sum;
+            while (true) {
+                const float msub = (m == -INFINITY) ? 0.f : m;
+                float mx = -INFINITY;
+                sum = 0.f;
+#pragma unroll 1
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    float v[32];
+                    tmem_ld32(sa + 32 * c4, v);
+                    uint32_t pk[16];
+                    float a[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY}, sm4[4] = {0.f, 0.f, 0.f, 0.f};
+                    if (masked) {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2) {
+                            float x0 = v[i], x1 = v[i + 1];
+                            float p0 = ex2_approx(fmaf(x0, c, -msub)), p1 = ex2_approx(fmaf(x1, c, -msub));
+                            if (static_cast<uint32_t>(rel + 32 * c4 + i) > span) { p0 = 0.f; x0 = -INFINITY; }
+                            if (static_cast<uint32_t>(rel + 32 * c4 + i + 1) > span) { p1 = 0.f; x1 = -INFINITY; }
+                            a[(i >> 1) & 3] = fmaxf(a[(i >> 1) & 3], fmaxf(x0, x1));
+                            sm4[(i >> 1) & 3] += p0 + p1;
+                            pk[i >> 1] = pack_bf16(p0, p1);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2) {
+                            const float p0 = ex2_approx(fmaf(v[i], c, -msub)), p1 = ex2_approx(fmaf(v[i + 1], c, -msub));
+                            a[(i >> 1) & 3] = fmaxf(a[(i >> 1) & 3], fmaxf(v[i], v[i + 1]));
+                            sm4[(i >> 1) & 3] += p0 + p1;
+                            pk[i >> 1] = pack_bf16(p0, p1);
+                        }
+                    }
+                    tmem_st16u(pa + 16 * c4, pk);
+                    mx = fmaxf(mx, fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])));
+                    sum += (sm4[0] + sm4[1]) + (sm4[2] + sm4[3]);
+                }
+                const float mb = mx * c;
+                const bool up = mb > m + kRescaleThreshold;
+                if (!__any_sync(kAll, up)) break;
+                raise(mb);
             }
             l = l * alpha + sum;
-            if (j > 0) {
-                // P_{j-1} V_{j-1} has completed: O is stable and P buffer b is free
-                ok = __all_sync(0xffffffffu, mbar_wait(bar(BR_PVDONE), (j - 1) & 1, lim, abort_flag));
+            if (__any_sync(kAll, rescale)) {
+                // O holds the sum over blocks < j: wait for P_{j-1} V_{j-1}, then scale it
+                ok = __all_sync(kAll, mbar_wait(bar(BR_PVDONE + (b ^ 1)), ((j - 1) >> 1) & 1, lim, abort_flag));
                 if (!ok) { fail(88); break; }
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    float v[32];
+                    tmem_ld32(tm + lane_off + TM_O + 32 * c4, v);
 #pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        float v[32];
-                        tmem_ld32(tm + lane_off + TM_O + 32 * c4, v);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] *= alpha;
-                        tmem_st32(tm + lane_off + TM_O + 32 * c4, v);
-                    }
+                    for (int i = 0; i < 32; ++i) v[i] *= alpha;
+                    tmem_st32(tm + lane_off + TM_O + 32 * c4, v);
                 }
             }
-            tmem_st32u(tm + lane_off + TM_P + b * (kBN / 2), pk[0]);
-            tmem_st32u(tm + lane_off + TM_P + b * (kBN / 2) + 32, pk[1]);
             tc_fence_before();
             mbar_arrive(bar(BR_PREADY + b));
         }
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(BR_PVDONE), (nkb - 1) & 1, lim, abort_flag));
+        if (ok)
+            ok = __all_sync(kAll, mbar_wait(bar(BR_PVDONE + ((nkb - 1) & 1)), ((nkb - 1) >> 1) & 1, lim, abort_flag));
         if (ok) {
             tc_fence_after();
             const float inv = 1.f / l;
             uint4 *dst = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(t) * p.Hq + h) * kD);
-#pragma unroll
+#pragma unroll 1
             for (int c4 = 0; c4 < 4; ++c4) {
                 float v[32];
                 tmem_ld32(tm + lane_off + TM_O + 32 * c4, v);
@@ -382,25 +412,25 @@ template <> struct Vec4<__nv_bfloat16> {
     }
 };
 
-// Rotate-half RoPE.  A thread rotates 4 consecutive pairs (i, i + d/2) of one
-// (token, head) row; rows are walked grid-stride.  The angle p * theta_i is
-// formed and reduced to [-pi, pi] in double (theta_i = base^(-2i/d) kept per
-// block in shared memory), so the fp32 sine and cosine see an exact argument
-// even at positions of 10^5 and beyond.
+// Rotate-half RoPE.  A thread owns 4 consecutive pairs (i, i + d/2) of one
+// token and rotates them in every head, so each angle is formed once per
+// token: p * theta_i is computed and reduced to [-pi, pi] in double
+// (theta_i = base^(-2i/d) kept per block in shared memory), so the fp32 sine
+// and cosine see an exact argument even at positions of 10^5 and beyond.
+// Tokens are walked grid-stride.
 template <typename T>
 __global__ void __launch_bounds__(kRopeThreads)
     rope_kernel(const T *__restrict__ x, T *out, const int32_t *__restrict__ cu, int num_seqs, int64_t uniform_len,
-                int64_t rows, int H, int d, int offset, double log2_base) {
+                int64_t tokens, int H, int d, int offset, double log2_base) {
     __shared__ double theta[128];
     const int half = d >> 1, groups = half >> 2;
     for (int i = threadIdx.x; i < half; i += blockDim.x) theta[i] = exp2(-(2.0 * i / d) * log2_base);
     __syncthreads();
-    const int rows_per_block = kRopeThreads / groups;
-    const int g = threadIdx.x % groups, rb = threadIdx.x / groups;
-    if (rb >= rows_per_block) return;
+    const int tok_per_block = kRopeThreads / groups;
+    const int g = threadIdx.x % groups, tb = threadIdx.x / groups;
+    if (tb >= tok_per_block) return;
     constexpr double kTwoPi = 6.283185307179586476925286766559;
-    for (int64_t row = (int64_t)blockIdx.x * rows_per_block + rb; row < rows; row += (int64_t)gridDim.x * rows_per_block) {
-        const int64_t t = row / H;
+    for (int64_t t = (int64_t)blockIdx.x * tok_per_block + tb; t < tokens; t += (int64_t)gridDim.x * tok_per_block) {
         int64_t bos;
         if (cu) {
             int a = 0, b = num_seqs;   // cu[a] <= t < cu[b]
@@ -414,22 +444,26 @@ __global__ void __launch_bounds__(kRopeThreads)
             bos = t - t % uniform_len;
         }
         const double pos = static_cast<double>(t - bos + offset);
-        const T *src = x + row * d + 4 * g;
-        T *dst = out + row * d + 4 * g;
-        float x1[4], x2[4], y1[4], y2[4];
-        Vec4<T>::load(src, x1);
-        Vec4<T>::load(src + half, x2);
+        float cs[4], sn[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const double ang = pos * theta[4 * g + e];
-            const float r = static_cast<float>(ang - kTwoPi * rint(ang / kTwoPi));
-            float sn, cs;
-            sincosf(r, &sn, &cs);
-            y1[e] = x1[e] * cs - x2[e] * sn;
-            y2[e] = x2[e] * cs + x1[e] * sn;
+            sincosf(static_cast<float>(ang - kTwoPi * rint(ang / kTwoPi)), &sn[e], &cs[e]);
         }
-        Vec4<T>::store(dst, y1);
-        Vec4<T>::store(dst + half, y2);
+        const T *src = x + t * H * d + 4 * g;
+        T *dst = out + t * H * d + 4 * g;
+        for (int h = 0; h < H; ++h, src += d, dst += d) {
+            float x1[4], x2[4], y1[4], y2[4];
+            Vec4<T>::load(src, x1);
+            Vec4<T>::load(src + half, x2);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                y1[e] = x1[e] * cs[e] - x2[e] * sn[e];
+                y2[e] = x2[e] * cs[e] + x1[e] * sn[e];
+            }
+            Vec4<T>::store(dst, y1);
+            Vec4<T>::store(dst + half, y2);
+        }
     }
 }
 
@@ -506,12 +540,11 @@ cudaError_t launch_swa(const SwaLaunch &L, cudaStream_t stream) {
 
 cudaError_t launch_rope(int dtype, const void *x, void *out, const int32_t *cu_seqlens, int num_seqs,
                         int64_t total_tokens, int H, int d, int offset, double base, cudaStream_t stream) {
-    const int64_t rows = total_tokens * H;
-    if (rows == 0) return cudaSuccess;
-    const int groups = d / 8, rows_per_block = kRopeThreads / groups;
+    if (total_tokens == 0 || H == 0) return cudaSuccess;
+    const int groups = d / 8, tok_per_block = kRopeThreads / groups;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int64_t blocks = (rows + rows_per_block - 1) / rows_per_block;
+    int64_t blocks = (total_tokens + tok_per_block - 1) / tok_per_block;
     const int64_t cap = (int64_t)sms * 8;
     if (blocks > cap) blocks = cap;
     const int64_t uniform_len = cu_seqlens ? 1 : total_tokens / num_seqs;
@@ -519,11 +552,12 @@ cudaError_t launch_rope(int dtype, const void *x, void *out, const int32_t *cu_s
     if (dtype == GDN_BF16)
         rope_kernel<__nv_bfloat16><<<(unsigned)blocks, kRopeThreads, 0, stream>>>(
             static_cast<const __nv_bfloat16 *>(x), static_cast<__nv_bfloat16 *>(out), cu_seqlens, num_seqs,
-            uniform_len, rows, H, d, offset, lb);
+            uniform_len, total_tokens, H, d, offset, lb);
     else
         rope_kernel<float><<<(unsigned)blocks, kRopeThreads, 0, stream>>>(static_cast<const float *>(x),
                                                                            static_cast<float *>(out), cu_seqlens,
-                                                                           num_seqs, uniform_len, rows, H, d, offset, lb);
+                                                                           num_seqs, uniform_len, total_tokens, H, d, offset,
+                                                                           lb);
     return cudaGetLastError();
 }
 
