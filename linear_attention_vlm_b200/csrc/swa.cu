@@ -12,10 +12,13 @@
 // position inside its sequence plus an offset.
 //
 // Attention kernel: one CTA per (128 query tokens, query head), 192 threads.
-//   warps 0-3  softmax: one thread per query row (= TMEM lane)
-//   warp 4     TMA producer: the Q tile once, then K and V blocks of 128 keys
+//   warps 0-7  softmax: warps w and w + 4 share query rows 32(w%4) ..
+//              32(w%4) + 31 (TMEM lanes); each takes one 64-column half of a
+//              score block, and the pair agrees on the row maximum through
+//              shared memory once per block
+//   warp 8     TMA producer: the Q tile once, then K and V blocks of 128 keys
 //              through two 3-stage rings
-//   warp 5     MMA issuer (one lane)
+//   warp 9     MMA issuer (one lane)
 // Per key block j: S_j = Q K_j^T on the tensor core (fp32 in TMEM, two
 // buffers), the softmax threads turn S_j into P_j = 2^(c S_j - m) (bf16, in
 // TMEM) and the tensor core accumulates O += P_j V_j in TMEM with P_j as the
@@ -71,10 +74,11 @@ enum : int {
 };
 constexpr uint32_t SM_TMEM_SLOT = SM_BAR + 8 * BR_NUM;
 constexpr uint32_t SM_ABORT = SM_TMEM_SLOT + 4;
-constexpr uint32_t SM_ALLOC = SM_BAR + 256;
-constexpr size_t kSwaSmem = SM_ALLOC + 1024;   // + alignment slack
-static_assert(8 * BR_NUM + 8 <= 256, "barrier area");
-static_assert(kSwaSmem <= 232448, "shared memory per CTA");
+constexpr uint32_t SM_XCH = SM_BAR + 176;       // [2 parities][2 column halves][128 rows] fp32
+constexpr uint32_t SM_ALLOC = SM_XCH + 2 * 2 * 128 * 4;
+constexpr size_t kSwaSmem = 232448;             // the per-CTA maximum; the rest is alignment slack
+static_assert(8 * BR_NUM + 8 <= 176, "barrier area");
+static_assert(SM_ALLOC <= kSwaSmem, "shared memory per CTA");
 
 // tensor memory columns (512 allocated: the CTA owns the SM)
 constexpr uint32_t TM_S = 0;      // 2 x 128: scores
@@ -82,7 +86,9 @@ constexpr uint32_t TM_P = 256;    // 2 x 64: bf16 probabilities (2 per column)
 constexpr uint32_t TM_O = 384;    // 128: output accumulator
 constexpr uint32_t kTmemCols = 512;
 
-constexpr int kThreads = 192;
+constexpr int kSoftmaxWarps = 8;       // two per TMEM lane quarter: one per 64-column half
+constexpr int kProducerWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
+constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.f;   // log2 units
 
@@ -112,8 +118,13 @@ __device__ __forceinline__ int seq_start(const SwaParams &p, int t) {
 __global__ void __launch_bounds__(kThreads, 1)
     swa_fwd_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                    const __grid_constant__ CUtensorMap mV, const SwaParams p) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    if (pad + SM_ALLOC > kSwaSmem) {   // cannot happen with an aligned dynamic base; never touch past the end
+        if (threadIdx.x == 0 && p.err) atomicCAS(p.err, 0, 80);
+        return;
+    }
+    uint8_t *sm = smem_raw + pad;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     auto bar = [&](int i) { return smem_u32(sm + SM_BAR + 8 * i); };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + SM_TMEM_SLOT);
@@ -137,7 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
         tmem_relinquish();
     }
-    if (tid == 128) {
+    if (tid == 32 * kProducerWarp) {
         mbar_init(bar(BR_Q), 1);
         for (int s = 0; s < kKVStages; ++s) {
             mbar_init(bar(BR_KFULL + s), 1);
@@ -147,7 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar(BR_SFULL + b), 1);
-            mbar_init(bar(BR_PREADY + b), 128);
+            mbar_init(bar(BR_PREADY + b), 32 * kSoftmaxWarps);
         }
         mbar_init(bar(BR_PVDONE), 1);
         mbar_init(bar(BR_PVDONE + 1), 1);
@@ -164,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tm = *tmem_slot;
     const uint64_t lim = p.timeout_ns;
 
-    if (warp == 4) {
+    if (warp == kProducerWarp) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             int issued_k[kKVStages] = {}, issued_v[kKVStages] = {};
@@ -193,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (issued_v[s]) mbar_wait(bar(BR_VFULL + s), (issued_v[s] - 1) & 1, lim, &zero);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t id_s = idesc_bf16(kBM, kBN, false, false);   // Q (K-major) x K (K-major)
@@ -240,8 +251,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // ------------------------------------------------------------ softmax (warps 0-3)
-        const int t = t0 + tid;
+        // ------------------------------------------------------------ softmax (warps 0-7)
+        const int quarter = warp & 3, half = warp >> 2;
+        const int r = 32 * quarter + lane;           // query row = TMEM lane
+        const int t = t0 + r;
         const bool vrow = t < p.T;
         int lo_t = kstart, hi_t = kstart;   // rows past the end: one key, never stored
         if (vrow) {
@@ -249,24 +262,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             hi_t = t;
         }
         const uint32_t span = static_cast<uint32_t>(hi_t - lo_t);
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+        const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
         const float c = p.c;
         constexpr unsigned kAll = 0xffffffffu;
-        float m = -INFINITY, l = 0.f;
+        float *xch = reinterpret_cast<float *>(sm + SM_XCH);
+        // this row's value from the other half of the pair (a named barrier
+        // per lane quarter; two parities keep consecutive exchanges apart)
+        auto partner = [&](float v, int parity) -> float {
+            xch[(parity * 2 + half) * 128 + r] = v;
+            named_bar_sync(1 + quarter, 64);
+            return xch[(parity * 2 + (half ^ 1)) * 128 + r];
+        };
+        // Both halves of a row hold the same m at all times, and the two warps
+        // of a pair take the same branches and exchanges: every decision
+        // between them is made from exchanged values.  A wait that gives up
+        // therefore does not leave the loop (the partner could be waiting at
+        // an exchange); with the abort flag set the remaining waits return at
+        // once and the results are dropped.
+        float m = -INFINITY, l = 0.f;   // l: this half's share of the row sum
         bool ok = true;
         for (int j = 0; j < nkb; ++j) {
-            const int b = j & 1, kb = kstart + j * kBN;
-            const bool masked = !(kb + kBN - 1 <= t0 && kb >= lo_all);
+            const int b = j & 1, kb = kstart + j * kBN + 64 * half;
+            const bool masked = !(kstart + j * kBN + kBN - 1 <= t0 && kstart + j * kBN >= lo_all);
             const int rel = kb - lo_t;   // key kb + i is visible iff (rel + i) in [0, span]
-            ok = __all_sync(kAll, mbar_wait(bar(BR_SFULL + b), (j >> 1) & 1, lim, abort_flag));
-            if (!ok) { fail(87); break; }
-            if (j >= 2) {   // P buffer b was last read by P_{j-2} V_{j-2}
-                ok = __all_sync(kAll, mbar_wait(bar(BR_PVDONE + b), ((j - 2) >> 1) & 1, lim, abort_flag));
-                if (!ok) { fail(88); break; }
+            if (!__all_sync(kAll, mbar_wait(bar(BR_SFULL + b), (j >> 1) & 1, lim, abort_flag))) {
+                fail(87);
+                ok = false;
+            }
+            // P buffer b was last read by P_{j-2} V_{j-2}
+            if (j >= 2 && !__all_sync(kAll, mbar_wait(bar(BR_PVDONE + b), ((j - 2) >> 1) & 1, lim, abort_flag))) {
+                fail(88);
+                ok = false;
             }
             tc_fence_after();
-            const uint32_t sa = tm + lane_off + TM_S + b * kBN;
-            const uint32_t pa = tm + lane_off + TM_P + b * (kBN / 2);
+            const uint32_t sa = tm + lane_off + TM_S + b * kBN + 64 * half;
+            const uint32_t pa = tm + lane_off + TM_P + b * (kBN / 2) + 32 * half;
             float alpha = 1.f;
             bool rescale = false;
             // move m up to mb when that raises it by more than the threshold
@@ -279,11 +309,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m = mb;
                 }
             };
-            if (__any_sync(kAll, m == -INFINITY)) {
+            const bool need_max = __any_sync(kAll, m == -INFINITY);   // the same in both warps of the pair
+            if (need_max) {
                 // a row without a maximum yet: find this block's first
                 float mx = -INFINITY;
 #pragma unroll 1
-                for (int c4 = 0; c4 < 4; ++c4) {
+                for (int c4 = 0; c4 < 2; ++c4) {
                     float v[32];
                     tmem_ld32(sa + 32 * c4, v);
                     float a[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -292,17 +323,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!masked || static_cast<uint32_t>(rel + 32 * c4 + i) <= span) a[i & 3] = fmaxf(a[i & 3], v[i]);
                     mx = fmaxf(mx, fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])));
                 }
-                raise(mx * c);
+                raise(fmaxf(mx, partner(mx, j & 1)) * c);
             }
             // probabilities against the current maximum, written to P chunk by
-            // chunk; rerun (rarely) when this block raises the maximum too far
+            // chunk; formed again (rarely) when this block raises the maximum
+            // too far
             float sum;
-            while (true) {
+            for (int attempt = 0;; ++attempt) {
                 const float msub = (m == -INFINITY) ? 0.f : m;
                 float mx = -INFINITY;
                 sum = 0.f;
 #pragma unroll 1
-                for (int c4 = 0; c4 < 4; ++c4) {
+                for (int c4 = 0; c4 < 2; ++c4) {
                     float v[32];
                     tmem_ld32(sa + 32 * c4, v);
                     uint32_t pk[16];
@@ -331,39 +363,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mx = fmaxf(mx, fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])));
                     sum += (sm4[0] + sm4[1]) + (sm4[2] + sm4[3]);
                 }
-                const float mb = mx * c;
-                const bool up = mb > m + kRescaleThreshold;
-                if (!__any_sync(kAll, up)) break;
+                // after a max pass, or on the second attempt, m already covers the block
+                if (need_max || attempt > 0) break;
+                const float mb = fmaxf(mx, partner(mx, j & 1)) * c;
+                if (!__any_sync(kAll, mb > m + kRescaleThreshold)) break;   // the same in both warps
                 raise(mb);
             }
             l = l * alpha + sum;
             if (__any_sync(kAll, rescale)) {
-                // O holds the sum over blocks < j: wait for P_{j-1} V_{j-1}, then scale it
-                ok = __all_sync(kAll, mbar_wait(bar(BR_PVDONE + (b ^ 1)), ((j - 1) >> 1) & 1, lim, abort_flag));
-                if (!ok) { fail(88); break; }
+                // O holds the sum over blocks < j: wait for P_{j-1} V_{j-1}, then scale this half
+                if (!__all_sync(kAll, mbar_wait(bar(BR_PVDONE + (b ^ 1)), ((j - 1) >> 1) & 1, lim, abort_flag))) {
+                    fail(88);
+                    ok = false;
+                }
                 tc_fence_after();
 #pragma unroll 1
-                for (int c4 = 0; c4 < 4; ++c4) {
+                for (int c4 = 0; c4 < 2; ++c4) {
+                    const uint32_t oa = tm + lane_off + TM_O + 64 * half + 32 * c4;
                     float v[32];
-                    tmem_ld32(tm + lane_off + TM_O + 32 * c4, v);
+                    tmem_ld32(oa, v);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] *= alpha;
-                    tmem_st32(tm + lane_off + TM_O + 32 * c4, v);
+                    tmem_st32(oa, v);
                 }
             }
             tc_fence_before();
             mbar_arrive(bar(BR_PREADY + b));
         }
-        if (ok)
-            ok = __all_sync(kAll, mbar_wait(bar(BR_PVDONE + ((nkb - 1) & 1)), ((nkb - 1) >> 1) & 1, lim, abort_flag));
-        if (ok) {
+        if (ok && !__all_sync(kAll, mbar_wait(bar(BR_PVDONE + ((nkb - 1) & 1)), ((nkb - 1) >> 1) & 1, lim,
+                                               abort_flag)))
+            ok = false;
+        // the pair meets here in every case and skips the output together
+        const bool pair_ok = !named_bar_any(5 + quarter, 64, !ok);
+        if (pair_ok) {
             tc_fence_after();
-            const float inv = 1.f / l;
-            uint4 *dst = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(t) * p.Hq + h) * kD);
+            xch[((nkb & 1) * 2 + half) * 128 + r] = l;
+            named_bar_sync(5 + quarter, 64);
+            const float inv = 1.f / (l + xch[((nkb & 1) * 2 + (half ^ 1)) * 128 + r]);
+            uint4 *dst = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(t) * p.Hq + h) * kD + 64 * half);
 #pragma unroll 1
-            for (int c4 = 0; c4 < 4; ++c4) {
+            for (int c4 = 0; c4 < 2; ++c4) {
                 float v[32];
-                tmem_ld32(tm + lane_off + TM_O + 32 * c4, v);
+                tmem_ld32(tm + lane_off + TM_O + 64 * half + 32 * c4, v);
                 if (vrow) {
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4)
