@@ -58,6 +58,7 @@ typedef enum gdn_status {
     GDN_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, bad cu_seqlens length */
     GDN_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement (dk, dv, chunk, dtype) */
     GDN_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed */
+    GDN_ERR_TIMEOUT = 4,       /* a wait inside a kernel gave up (gdn_read_status) */
     GDN_ERR_WORKSPACE = 5      /* workspace NULL or smaller than gdn_prefill_workspace_size() */
 } gdn_status;
 
@@ -167,6 +168,21 @@ int gdn_prefill_noalloc(const void *q, const void *k, const void *v, const float
 
 /* Static, human-readable name of a gdn_status value. */
 const char *gdn_status_string(int status);
+
+/*
+ * Device status word of the tensor-core kernels.  Every wait inside them
+ * (on a copy, an MMA or another role of the CTA) gives up after 2 s; the
+ * kernel then records a nonzero code in a device int32 and returns, leaving
+ * its outputs invalid but the GPU usable.  The word is the first int32 of the
+ * workspace of gdn_prefill (and of a session's workspace; cleared by every
+ * call that uses the tensor-core path) and the `status` argument of
+ * gdn_swa_attention (cleared by the caller).
+ *
+ * gdn_read_status waits for `stream`, then reads the int32 at `word` (device,
+ * 4-byte aligned): GDN_OK if it is 0, GDN_ERR_TIMEOUT otherwise; *code (may
+ * be NULL) receives the word.  It is the one entry point that synchronises.
+ */
+int gdn_read_status(const int32_t *word, void *stream, int32_t *code);
 
 /* Text of the most recent CUDA error seen by this host thread inside the
  * library ("" if none).  Valid until the next call on this thread. */

@@ -75,12 +75,25 @@ const char *gdn_status_string(int status) {
         case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG: invalid argument";
         case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: shape, chunk or dtype not implemented";
         case GDN_ERR_CUDA: return "GDN_ERR_CUDA: CUDA runtime error";
+        case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT: a wait inside a kernel gave up";
         case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE: workspace missing or too small";
         default: return "unknown gdn_status";
     }
 }
 
 const char *gdn_last_cuda_error(void) { return g_last_cuda_error; }
+
+int gdn_read_status(const int32_t *word, void *stream, int32_t *code) {
+    if (code) *code = 0;
+    if (!word || (reinterpret_cast<uintptr_t>(word) & 3u)) return GDN_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t h = 0;
+    cudaError_t e = cudaMemcpyAsync(&h, word, sizeof(h), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (code) *code = h;
+    return h == 0 ? GDN_OK : GDN_ERR_TIMEOUT;
+}
 
 size_t gdn_prefill_workspace_size(int num_seqs, int64_t total_tokens, int H, int dk, int dv,
                                   int chunk, int dtype) {

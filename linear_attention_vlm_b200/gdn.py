@@ -19,7 +19,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libgdn.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "gdn.h")
 
-GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_WORKSPACE = 0, 1, 2, 3, 5
+GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT, GDN_ERR_WORKSPACE = 0, 1, 2, 3, 4, 5
 GDN_F32, GDN_BF16 = 0, 1
 ACT_NONE, ACT_SILU = 0, 1
 GATE_SIGMOID, GATE_SILU = 0, 1
@@ -85,6 +85,8 @@ def _load():
     lib.gdn_session_destroy.restype = None
     lib.gdn_status_string.argtypes = [i32]
     lib.gdn_status_string.restype = ctypes.c_char_p
+    lib.gdn_read_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int32)]
+    lib.gdn_read_status.restype = i32
     lib.gdn_last_cuda_error.argtypes = []
     lib.gdn_last_cuda_error.restype = ctypes.c_char_p
     _lib = lib
@@ -105,6 +107,21 @@ def declared_symbols():
 
 def status_string(status: int) -> str:
     return _load().gdn_status_string(int(status)).decode()
+
+
+def gdn_read_status(word: torch.Tensor) -> int:
+    """Wait for the current stream and return the device status word the
+    tensor-core kernels leave (include/gdn.h, gdn_read_status): 0 when every
+    wait inside them completed, else the kernel's code.  ``word`` is an int32
+    view of the prefill workspace's first word, or gdn_swa_attention's status
+    tensor."""
+    if word.device.type != "cuda" or word.dtype != torch.int32 or word.numel() < 1:
+        raise ValueError("word must be a CUDA int32 tensor")
+    code = ctypes.c_int32(0)
+    st = _load().gdn_read_status(_ptr(word), _stream(word.device), ctypes.byref(code))
+    if st not in (GDN_OK, GDN_ERR_TIMEOUT):
+        raise GdnError(st, "gdn_read_status")
+    return int(code.value)
 
 
 def _dtype_code(t: torch.dtype) -> int:

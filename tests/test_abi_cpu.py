@@ -23,7 +23,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in (0, 1, 2, 3, 5):
+    for code in (0, 1, 2, 3, 4, 5):
         assert gdn.status_string(code).startswith("GDN_")
     assert "unknown" in gdn.status_string(99)
     assert binding._load().gdn_last_cuda_error() == b""
@@ -180,3 +180,10 @@ def test_swa_attention_rejects_bad_arguments(lib):
     assert f(o=base + 4096) == inv                                # output over q
     assert f(status=4 * base + 2) == inv
     assert f(T=0) == binding.GDN_OK
+
+
+def test_read_status_rejects_bad_words(lib):
+    code = ctypes.c_int32(7)
+    assert lib.gdn_read_status(None, None, ctypes.byref(code)) == binding.GDN_ERR_INVALID_ARG
+    assert code.value == 0                                        # cleared before anything else
+    assert lib.gdn_read_status(4098, None, None) == binding.GDN_ERR_INVALID_ARG   # not 4-byte aligned

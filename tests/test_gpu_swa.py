@@ -50,8 +50,7 @@ def run_attn(x, lens, window, uniform_n=None, scale=None):
     cu = None if uniform_n else torch.tensor(cu_of(lens), dtype=torch.int32, device=DEV)
     o = gdn.gdn_swa_attention(x["q"].to(DEV), x["k"].to(DEV), x["v"].to(DEV), cu, num_seqs=uniform_n,
                               window=window, scale=scale, status=status)
-    torch.cuda.synchronize()
-    assert int(status.item()) == 0
+    assert gdn.gdn_read_status(status) == 0   # no wait inside the kernel gave up
     return o
 
 
