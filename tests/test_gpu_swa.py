@@ -146,3 +146,25 @@ def test_attention_full_size_sampled_rows():
     ref = oracle.swa_attention(np64(x["q"]), np64(x["k"]), np64(x["v"]), None, window=workloads.SWA_WINDOW,
                                rows=rows)
     check_attn(o, ref, x["v"], rows=rows)
+
+
+def test_attention_packed_long_sequences_sampled_rows():
+    # three packed sequences (32768 tokens in all), window 8192: rows on both
+    # sides of each sequence start, at the window length and at the ends
+    lens = [5000, 20000, 7768]
+    T = sum(lens)
+    x = workloads.attention_inputs(T, seed=3)
+    o = run_attn(x, lens, workloads.SWA_WINDOW)
+    rows = [0, 4999, 5000, 5001, 5127, 5128, 13191, 13192, 13193, 24999, 25000, 25001, 25100, 32767]
+    ref = oracle.swa_attention(np64(x["q"]), np64(x["k"]), np64(x["v"]), cu_of(lens), window=workloads.SWA_WINDOW,
+                               rows=rows)
+    check_attn(o, ref, x["v"], rows=rows)
+
+
+def test_attention_without_grouping():
+    lens = [260, 3]
+    T = sum(lens)
+    x = workloads.attention_inputs(T, Hq=3, Hkv=3, d=128, seed=8)
+    o = run_attn(x, lens, 130)
+    ref = oracle.swa_attention(np64(x["q"]), np64(x["k"]), np64(x["v"]), cu_of(lens), window=130)
+    check_attn(o, ref, x["v"])
