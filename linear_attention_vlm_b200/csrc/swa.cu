@@ -426,6 +426,328 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// ------------------------------------------------------------------ head-pair kernel
+//
+// For grouped heads (an even number of query heads per key/value head) a CTA
+// takes the same 128 tokens of two query heads that read the same key/value
+// head, as two tiles A and B.  Every K and V block is loaded once for both,
+// and the tensor core works on one tile's products while the other tile's
+// softmax runs, so the softmax round trip of one tile no longer leaves the
+// tensor pipe idle.
+//   warps 0-3  softmax of tile A, warps 4-7 tile B (one thread per row)
+//   warp 8     TMA producer (both Q tiles, then K and V through 2-stage rings)
+//   warp 9     MMA issuer
+// Tensor memory: S_A, S_B (128 columns each; P_X is written as bf16 over the
+// first 64 columns of S_X once they are read) and O_A, O_B (128 each).  The
+// softmax makes a max pass over the block first, so P never has to be formed
+// twice; the rescale rule is that of the single-tile kernel.  QK_X(j+1) goes
+// into S_X only after P_X(j) V_j has completed, which also means O_X is
+// stable whenever the softmax of tile X runs.
+constexpr int kPairKV = 2;                       // K and V ring stages
+constexpr uint32_t PS_Q = 0;                     // Q_A, Q_B
+constexpr uint32_t PS_K = 2 * kBlk;
+constexpr uint32_t PS_V = PS_K + kPairKV * kBlk;
+constexpr uint32_t PS_BAR = PS_V + kPairKV * kBlk;
+enum : int {
+    PB_Q = 0,
+    PB_KFULL = 1,
+    PB_KEMPTY = PB_KFULL + kPairKV,
+    PB_VFULL = PB_KEMPTY + kPairKV,
+    PB_VEMPTY = PB_VFULL + kPairKV,
+    PB_SFULL = PB_VEMPTY + kPairKV,   // + tile
+    PB_PREADY = PB_SFULL + 2,         // + tile
+    PB_PVDONE = PB_PREADY + 2,        // + tile
+    PB_FIN = PB_PVDONE + 2,
+    PB_NUM = PB_FIN + 1
+};
+constexpr uint32_t PS_TMEM_SLOT = PS_BAR + 8 * PB_NUM;
+constexpr uint32_t PS_ABORT = PS_TMEM_SLOT + 4;
+constexpr uint32_t PS_ALLOC = PS_BAR + 256;
+constexpr size_t kPairSmem = PS_ALLOC + 1024;
+static_assert(8 * PB_NUM + 8 <= 256, "barrier area");
+static_assert(kPairSmem <= 232448, "shared memory per CTA");
+constexpr uint32_t PT_S = 0;      // + 128 * tile
+constexpr uint32_t PT_O = 256;    // + 128 * tile
+
+__global__ void __launch_bounds__(kThreads, 1)
+    swa_fwd_pair_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
+                        const __grid_constant__ CUtensorMap mV, const SwaParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    uint8_t *sm = smem_raw + pad;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    auto bar = [&](int i) { return smem_u32(sm + PS_BAR + 8 * i); };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + PS_TMEM_SLOT);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + PS_ABORT);
+    auto fail = [&](int code) {
+        *abort_flag = 1;
+        if (p.err) atomicCAS(p.err, 0, code);
+    };
+
+    const int qb = gridDim.x - 1 - blockIdx.x;
+    const int h0 = 2 * blockIdx.y, kvh = h0 / (p.Hq / p.Hkv);   // heads h0, h0 + 1 share kvh
+    const int t0 = qb * kBM;
+    const int tlast = min(t0 + kBM - 1, p.T - 1);
+    const int kstart = max(seq_start(p, t0), t0 - p.window + 1);
+    const int nkb = (tlast + 1 - kstart + kBN - 1) / kBN;
+    const int lo_all = max(seq_start(p, tlast), tlast - p.window + 1);
+
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    if (tid == 32 * kProducerWarp) {
+        mbar_init(bar(PB_Q), 1);
+        for (int s = 0; s < kPairKV; ++s) {
+            mbar_init(bar(PB_KFULL + s), 1);
+            mbar_init(bar(PB_KEMPTY + s), 1);
+            mbar_init(bar(PB_VFULL + s), 1);
+            mbar_init(bar(PB_VEMPTY + s), 1);
+        }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(bar(PB_SFULL + x), 1);
+            mbar_init(bar(PB_PREADY + x), 128);
+            mbar_init(bar(PB_PVDONE + x), 1);
+        }
+        mbar_init(bar(PB_FIN), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&mQ);
+        tma_prefetch_desc(&mK);
+        tma_prefetch_desc(&mV);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tmem_slot;
+    const uint64_t lim = p.timeout_ns;
+
+    if (warp == kProducerWarp) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int issued_k[kPairKV] = {}, issued_v[kPairKV] = {};
+            mbar_arrive_expect_tx(bar(PB_Q), 2 * kBlk);
+            for (int x = 0; x < 2; ++x) {
+                tma_load_3d(smem_u32(sm + PS_Q + x * kBlk), &mQ, 0, h0 + x, t0, bar(PB_Q));
+                tma_load_3d(smem_u32(sm + PS_Q + x * kBlk + kHalf), &mQ, 64, h0 + x, t0, bar(PB_Q));
+            }
+            for (int j = 0; j < nkb; ++j) {
+                const int s = j % kPairKV, kb = kstart + j * kBN;
+                const uint32_t ph = ((j - kPairKV) / kPairKV) & 1;
+                if (j >= kPairKV && !mbar_wait(bar(PB_KEMPTY + s), ph, lim, abort_flag)) { fail(91); break; }
+                mbar_arrive_expect_tx(bar(PB_KFULL + s), kBlk);
+                tma_load_3d(smem_u32(sm + PS_K + s * kBlk), &mK, 0, kvh, kb, bar(PB_KFULL + s));
+                tma_load_3d(smem_u32(sm + PS_K + s * kBlk + kHalf), &mK, 64, kvh, kb, bar(PB_KFULL + s));
+                ++issued_k[s];
+                if (j >= kPairKV && !mbar_wait(bar(PB_VEMPTY + s), ph, lim, abort_flag)) { fail(92); break; }
+                mbar_arrive_expect_tx(bar(PB_VFULL + s), kBlk);
+                tma_load_3d(smem_u32(sm + PS_V + s * kBlk), &mV, 0, kvh, kb, bar(PB_VFULL + s));
+                tma_load_3d(smem_u32(sm + PS_V + s * kBlk + kHalf), &mV, 64, kvh, kb, bar(PB_VFULL + s));
+                ++issued_v[s];
+            }
+            const int zero = 0;   // no copy may still be landing in shared memory at exit
+            mbar_wait(bar(PB_Q), 0, lim, &zero);
+            for (int s = 0; s < kPairKV; ++s) {
+                if (issued_k[s]) mbar_wait(bar(PB_KFULL + s), (issued_k[s] - 1) & 1, lim, &zero);
+                if (issued_v[s]) mbar_wait(bar(PB_VFULL + s), (issued_v[s] - 1) & 1, lim, &zero);
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t id_s = idesc_bf16(kBM, kBN, false, false);
+            const uint32_t id_o = idesc_bf16(kBM, kD, false, true);
+            const uint64_t dKm = desc_sw128(smem_u32(sm), 16, 1024);
+            const uint64_t dMN = desc_sw128(smem_u32(sm), kHalf, 1024);
+            auto qk = [&](int x, int j) {   // S_x = Q_x K_j^T (K_j already waited for)
+                const uint32_t kofs = PS_K + (j % kPairKV) * kBlk, qofs = PS_Q + x * kBlk;
+#pragma unroll
+                for (int ks = 0; ks < kD / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
+                    mma_bf16_ss(tm + PT_S + x * kBN, dKm + ((qofs + off) >> 4), dKm + ((kofs + off) >> 4), id_s,
+                                ks > 0);
+                }
+                mma_commit(bar(PB_SFULL + x));
+            };
+            auto pv = [&](int x, int j) {   // O_x += P_x V_j (P_x over the first 64 columns of S_x)
+                const uint32_t vofs = PS_V + (j % kPairKV) * kBlk;
+#pragma unroll
+                for (int ks = 0; ks < kBN / 16; ++ks)
+                    mma_bf16_ts(tm + PT_O + x * kD, tm + PT_S + x * kBN + 8 * ks, dMN + ((vofs + ks * 2048) >> 4),
+                                id_o, (j > 0 || ks > 0) ? 1u : 0u);
+                mma_commit(bar(PB_PVDONE + x));
+            };
+            bool ok = mbar_wait(bar(PB_Q), 0, lim, abort_flag) && mbar_wait(bar(PB_KFULL), 0, lim, abort_flag);
+            if (!ok) fail(93);
+            if (ok) {
+                tc_fence_after();
+                qk(0, 0);
+                qk(1, 0);
+                mma_commit(bar(PB_KEMPTY));
+            }
+            for (int j = 0; ok && j < nkb; ++j) {
+                const int s = j % kPairKV, sn = (j + 1) % kPairKV;
+                const uint32_t par = j & 1;
+                const bool more = j + 1 < nkb;
+                for (int x = 0; x < 2; ++x) {
+                    if (!mbar_wait(bar(PB_PREADY + x), par, lim, abort_flag)) { fail(94); ok = false; break; }
+                    if (x == 0 && !mbar_wait(bar(PB_VFULL + s), (j / kPairKV) & 1, lim, abort_flag)) {
+                        fail(95);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    pv(x, j);
+                    if (x == 1) mma_commit(bar(PB_VEMPTY + s));
+                    if (more) {
+                        if (x == 0 && !mbar_wait(bar(PB_KFULL + sn), ((j + 1) / kPairKV) & 1, lim, abort_flag)) {
+                            fail(96);
+                            ok = false;
+                            break;
+                        }
+                        // S_x is overwritten only after P_x V_j has read it
+                        if (!mbar_wait(bar(PB_PVDONE + x), par, lim, abort_flag)) { fail(97); ok = false; break; }
+                        tc_fence_after();
+                        qk(x, j + 1);
+                        if (x == 1) mma_commit(bar(PB_KEMPTY + sn));
+                    }
+                }
+            }
+            mma_commit(bar(PB_FIN));
+            if (!mbar_wait(bar(PB_FIN), 0, lim, abort_flag)) {
+                const int zero = 0;
+                mbar_wait(bar(PB_FIN), 0, lim, &zero);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ softmax (warps 0-7)
+        const int x = warp >> 2, quarter = warp & 3;
+        const int r = 32 * quarter + lane;
+        const int t = t0 + r;
+        const bool vrow = t < p.T;
+        int lo_t = kstart, hi_t = kstart;
+        if (vrow) {
+            lo_t = max(seq_start(p, t), t - p.window + 1);
+            hi_t = t;
+        }
+        const uint32_t span = static_cast<uint32_t>(hi_t - lo_t);
+        const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
+        const uint32_t sa = tm + lane_off + PT_S + x * kBN, oa = tm + lane_off + PT_O + x * kD;
+        const float c = p.c;
+        constexpr unsigned kAll = 0xffffffffu;
+        float m = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nkb; ++j) {
+            const int kb = kstart + j * kBN;
+            const bool masked = !(kb + kBN - 1 <= t0 && kb >= lo_all);
+            const int rel = kb - lo_t;
+            // S_x(j) written (which also means P_x(j-1) V_{j-1} has completed)
+            if (!__all_sync(kAll, mbar_wait(bar(PB_SFULL + x), j & 1, lim, abort_flag))) {
+                fail(98);
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            float mx = -INFINITY;
+#pragma unroll 1
+            for (int c4 = 0; c4 < 4; ++c4) {
+                float v[32];
+                tmem_ld32(sa + 32 * c4, v);
+                float a[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                if (masked) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (static_cast<uint32_t>(rel + 32 * c4 + i) <= span) a[i & 3] = fmaxf(a[i & 3], v[i]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) a[i & 3] = fmaxf(a[i & 3], v[i]);
+                }
+                mx = fmaxf(mx, fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])));
+            }
+            const float mb = mx * c;
+            float alpha = 1.f;
+            bool rescale = false;
+            if (mb > m + kRescaleThreshold) {
+                if (m != -INFINITY) {
+                    alpha = ex2_approx(m - mb);
+                    rescale = true;
+                }
+                m = mb;
+            }
+            const float msub = (m == -INFINITY) ? 0.f : m;
+            float sum = 0.f;
+            // P chunk c4 goes over columns 16 c4 .. 16 c4 + 15, all read by then
+#pragma unroll 1
+            for (int c4 = 0; c4 < 4; ++c4) {
+                float v[32];
+                tmem_ld32(sa + 32 * c4, v);
+                uint32_t pk[16];
+                float sm4[4] = {0.f, 0.f, 0.f, 0.f};
+                if (masked) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        float p0 = ex2_approx(fmaf(v[i], c, -msub)), p1 = ex2_approx(fmaf(v[i + 1], c, -msub));
+                        if (static_cast<uint32_t>(rel + 32 * c4 + i) > span) p0 = 0.f;
+                        if (static_cast<uint32_t>(rel + 32 * c4 + i + 1) > span) p1 = 0.f;
+                        sm4[(i >> 1) & 3] += p0 + p1;
+                        pk[i >> 1] = pack_bf16(p0, p1);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        const float p0 = ex2_approx(fmaf(v[i], c, -msub)), p1 = ex2_approx(fmaf(v[i + 1], c, -msub));
+                        sm4[(i >> 1) & 3] += p0 + p1;
+                        pk[i >> 1] = pack_bf16(p0, p1);
+                    }
+                }
+                tmem_st16u(sa + 16 * c4, pk);
+                sum += (sm4[0] + sm4[1]) + (sm4[2] + sm4[3]);
+            }
+            l = l * alpha + sum;
+            if (__any_sync(kAll, rescale)) {
+#pragma unroll 1
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    float v[32];
+                    tmem_ld32(oa + 32 * c4, v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] *= alpha;
+                    tmem_st32(oa + 32 * c4, v);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar(PB_PREADY + x));
+        }
+        if (ok && !__all_sync(kAll, mbar_wait(bar(PB_PVDONE + x), (nkb - 1) & 1, lim, abort_flag))) {
+            fail(99);
+            ok = false;
+        }
+        if (ok) {
+            tc_fence_after();
+            const float inv = 1.f / l;
+            uint4 *dst = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(t) * p.Hq + h0 + x) * kD);
+#pragma unroll 1
+            for (int c4 = 0; c4 < 4; ++c4) {
+                float v[32];
+                tmem_ld32(oa + 32 * c4, v);
+                if (vrow) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        dst[c4 * 4 + q4] = make_uint4(pack_bf16(v[8 * q4] * inv, v[8 * q4 + 1] * inv),
+                                                      pack_bf16(v[8 * q4 + 2] * inv, v[8 * q4 + 3] * inv),
+                                                      pack_bf16(v[8 * q4 + 4] * inv, v[8 * q4 + 5] * inv),
+                                                      pack_bf16(v[8 * q4 + 6] * inv, v[8 * q4 + 7] * inv));
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tm, kTmemCols);
+    }
+}
+
 // ------------------------------------------------------------------ RoPE
 
 constexpr int kRopeThreads = 256;
@@ -549,6 +871,8 @@ cudaError_t swa_setup() {
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
     e = cudaFuncSetAttribute(swa_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSwaSmem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(swa_fwd_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmem);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) done[dev] = true;
     return cudaSuccess;
@@ -574,8 +898,13 @@ cudaError_t launch_swa(const SwaLaunch &L, cudaStream_t stream) {
     p.c = L.scale * kLog2e;
     p.err = L.err;
     p.timeout_ns = L.timeout_ns;
-    const dim3 grid((T + kBM - 1) / kBM, L.Hq);
-    swa_fwd_kernel<<<grid, kThreads, kSwaSmem, stream>>>(mq, mk, mv, p);
+    if ((L.Hq / L.Hkv) % 2 == 0) {   // head pairs that share a key/value head
+        const dim3 grid((T + kBM - 1) / kBM, L.Hq / 2);
+        swa_fwd_pair_kernel<<<grid, kThreads, kPairSmem, stream>>>(mq, mk, mv, p);
+    } else {
+        const dim3 grid((T + kBM - 1) / kBM, L.Hq);
+        swa_fwd_kernel<<<grid, kThreads, kSwaSmem, stream>>>(mq, mk, mv, p);
+    }
     return cudaGetLastError();
 }
 
