@@ -434,13 +434,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 // and the tensor core works on one tile's products while the other tile's
 // softmax runs, so the softmax round trip of one tile no longer leaves the
 // tensor pipe idle.
-//   warps 0-3  softmax of tile A, warps 4-7 tile B (one thread per row)
-//   warp 8     TMA producer (both Q tiles, then K and V through 2-stage rings)
-//   warp 9     MMA issuer
-// Tensor memory: S_A, S_B (128 columns each; P_X is written as bf16 over the
-// first 64 columns of S_X once they are read) and O_A, O_B (128 each).  The
-// softmax makes a max pass over the block first, so P never has to be formed
-// twice; the rescale rule is that of the single-tile kernel.  QK_X(j+1) goes
+//   warps 0-7  softmax of tile A, warps 8-15 tile B; as in the single-tile
+//              kernel, warps w and w + 4 of a tile split the columns of the
+//              rows of TMEM lane quarter w%4 and agree on the row maximum
+//              through shared memory
+//   warp 16    TMA producer (both Q tiles, then K and V through 2-stage rings)
+//   warp 17    MMA issuer
+// Tensor memory: S_A, S_B (128 columns each) and O_A, O_B (128 each).  The
+// column half h of S_X (columns 64h .. 64h + 63) receives, once read, the bf16
+// probabilities of its 64 keys in its first 32 columns.  The softmax makes a
+// max pass over the block first, so P never has to be formed twice; the
+// rescale rule is that of the single-tile kernel.  QK_X(j+1) goes
 // into S_X only after P_X(j) V_j has completed, which also means O_X is
 // stable whenever the softmax of tile X runs.
 constexpr int kPairKV = 2;                       // K and V ring stages
@@ -462,14 +466,18 @@ enum : int {
 };
 constexpr uint32_t PS_TMEM_SLOT = PS_BAR + 8 * PB_NUM;
 constexpr uint32_t PS_ABORT = PS_TMEM_SLOT + 4;
-constexpr uint32_t PS_ALLOC = PS_BAR + 256;
+constexpr uint32_t PS_XCH = PS_BAR + 256;   // [2 tiles][2 parities][2 halves][128 rows] fp32
+constexpr uint32_t PS_ALLOC = PS_XCH + 2 * 2 * 2 * 128 * 4;
 constexpr size_t kPairSmem = PS_ALLOC + 1024;
 static_assert(8 * PB_NUM + 8 <= 256, "barrier area");
 static_assert(kPairSmem <= 232448, "shared memory per CTA");
 constexpr uint32_t PT_S = 0;      // + 128 * tile
 constexpr uint32_t PT_O = 256;    // + 128 * tile
+constexpr int kPairSoftmaxWarps = 16;
+constexpr int kPairProducerWarp = kPairSoftmaxWarps, kPairMmaWarp = kPairSoftmaxWarps + 1;
+constexpr int kPairThreads = 32 * (kPairSoftmaxWarps + 2);
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kPairThreads, 1)
     swa_fwd_pair_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                         const __grid_constant__ CUtensorMap mV, const SwaParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -496,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
         tmem_relinquish();
     }
-    if (tid == 32 * kProducerWarp) {
+    if (tid == 32 * kPairProducerWarp) {
         mbar_init(bar(PB_Q), 1);
         for (int s = 0; s < kPairKV; ++s) {
             mbar_init(bar(PB_KFULL + s), 1);
@@ -506,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(bar(PB_SFULL + x), 1);
-            mbar_init(bar(PB_PREADY + x), 128);
+            mbar_init(bar(PB_PREADY + x), 32 * kPairSoftmaxWarps / 2);
             mbar_init(bar(PB_PVDONE + x), 1);
         }
         mbar_init(bar(PB_FIN), 1);
@@ -522,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tm = *tmem_slot;
     const uint64_t lim = p.timeout_ns;
 
-    if (warp == kProducerWarp) {
+    if (warp == kPairProducerWarp) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             int issued_k[kPairKV] = {}, issued_v[kPairKV] = {};
@@ -552,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (issued_v[s]) mbar_wait(bar(PB_VFULL + s), (issued_v[s] - 1) & 1, lim, &zero);
             }
         }
-    } else if (warp == kMmaWarp) {
+    } else if (warp == kPairMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t id_s = idesc_bf16(kBM, kBN, false, false);
@@ -569,12 +577,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 mma_commit(bar(PB_SFULL + x));
             };
-            auto pv = [&](int x, int j) {   // O_x += P_x V_j (P_x over the first 64 columns of S_x)
+            auto pv = [&](int x, int j) {   // O_x += P_x V_j (keys 0..63 in columns 0..31, 64..127 in 64..95)
                 const uint32_t vofs = PS_V + (j % kPairKV) * kBlk;
 #pragma unroll
                 for (int ks = 0; ks < kBN / 16; ++ks)
-                    mma_bf16_ts(tm + PT_O + x * kD, tm + PT_S + x * kBN + 8 * ks, dMN + ((vofs + ks * 2048) >> 4),
-                                id_o, (j > 0 || ks > 0) ? 1u : 0u);
+                    mma_bf16_ts(tm + PT_O + x * kD, tm + PT_S + x * kBN + (ks >> 2) * 64 + (ks & 3) * 8,
+                                dMN + ((vofs + ks * 2048) >> 4), id_o, (j > 0 || ks > 0) ? 1u : 0u);
                 mma_commit(bar(PB_PVDONE + x));
             };
             bool ok = mbar_wait(bar(PB_Q), 0, lim, abort_flag) && mbar_wait(bar(PB_KFULL), 0, lim, abort_flag);
@@ -620,8 +628,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // ------------------------------------------------------------ softmax (warps 0-7)
-        const int x = warp >> 2, quarter = warp & 3;
+        // ------------------------------------------------------------ softmax (warps 0-15)
+        const int x = warp >> 3, quarter = warp & 3, half = (warp >> 2) & 1;
         const int r = 32 * quarter + lane;
         const int t = t0 + r;
         const bool vrow = t < p.T;
@@ -632,25 +640,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const uint32_t span = static_cast<uint32_t>(hi_t - lo_t);
         const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
-        const uint32_t sa = tm + lane_off + PT_S + x * kBN, oa = tm + lane_off + PT_O + x * kD;
+        const uint32_t sa = tm + lane_off + PT_S + x * kBN + 64 * half;
+        const uint32_t oa = tm + lane_off + PT_O + x * kD + 64 * half;
         const float c = p.c;
         constexpr unsigned kAll = 0xffffffffu;
-        float m = -INFINITY, l = 0.f;
+        float *xch = reinterpret_cast<float *>(sm + PS_XCH) + x * (2 * 2 * 128);
+        const int bar_id = 1 + 4 * x + quarter;
+        // the row's value from the other column half (two parities keep
+        // consecutive exchanges apart); both warps of a pair call this the
+        // same number of times, whatever happens to their waits
+        auto partner = [&](float v, int parity) -> float {
+            xch[(parity * 2 + half) * 128 + r] = v;
+            named_bar_sync(bar_id, 64);
+            return xch[(parity * 2 + (half ^ 1)) * 128 + r];
+        };
+        float m = -INFINITY, l = 0.f;   // m: the same in both halves of a row; l: this half's share
         bool ok = true;
         for (int j = 0; j < nkb; ++j) {
-            const int kb = kstart + j * kBN;
-            const bool masked = !(kb + kBN - 1 <= t0 && kb >= lo_all);
-            const int rel = kb - lo_t;
+            const int kb0 = kstart + j * kBN;
+            const bool masked = !(kb0 + kBN - 1 <= t0 && kb0 >= lo_all);
+            const int rel = kb0 + 64 * half - lo_t;
             // S_x(j) written (which also means P_x(j-1) V_{j-1} has completed)
             if (!__all_sync(kAll, mbar_wait(bar(PB_SFULL + x), j & 1, lim, abort_flag))) {
                 fail(98);
                 ok = false;
-                break;
             }
             tc_fence_after();
             float mx = -INFINITY;
 #pragma unroll 1
-            for (int c4 = 0; c4 < 4; ++c4) {
+            for (int c4 = 0; c4 < 2; ++c4) {
                 float v[32];
                 tmem_ld32(sa + 32 * c4, v);
                 float a[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -664,7 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 mx = fmaxf(mx, fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])));
             }
-            const float mb = mx * c;
+            const float mb = fmaxf(mx, partner(mx, j & 1)) * c;
             float alpha = 1.f;
             bool rescale = false;
             if (mb > m + kRescaleThreshold) {
@@ -676,9 +694,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const float msub = (m == -INFINITY) ? 0.f : m;
             float sum = 0.f;
-            // P chunk c4 goes over columns 16 c4 .. 16 c4 + 15, all read by then
+            // P chunk c4 of this half goes over its columns 16 c4 .. 16 c4 + 15, read by then
 #pragma unroll 1
-            for (int c4 = 0; c4 < 4; ++c4) {
+            for (int c4 = 0; c4 < 2; ++c4) {
                 float v[32];
                 tmem_ld32(sa + 32 * c4, v);
                 uint32_t pk[16];
@@ -706,7 +724,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             l = l * alpha + sum;
             if (__any_sync(kAll, rescale)) {
 #pragma unroll 1
-                for (int c4 = 0; c4 < 4; ++c4) {
+                for (int c4 = 0; c4 < 2; ++c4) {
                     float v[32];
                     tmem_ld32(oa + 32 * c4, v);
 #pragma unroll
@@ -721,12 +739,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             fail(99);
             ok = false;
         }
+        // the halves' row sums (an exchange both warps always make)
+        xch[((nkb & 1) * 2 + half) * 128 + r] = l;
+        named_bar_sync(bar_id, 64);
+        const float lsum = l + xch[((nkb & 1) * 2 + (half ^ 1)) * 128 + r];
         if (ok) {
             tc_fence_after();
-            const float inv = 1.f / l;
-            uint4 *dst = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(t) * p.Hq + h0 + x) * kD);
+            const float inv = 1.f / lsum;
+            uint4 *dst = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(t) * p.Hq + h0 + x) * kD + 64 * half);
 #pragma unroll 1
-            for (int c4 = 0; c4 < 4; ++c4) {
+            for (int c4 = 0; c4 < 2; ++c4) {
                 float v[32];
                 tmem_ld32(oa + 32 * c4, v);
                 if (vrow) {
@@ -900,7 +922,7 @@ cudaError_t launch_swa(const SwaLaunch &L, cudaStream_t stream) {
     p.timeout_ns = L.timeout_ns;
     if ((L.Hq / L.Hkv) % 2 == 0) {   // head pairs that share a key/value head
         const dim3 grid((T + kBM - 1) / kBM, L.Hq / 2);
-        swa_fwd_pair_kernel<<<grid, kThreads, kPairSmem, stream>>>(mq, mk, mv, p);
+        swa_fwd_pair_kernel<<<grid, kPairThreads, kPairSmem, stream>>>(mq, mk, mv, p);
     } else {
         const dim3 grid((T + kBM - 1) / kBM, L.Hq);
         swa_fwd_kernel<<<grid, kThreads, kSwaSmem, stream>>>(mq, mk, mv, p);
