@@ -398,7 +398,7 @@ def run_native(args):
                           % (SWA_T, W.SWA_WINDOW, W.SWA_HQ, W.SWA_HKV, W.SWA_D),
                 "value": aggregate_throughput(SWA_T, world, ms_swa_layer), "unit": "tokens/s",
                 "ms_per_step": ms_swa_layer, "attention_ms": ms_swa_attn,
-                "roofline": {"kernel": "swa_fwd_kernel", "bound": "tensor", "achieved": swa_tf,
+                "roofline": {"kernel": "swa_fwd_pair_kernel", "bound": "tensor", "achieved": swa_tf,
                              "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": swa_tf / pk["bf16_tflops"],
                              "traffic": None, "algorithmic_flops": swa_flops},
                 "l2": "flushed before every step"},

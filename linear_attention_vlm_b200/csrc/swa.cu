@@ -11,7 +11,11 @@
 // key/value head h / (Hq / Hkv); RoPE is the rotate-half form at the token's
 // position inside its sequence plus an offset.
 //
-// Attention kernel: one CTA per (128 query tokens, query head), 192 threads.
+// Two attention kernels.  For grouped heads with an even group size the
+// head-pair kernel further down (two query heads of one key/value group per
+// CTA) is used; this one covers the rest.
+//
+// Single-tile kernel: one CTA per (128 query tokens, query head), 320 threads.
 //   warps 0-7  softmax: warps w and w + 4 share query rows 32(w%4) ..
 //              32(w%4) + 31 (TMEM lanes); each takes one 64-column half of a
 //              score block, and the pair agrees on the row maximum through
