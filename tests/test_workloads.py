@@ -75,3 +75,19 @@ def test_random_prefill_allows_empty():
     assert x["cu_seqlens"].tolist() == [0, 0, 3, 3, 73]
     assert x["q"].shape == (73, 2, 64)
     assert x["state_in"].shape == (4, 2, 64, 64)
+
+
+def test_attention_flop_count_matches_brute_force():
+    import bench
+    for T, W in ((1, 8192), (7, 3), (300, 128), (1000, 1000), (1000, 1)):
+        pairs = sum(min(t + 1, W) for t in range(T))
+        assert bench.swa_attention_flops(T, 16, 128, W) == 4 * 128 * 16 * pairs
+
+
+def test_attention_inputs_recipe():
+    x = W.attention_inputs(64, Hq=4, Hkv=2, d=128, seed=1, q_scale=3.0)
+    assert x["q"].shape == (64, 4, 128) and x["k"].shape == (64, 2, 128) and x["v"].shape == (64, 2, 128)
+    assert all(t.dtype == torch.bfloat16 for t in x.values())
+    assert 2.5 < float(x["q"].float().std()) < 3.5 and 0.8 < float(x["k"].float().std()) < 1.2
+    y = W.attention_inputs(64, Hq=4, Hkv=2, d=128, seed=1, q_scale=3.0)
+    assert all(torch.equal(x[n], y[n]) for n in x)
