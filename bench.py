@@ -57,6 +57,14 @@ def peaks():
 
 # ------------------------------------------------------------------ algorithmic work
 
+# DRAM bytes (read + write) per launch measured by ncu on this build, cold L2
+# (ncu flushes it before every captured launch): the four launches of one
+# prefill_bf16 call, and the head-pair attention kernel on the 32768-token
+# layer.  To be set to None whenever those kernels change.
+PREFILL_CALL_DRAM_BYTES = 434.0e6
+SWA_LAUNCH_DRAM_BYTES = 267.3e6
+
+
 def prefill_bytes(T, H, dk, dv, num_seqs, with_state_in, elem=2):
     """Bytes the prefill must move at minimum: q, k, v, g, beta in; out and
     the final state out (and the initial state in, when given)."""
@@ -363,7 +371,8 @@ def run_native(args):
                    "l2": "flushed before every step (512 MiB write)"},
         "roofline": {"kernel": "gdn_prefill (all %d launches of one call)" % launches_per_prefill,
                      "bound": "hbm", "achieved": ach_gbs, "peak": hbm, "unit": "GB/s",
-                     "frac": ach_gbs / hbm, "traffic": None,
+                     "frac": ach_gbs / hbm, "traffic": PREFILL_CALL_DRAM_BYTES,
+                     "traffic_note": "ncu dram bytes of the call's 4 launches, each from a cold L2",
                      "peak_source": pk_kind,
                      "algorithmic_bytes": pbytes, "algorithmic_flops": pflops,
                      "tensor_frac": (pflops / (ms_prefill * 1e-3) / 1e12) / pk["bf16_tflops"]},
@@ -400,7 +409,7 @@ def run_native(args):
                 "ms_per_step": ms_swa_layer, "attention_ms": ms_swa_attn,
                 "roofline": {"kernel": "swa_fwd_pair_kernel", "bound": "tensor", "achieved": swa_tf,
                              "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": swa_tf / pk["bf16_tflops"],
-                             "traffic": None, "algorithmic_flops": swa_flops},
+                             "traffic": SWA_LAUNCH_DRAM_BYTES, "algorithmic_flops": swa_flops},
                 "l2": "flushed before every step"},
         "e2e": {"value": aggregate_throughput(T, world, ms_e2e), "unit": "tokens/s",
                 "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
