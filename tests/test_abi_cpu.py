@@ -187,3 +187,15 @@ def test_read_status_rejects_bad_words(lib):
     assert lib.gdn_read_status(None, None, ctypes.byref(code)) == binding.GDN_ERR_INVALID_ARG
     assert code.value == 0                                        # cleared before anything else
     assert lib.gdn_read_status(4098, None, None) == binding.GDN_ERR_INVALID_ARG   # not 4-byte aligned
+
+
+def test_attention_bindings_refuse_bad_tensors():
+    import torch
+    q = torch.zeros(16, 4, 128, dtype=torch.bfloat16)
+    kv = torch.zeros(16, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        gdn.gdn_rope(q)                                   # CPU tensor
+    with pytest.raises(ValueError):
+        gdn.gdn_swa_attention(q, kv, kv)                  # CPU tensors
+    with pytest.raises(ValueError):
+        gdn.gdn_read_status(torch.zeros(1, dtype=torch.int32))
