@@ -7,10 +7,22 @@ One step = one gdn_prefill call over the bf16 prefill workload (1 sequence,
 16 heads, 8192 tokens, d_k = d_v = 128, chunk 64, zero initial state) with
 its inputs resident in HBM.  The L2 (126 MB) is flushed before every step by
 writing a 512 MiB buffer; only the prefill launches are inside the CUDA-event
-intervals.  The same run also times the decode step (64 sequences x 16 heads,
-fp32 state, one bf16 token each; L2 flushed before every step) and an
-end-to-end prefill through the public API with pinned host buffers (inputs
-copied in and out, result read back, inside the timed region).
+intervals.  The same run times every other workload of the method, one JSON
+object each:
+
+  long_prefill   262144 tokens x 16 heads, one call and 64 carried-state
+                 calls of 4096 tokens (inputs of 3.2 GB: larger than L2)
+  varlen         8 packed sequences of 1024..32768 tokens with their own
+                 initial states (inputs larger than L2)
+  decode         64 sequences x 16 heads, 1024 one-token steps captured in
+                 one CUDA graph; the state ping-pongs between two buffers
+                 (128 MiB, larger than L2) so every step streams it from HBM;
+                 decode_inplace is the same graph updating one 64 MiB state
+  e2e            the prefill through the public API with pinned host buffers
+                 (inputs copied in and out, result read back, all timed)
+
+plus the layer steps around the recurrence, the streaming session and the
+sliding-window attention layer of the hybrid block.
 
 Multi-GPU (torchrun): every rank runs its own replica of the workload (the
 units are independent sequences; there is no data-path collective); the
@@ -23,6 +35,8 @@ of the method) on a bounded sample of the same workload on the host cores.
 from __future__ import annotations
 
 import argparse
+import dataclasses
+import hashlib
 import json
 import os
 import statistics
@@ -44,6 +58,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 L2_FLUSH_BYTES = 512 << 20
 
 PREFILL = W.WORKLOADS["prefill_bf16"]
+ALL_LEGS = ("prefill", "long_prefill", "varlen", "decode", "e2e", "layer", "streaming", "swa")
 DECODE = W.WORKLOADS["decode_bf16"]
 
 
@@ -57,12 +72,39 @@ def peaks():
 
 # ------------------------------------------------------------------ algorithmic work
 
-# DRAM bytes (read + write) per launch measured by ncu on this build, cold L2
-# (ncu flushes it before every captured launch): the four launches of one
-# prefill_bf16 call, and the head-pair attention kernel on the 32768-token
-# layer.  To be set to None whenever those kernels change.
-PREFILL_CALL_DRAM_BYTES = 434.0e6
-SWA_LAUNCH_DRAM_BYTES = 267.3e6
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per call or
+# launch, measured by ncu and recorded in profiles/dram_traffic.txt together
+# with a hash of the kernel's sources at the time of the capture.  A figure
+# whose sources have changed since is not reported (traffic: null).
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+_CSRC = os.path.join("linear_attention_vlm_b200", "csrc")
+KERNEL_SOURCES = {
+    "prefill": [os.path.join(_CSRC, f) for f in ("prefill_tc.cu", "prefill_tc.h", "sm100.cuh")],
+    "swa": [os.path.join(_CSRC, f) for f in ("swa.cu", "sm100.cuh")],
+    "decode": [os.path.join(_CSRC, "decode.cu")],
+}
+
+
+def source_hash(kind):
+    """First 16 hex digits of the SHA-256 of a kernel family's sources."""
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES[kind]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(key, kind):
+    """Recorded DRAM bytes for `key`, or None if absent or stale."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    want = source_hash(kind)
+    with open(TRAFFIC_FILE) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 3 and not line.startswith("#") and parts[0] == key:
+                return float(parts[2]) if parts[1] == want else None
+    return None
 
 
 def prefill_bytes(T, H, dk, dv, num_seqs, with_state_in, elem=2):
@@ -200,8 +242,19 @@ def run_native(args):
     rank, world, local = dist_setup(args.gpus)
     dev = torch.device("cuda", torch.cuda.current_device())
     pk, pk_kind = peaks()
+    hbm = pk["hbm_gbs"]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    launches = {}   # leg -> kernel launches inside its timed region
+    legs = set(args.legs.split(",")) if args.legs else set(ALL_LEGS)
+    want = lambda leg: leg in legs
+
+    def hbm_roofline(kernel, nbytes, ms, traffic=None, **extra):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        r = {"kernel": kernel, "bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+             "frac": gbs / hbm, "traffic": traffic, "peak_source": pk_kind, "algorithmic_bytes": nbytes}
+        r.update(extra)
+        return r
 
     # ---- prefill inputs (seed per rank: independent replicas)
     w = PREFILL
@@ -218,28 +271,92 @@ def run_native(args):
         gdn.gdn_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], None, None, out=out,
                         state_out=st_out, workspace=ws)
 
-    # ---- decode inputs
-    dw = DECODE
-    S = W.decode_state(dw, seed=rank).to(dev)
-    ntok = args.steps + args.warmup
-    toks = [{k: v.to(dev) for k, v in W.decode_tokens(dw, i % dw.steps, seed=rank).items()}
-            for i in range(min(ntok, 64))]
-    dout = torch.empty((dw.num_seqs, dw.H, dw.dv), dtype=dw.dtype, device=dev)
+    # ---- long prefill: 262144 tokens, one call and 64 carried-state segments
+    lw = W.WORKLOADS["long_prefill_bf16"]
+    if not want("long_prefill"):
+        lw = dataclasses.replace(lw, T=lw.segments * 64)   # a token-sized stand-in, never timed
+    lx = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v)
+          for k, v in W.prefill_inputs(lw, seed=rank).items()}
+    LT = lw.T
+    l_out = torch.empty((LT, H, dv), dtype=lw.dtype, device=dev)
+    l_st = torch.empty((1, H, dv, dk), dtype=torch.float32, device=dev)
+    l_ws = torch.empty(max(gdn.gdn_prefill_workspace_size(1, LT, H, dk, dv), 16), dtype=torch.uint8, device=dev)
+    seg = LT // lw.segments
+    s_ws = torch.empty(max(gdn.gdn_prefill_workspace_size(1, seg, H, dk, dv), 16), dtype=torch.uint8, device=dev)
+    l_launch_whole = gdn.gdn_prefill_kernel_count(1, LT, H, dk, dv, packed=False)
+    l_launch_seg = gdn.gdn_prefill_kernel_count(1, seg, H, dk, dv, packed=False) * lw.segments
 
-    def decode_once(i):
-        t = toks[i % len(toks)]
-        gdn.gdn_decode_step(t["q"], t["k"], t["v"], t["g"], t["beta"], S, S, out=dout)
+    def long_whole_once():
+        gdn.gdn_prefill(lx["q"], lx["k"], lx["v"], lx["g"], lx["beta"], None, None, out=l_out,
+                        state_out=l_st, workspace=l_ws)
+
+    def long_segmented_once():
+        l_st.zero_()
+        for s0 in range(0, LT, seg):
+            sl = slice(s0, s0 + seg)
+            gdn.gdn_prefill(lx["q"][sl], lx["k"][sl], lx["v"][sl], lx["g"][sl], lx["beta"][sl], l_st, None,
+                            out=l_out[sl], state_out=l_st, workspace=s_ws)
+
+    # ---- varlen: 8 packed sequences, per-sequence initial states
+    vw = W.WORKLOADS["varlen_bf16"]
+    if not want("varlen"):
+        vw = dataclasses.replace(vw, varlen=(2, 64, 64))
+    vx = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v)
+          for k, v in W.prefill_inputs(vw, seed=rank).items()}
+    VT = int(vx["q"].shape[0])
+    VN = vx["cu_seqlens"].numel() - 1
+    v_out = torch.empty((VT, H, dv), dtype=vw.dtype, device=dev)
+    v_st = torch.empty((VN, H, dv, dk), dtype=torch.float32, device=dev)
+    v_ws = torch.empty(max(gdn.gdn_prefill_workspace_size(VN, VT, H, dk, dv), 16), dtype=torch.uint8, device=dev)
+    v_launch = gdn.gdn_prefill_kernel_count(VN, VT, H, dk, dv, packed=True)
+
+    def varlen_once():
+        gdn.gdn_prefill(vx["q"], vx["k"], vx["v"], vx["g"], vx["beta"], vx["state_in"], vx["cu_seqlens"],
+                        out=v_out, state_out=v_st, workspace=v_ws)
+
+    # ---- decode: 1024 one-token steps of 64 sequences x 16 heads in one CUDA graph
+    dw = DECODE
+    nsteps = dw.steps if want("decode") else 2
+    steps_host = [W.decode_tokens(dw, i, seed=rank) for i in range(nsteps)]
+    tok = {k: torch.stack([x[k] for x in steps_host]).to(dev) for k in ("q", "k", "v", "g", "beta")}
+    del steps_host
+    S0 = W.decode_state(dw, seed=rank).to(dev)
+    S_a, S_b = S0.clone(), torch.empty_like(S0)
+    dout = torch.empty((nsteps, dw.num_seqs, dw.H, dw.dv), dtype=dw.dtype, device=dev)
+
+    def decode_steps(pingpong):
+        for i in range(nsteps):
+            src = S_a if (not pingpong or i % 2 == 0) else S_b
+            dst = S_a if not pingpong else (S_b if i % 2 == 0 else S_a)
+            gdn.gdn_decode_step(tok["q"][i], tok["k"][i], tok["v"][i], tok["g"][i], tok["beta"][i], src, dst,
+                                out=dout[i])
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream(dev)
+        s.wait_stream(stream)
+        with torch.cuda.stream(s):
+            fn()   # warm-up outside the capture (one-time set-up of the kernels)
+        stream.wait_stream(s)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            fn()
+        torch.cuda.synchronize()
+        return g
+
+    graph_pp = capture(lambda: decode_steps(True))
+    graph_ip = capture(lambda: decode_steps(False))
 
     # ---- layer steps around the recurrence, on the prefill shapes
-    lx = {k: v.to(dev) for k, v in W.layer_inputs(T, H, dk, w.dtype, seed=rank).items()}
-    gate_out = torch.empty_like(lx["z"])
+    lay = {k: v.to(dev) for k, v in W.layer_inputs(T, H, dk, w.dtype, seed=rank).items()}
+    gate_out = torch.empty_like(lay["z"])
 
     def preprocess_once():
-        gdn.gdn_preprocess(lx["xq"], lx["xk"], lx["xv"], lx["conv_w"], lx["a"], lx["b"], None, None,
+        gdn.gdn_preprocess(lay["xq"], lay["xk"], lay["xv"], lay["conv_w"], lay["a"], lay["b"], None, None,
                            activation=gdn.ACT_SILU, want_state=False)
 
     def gate_once():
-        gdn.gdn_output_gate(out, lx["z"], lx["norm_w"], gate=gdn.GATE_SIGMOID, out=gate_out)
+        gdn.gdn_output_gate(out, lay["z"], lay["norm_w"], gate=gdn.GATE_SIGMOID, out=gate_out)
 
     # ---- streaming session: one GDN layer step per video frame (~274 tokens per
     # frame in the pages' streaming measurement), state carried, graph replay
@@ -254,7 +371,7 @@ def run_native(args):
 
     # ---- sliding-window attention layer of the hybrid block: RoPE on q and k,
     # then causal attention over an 8K window with 16 query / 2 key-value heads
-    SWA_T = 32768
+    SWA_T = 32768 if want("swa") else 256
     ax = {k: v.to(dev) for k, v in W.attention_inputs(SWA_T, seed=rank).items()}
     swa_q, swa_k = torch.empty_like(ax["q"]), torch.empty_like(ax["k"])
     swa_o = torch.empty_like(ax["q"])
@@ -285,18 +402,30 @@ def run_native(args):
 
     # ---- warm-up
     for i in range(args.warmup):
-        prefill_once()
-        decode_once(i)
-        e2e_once()
-        preprocess_once()
-        gate_once()
-        sess.prefill(FRAME)
-        sess.prefill(FRAME, eager=True)
-        sess.decode()
-        swa_layer_once()
+        if want("prefill"):
+            prefill_once()
+        if want("long_prefill"):
+            long_whole_once()
+            long_segmented_once()
+        if want("varlen"):
+            varlen_once()
+        if want("decode"):
+            graph_pp.replay()
+            graph_ip.replay()
+        if want("e2e"):
+            e2e_once()
+        if want("layer"):
+            preprocess_once()
+            gate_once()
+        if want("streaming"):
+            sess.prefill(FRAME)
+            sess.prefill(FRAME, eager=True)
+            sess.decode()
+        if want("swa"):
+            swa_layer_once()
     torch.cuda.synchronize()
 
-    def timed(fn, steps, do_flush=True):
+    def timed(fn, steps, do_flush=True, reduce="mean"):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(steps)]
         barrier(world)
@@ -310,46 +439,68 @@ def run_native(args):
         torch.cuda.synchronize()
         barrier(world)
         ms = [a.elapsed_time(b) for a, b in evs]
-        return sum(ms) / len(ms)
+        return statistics.median(ms) if reduce == "median" else sum(ms) / len(ms)
 
     K = args.steps
+    KL = max(3, min(K, 10))          # repeats of the long legs (milliseconds each)
+    KG = max(20, min(K, 20))         # graph replays of the 1024 decode steps (median)
+    ms = {}
+    nan = float("nan")
     with ClockSampler(local) as clk:
         t_wall0 = time.time()
-        ms_prefill = timed(lambda i: prefill_once(), K)
-        ms_decode = timed(decode_once, K)
-        ms_e2e = timed(lambda i: e2e_once(), max(3, K // 10), do_flush=False)
-        ms_pre = timed(lambda i: preprocess_once(), K)
-        ms_gate = timed(lambda i: gate_once(), K)
-        ms_frame_graph = timed(lambda i: sess.prefill(FRAME), K)
-        ms_frame_eager = timed(lambda i: sess.prefill(FRAME, eager=True), K)
-        ms_dec_graph = timed(lambda i: sess.decode(), K)
-        ms_swa_attn = timed(lambda i: swa_attn_once(), K)
-        ms_swa_layer = timed(lambda i: swa_layer_once(), K)
+        if want("prefill"):
+            ms["prefill"] = timed(lambda i: prefill_once(), K)
+            launches["prefill"] = K * launches_per_prefill
+        if want("long_prefill"):
+            ms["long"] = timed(lambda i: long_whole_once(), KL, do_flush=False)
+            launches["long"] = KL * l_launch_whole
+            ms["long_seg"] = timed(lambda i: long_segmented_once(), KL, do_flush=False)
+            launches["long_seg"] = KL * l_launch_seg
+        if want("varlen"):
+            ms["varlen"] = timed(lambda i: varlen_once(), KL, do_flush=False)
+            launches["varlen"] = KL * v_launch
+        if want("decode"):
+            ms["dec_pp"] = timed(lambda i: graph_pp.replay(), KG, do_flush=False, reduce="median")
+            ms["dec_ip"] = timed(lambda i: graph_ip.replay(), KG, do_flush=False, reduce="median")
+            launches["decode"] = 2 * KG * nsteps
+        if want("e2e"):
+            KE = max(3, K // 10)
+            ms["e2e"] = timed(lambda i: e2e_once(), KE, do_flush=False)
+            launches["e2e"] = KE * launches_per_prefill
+        if want("layer"):
+            ms["pre"] = timed(lambda i: preprocess_once(), K)
+            ms["gate"] = timed(lambda i: gate_once(), K)
+            launches["layer"] = 2 * K + K
+        if want("streaming"):
+            ms["frame_graph"] = timed(lambda i: sess.prefill(FRAME), K)
+            ms["frame_eager"] = timed(lambda i: sess.prefill(FRAME, eager=True), K)
+            ms["dec_graph"] = timed(lambda i: sess.decode(), K)
+            launches["session"] = 2 * K * frame_launches + K * decode_launches
+        if want("swa"):
+            ms["swa_attn"] = timed(lambda i: swa_attn_once(), K)
+            ms["swa_layer"] = timed(lambda i: swa_layer_once(), K)
+            launches["swa"] = K + 3 * K
         wall = time.time() - t_wall0
-    ms_prefill = max_over_ranks(ms_prefill, world)
-    ms_decode = max_over_ranks(ms_decode, world)
-    ms_e2e = max_over_ranks(ms_e2e, world)
-    ms_pre = max_over_ranks(ms_pre, world)
-    ms_gate = max_over_ranks(ms_gate, world)
-    ms_frame_graph = max_over_ranks(ms_frame_graph, world)
-    ms_frame_eager = max_over_ranks(ms_frame_eager, world)
-    ms_dec_graph = max_over_ranks(ms_dec_graph, world)
-    ms_swa_attn = max_over_ranks(ms_swa_attn, world)
-    ms_swa_layer = max_over_ranks(ms_swa_layer, world)
+    keys = ("prefill", "long", "long_seg", "varlen", "dec_pp", "dec_ip", "e2e", "pre", "gate",
+            "frame_graph", "frame_eager", "dec_graph", "swa_attn", "swa_layer")
+    (ms_prefill, ms_long, ms_long_seg, ms_varlen, ms_dec_pp, ms_dec_ip, ms_e2e, ms_pre, ms_gate,
+     ms_frame_graph, ms_frame_eager, ms_dec_graph, ms_swa_attn, ms_swa_layer) = (
+        max_over_ranks(ms.get(k, nan), world) for k in keys)
     swa_flops = swa_attention_flops(SWA_T, W.SWA_HQ, W.SWA_D, W.SWA_WINDOW)
     swa_tf = swa_flops / (ms_swa_attn * 1e-3) / 1e12
     el = 2 if w.dtype == torch.bfloat16 else 4
     pre_bytes = 6 * T * H * dk * el + 4 * T * H * 4 + 3 * H * dk * 16    # x in, q/k/v out, a/b in, g/beta out, taps
     gate_bytes = 3 * T * H * dv * el + dv * 4                             # o, z in, y out, norm weight
 
-    tokens = T * world
     value = aggregate_throughput(T, world, ms_prefill)
     pbytes = prefill_bytes(T, H, dk, dv, 1, with_state_in=False)
     pflops = prefill_flops(T, H, dk)
-    ach_gbs = pbytes / (ms_prefill * 1e-3) / 1e9
-    dbytes = decode_bytes(dw.num_seqs, dw.H, dw.dk, dw.dv)
-    d_gbs = dbytes / (ms_decode * 1e-3) / 1e9
-    hbm = pk["hbm_gbs"]
+    lbytes = prefill_bytes(LT, H, dk, dv, 1, with_state_in=False)
+    lseg_bytes = (prefill_bytes(seg, H, dk, dv, 1, with_state_in=True)) * lw.segments
+    vbytes = prefill_bytes(VT, H, dk, dv, VN, with_state_in=True)
+    dbytes = decode_bytes(dw.num_seqs, dw.H, dw.dk, dw.dv) * nsteps
+    tensor_frac = lambda flops, ms: (flops / (ms * 1e-3) / 1e12) / pk["bf16_tflops"]
+    prefill_kernel = "gdn_prefill (all %d launches of one call)"
     line = {
         "metric": "GDN prefill tokens/s and decode tokens/s on 1 B200; % of TC / HBM roofline",
         "value": value,
@@ -369,32 +520,53 @@ def run_native(args):
                    "global_batch": world, "seq_len": T, "heads": H, "head_dim": dk,
                    "parallelism": "replicas x%d (independent sequences)" % world,
                    "l2": "flushed before every step (512 MiB write)"},
-        "roofline": {"kernel": "gdn_prefill (all %d launches of one call)" % launches_per_prefill,
-                     "bound": "hbm", "achieved": ach_gbs, "peak": hbm, "unit": "GB/s",
-                     "frac": ach_gbs / hbm, "traffic": PREFILL_CALL_DRAM_BYTES,
-                     "traffic_note": "ncu dram bytes of the call's 4 launches, each from a cold L2",
-                     "peak_source": pk_kind,
-                     "algorithmic_bytes": pbytes, "algorithmic_flops": pflops,
-                     "tensor_frac": (pflops / (ms_prefill * 1e-3) / 1e12) / pk["bf16_tflops"]},
-        "decode": {"metric": "decode tokens/s (64 sequences x 16 heads, one token each)",
-                   "value": aggregate_throughput(dw.num_seqs, world, ms_decode), "unit": "tokens/s",
-                   "ms_per_step": ms_decode,
-                   "roofline": {"kernel": "gdn_decode_kernel", "bound": "hbm",
-                                "achieved": d_gbs, "peak": hbm, "unit": "GB/s",
-                                "frac": d_gbs / hbm, "traffic": None,
-                                "algorithmic_bytes": dbytes}},
+        "roofline": hbm_roofline(prefill_kernel % launches_per_prefill, pbytes, ms_prefill,
+                                 traffic=measured_traffic("prefill_bf16_call", "prefill"),
+                                 traffic_note="ncu dram bytes of one call's launches, each from a cold L2",
+                                 algorithmic_flops=pflops, tensor_frac=tensor_frac(pflops, ms_prefill)),
+        "long_prefill": {
+            "metric": "prefill tokens/s, 262144 tokens x 16 heads in one call",
+            "value": aggregate_throughput(LT, world, ms_long), "unit": "tokens/s", "ms_per_step": ms_long,
+            "roofline": hbm_roofline(prefill_kernel % l_launch_whole, lbytes, ms_long,
+                                     traffic=measured_traffic("long_prefill_call", "prefill"),
+                                     algorithmic_flops=prefill_flops(LT, H, dk),
+                                     tensor_frac=tensor_frac(prefill_flops(LT, H, dk), ms_long)),
+            "segmented": {"metric": "the same tokens as 64 calls of 4096 with the state carried",
+                          "value": aggregate_throughput(LT, world, ms_long_seg), "unit": "tokens/s",
+                          "ms_per_step": ms_long_seg,
+                          "roofline": hbm_roofline("gdn_prefill x %d calls" % lw.segments, lseg_bytes,
+                                                   ms_long_seg)},
+            "l2": "not flushed: the inputs (3.2 GB) exceed the L2"},
+        "varlen": {
+            "metric": "packed prefill tokens/s, %d sequences (lengths uniform in [1024, 32768], %d tokens) x 16 "
+                      "heads, per-sequence initial states" % (VN, VT),
+            "value": aggregate_throughput(VT, world, ms_varlen), "unit": "tokens/s", "ms_per_step": ms_varlen,
+            "roofline": hbm_roofline(prefill_kernel % v_launch, vbytes, ms_varlen,
+                                     traffic=measured_traffic("varlen_call", "prefill"),
+                                     algorithmic_flops=prefill_flops(VT, H, dk),
+                                     tensor_frac=tensor_frac(prefill_flops(VT, H, dk), ms_varlen)),
+            "l2": "not flushed: the inputs (%.0f MB) exceed the L2" % (VT * H * (2 * dk + dv) * 2 / 1e6)},
+        "decode": {
+            "metric": "decode tokens/s: 1024 one-token steps of 64 sequences x 16 heads in one CUDA graph, "
+                      "state ping-ponged between two buffers (128 MiB, larger than the L2)",
+            "value": aggregate_throughput(dw.num_seqs * nsteps, world, ms_dec_pp), "unit": "tokens/s",
+            "ms_per_graph": ms_dec_pp, "us_per_step": 1e3 * ms_dec_pp / nsteps,
+            "roofline": hbm_roofline("gdn_decode_kernel", dbytes, ms_dec_pp,
+                                     traffic=measured_traffic("decode_pingpong_1024", "decode")),
+            "timing": "median of %d graph replays" % KG},
+        "decode_inplace": {
+            "metric": "the same 1024 steps updating one 64 MiB state in place",
+            "value": aggregate_throughput(dw.num_seqs * nsteps, world, ms_dec_ip), "unit": "tokens/s",
+            "ms_per_graph": ms_dec_ip, "us_per_step": 1e3 * ms_dec_ip / nsteps,
+            "roofline": hbm_roofline("gdn_decode_kernel", dbytes, ms_dec_ip,
+                                     traffic=measured_traffic("decode_inplace_1024", "decode"),
+                                     note="part of the state can stay in the 126 MB L2 between steps")},
         "preprocess": {"metric": "pre-processing tokens/s (conv4 + SiLU + q/k L2 norm + gates), prefill shapes",
                        "value": aggregate_throughput(T, world, ms_pre), "unit": "tokens/s", "ms_per_step": ms_pre,
-                       "roofline": {"kernel": "gdn_preprocess_kernel", "bound": "hbm",
-                                    "achieved": pre_bytes / (ms_pre * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
-                                    "frac": pre_bytes / (ms_pre * 1e-3) / 1e9 / hbm, "traffic": None,
-                                    "algorithmic_bytes": pre_bytes}},
+                       "roofline": hbm_roofline("gdn_preprocess_kernel", pre_bytes, ms_pre)},
         "output_gate": {"metric": "output gate tokens/s (RMS norm + sigmoid gate), prefill shapes",
                         "value": aggregate_throughput(T, world, ms_gate), "unit": "tokens/s", "ms_per_step": ms_gate,
-                        "roofline": {"kernel": "gdn_output_gate_kernel", "bound": "hbm",
-                                     "achieved": gate_bytes / (ms_gate * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
-                                     "frac": gate_bytes / (ms_gate * 1e-3) / 1e9 / hbm, "traffic": None,
-                                     "algorithmic_bytes": gate_bytes}},
+                        "roofline": hbm_roofline("gdn_output_gate_kernel", gate_bytes, ms_gate)},
         "streaming": {"metric": "GDN layer frames/s: pre-processing + recurrence with carried state + "
                                 "output gate per %d-token frame x %d heads, CUDA-graph replay" % (FRAME, H),
                       "value": 1e3 / ms_frame_graph * world, "unit": "frames/s",
@@ -409,19 +581,31 @@ def run_native(args):
                 "ms_per_step": ms_swa_layer, "attention_ms": ms_swa_attn,
                 "roofline": {"kernel": "swa_fwd_pair_kernel", "bound": "tensor", "achieved": swa_tf,
                              "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": swa_tf / pk["bf16_tflops"],
-                             "traffic": SWA_LAUNCH_DRAM_BYTES, "algorithmic_flops": swa_flops},
+                             "traffic": measured_traffic("swa_T32768_W8192", "swa"),
+                             "peak_source": pk_kind, "algorithmic_flops": swa_flops},
                 "l2": "flushed before every step"},
         "e2e": {"value": aggregate_throughput(T, world, ms_e2e), "unit": "tokens/s",
                 "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": (K * launches_per_prefill + K + max(3, K // 10) * launches_per_prefill + 2 * K
-                         + 2 * K * frame_launches + K * decode_launches + K + 3 * K),
+        "gpu_launches": sum(launches.values()),
+        "gpu_launches_by_leg": launches,
         "clocks": clk.summary(),
         "timed_wall_s": wall,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    leg_keys = {"long_prefill": "long_prefill", "varlen": "varlen", "decode": "decode",
+                "decode_inplace": "decode", "preprocess": "layer", "output_gate": "layer",
+                "streaming": "streaming", "swa": "swa", "e2e": "e2e"}
+    for key, leg in leg_keys.items():
+        if not want(leg):
+            line.pop(key, None)
+    if not want("prefill"):
+        line["value"] = None
+        line["ms_per_step"] = None
+        line["roofline"] = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and want("prefill"):
         line["cpu_baseline"] = cpu_baseline()
     if rank == 0:
         print(json.dumps(line), flush=True)
+    del graph_pp, graph_ip
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -449,7 +633,7 @@ def cpu_baseline(tokens=8192, target_s=10.0):
         total += time.perf_counter() - t0
         reps += 1
     return {"value": reps * tokens / total, "unit": "tokens/s", "cores": min(n, PREFILL.H),
-            "kind": "oracle",
+            "host_cores": os.cpu_count(), "kind": "oracle",
             "sample": "full prefill_bf16 workload (%d tokens x 16 heads) run %d times, %.1f s; "
                       "threads over the 16 (sequence, head) units" % (tokens, reps, total)}
 
@@ -482,7 +666,7 @@ def run_reference(args):
         "config": {"workload": "prefill_bf16: B=1, H=16, T=8192, d_k=d_v=128, chunk=64 "
                                "(bounded sample per step)", "seq_len": tokens},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": min(n, PREFILL.H),
-                         "kind": "oracle", "sample": sample},
+                         "host_cores": os.cpu_count(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
@@ -497,6 +681,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--legs", default="",
+                    help="comma-separated subset of %s (default: all); for profiling one workload" % (ALL_LEGS,))
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

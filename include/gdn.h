@@ -166,6 +166,18 @@ int gdn_prefill_noalloc(const void *q, const void *k, const void *v, const float
                         int64_t total_tokens, int H, int dk, int dv, int chunk,
                         int dtype, void *stream);
 
+/*
+ * Status word of gdn_prefill_noalloc on the current device.  The tensor-core
+ * kernels of a no-alloc call record a wait that gave up in the first int32 of
+ * the library's scratch array, whose address callers cannot see; this reads
+ * that word exactly as gdn_read_status reads a caller's workspace: it waits
+ * for `stream`, returns GDN_OK when the word is 0 and GDN_ERR_TIMEOUT
+ * otherwise, and stores the word in *code (may be NULL).  Read it before the
+ * next no-alloc call on the device, which clears the word.  Like the
+ * no-alloc call itself it allocates nothing; it synchronises with `stream`.
+ */
+int gdn_noalloc_read_status(void *stream, int32_t *code);
+
 /* Static, human-readable name of a gdn_status value. */
 const char *gdn_status_string(int status);
 

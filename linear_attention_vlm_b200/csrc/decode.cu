@@ -129,8 +129,6 @@ gdn_decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
 
 }  // namespace
 
-// Variant selector, also used by the tuning harness: unr in {1,2,4,8}
-// (dividing the pass count), nw in {4,8}, coal in {0,1}.
 template <typename T, int D, int UNR, int NW, bool COAL>
 static cudaError_t launch_decode_v(const void *q, const void *k, const void *v, const float *g,
                                    const float *beta, const float *state_in, float *state_out,
@@ -142,25 +140,12 @@ static cudaError_t launch_decode_v(const void *q, const void *k, const void *v, 
     return cudaGetLastError();
 }
 
-cudaError_t launch_decode_variant(int variant, int dtype, int dk, const void *q, const void *k,
-                                  const void *v, const float *g, const float *beta,
-                                  const float *state_in, float *state_out, void *out, int B, int H,
-                                  cudaStream_t stream) {
+cudaError_t launch_decode(int dtype, int dk, const void *q, const void *k, const void *v,
+                          const float *g, const float *beta, const float *state_in,
+                          float *state_out, void *out, int B, int H, cudaStream_t stream) {
 #define GDN_DEC(T, D, U, W, C) \
     return launch_decode_v<T, D, U, W, C>(q, k, v, g, beta, state_in, state_out, out, B, H, stream)
-    if (dtype == 1 && dk == 128) {
-        switch (variant) {
-            case 0: GDN_DEC(__nv_bfloat16, 128, 4, 4, false);
-            case 1: GDN_DEC(__nv_bfloat16, 128, 4, 4, true);
-            case 2: GDN_DEC(__nv_bfloat16, 128, 2, 4, true);
-            case 3: GDN_DEC(__nv_bfloat16, 128, 2, 8, true);
-            case 4: GDN_DEC(__nv_bfloat16, 128, 4, 8, true);
-            case 5: GDN_DEC(__nv_bfloat16, 128, 1, 8, true);
-            case 6: GDN_DEC(__nv_bfloat16, 128, 8, 4, true);
-            default: break;
-        }
-    }
-    // defaults, from a sweep on B200 (64 x 16 heads, L2 flushed): coalesced
+    // from a sweep on B200 (64 sequences x 16 heads, L2 flushed): coalesced
     // 128-byte row pieces, 8 warps, 4 passes in flight
     if (dtype == 0) {
         if (dk == 128) GDN_DEC(float, 128, 4, 8, true);
@@ -169,13 +154,6 @@ cudaError_t launch_decode_variant(int variant, int dtype, int dk, const void *q,
     if (dk == 128) GDN_DEC(__nv_bfloat16, 128, 4, 8, true);
     GDN_DEC(__nv_bfloat16, 64, 2, 4, true);
 #undef GDN_DEC
-}
-
-cudaError_t launch_decode(int dtype, int dk, const void *q, const void *k, const void *v,
-                          const float *g, const float *beta, const float *state_in,
-                          float *state_out, void *out, int B, int H, cudaStream_t stream) {
-    return launch_decode_variant(-1, dtype, dk, q, k, v, g, beta, state_in, state_out, out, B, H,
-                                 stream);
 }
 
 }  // namespace gdn

@@ -63,3 +63,13 @@ extern "C" int gdn_prefill_noalloc(const void *q, const void *k, const void *v, 
                        total_tokens, H, dk, dv, chunk, dtype, ws, need > 0 ? kScratchBytes : 0,
                        stream);
 }
+
+extern "C" int gdn_noalloc_read_status(void *stream, int32_t *code) {
+    if (code) *code = 0;
+    void *ws = nullptr;
+    const int st = scratch_on_current_device(&ws);
+    if (st != GDN_OK) return st;
+    // the status word is the first int32 of the scratch, as it is the first
+    // int32 of a caller-owned workspace for gdn_prefill
+    return gdn_read_status(static_cast<const int32_t *>(ws), stream, code);
+}

@@ -87,6 +87,8 @@ def _load():
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_read_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int32)]
     lib.gdn_read_status.restype = i32
+    lib.gdn_noalloc_read_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
+    lib.gdn_noalloc_read_status.restype = i32
     lib.gdn_last_cuda_error.argtypes = []
     lib.gdn_last_cuda_error.restype = ctypes.c_char_p
     _lib = lib
@@ -240,6 +242,20 @@ def gdn_prefill_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: to
     if st != GDN_OK:
         raise GdnError(st, "gdn_prefill_noalloc")
     return out, state_out
+
+
+def gdn_noalloc_read_status(device=None) -> int:
+    """Wait for the current stream and return the status word that
+    gdn_prefill_noalloc's kernels leave in the library's scratch on
+    ``device`` (include/gdn.h, gdn_noalloc_read_status): 0 when every wait
+    inside them completed, else the kernel's code."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    code = ctypes.c_int32(0)
+    with torch.cuda.device(dev):
+        st = _load().gdn_noalloc_read_status(_stream(dev), ctypes.byref(code))
+    if st not in (GDN_OK, GDN_ERR_TIMEOUT):
+        raise GdnError(st, "gdn_noalloc_read_status")
+    return int(code.value)
 
 
 def gdn_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,

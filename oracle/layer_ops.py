@@ -4,7 +4,7 @@ one layer -- TEST INFRASTRUCTURE ONLY (same rules as the rest of ``oracle``).
 The explainer page (InfiniteVL, "Step 2: Process tokens with Hybrid Blocks")
 states that every Gated DeltaNet layer has 16 heads, a 1-D convolution of
 window 4 and an output gate.  It fixes nothing else, so the plainest readings
-are taken (and listed in the design notes):
+are taken:
 
 * pre-processing (``preprocess``): a causal depthwise convolution of window 4
   over each of the q, k and v channels, restarted at every sequence start

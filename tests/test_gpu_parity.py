@@ -144,8 +144,11 @@ def test_long_prefill_segmented(cuda_device):
     # Segmented and whole runs agree.  Not bit for bit: a long sequence is cut
     # into sequence-parallel chunk ranges, and a 4096-token segment is cut at
     # other places than the whole run, so bf16 operand roundings differ.
-    assert rel_err(np64(st), np64(st_whole)) <= 2e-2
-    assert rel_err(np64(outs[-1]), np64(out_whole[-64:])) <= 2e-2
+    gap_s = rel_err(np64(st), np64(st_whole))
+    gap_o = rel_err(np64(outs[-1]), np64(out_whole[-64:]))
+    print("segmented vs whole: state gap %.3g, last-chunk output gap %.3g" % (gap_s, gap_o))
+    assert gap_s <= 2e-2
+    assert gap_o <= 2e-2
     heads = [5]
     sub = W.prefill_inputs(w, seed=0, heads=heads)
     ro, rs = run_oracle(sub)

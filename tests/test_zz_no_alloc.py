@@ -44,6 +44,31 @@ def test_noalloc_matches_prefill_on_two_calls(cuda_device):
     e2 = _one_call(cuda_device, [600], 16, 0.0, seed=22)
     for eo, es in (e1, e2):
         assert eo <= TOL and es <= TOL, (e1, e2)
+    # the kernels' status word lives in the scratch, out of the caller's
+    # sight; the accessor reads it: every wait of the two calls completed
+    assert gdn.gdn_noalloc_read_status() == 0
+
+
+def _largest_fitting_tokens(H):
+    """Longest single sequence of H heads whose workspace fits the scratch."""
+    best = 0
+    for T in range(256, 262145, 256):
+        if gdn.gdn_prefill_workspace_size(1, T, H, 128, 128) <= binding.NOALLOC_SCRATCH_BYTES:
+            best = T
+    return best
+
+
+def test_noalloc_near_the_scratch_limit(cuda_device):
+    # one long sequence of 16 heads, as long as the scratch allows: few
+    # sequences of many chunks take the sequence-parallel chunk ranges, so
+    # the range transitions and start states sit near the end of the array
+    H = 16
+    T = _largest_fitting_tokens(H)
+    need = gdn.gdn_prefill_workspace_size(1, T, H, 128, 128)
+    assert T >= 1024 and binding.NOALLOC_SCRATCH_BYTES // 2 < need <= binding.NOALLOC_SCRATCH_BYTES
+    eo, es = _one_call(cuda_device, [T], H, 0.02, seed=23)
+    assert eo <= TOL and es <= TOL, (T, eo, es)
+    assert gdn.gdn_noalloc_read_status() == 0
 
 
 def test_noalloc_rejects_requests_beyond_the_scratch(cuda_device):

@@ -26,7 +26,9 @@ full-size workloads.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
+import os
 from typing import Dict, Optional, Sequence
 
 import numpy as np
@@ -112,16 +114,31 @@ def seqlens(w: Workload, seed: int = 0) -> np.ndarray:
     return np.full(w.num_seqs, w.T, dtype=np.int64)
 
 
+def _workers() -> int:
+    return max(1, min(16, os.cpu_count() or 1))
+
+
 def _token_tensor(seed: int, tid: int, T: int, heads: Sequence[int], d: int,
                   unit: bool, dtype: torch.dtype) -> torch.Tensor:
     out = torch.empty((T, len(heads), d), dtype=dtype)
-    for j, h in enumerate(heads):
-        for b0 in range(0, T, BLOCK):
-            n = min(BLOCK, T - b0)
-            x = _rng(seed, tid, h, b0 // BLOCK).standard_normal((n, d), dtype=np.float32)
-            if unit:
-                x = _unit_rows(x)
-            out[b0:b0 + n, j, :] = _round(x, dtype)
+
+    def fill(job):
+        j, h, b0 = job
+        n = min(BLOCK, T - b0)
+        x = _rng(seed, tid, h, b0 // BLOCK).standard_normal((n, d), dtype=np.float32)
+        if unit:
+            x = _unit_rows(x)
+        out[b0:b0 + n, j, :] = _round(x, dtype)
+
+    # every (head, block) has its own stream and its own slice of `out`, so
+    # the blocks are drawn on a thread pool; the result does not depend on it
+    jobs = [(j, h, b0) for j, h in enumerate(heads) for b0 in range(0, T, BLOCK)]
+    if len(jobs) > 8:
+        with concurrent.futures.ThreadPoolExecutor(_workers()) as ex:
+            list(ex.map(fill, jobs))
+    else:
+        for job in jobs:
+            fill(job)
     return out
 
 
