@@ -551,15 +551,15 @@ def run_native(args):
                       "state ping-ponged between two buffers (128 MiB, larger than the L2)",
             "value": aggregate_throughput(dw.num_seqs * nsteps, world, ms_dec_pp), "unit": "tokens/s",
             "ms_per_graph": ms_dec_pp, "us_per_step": 1e3 * ms_dec_pp / nsteps,
-            "roofline": hbm_roofline("gdn_decode_kernel", dbytes, ms_dec_pp,
-                                     traffic=measured_traffic("decode_pingpong_1024", "decode")),
+            "roofline": hbm_roofline("gdn_decode_kernel (per step)", dbytes // nsteps, ms_dec_pp / nsteps,
+                                     traffic=measured_traffic("decode_pingpong_step", "decode")),
             "timing": "median of %d graph replays" % KG},
         "decode_inplace": {
             "metric": "the same 1024 steps updating one 64 MiB state in place",
             "value": aggregate_throughput(dw.num_seqs * nsteps, world, ms_dec_ip), "unit": "tokens/s",
             "ms_per_graph": ms_dec_ip, "us_per_step": 1e3 * ms_dec_ip / nsteps,
-            "roofline": hbm_roofline("gdn_decode_kernel", dbytes, ms_dec_ip,
-                                     traffic=measured_traffic("decode_inplace_1024", "decode"),
+            "roofline": hbm_roofline("gdn_decode_kernel (per step)", dbytes // nsteps, ms_dec_ip / nsteps,
+                                     traffic=measured_traffic("decode_inplace_step", "decode"),
                                      note="part of the state can stay in the 126 MB L2 between steps")},
         "preprocess": {"metric": "pre-processing tokens/s (conv4 + SiLU + q/k L2 norm + gates), prefill shapes",
                        "value": aggregate_throughput(T, world, ms_pre), "unit": "tokens/s", "ms_per_step": ms_pre,

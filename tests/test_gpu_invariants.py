@@ -75,6 +75,9 @@ IDS = ["tc-packed", "tc-ranges", "f32"]
 def test_beta_zero_only_decays(cuda_device, lens, H, d, dtype, unpacked):
     inp = W.random_prefill(lens, H=H, dk=d, dv=d, dtype=dtype, seed=31, state_std=0.5)
     inp["beta"].zero_()
+    # milder gates, so that the decay over 4096 tokens (exp(sum g)) stays
+    # inside the fp32 range the kernels keep the state in
+    inp["g"].mul_(0.1)
     out, st = run(inp, cuda_device, cu=not unpacked)
     cu = inp["cu_seqlens"].numpy()
     g = np64(inp["g"])
