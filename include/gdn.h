@@ -196,6 +196,21 @@ const char *gdn_status_string(int status);
  */
 int gdn_read_status(const int32_t *word, void *stream, int32_t *code);
 
+/*
+ * Test hook of those bounded waits.  Sets, for the calling host thread, the
+ * bound on the waits of the work loops of the tensor-core kernels that its
+ * later calls launch (gdn_prefill, gdn_prefill_noalloc, gdn_swa_attention,
+ * and the prefill steps a session captures).  With ns = 0 a wait gives up as
+ * soon as the phase it waits for is not already complete, so a call's first
+ * wait on a copy or an MMA in flight gives up; GDN_WAIT_LIMIT_DEFAULT
+ * restores the 2 s default.  Whatever the bound, the waits that drain a
+ * kernel's copies and MMAs before it exits keep 2 s: a kernel whose waits
+ * gave up records its code in the status word and returns with no work in
+ * flight and its outputs invalid, and later calls on the device run normally.
+ */
+#define GDN_WAIT_LIMIT_DEFAULT ((uint64_t)2000000000)
+void gdn_set_wait_limit(uint64_t ns);
+
 /* Text of the most recent CUDA error seen by this host thread inside the
  * library ("" if none).  Valid until the next call on this thread. */
 const char *gdn_last_cuda_error(void);

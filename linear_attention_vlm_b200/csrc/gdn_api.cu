@@ -31,7 +31,11 @@ bool use_tc(int64_t total_tokens, int dk, int dtype) {
     return dtype == GDN_BF16 && dk == 128 && total_tokens > 0;
 }
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s bound on any in-kernel wait
+constexpr uint64_t kWaitLimitNs = GDN_WAIT_LIMIT_DEFAULT;   // 2 s bound on any in-kernel wait
+
+// Bound on the work-loop waits of the kernels this host thread launches
+// (gdn_set_wait_limit); the drains before a kernel exits always keep 2 s.
+thread_local uint64_t g_wait_limit_ns = kWaitLimitNs;
 
 // Common validation of gdn_prefill's arguments (without workspace).
 int check_prefill(const void *q, const void *k, const void *v, const float *g,
@@ -83,6 +87,8 @@ const char *gdn_status_string(int status) {
 
 const char *gdn_last_cuda_error(void) { return g_last_cuda_error; }
 
+void gdn_set_wait_limit(uint64_t ns) { g_wait_limit_ns = ns; }
+
 int gdn_read_status(const int32_t *word, void *stream, int32_t *code) {
     if (code) *code = 0;
     if (!word || (reinterpret_cast<uintptr_t>(word) & 3u)) return GDN_ERR_INVALID_ARG;
@@ -132,7 +138,7 @@ int gdn_prefill(const void *q, const void *k, const void *v, const float *g, con
         cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), s);
         if (e != cudaSuccess) return cuda_fail(e);
         gdn::TcLaunch L{q, k, v, g, beta, state_in, out, state_out, cu_seqlens, uniform_len,
-                        total_tokens, num_seqs, H, workspace, err, kWaitLimitNs};
+                        total_tokens, num_seqs, H, workspace, err, g_wait_limit_ns, kWaitLimitNs};
         e = gdn::launch_prefill_tc(L, s);
         return e == cudaSuccess ? GDN_OK : cuda_fail(e);
     }
@@ -284,7 +290,8 @@ int gdn_swa_attention(const void *q, const void *k, const void *v, void *o, cons
     L.Hq = Hq; L.Hkv = Hkv; L.window = window;
     L.scale = scale > 0.f ? scale : 1.f / sqrtf((float)d);
     L.err = status;
-    L.timeout_ns = kWaitLimitNs;
+    L.timeout_ns = g_wait_limit_ns;
+    L.drain_ns = kWaitLimitNs;
     const cudaError_t e = gdn::launch_swa(L, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GDN_OK : cuda_fail(e);
 }

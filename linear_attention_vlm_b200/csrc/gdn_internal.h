@@ -82,7 +82,8 @@ struct SwaLaunch {
     int Hq, Hkv, window;
     float scale;
     int *err;                          // device status word, or null
-    uint64_t timeout_ns;               // bound on every wait inside the kernel
+    uint64_t timeout_ns;               // bound on the waits of the kernel's work loops
+    uint64_t drain_ns;                 // bound on the waits that drain copies and MMAs before exit
 };
 cudaError_t launch_swa(const SwaLaunch &L, cudaStream_t stream);
 cudaError_t swa_setup();

@@ -18,16 +18,20 @@
 //   TMA brings K and Q; p1 = [K;Q] K^T on tcgen05 (TMEM); four warps form A
 //   and Phat, invert I + A (16x16 diagonal blocks by substitution, the
 //   off-diagonal blocks with tf32 mma.sync), scale T' and T''; p2 = K^T T'^T
-//   on tcgen05 gives W^T, which is transposed into W.  W, Qg, T'' and Pt are
-//   written to the workspace in the 128-byte-swizzled layout the chain
-//   kernel's MMAs read, so it copies them with one bulk copy per chunk.
+//   on tcgen05 gives W.  Qg and -W (interleaved per 64-column block, so that
+//   they form one 128-row operand), T'' and Pt are written to the workspace in
+//   the 128-byte-swizzled layout the chain kernel's MMAs read, so it copies
+//   them with one bulk copy per chunk.
 // gdn_chunk_chain_kernel: one CTA per (sequence, head), fp32 state in TMEM:
-//   p3 U^T = V^T T''^T, (a) U^T -= S W^T, (b) S += U^T K, c1 O^T = S Qg^T,
-//   c2 O^T += U^T Pt^T -- five M = 128 tcgen05 MMAs per chunk, the S and U^T
-//   operands read from TMEM -- with a four-warp state group (residual and
-//   state epilogues, the serial chain), a four-warp output group (output
+//   p3 U^T = V^T T''^T, (a + c1) [O^T | U^T] += S [Qg; -W]^T as ONE N = 128
+//   MMA, (b) S += U^T K, c2 O^T += U^T Pt^T -- M = 128 tcgen05 MMAs, the S
+//   and U^T operands read from TMEM -- with a four-warp state group (residual
+//   and state epilogues, the serial chain), a four-warp output group (output
 //   epilogue, off the chain), one MMA thread and one TMA thread.  The state
-//   never leaves the SM between chunks.
+//   never leaves the SM between chunks.  A tcgen05.mma costs its issuing
+//   thread some 60 cycles whatever its width, while an M = 128, N = 64 MMA
+//   computes for 32: merging the two MMAs that share the A operand S into one
+//   of twice the width removes eight issues per chunk.
 //
 // Tokens past the end of a sequence inside its last chunk get g = 0 and
 // beta = 0, which zeroes their rows of W and T'' and keeps the state
@@ -84,24 +88,29 @@ __device__ __forceinline__ float *t_blk(uint8_t *sm, int i, int j) {
 }
 
 // ------------------------------------------------------------ chain kernel layout
-constexpr int kChainThreads = 320;                     // warps 0-3 chain, 4-7 output, 8 MMA, 9 TMA
+constexpr int kChainThreads = 352;                     // warps 0-3 chain, 4-7 output / chain X, 8 MMA, 9 TMA, 10 MMA of chain X
 // Stages of the load pipeline.  An output range needs all of a chunk's data
 // (K, V and the 48 KB prep tile: two stages of 80 KB); a transition range
 // needs K, V, W and T'' only, and runs three stages of 56 KB so that a chunk's
 // loads are issued two chunks ahead.
 template <int MODE> struct ChainLayout;
+// WQ is the tile's [Qg | -W] operand: per 64-column block, 64 rows of Qg then
+// 64 rows of -W (a 128-row K-major operand, blocks 16 KB apart).  A
+// transition range reads -W alone, as 64 rows per block (blocks 8 KB apart).
 template <> struct ChainLayout<0> {   // MODE_OUT
     static constexpr int NST = 2;
     static constexpr uint32_t STAGE = 81920;
-    static constexpr uint32_t K = 0, V = 16384, W = 32768, QG = 49152, TPP = 65536, PT = 73728;
+    static constexpr uint32_t K = 0, V = 16384, WQ = 32768, TPP = 65536, PT = 73728;
 };
 template <> struct ChainLayout<1> {   // MODE_TRANS
     static constexpr int NST = 3;
     static constexpr uint32_t STAGE = 57344;
-    static constexpr uint32_t K = 0, V = 16384, W = 32768, QG = 0, TPP = 49152, PT = 0;
+    static constexpr uint32_t K = 0, V = 16384, W = 32768, TPP = 49152;
 };
 static_assert(ChainLayout<0>::PT + 8192 == ChainLayout<0>::STAGE &&
-              ChainLayout<0>::STAGE - ChainLayout<0>::W == kTileBytes, "stage layout");
+              ChainLayout<0>::STAGE - ChainLayout<0>::WQ == kTileBytes, "stage layout");
+// offsets inside a tile: [Qg | -W] per block (32 KB), T'' (8 KB), Pt (8 KB)
+constexpr uint32_t TILE_NEGW = 8192, TILE_TPP = 32768, TILE_PT = 40960;
 static_assert(ChainLayout<1>::TPP + 8192 == ChainLayout<1>::STAGE, "stage layout");
 // After the stages: output staging [64 t][128 dv] bf16, ChainScalars x 3 per
 // chain, mbarriers + TMEM base + abort flag.
@@ -114,18 +123,21 @@ static_assert(c_alloc<0>() <= 232448 && c_alloc<1>() <= 232448, "chain kernel sh
 // TMEM columns of the chain kernel.  The MMA A operands produced by the chain
 // itself (bf16 S and bf16 U^T) stay in TMEM: shared-memory bandwidth, not the
 // tensor core, bounds these small-N MMAs, so only B is read from shared memory.
-constexpr uint32_t TM_SBF = 0;     // S bf16, two per column (64)
-constexpr uint32_t TM_U = 64;      // U^T accumulator (64); then U^T bf16 in its first 32
-constexpr uint32_t TM_S = 128;     // state S (128)
-constexpr uint32_t TM_O = 256;     // O^T [2 bufs] at 256, 320 (64 each)
-constexpr uint32_t TM_X = 256;     // identity chain (transition ranges): its S bf16, U^T, S at +0, +64, +128
+// O^T sits right before U^T, so that the merged MMA writes [O^T | U^T] as one
+// 128-column accumulator.
+constexpr uint32_t TM_S = 0;       // state S (128)
+constexpr uint32_t TM_O = 128;     // O^T (64)
+constexpr uint32_t TM_U = 192;     // U^T accumulator (64); then U^T bf16 in its first 32
+constexpr uint32_t TM_SBF = 256;   // S bf16, two per column (64)
+// the identity chain of a transition range: its bf16 copy, U^T and state
+constexpr uint32_t TM_XSBF = 128, TM_XU = 320, TM_XS = 384;
 constexpr uint32_t TM_COLS = 512;
 // Barriers that a role may complete twice before its consumer waits once are
-// per buffer (FULL/EMPTY per stage, C/OFREE per output buffer) and waited with
+// per buffer (FULL/EMPTY per stage) and waited with
 // the parity of the buffer's use count, so that no phase can be skipped.
 enum { CB_FULL = 0, CB_EMPTY = 3, CB_A = 6, CB_B = 7, CB_C = 8, CB_SREADY = 10, CB_UREADY = 11,
        CB_FIN = 12, CB_OFREE = 13, CB_A2 = 15, CB_B2 = 16, CB_SREADY2 = 17, CB_UREADY2 = 18,
-       CB_NUM = 19 };   // FULL, EMPTY: one per stage (up to 3); C, OFREE: one per output buffer
+       CB_FIN2 = 19, CB_NUM = 20 };   // FULL, EMPTY: one per stage (up to 3)
 
 struct ChainScalars {   // per chunk, state group
     float gC;           // exp(G_C)
@@ -154,7 +166,8 @@ struct PrepParams {
     int num_seqs, H;
     uint8_t *tiles;
     int *err;
-    uint64_t timeout_ns;
+    uint64_t timeout_ns;         // bound on the waits of the work loops
+    uint64_t drain_ns;           // bound on the waits that drain copies and MMAs before exit
 };
 
 struct ChainParams {
@@ -174,7 +187,8 @@ struct ChainParams {
     int wait_tiles;              // the prep kernel may still run: wait before reading tiles
     int wait_start;              // the combine may still run: wait before reading seg_start
     int *err;
-    uint64_t timeout_ns;
+    uint64_t timeout_ns;         // bound on the waits of the work loops
+    uint64_t drain_ns;           // bound on the waits that drain copies and MMAs before exit
 };
 
 __device__ __forceinline__ uint8_t *aligned_smem(uint8_t *raw) {
@@ -429,7 +443,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
     const int no_abort = 0;   // CTA-local failures end each wait by its own bound
     bool ok = true;
     PrepScalars *sc = reinterpret_cast<PrepScalars *>(sm + P_SC);
-    uint8_t *tile = p.tiles + ((size_t)gc * H + h) * kTileBytes;   // [W 16K][Qg 16K][T'' 8K][Pt 8K]
+    uint8_t *tile = p.tiles + ((size_t)gc * H + h) * kTileBytes;   // [Qg|-W 32K][T'' 8K][Pt 8K]
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     float *mm = reinterpret_cast<float *>(sm + P_MM);          // 4 warps x 16 x 20 fp32
 
@@ -480,7 +494,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
                     const float2 f = __bfloat1622float2(hv[e]);
                     hv[e] = __floats2bfloat162_rn(gr * f.x, gr * f.y);
                 }
-                *reinterpret_cast<uint4 *>(tile + 16384 + kb * 8192 + r * 128 + pc * 16) = v;
+                *reinterpret_cast<uint4 *>(tile + kb * 16384 + r * 128 + pc * 16) = v;
             }
         }
         ok = mbar_wait(bar(PB_P1), 0, lim, &no_abort) && ok;
@@ -561,7 +575,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
         const uint32_t off = r * 128 + pc * 16;
         st_shared_v4(smem_u32(sm + P_TP + off), a0, a1, a2, a3);
         st_shared_v4(smem_u32(sm + P_TP + 8192 + off), a0, a1, a2, a3);
-        *reinterpret_cast<uint4 *>(tile + 32768 + off) = make_uint4(b0, b1, b2, b3);
+        *reinterpret_cast<uint4 *>(tile + TILE_TPP + off) = make_uint4(b0, b1, b2, b3);
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -596,7 +610,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
         }
     }
     {
-        // W row t staged over the T' tile (p2, its last reader, has completed):
+        // -W row t staged over the T' tile (p2, its last reader, has completed):
         // warps 0-1 stage d_k 0..63 (kb 0), warps 2-3 d_k 64..127 (kb 1)
         ok = mbar_wait(bar(PB_P2), 0, lim, &no_abort) && ok;
         tc_fence_after();
@@ -609,20 +623,26 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) {
                 const float *e = y + 8 * c4;
-                st_shared_v4(w_s + sw128_chunk(t, 4 * h2 + c4), pack_bf16(e[0], e[1]), pack_bf16(e[2], e[3]),
-                             pack_bf16(e[4], e[5]), pack_bf16(e[6], e[7]));
+                st_shared_v4(w_s + sw128_chunk(t, 4 * h2 + c4), pack_bf16(-e[0], -e[1]), pack_bf16(-e[2], -e[3]),
+                             pack_bf16(-e[4], -e[5]), pack_bf16(-e[6], -e[7]));
             }
         }
     }
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
-        bulk_store(tile, smem_u32(sm + P_TP), 16384);                // W
-        bulk_store(tile + 40960, smem_u32(sm + P_KQ + 8192), 8192);  // Pt
+        bulk_store(tile + TILE_NEGW, smem_u32(sm + P_TP), 8192);              // -W, first block
+        bulk_store(tile + 16384 + TILE_NEGW, smem_u32(sm + P_TP + 8192), 8192); // -W, second block
+        bulk_store(tile + TILE_PT, smem_u32(sm + P_KQ + 8192), 8192);         // Pt
         bulk_commit_wait_read();
     }
     if (!ok && p.err) atomicCAS(p.err, 0, 52);
-    if (tid == 0) mbar_wait(bar(PB_FULL), 0, lim, &no_abort);   // no TMA copy still landing at exit
+    if (tid == 0) {
+        // no TMA copy still landing and no MMA still running at exit (p2's
+        // commit covers p1 too), whatever became of the waits above
+        mbar_wait(bar(PB_FULL), 0, p.drain_ns, &no_abort);
+        mbar_wait(bar(PB_P2), 0, p.drain_ns, &no_abort);
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -679,9 +699,12 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
     float *finish = MODE == MODE_TRANS ? nullptr : (seg == p.nseg - 1 ? p.state_out : nullptr);
 
     if (tid == 0) {
-        for (int i = 0; i < CB_NUM; ++i)
-            mbar_init(bar(i), (i == CB_SREADY || i == CB_UREADY || i == CB_SREADY2 || i == CB_UREADY2 ||
-                               i == CB_OFREE || i == CB_OFREE + 1) ? 128 : 1);
+        for (int i = 0; i < CB_NUM; ++i) {
+            uint32_t cnt = (i == CB_SREADY || i == CB_UREADY || i == CB_SREADY2 || i == CB_UREADY2 ||
+                            i == CB_OFREE) ? 128 : 1;
+            if (MODE == MODE_TRANS && i >= CB_EMPTY && i < CB_EMPTY + 3) cnt = 2;   // both chains' MMAs
+            mbar_init(bar(i), cnt);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -737,8 +760,8 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                 }
                 const uint8_t *tm_ = p.tiles + ((size_t)(gc0 + m) * H + h) * kTileBytes;
                 if (MODE == MODE_TRANS) {
-                    bulk_prefetch_l2(tm_, 16384);
-                    bulk_prefetch_l2(tm_ + (ChainLayout<0>::TPP - ChainLayout<0>::W), 8192);
+                    bulk_prefetch_l2(tm_ + TILE_NEGW, 8192);
+                    bulk_prefetch_l2(tm_ + 16384 + TILE_NEGW, 16384);   // second -W block and T''
                 } else {
                     bulk_prefetch_l2(tm_, (uint32_t)kTileBytes);
                 }
@@ -753,103 +776,112 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                 }
                 const uint32_t full = bar(CB_FULL + s);
                 const uint8_t *tile = p.tiles + ((size_t)(gc0 + n) * H + h) * kTileBytes;
-                // a transition range reads W and T'' only
+                // a transition range reads -W and T'' only
                 mbar_arrive_expect_tx(full, Lay::STAGE);
                 for (int kb = 0; kb < 2; ++kb) {
                     tma_load_3d(st + Lay::K + kb * 8192, &p.map_k, kb * 64, h, z, full);
                     tma_load_3d(st + Lay::V + kb * 8192, &p.map_v, kb * 64, h, z, full);
                 }
                 if (n == 0 && p.wait_tiles) grid_dep_wait();   // tiles come from the prep kernel
-                if (MODE == MODE_TRANS) {   // W and T'' of the tile
-                    bulk_load(st + Lay::W, tile, 16384, full);
-                    bulk_load(st + Lay::TPP, tile + (ChainLayout<0>::TPP - ChainLayout<0>::W), 8192, full);
+                if (MODE == MODE_TRANS) {   // -W and T'' of the tile
+                    bulk_load(st + ChainLayout<1>::W, tile + TILE_NEGW, 8192, full);
+                    bulk_load(st + ChainLayout<1>::W + 8192, tile + 16384 + TILE_NEGW, 8192, full);
+                    bulk_load(st + ChainLayout<1>::TPP, tile + TILE_TPP, 8192, full);
                 } else {
-                    bulk_load(st + Lay::W, tile, (uint32_t)kTileBytes, full);
+                    bulk_load(st + ChainLayout<0>::WQ, tile, (uint32_t)kTileBytes, full);
                 }
                 ++issued[s];
             }
             const int zero = 0;   // no copy may still be landing in shared memory at exit
             for (int s = 0; s < NST; ++s)
-                if (issued[s]) mbar_wait(bar(CB_FULL + s), (issued[s] - 1) & 1, lim, &zero);
+                if (issued[s]) mbar_wait(bar(CB_FULL + s), (issued[s] - 1) & 1, p.drain_ns, &zero);
         }
-    } else if (warp == 8) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+    } else if (warp == 8 || warp == 10) {
+        // ------------------------------------------------------------ MMA issuers
+        // warp 8: the state chain (p3, the residual and state products and,
+        // for outputs, c1 and c2); warp 10 (MODE_TRANS): the identity chain,
+        // issued alongside so that the two chains' MMA issues overlap
+        const bool xissuer = warp == 10;
+        if (lane == 0 && (!xissuer || MODE == MODE_TRANS)) {
             const uint32_t id_n64 = idesc_bf16(128, 64, false, false);
+            const uint32_t id_n128 = idesc_bf16(128, 128, false, false);
             const uint32_t id_p3 = idesc_bf16(128, 64, true, false);
-            const uint32_t id_a = idesc_bf16(128, 64, false, false, true);
             const uint32_t id_b = idesc_bf16(128, 128, false, true);
-            // descriptors are built once; a byte offset o inside a tile adds o >> 4
+            // descriptors are built once; a byte offset o inside the stages adds o >> 4
             const uint64_t dSTk = desc_sw128(smem_u32(sm), 16, 1024);      // K-major views of stage data
             const uint64_t dSTm = desc_sw128(smem_u32(sm), 8192, 1024);    // MN-major views of K and V
+            const int zero = 0;
             bool ok = true;
-            // (a): U^T (+)= -S W^T for the chain whose tensor memory starts at `base`
-            auto issue_a = [&](uint32_t base, uint32_t st, uint32_t accumulate_first) {
+            // transition ranges: U^T (+)= S (-W)^T, -W as 64 rows per block, 8 KB apart
+            auto issue_a = [&](uint32_t col_u, uint32_t col_sbf, uint32_t st, uint32_t accumulate_first) {
                 for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t offw = st + Lay::W + (ks >> 2) * 8192 + (ks & 3) * 32;
-                    mma_bf16_ts(tm + base + TM_U, tm + base + TM_SBF + 8 * ks, dSTk + (offw >> 4), id_a,
+                    const uint32_t offw = st + ChainLayout<1>::W + (ks >> 2) * 8192 + (ks & 3) * 32;
+                    mma_bf16_ts(tm + col_u, tm + col_sbf + 8 * ks, dSTk + (offw >> 4), id_n64,
                                 ks > 0 ? 1u : accumulate_first);
                 }
             };
             // (b): S += U^T K  (A = U^T bf16 in TMEM; B = K tile MN-major)
-            auto issue_b = [&](uint32_t base, uint32_t st) {
+            auto issue_b = [&](uint32_t col_s, uint32_t col_u, uint32_t st) {
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ts(tm + base + TM_S, tm + base + TM_U + 8 * ks,
-                                dSTm + ((st + Lay::K + ks * 2048) >> 4), id_b, 1);
+                    mma_bf16_ts(tm + col_s, tm + col_u + 8 * ks, dSTm + ((st + Lay::K + ks * 2048) >> 4), id_b, 1);
             };
             for (int n = 0; ok && n < nloc; ++n) {
-                const int s = n % NST, ob = n & 1;   // stage, output buffer
+                const int s = n % NST;
                 const uint32_t st = s * Lay::STAGE;
                 if (!(ok = mbar_wait(bar(CB_FULL + s), (n / NST) & 1, lim, abort_flag))) { fail(62); break; }
                 tc_fence_after();
+                if (MODE == MODE_TRANS && xissuer) {
+                    // chain X: U_X^T = X (-W)^T (no values), then X += U_X^T K
+                    if (!(ok = mbar_wait(bar(CB_SREADY2), n & 1, lim, abort_flag))) { fail(66); break; }
+                    tc_fence_after();
+                    issue_a(TM_XU, TM_XSBF, st, 0);
+                    mma_commit(bar(CB_A2));
+                    if (!(ok = mbar_wait(bar(CB_UREADY2), n & 1, lim, abort_flag))) { fail(67); break; }
+                    tc_fence_after();
+                    issue_b(TM_XS, TM_XU, st);
+                    mma_commit(bar(CB_B2));
+                    mma_commit(bar(CB_EMPTY + s));
+                    continue;
+                }
                 // p3: U^T = V^T T''^T (the previous residual was consumed: U_READY(n-1))
                 for (int ks = 0; ks < 4; ++ks)
                     mma_bf16_ss(tm + TM_U, dSTm + ((st + Lay::V + ks * 2048) >> 4),
                                 dSTk + ((st + Lay::TPP + ks * 32) >> 4), id_p3, ks > 0);
                 if (!(ok = mbar_wait(bar(CB_SREADY), n & 1, lim, abort_flag))) { fail(63); break; }
+                // the output group has read O^T of chunk n-1 and cleared it
+                if (MODE == MODE_OUT && !(ok = mbar_wait(bar(CB_OFREE), n & 1, lim, abort_flag))) { fail(65); break; }
                 tc_fence_after();
-                issue_a(0, st, 1);
-                mma_commit(bar(CB_A));
                 if (MODE == MODE_TRANS) {
-                    if (!(ok = mbar_wait(bar(CB_SREADY2), n & 1, lim, abort_flag))) { fail(66); break; }
-                    tc_fence_after();
-                    issue_a(TM_X, st, 0);   // U_X^T = -X W^T (no values)
-                    mma_commit(bar(CB_A2));
+                    issue_a(TM_U, TM_SBF, st, 1);
+                    mma_commit(bar(CB_A));
                     if (!(ok = mbar_wait(bar(CB_UREADY), n & 1, lim, abort_flag))) { fail(64); break; }
                     tc_fence_after();
-                    issue_b(0, st);
+                    issue_b(TM_S, TM_U, st);
                     mma_commit(bar(CB_B));
-                    if (!(ok = mbar_wait(bar(CB_UREADY2), n & 1, lim, abort_flag))) { fail(67); break; }
-                    tc_fence_after();
-                    issue_b(TM_X, st);
-                    mma_commit(bar(CB_B2));
                     mma_commit(bar(CB_EMPTY + s));
                 } else {
-                    // the output group has read this output buffer for chunk n-2
-                    if (n >= 2 && !(ok = mbar_wait(bar(CB_OFREE + ob), ((n - 2) >> 1) & 1, lim, abort_flag))) { fail(65); break; }
-                    tc_fence_after();
-                    // c1: O^T = S Qg^T (off the state chain)
+                    // (a) and c1 share A = S: [O^T | U^T] += S [Qg; -W]^T as one N = 128 MMA per
+                    // K step (O^T starts cleared, U^T holds p3)
                     for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t off = st + Lay::QG + (ks >> 2) * 8192 + (ks & 3) * 32;
-                        mma_bf16_ts(tm + TM_O + ob * 64, tm + TM_SBF + 8 * ks, dSTk + (off >> 4), id_n64, ks > 0);
+                        const uint32_t off = st + ChainLayout<0>::WQ + (ks >> 2) * 16384 + (ks & 3) * 32;
+                        mma_bf16_ts(tm + TM_O, tm + TM_SBF + 8 * ks, dSTk + (off >> 4), id_n128, 1);
                     }
+                    mma_commit(bar(CB_A));
                     if (!(ok = mbar_wait(bar(CB_UREADY), n & 1, lim, abort_flag))) { fail(64); break; }
                     tc_fence_after();
-                    issue_b(0, st);
+                    issue_b(TM_S, TM_U, st);
                     mma_commit(bar(CB_B));
                     // c2: O^T += U^T Pt^T
                     for (int ks = 0; ks < 4; ++ks)
-                        mma_bf16_ts(tm + TM_O + ob * 64, tm + TM_U + 8 * ks, dSTk + ((st + Lay::PT + ks * 32) >> 4),
-                                    id_n64, 1);
-                    mma_commit(bar(CB_C + ob));
+                        mma_bf16_ts(tm + TM_O, tm + TM_U + 8 * ks,
+                                    dSTk + ((st + ChainLayout<0>::PT + ks * 32) >> 4), id_n64, 1);
+                    mma_commit(bar(CB_C));
                     mma_commit(bar(CB_EMPTY + s));
                 }
             }
-            mma_commit(bar(CB_FIN));   // every issued MMA completes before TMEM is released
-            if (!mbar_wait(bar(CB_FIN), 0, lim, abort_flag)) {
-                const int zero = 0;
-                mbar_wait(bar(CB_FIN), 0, lim, &zero);
-            }
+            const int fin = xissuer ? CB_FIN2 : CB_FIN;
+            mma_commit(bar(fin));   // every issued MMA completes before TMEM is released
+            mbar_wait(bar(fin), 0, p.drain_ns, &zero);
         }
     } else if (warp < 4 || MODE == MODE_TRANS) {
         // ------------------------------------------------------------ state group(s)
@@ -858,7 +890,8 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
         const int wg = warp & 3;
         const int dv = tid & 127;   // TMEM lane and state row
         const uint32_t lane_off = static_cast<uint32_t>(wg * 32) << 16;
-        const uint32_t base = xchain ? TM_X : 0;
+        const uint32_t col_u = xchain ? TM_XU : TM_U, col_s = xchain ? TM_XS : TM_S;
+        const uint32_t col_sbf = xchain ? TM_XSBF : TM_SBF;
         const int bA = xchain ? CB_A2 : CB_A, bB = xchain ? CB_B2 : CB_B;
         const int bS = xchain ? CB_SREADY2 : CB_SREADY, bU = xchain ? CB_UREADY2 : CB_UREADY;
         const int nb = xchain ? 3 : 2;    // named barrier of this group
@@ -883,7 +916,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                 pk[j] = pack_bf16(x0[2 * j], x0[2 * j + 1]);
                 pk[16 + j] = pack_bf16(x1[2 * j], x1[2 * j + 1]);
             }
-            tmem_st32u(tm + lane_off + base + col, pk);
+            tmem_st32u(tm + lane_off + col, pk);
         };
         compute_scalars(0);
         if (MODE == MODE_OUT && seg > 0 && p.wait_start) grid_dep_wait();   // start state from the combine
@@ -911,11 +944,11 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                         x1[j] = (dv == c0 + 32 + j) ? 1.f : 0.f;
                     }
                 }
-                st_bf16_cols(TM_SBF + c0 / 2, x0, x1);
+                st_bf16_cols(col_sbf + c0 / 2, x0, x1);
 #pragma unroll
                 for (int j = 0; j < 32; ++j) { x0[j] *= gC0; x1[j] *= gC0; }
-                tmem_st32(tm + lane_off + base + TM_S + c0, x0);
-                tmem_st32(tm + lane_off + base + TM_S + c0 + 32, x1);
+                tmem_st32(tm + lane_off + col_s + c0, x0);
+                tmem_st32(tm + lane_off + col_s + c0 + 32, x1);
             }
             tc_fence_before();
             mbar_arrive(bar(bS));
@@ -926,9 +959,9 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
             tc_fence_after();
             {
                 float x0[32], x1[32];
-                tmem_ld32(tm + lane_off + base + TM_U, x0);
-                tmem_ld32(tm + lane_off + base + TM_U + 32, x1);
-                st_bf16_cols(TM_U, x0, x1);
+                tmem_ld32(tm + lane_off + col_u, x0);
+                tmem_ld32(tm + lane_off + col_u + 32, x1);
+                st_bf16_cols(col_u, x0, x1);
             }
             tc_fence_before();
             mbar_arrive(bar(bU));
@@ -941,10 +974,10 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
             {
                 float x0[32], x1[32];
                 for (int c0 = 0; c0 < D; c0 += 64) {
-                    tmem_ld32(tm + lane_off + base + TM_S + c0, x0);
-                    tmem_ld32(tm + lane_off + base + TM_S + c0 + 32, x1);
+                    tmem_ld32(tm + lane_off + col_s + c0, x0);
+                    tmem_ld32(tm + lane_off + col_s + c0 + 32, x1);
                     if (!last) {
-                        st_bf16_cols(TM_SBF + c0 / 2, x0, x1);
+                        st_bf16_cols(col_sbf + c0 / 2, x0, x1);
                     }   // the last state stays in TMEM; it leaves at teardown (coalesced)
                 }
                 tc_fence_before();
@@ -954,10 +987,10 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                     mbar_arrive(bar(bS));
                     const float gnext = scb[(n + 1) % 3].gC;
                     for (int c0 = 0; c0 < D; c0 += 32) {
-                        tmem_ld32(tm + lane_off + base + TM_S + c0, x0);
+                        tmem_ld32(tm + lane_off + col_s + c0, x0);
 #pragma unroll
                         for (int j = 0; j < 32; ++j) x0[j] *= gnext;
-                        tmem_st32(tm + lane_off + base + TM_S + c0, x0);
+                        tmem_st32(tm + lane_off + col_s + c0, x0);
                     }
                     tc_fence_before();
                 }
@@ -969,17 +1002,30 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
         const int dv = tid - 128;   // TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>((warp - 4) * 32) << 16;
         __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(sm + c_u<MODE>());
+        float a[32], b[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) a[j] = 0.f;
+        // O^T starts cleared: the merged MMA accumulates c1 onto it
+        tmem_st32(tm + lane_off + TM_O, a);
+        tmem_st32(tm + lane_off + TM_O + 32, a);
+        tc_fence_before();
+        mbar_arrive(bar(CB_OFREE));
         for (int n = 0; n < nloc; ++n) {
-            const int s = n & 1;
             // all four warps are done with chunk n-1's staging buffer
             if (named_bar_any(3, 128, *abort_flag != 0)) break;
-            if (!mbar_wait(bar(CB_C + s), (n >> 1) & 1, lim, abort_flag)) fail(73);
+            if (!mbar_wait(bar(CB_C), n & 1, lim, abort_flag)) fail(73);
             tc_fence_after();
-            float a[32], b[32];
-            tmem_ld32(tm + lane_off + TM_O + s * 64, a);
-            tmem_ld32(tm + lane_off + TM_O + s * 64 + 32, b);
+            tmem_ld32(tm + lane_off + TM_O, a);
+            tmem_ld32(tm + lane_off + TM_O + 32, b);
+            {
+                float z[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) z[j] = 0.f;
+                tmem_st32(tm + lane_off + TM_O, z);
+                tmem_st32(tm + lane_off + TM_O + 32, z);
+            }
             tc_fence_before();
-            mbar_arrive(bar(CB_OFREE + s));   // the MMA thread may reuse this buffer
+            mbar_arrive(bar(CB_OFREE));   // the MMA thread may accumulate chunk n+1's O^T
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 stage[j * D + dv] = __float2bfloat16_rn(a[j]);
@@ -1023,7 +1069,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                 const int row = (warp & 3) * 32 + lane;
                 for (int c0 = 0; c0 < D; c0 += 32) {
                     float x[32];
-                    tmem_ld32(tm + lane_off + (c ? TM_X : 0) + TM_S + c0, x);
+                    tmem_ld32(tm + lane_off + (c ? TM_XS : TM_S) + c0, x);
 #pragma unroll
                     for (int j = 0; j < 32; j += 4)
                         *reinterpret_cast<float4 *>(stg + row * PITCH + c0 + j) = make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
@@ -1324,6 +1370,7 @@ cudaError_t launch_prefill_tc(const TcLaunch &L, cudaStream_t stream) {
     cp.tiles = tiles;
     pp.err = cp.err = L.err;
     pp.timeout_ns = cp.timeout_ns = L.timeout_ns;
+    pp.drain_ns = cp.drain_ns = L.drain_ns;
     cp.state_in = L.state_in;
     cp.state_out = L.state_out;
     cp.out = static_cast<__nv_bfloat16 *>(L.out);

@@ -25,7 +25,8 @@ struct TcLaunch {
     int num_seqs, H;
     void *workspace;             // tc_workspace_bytes(...) bytes, 16-byte aligned
     int *err;                    // device status word (0 = ok)
-    uint64_t timeout_ns;         // bound on every wait inside the kernels
+    uint64_t timeout_ns;         // bound on the waits of the kernels' work loops
+    uint64_t drain_ns;           // bound on the waits that drain copies and MMAs before exit
 };
 
 // Upper bound on the number of 64-token chunks of a packed batch.

@@ -69,13 +69,16 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 
 // Wait for the phase with the given parity to complete.  Gives up (returns
 // false) after `limit_ns` of wall time, or as soon as *abort becomes nonzero,
-// so that no role of a CTA can spin forever.
+// so that no role of a CTA can spin forever.  The hardware suspend hint never
+// exceeds the limit: with a limit of 0 the wait gives up at once unless the
+// phase has already completed.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns,
                                           const volatile int *abort) {
     if (mbar_try_wait(bar, parity)) return true;
+    const uint32_t hint = limit_ns < 200000u ? static_cast<uint32_t>(limit_ns) : 200000u;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-        if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
+        if (mbar_try_wait_sleep(bar, parity, hint)) return true;
         if (*abort) return false;
         if (globaltimer_ns() - t0 > limit_ns) return false;
     }

@@ -104,7 +104,8 @@ struct SwaParams {
     int T, Hq, Hkv, window;
     float c;                            // scale * log2(e)
     int *err;                           // device status word, or null
-    uint64_t timeout_ns;
+    uint64_t timeout_ns;                // bound on the waits of the work loops
+    uint64_t drain_ns;                  // bound on the waits that drain copies and MMAs before exit
 };
 
 // First token of the sequence that holds token t.
@@ -177,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = *tmem_slot;
-    const uint64_t lim = p.timeout_ns;
+    const uint64_t lim = p.timeout_ns, drain = p.drain_ns;
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------------------ TMA producer
@@ -202,10 +203,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // no copy may still be landing in shared memory at exit
             const int zero = 0;
-            mbar_wait(bar(BR_Q), 0, lim, &zero);
+            mbar_wait(bar(BR_Q), 0, drain, &zero);
             for (int s = 0; s < kKVStages; ++s) {
-                if (issued_k[s]) mbar_wait(bar(BR_KFULL + s), (issued_k[s] - 1) & 1, lim, &zero);
-                if (issued_v[s]) mbar_wait(bar(BR_VFULL + s), (issued_v[s] - 1) & 1, lim, &zero);
+                if (issued_k[s]) mbar_wait(bar(BR_KFULL + s), (issued_k[s] - 1) & 1, drain, &zero);
+                if (issued_v[s]) mbar_wait(bar(BR_VFULL + s), (issued_v[s] - 1) & 1, drain, &zero);
             }
         }
     } else if (warp == kMmaWarp) {
@@ -251,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(bar(BR_FIN));   // every issued MMA completes before TMEM is released
             if (!mbar_wait(bar(BR_FIN), 0, lim, abort_flag)) {
                 const int zero = 0;
-                mbar_wait(bar(BR_FIN), 0, lim, &zero);
+                mbar_wait(bar(BR_FIN), 0, drain, &zero);
             }
         }
     } else {
@@ -532,7 +533,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = *tmem_slot;
-    const uint64_t lim = p.timeout_ns;
+    const uint64_t lim = p.timeout_ns, drain = p.drain_ns;
 
     if (warp == kPairProducerWarp) {
         // ------------------------------------------------------------ TMA producer
@@ -558,10 +559,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 ++issued_v[s];
             }
             const int zero = 0;   // no copy may still be landing in shared memory at exit
-            mbar_wait(bar(PB_Q), 0, lim, &zero);
+            mbar_wait(bar(PB_Q), 0, drain, &zero);
             for (int s = 0; s < kPairKV; ++s) {
-                if (issued_k[s]) mbar_wait(bar(PB_KFULL + s), (issued_k[s] - 1) & 1, lim, &zero);
-                if (issued_v[s]) mbar_wait(bar(PB_VFULL + s), (issued_v[s] - 1) & 1, lim, &zero);
+                if (issued_k[s]) mbar_wait(bar(PB_KFULL + s), (issued_k[s] - 1) & 1, drain, &zero);
+                if (issued_v[s]) mbar_wait(bar(PB_VFULL + s), (issued_v[s] - 1) & 1, drain, &zero);
             }
         }
     } else if (warp == kPairMmaWarp) {
@@ -628,7 +629,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             mma_commit(bar(PB_FIN));
             if (!mbar_wait(bar(PB_FIN), 0, lim, abort_flag)) {
                 const int zero = 0;
-                mbar_wait(bar(PB_FIN), 0, lim, &zero);
+                mbar_wait(bar(PB_FIN), 0, drain, &zero);
             }
         }
     } else {
@@ -924,6 +925,7 @@ cudaError_t launch_swa(const SwaLaunch &L, cudaStream_t stream) {
     p.c = L.scale * kLog2e;
     p.err = L.err;
     p.timeout_ns = L.timeout_ns;
+    p.drain_ns = L.drain_ns;
     if ((L.Hq / L.Hkv) % 2 == 0) {   // head pairs that share a key/value head
         const dim3 grid((T + kBM - 1) / kBM, L.Hq / 2);
         swa_fwd_pair_kernel<<<grid, kPairThreads, kPairSmem, stream>>>(mq, mk, mv, p);

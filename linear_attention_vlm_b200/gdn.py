@@ -89,6 +89,8 @@ def _load():
     lib.gdn_read_status.restype = i32
     lib.gdn_noalloc_read_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
     lib.gdn_noalloc_read_status.restype = i32
+    lib.gdn_set_wait_limit.argtypes = [ctypes.c_uint64]
+    lib.gdn_set_wait_limit.restype = None
     lib.gdn_last_cuda_error.argtypes = []
     lib.gdn_last_cuda_error.restype = ctypes.c_char_p
     _lib = lib
@@ -124,6 +126,16 @@ def gdn_read_status(word: torch.Tensor) -> int:
     if st not in (GDN_OK, GDN_ERR_TIMEOUT):
         raise GdnError(st, "gdn_read_status")
     return int(code.value)
+
+
+WAIT_LIMIT_DEFAULT = 2000000000
+
+
+def gdn_set_wait_limit(ns: int) -> None:
+    """Bound (ns) on the work-loop waits of the tensor-core kernels this host
+    thread launches next (include/gdn.h, gdn_set_wait_limit); 0 makes the
+    first wait on work in flight give up, WAIT_LIMIT_DEFAULT restores 2 s."""
+    _load().gdn_set_wait_limit(int(ns))
 
 
 def _dtype_code(t: torch.dtype) -> int:
