@@ -205,6 +205,15 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
         : "memory");
 }
 
+// bulk_load with an L2 eviction-priority policy for the lines it reads.
+__device__ __forceinline__ void bulk_load_hint(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar,
+                                               uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar), "l"(policy)
+        : "memory");
+}
+
 // 1-D bulk copy shared -> global (bulk async-group completion).
 __device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t bytes) {
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
@@ -747,6 +756,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
     } else if (warp == 9) {
         // ------------------------------------------------------------ TMA / bulk producer
         if (lane == 0) {
+            const uint64_t l2pol = MODE == MODE_TRANS ? l2_evict_last_policy() : l2_evict_first_policy();
             int issued[NST] = {};
             // Pull chunk m's data into L2 while its stage is still in use, so
             // that the copy into shared memory, once the stage frees up, is an
@@ -776,19 +786,23 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                 }
                 const uint32_t full = bar(CB_FULL + s);
                 const uint8_t *tile = p.tiles + ((size_t)(gc0 + n) * H + h) * kTileBytes;
+                // A transition range reads K, V, -W and T'' of chunks that the
+                // output pass reads again after the combine: keep them in L2
+                // (evict_last).  The output pass reads them for the last time.
+                const uint64_t pol = l2pol;
                 // a transition range reads -W and T'' only
                 mbar_arrive_expect_tx(full, Lay::STAGE);
                 for (int kb = 0; kb < 2; ++kb) {
-                    tma_load_3d(st + Lay::K + kb * 8192, &p.map_k, kb * 64, h, z, full);
-                    tma_load_3d(st + Lay::V + kb * 8192, &p.map_v, kb * 64, h, z, full);
+                    tma_load_3d_hint(st + Lay::K + kb * 8192, &p.map_k, kb * 64, h, z, full, pol);
+                    tma_load_3d_hint(st + Lay::V + kb * 8192, &p.map_v, kb * 64, h, z, full, pol);
                 }
                 if (n == 0 && p.wait_tiles) grid_dep_wait();   // tiles come from the prep kernel
                 if (MODE == MODE_TRANS) {   // -W and T'' of the tile
-                    bulk_load(st + ChainLayout<1>::W, tile + TILE_NEGW, 8192, full);
-                    bulk_load(st + ChainLayout<1>::W + 8192, tile + 16384 + TILE_NEGW, 8192, full);
-                    bulk_load(st + ChainLayout<1>::TPP, tile + TILE_TPP, 8192, full);
+                    bulk_load_hint(st + ChainLayout<1>::W, tile + TILE_NEGW, 8192, full, pol);
+                    bulk_load_hint(st + ChainLayout<1>::W + 8192, tile + 16384 + TILE_NEGW, 8192, full, pol);
+                    bulk_load_hint(st + ChainLayout<1>::TPP, tile + TILE_TPP, 8192, full, pol);
                 } else {
-                    bulk_load(st + ChainLayout<0>::WQ, tile, (uint32_t)kTileBytes, full);
+                    bulk_load_hint(st + ChainLayout<0>::WQ, tile, (uint32_t)kTileBytes, full, pol);
                 }
                 ++issued[s];
             }
