@@ -183,7 +183,8 @@ struct ChainParams {
     int nseg, seg_len;           // chunk ranges per sequence, chunks per range
     const uint8_t *tiles;
     const float *seg_start;      // start states of ranges 1.. [N][H][nseg-1][D][D]
-    float *trans_r, *trans_m;    // transitions R, M of ranges 0..nseg-2, same layout
+    float *trans_r;              // transitions R of ranges 0..nseg-2, same layout
+    float *trans_m;              // transitions M, same units; each as bf16 rows [k][n], hi then lo (M = hi + lo)
     int wait_tiles;              // the prep kernel may still run: wait before reading tiles
     int wait_start;              // the combine may still run: wait before reading seg_start
     int *err;
@@ -350,6 +351,14 @@ __device__ __forceinline__ void merge_level2b(uint8_t *sm, float *scratch0, int 
     store16(t_blk(sm, i, j), TB_P, acc, true, lane);
 }
 
+
+// (x, y) -> packed bf16 hi = rn(x, y) and lo = rn(x - hi_x, y - hi_y)
+__device__ __forceinline__ void split2(float x, float y, uint32_t &hi, uint32_t &lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+    const float2 hf = __bfloat1622float2(h);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    lo = pack_bf16(x - hf.x, y - hf.y);
+}
 
 // ---------------------------------------------------------------- chunk offsets
 
@@ -747,9 +756,13 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                 }
                 if (MODE == MODE_TRANS) {
                     *reinterpret_cast<float4 *>(p.trans_r + unit * D * D + (size_t)tid * D + j) = make_float4(0.f, 0.f, 0.f, 0.f);
-                    float4 e = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (tid >= j && tid < j + 4) (&e.x)[tid - j] = 1.f;
-                    *reinterpret_cast<float4 *>(p.trans_m + unit * D * D + (size_t)tid * D + j) = e;
+                    // M = I: hi = I, lo = 0; row tid, column pairs j/2, j/2 + 1
+                    uint32_t *hi = reinterpret_cast<uint32_t *>(p.trans_m + unit * D * D) + (size_t)tid * (D / 2) + j / 2;
+                    uint32_t *lo = hi + D * D / 2;
+                    hi[0] = pack_bf16(tid == j ? 1.f : 0.f, tid == j + 1 ? 1.f : 0.f);
+                    hi[1] = pack_bf16(tid == j + 2 ? 1.f : 0.f, tid == j + 3 ? 1.f : 0.f);
+                    lo[0] = 0u;
+                    lo[1] = 0u;
                 }
             }
         }
@@ -1070,7 +1083,9 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
     // idle now: each state warp writes its rows (padded pitch, conflict-free),
     // then all threads store 16-byte pieces in row order.
     if (nloc > 0 && *abort_flag == 0) {
-        constexpr int PITCH = D + 4;
+        constexpr int PITCH = D + 4;   // fp32 rows
+        constexpr int MPW = D / 2 + 4;  // 32-bit words per bf16 row (M of a transition range)
+        static_assert(4 * (D * PITCH + 2 * D * MPW) <= Lay::NST * Lay::STAGE, "staging fits the idle stages");
         const int nchains = MODE == MODE_TRANS ? 2 : 1;
         for (int c = 0; c < nchains; ++c) {
             float *dst = MODE == MODE_TRANS ? (c ? p.trans_m : p.trans_r) + unit * D * D
@@ -1084,6 +1099,21 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                 for (int c0 = 0; c0 < D; c0 += 32) {
                     float x[32];
                     tmem_ld32(tm + lane_off + (c ? TM_XS : TM_S) + c0, x);
+                    if (MODE == MODE_TRANS && c == 1) {
+                        // M leaves as bf16 hi and lo rows (M = hi + lo to about
+                        // 16 mantissa bits), the form the combine's mma.sync
+                        // consumes: rows of MPW words, hi rows then lo rows
+                        uint32_t *sh = reinterpret_cast<uint32_t *>(stg);
+#pragma unroll
+                        for (int j = 0; j < 32; j += 8) {
+                            uint32_t h_[4], l_[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) split2(x[j + 2 * e], x[j + 2 * e + 1], h_[e], l_[e]);
+                            *reinterpret_cast<uint4 *>(sh + row * MPW + (c0 + j) / 2) = make_uint4(h_[0], h_[1], h_[2], h_[3]);
+                            *reinterpret_cast<uint4 *>(sh + (D + row) * MPW + (c0 + j) / 2) = make_uint4(l_[0], l_[1], l_[2], l_[3]);
+                        }
+                        continue;
+                    }
 #pragma unroll
                     for (int j = 0; j < 32; j += 4)
                         *reinterpret_cast<float4 *>(stg + row * PITCH + c0 + j) = make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
@@ -1096,6 +1126,14 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                                             : (finish ? finish + state_off : nullptr);
             if (!dst) break;
             const float *stg = reinterpret_cast<const float *>(sm) + c * D * PITCH;
+            if (MODE == MODE_TRANS && c == 1) {   // 2 D rows of 16 pieces (hi, then lo)
+                const uint32_t *sh = reinterpret_cast<const uint32_t *>(stg);
+                for (int i = threadIdx.x; i < 2 * D * 16; i += blockDim.x) {
+                    const int row = i >> 4, piece = i & 15;
+                    reinterpret_cast<uint4 *>(dst)[i] = *reinterpret_cast<const uint4 *>(sh + row * MPW + 4 * piece);
+                }
+                continue;
+            }
             for (int i = threadIdx.x; i < D * D / 4; i += blockDim.x) {
                 const int row = i >> 5, c4 = i & 31;
                 *reinterpret_cast<float4 *>(dst + row * D + 4 * c4) =
@@ -1120,18 +1158,28 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
 // M_j; the four k-slice partials meet in shared memory, where R_j is added.
 // The products run on bf16 mma.sync with each fp32 operand split in two
 // (x = hi + lo, both bf16; S M ~= S_hi M_hi + S_hi M_lo + S_lo M_hi), which
-// keeps about 16 mantissa bits; accumulation is fp32.  M_{j+1} streams into
-// the other half of a double buffer (cp.async) while step j computes.
+// keeps about 16 mantissa bits; accumulation is fp32.  M_j arrives already
+// split from the transition ranges (bf16 hi and lo rows [k][n]), ldmatrix
+// (.trans) turns its rows into B fragments, and it streams into the other
+// half of a double buffer (cp.async) while step j computes.
 constexpr int kCombRows = 16;
 constexpr int kCombThreads = 256;
-constexpr int kCombMP = 132, kCombSP = 136, kCombPP = 132;   // row pitches: conflict-free fragments
+constexpr int kCombMB = 136, kCombSP = 136, kCombPP = 132;   // row pitches: conflict-free fragments
+constexpr size_t kCombMBuf = (size_t)2 * D * kCombMB;         // bf16 per buffer: hi then lo
 constexpr size_t kCombSmem =
-    (size_t)(2 * D * kCombMP + kCombRows * kCombSP + 4 * kCombRows * kCombPP) * sizeof(float);
+    (size_t)2 * kCombMBuf * sizeof(__nv_bfloat16) + (size_t)(kCombRows * kCombSP + 4 * kCombRows * kCombPP) * sizeof(float);
 
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)),
                  "l"(reinterpret_cast<uint64_t>(src))
                  : "memory");
+}
+
+// four 8x8 bf16 blocks, transposed on the way: the col-major B fragments of mma.sync
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const __nv_bfloat16 *row) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(row)));
 }
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -1143,14 +1191,6 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// (x, y) -> packed bf16 hi = rn(x, y) and lo = rn(x - hi_x, y - hi_y)
-__device__ __forceinline__ void split2(float x, float y, uint32_t &hi, uint32_t &lo) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
-    const float2 hf = __bfloat1622float2(h);
-    hi = *reinterpret_cast<const uint32_t *>(&h);
-    lo = pack_bf16(x - hf.x, y - hf.y);
-}
-
 __global__ void __launch_bounds__(kCombThreads, 1)
 gdn_scan_combine_kernel(const float *__restrict__ state_in, const float *__restrict__ trans_r,
                         const float *__restrict__ trans_m, float *__restrict__ seg_start, int nseg,
@@ -1158,19 +1198,22 @@ gdn_scan_combine_kernel(const float *__restrict__ state_in, const float *__restr
     (void)err;
     (void)timeout_ns;
     extern __shared__ float smf[];
-    float *Ms = smf;                              // M_j [k][n], two buffers
-    float *Ss = Ms + 2 * D * kCombMP;             // S_j rows [16][D]
-    float *Ps = Ss + kCombRows * kCombSP;         // k-slice partials [4][16][D]
+    __nv_bfloat16 *Mb = reinterpret_cast<__nv_bfloat16 *>(smf);   // M_j hi, lo rows [k][n], two buffers
+    float *Ss = reinterpret_cast<float *>(Mb + 2 * kCombMBuf);    // S_j rows [16][D]
+    float *Ps = Ss + kCombRows * kCombSP;                          // k-slice partials [4][16][D]
     const int nh = blockIdx.x, r0 = blockIdx.y * kCombRows;
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31, g = lane >> 2, q = lane & 3;
     const int kg = warp >> 1, ch = warp & 1;
     grid_dep_wait();     // the transitions come from the previous kernel
     grid_dep_launch();   // the output pass may launch; its first ranges do not need this grid
     auto stage = [&](int j) {
-        const float *src = trans_m + ((size_t)nh * (nseg - 1) + j) * D * D;
-        float *dst = Ms + (j & 1) * D * kCombMP;
-        for (int i = t; i < D * D / 4; i += kCombThreads)
-            cp_async16(dst + (i >> 5) * kCombMP + 4 * (i & 31), src + 4 * i);
+        // 2 x 128 rows of 256 bytes (16 pieces each) into rows of kCombMB bf16
+        const __nv_bfloat16 *src = reinterpret_cast<const __nv_bfloat16 *>(trans_m + ((size_t)nh * (nseg - 1) + j) * D * D);
+        __nv_bfloat16 *dst = Mb + (j & 1) * kCombMBuf;
+        for (int i = t; i < 2 * D * 16; i += kCombThreads) {
+            const int row = i >> 4, piece = i & 15;   // row: hi rows 0..127, then lo rows
+            cp_async16(dst + row * kCombMB + piece * 8, src + row * D + piece * 8);
+        }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
     if (nseg > 1) stage(0);
@@ -1190,7 +1233,7 @@ gdn_scan_combine_kernel(const float *__restrict__ state_in, const float *__restr
         asm volatile("cp.async.wait_group 0;" ::: "memory");
         __syncthreads();   // M_j landed for every thread; S_j rows are written
         if (j + 2 < nseg) stage(j + 1);
-        const float *M = Ms + (j & 1) * D * kCombMP;
+        const __nv_bfloat16 *Mh = Mb + (j & 1) * kCombMBuf, *Ml = Mh + D * kCombMB;
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks) {
             const int k0 = 32 * kg + 16 * ks;
@@ -1203,16 +1246,23 @@ gdn_scan_combine_kernel(const float *__restrict__ state_in, const float *__restr
             split2(s10.x, s10.y, ah[1], al[1]);
             split2(s01.x, s01.y, ah[2], al[2]);
             split2(s11.x, s11.y, ah[3], al[3]);
-            const float *m0 = M + (k0 + 2 * q) * kCombMP, *m8 = m0 + 8 * kCombMP;
+            // lane -> row of one of four 8x8 blocks: k0 + (lane & 7) + 8 ((lane >> 3) & 1),
+            // columns n0 + 8 (lane >> 4); .trans turns them into the B fragments
+            // {b0, b1} of n-tiles 2 pr and 2 pr + 1
+            const int krow = k0 + (lane & 7) + 8 * ((lane >> 3) & 1), ncol = 8 * (lane >> 4);
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-                const int n = 64 * ch + 8 * nt + g;
-                uint32_t bh0, bl0, bh1, bl1;
-                split2(m0[n], m0[kCombMP + n], bh0, bl0);
-                split2(m8[n], m8[kCombMP + n], bh1, bl1);
-                mma_bf16_16816(accx[nt], al[0], al[1], al[2], al[3], bh0, bh1);
-                mma_bf16_16816(accx[nt], ah[0], ah[1], ah[2], ah[3], bl0, bl1);
-                mma_bf16_16816(acc[nt], ah[0], ah[1], ah[2], ah[3], bh0, bh1);
+            for (int pr = 0; pr < 4; ++pr) {
+                const int n0 = 64 * ch + 16 * pr;
+                uint32_t bh[4], bl[4];
+                ldmatrix_x4_trans(bh, Mh + krow * kCombMB + n0 + ncol);
+                ldmatrix_x4_trans(bl, Ml + krow * kCombMB + n0 + ncol);
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int nt = 2 * pr + u;
+                    mma_bf16_16816(accx[nt], al[0], al[1], al[2], al[3], bh[2 * u], bh[2 * u + 1]);
+                    mma_bf16_16816(accx[nt], ah[0], ah[1], ah[2], ah[3], bl[2 * u], bl[2 * u + 1]);
+                    mma_bf16_16816(acc[nt], ah[0], ah[1], ah[2], ah[3], bh[2 * u], bh[2 * u + 1]);
+                }
             }
         }
         float *P = Ps + kg * kCombRows * kCombPP;
