@@ -358,6 +358,21 @@ def run_native(args):
     def gate_once():
         gdn.gdn_output_gate(out, lay["z"], lay["norm_w"], gate=gdn.GATE_SIGMOID, out=gate_out)
 
+    # the whole token mixer of one layer: one fused call, and the three calls
+    lay_state = torch.zeros((1, H, dv, dk), dtype=torch.float32, device=dev)
+    lay_ws = torch.empty(gdn.gdn_layer_prefill_workspace_size(1, T, H, dk, w.dtype), dtype=torch.uint8, device=dev)
+
+    def layer_fused_once():
+        gdn.gdn_layer_prefill(lay["xq"], lay["xk"], lay["xv"], lay["conv_w"], lay["a"], lay["b"], lay["z"], None, None,
+                              lay["norm_w"], activation=gdn.ACT_SILU, gate=gdn.GATE_SIGMOID, y=gate_out,
+                              state_out=lay_state, workspace=lay_ws, want_conv_state=False)
+
+    def layer_unfused_once():
+        q_, k_, v_, g_, b_, _ = gdn.gdn_preprocess(lay["xq"], lay["xk"], lay["xv"], lay["conv_w"], lay["a"], lay["b"],
+                                                   None, None, activation=gdn.ACT_SILU, want_state=False)
+        gdn.gdn_prefill(q_, k_, v_, g_, b_, None, out=out, state_out=lay_state, workspace=ws)
+        gdn.gdn_output_gate(out, lay["z"], lay["norm_w"], gate=gdn.GATE_SIGMOID, out=gate_out)
+
     # ---- streaming session: one GDN layer step per video frame (~274 tokens per
     # frame in the pages' streaming measurement), state carried, graph replay
     FRAME = 274
@@ -366,7 +381,8 @@ def run_native(args):
                           activation=gdn.ACT_SILU)
     for name in ("xq", "xk", "xv", "a", "b", "z"):
         getattr(sess, name)[:FRAME].copy_(P[name].to(dev))
-    frame_launches = 2 + gdn.gdn_prefill_kernel_count(1, FRAME, H, dk, dv, w.chunk, w.dtype) + 1
+    # a frame: the fused layer call's kernels + the convolution-state update
+    frame_launches = gdn.gdn_prefill_kernel_count(1, FRAME, H, dk, dv, w.chunk, w.dtype) + 1
     decode_launches = 2 + 1 + 1
 
     # ---- sliding-window attention layer of the hybrid block: RoPE on q and k,
@@ -417,6 +433,8 @@ def run_native(args):
         if want("layer"):
             preprocess_once()
             gate_once()
+            layer_fused_once()
+            layer_unfused_once()
         if want("streaming"):
             sess.prefill(FRAME)
             sess.prefill(FRAME, eager=True)
@@ -470,7 +488,9 @@ def run_native(args):
         if want("layer"):
             ms["pre"] = timed(lambda i: preprocess_once(), K)
             ms["gate"] = timed(lambda i: gate_once(), K)
-            launches["layer"] = 2 * K + K
+            ms["layer_fused"] = timed(lambda i: layer_fused_once(), K)
+            ms["layer_unfused"] = timed(lambda i: layer_unfused_once(), K)
+            launches["layer"] = 2 * K + K + K * launches_per_prefill + K * (2 + launches_per_prefill)
         if want("streaming"):
             ms["frame_graph"] = timed(lambda i: sess.prefill(FRAME), K)
             ms["frame_eager"] = timed(lambda i: sess.prefill(FRAME, eager=True), K)
@@ -482,9 +502,9 @@ def run_native(args):
             launches["swa"] = K + 3 * K
         wall = time.time() - t_wall0
     keys = ("prefill", "long", "long_seg", "varlen", "dec_pp", "dec_ip", "e2e", "pre", "gate",
-            "frame_graph", "frame_eager", "dec_graph", "swa_attn", "swa_layer")
+            "frame_graph", "frame_eager", "dec_graph", "swa_attn", "swa_layer", "layer_fused", "layer_unfused")
     (ms_prefill, ms_long, ms_long_seg, ms_varlen, ms_dec_pp, ms_dec_ip, ms_e2e, ms_pre, ms_gate,
-     ms_frame_graph, ms_frame_eager, ms_dec_graph, ms_swa_attn, ms_swa_layer) = (
+     ms_frame_graph, ms_frame_eager, ms_dec_graph, ms_swa_attn, ms_swa_layer, ms_layer_fused, ms_layer_unfused) = (
         max_over_ranks(ms.get(k, nan), world) for k in keys)
     swa_flops = swa_attention_flops(SWA_T, W.SWA_HQ, W.SWA_D, W.SWA_WINDOW)
     swa_tf = swa_flops / (ms_swa_attn * 1e-3) / 1e12
@@ -567,6 +587,14 @@ def run_native(args):
         "output_gate": {"metric": "output gate tokens/s (RMS norm + sigmoid gate), prefill shapes",
                         "value": aggregate_throughput(T, world, ms_gate), "unit": "tokens/s", "ms_per_step": ms_gate,
                         "roofline": hbm_roofline("gdn_output_gate_kernel", gate_bytes, ms_gate)},
+        "layer": {"metric": "GDN layer token mixer tokens/s at the prefill shapes: raw projections -> "
+                            "pre-processing -> recurrence -> output gate",
+                  "value": aggregate_throughput(T, world, ms_layer_fused), "unit": "tokens/s",
+                  "ms_per_step": ms_layer_fused, "kernels": launches_per_prefill,
+                  "unfused": {"metric": "the same as gdn_preprocess + gdn_prefill + gdn_output_gate",
+                              "value": aggregate_throughput(T, world, ms_layer_unfused), "unit": "tokens/s",
+                              "ms_per_step": ms_layer_unfused, "kernels": 2 + launches_per_prefill},
+                  "l2": "flushed before every step"},
         "streaming": {"metric": "GDN layer frames/s: pre-processing + recurrence with carried state + "
                                 "output gate per %d-token frame x %d heads, CUDA-graph replay" % (FRAME, H),
                       "value": 1e3 / ms_frame_graph * world, "unit": "frames/s",
@@ -592,7 +620,7 @@ def run_native(args):
         "timed_wall_s": wall,
     }
     leg_keys = {"long_prefill": "long_prefill", "varlen": "varlen", "decode": "decode",
-                "decode_inplace": "decode", "preprocess": "layer", "output_gate": "layer",
+                "decode_inplace": "decode", "preprocess": "layer", "output_gate": "layer", "layer": "layer",
                 "streaming": "streaming", "swa": "swa", "e2e": "e2e"}
     for key, leg in leg_keys.items():
         if not want(leg):

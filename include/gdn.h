@@ -277,6 +277,49 @@ int gdn_preprocess(const void *xq, const void *xk, const void *xv, const float *
 int gdn_output_gate(const void *o, const void *z, const float *norm_w, void *y, int64_t rows, int dv,
                     int gate, float eps, int dtype, void *stream);
 
+/*
+ * One Gated DeltaNet layer's token mixer over a packed batch, from the raw
+ * projections to the gated output: gdn_preprocess, gdn_prefill and
+ * gdn_output_gate in one call, with their arguments and their results (up to
+ * the rounding order of sums):
+ *
+ *   (q, k, v, g, beta) = pre-processing of (xq, xk, xv, a_logit, b_logit)
+ *   (o, state_out)     = the chunkwise recurrence from state_in
+ *   y                  = n(o) * act(z)
+ *
+ * On the tensor-core path (GDN_BF16, d = 128, total_tokens > 0) the steps
+ * are fused: the chunk-prep kernel forms q, k, v, g and beta from its chunk's
+ * raw projections (q never leaves the chip; k, v, g and beta go to the
+ * workspace for the state and output passes), and the output pass writes y
+ * in place of o.  Otherwise the three steps run one after another through
+ * the workspace.
+ *
+ *   xq, xk, xv, conv_w, a_logit, b_logit, conv_state_in, conv_state_out,
+ *   activation   as in gdn_preprocess (conv_state_out may equal
+ *                conv_state_in, or be NULL)
+ *   state_in, state_out, cu_seqlens, num_seqs, total_tokens, H   as in
+ *                gdn_prefill, with d_k = d_v = d (state_out may equal
+ *                state_in, or be NULL)
+ *   z            [total_tokens, H, d] dtype; norm_w [d] fp32 or NULL; gate
+ *                as in gdn_output_gate
+ *   y            [total_tokens, H, d] dtype (written)
+ *   eps          of the q/k L2 norm and of the RMS norm, in [0, 1]
+ *   workspace    gdn_layer_prefill_workspace_size(...) bytes, 16-byte aligned,
+ *                owned by the caller; its first int32 is the status word of
+ *                the tensor-core kernels (gdn_read_status)
+ * y, the workspace and the output states may not overlap the inputs or one
+ * another, except that each state may be updated in place
+ * (GDN_ERR_INVALID_ARG).  Supported: d in {64, 128}; dtype GDN_F32 or
+ * GDN_BF16.
+ */
+size_t gdn_layer_prefill_workspace_size(int num_seqs, int64_t total_tokens, int H, int d, int dtype);
+int gdn_layer_prefill(const void *xq, const void *xk, const void *xv, const float *conv_w,
+                      const float *a_logit, const float *b_logit, const void *conv_state_in,
+                      void *conv_state_out, const float *state_in, float *state_out, const void *z,
+                      const float *norm_w, void *y, const int32_t *cu_seqlens, int num_seqs,
+                      int64_t total_tokens, int H, int d, int activation, int gate, float eps,
+                      int dtype, void *workspace, size_t workspace_bytes, void *stream);
+
 /* ------------------------------------------------------------------ sliding-window attention
  *
  * The hybrid block's other token mixer (InfiniteVL explainer page, "Step 2:
@@ -338,10 +381,11 @@ int gdn_swa_attention(const void *q, const void *k, const void *v, void *o, cons
  * be captured once and replayed without launch overhead; a video is fed
  * segment by segment while the state is carried).
  *
- * A step, for each of num_streams independent streams:
- *   gdn_preprocess (convolution state carried in place) ->
- *   gdn_prefill (tokens > 0; recurrent state carried in place) or
- *   gdn_decode_step (one token) -> gdn_output_gate.
+ * A step, for each of num_streams independent streams, with the convolution
+ * and recurrent states carried in place:
+ *   tokens > 0:  gdn_layer_prefill (pre-processing, recurrence and output
+ *                gate; fused on the tensor-core path);
+ *   one token:   gdn_preprocess -> gdn_decode_step -> gdn_output_gate.
  *
  * The caller owns every buffer and keeps it in place for the session's
  * lifetime (the graphs hold the addresses).  Sizes, with R = num_streams *

@@ -67,6 +67,28 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
     return x < y + nb && y < x + na;
 }
 
+size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
+
+// Workspace of gdn_layer_prefill.  Tensor-core path: [prefill workspace]
+// [k][v] (processed, dtype) [g][beta] (fp32); otherwise [q][k][v][o][g][beta].
+struct LayerWs {
+    size_t prefill, tens, gates, total;
+};
+
+LayerWs layer_ws(int num_seqs, int64_t total_tokens, int H, int d, int dtype) {
+    LayerWs w{0, 0, 0, 0};
+    const size_t es = dtype == GDN_BF16 ? 2 : 4;
+    w.tens = align256((size_t)total_tokens * H * d * es);
+    w.gates = align256((size_t)total_tokens * H * 4);
+    if (use_tc(total_tokens, d, dtype)) {
+        w.prefill = align256(gdn::tc_workspace_bytes(num_seqs, total_tokens, H, /*varlen=*/true));
+        w.total = w.prefill + 2 * w.tens + 2 * w.gates;
+    } else {
+        w.total = 4 * w.tens + 2 * w.gates;
+    }
+    return w;
+}
+
 }  // namespace
 
 int gdn::note_cuda_error(cudaError_t e) { return cuda_fail(e); }
@@ -138,7 +160,7 @@ int gdn_prefill(const void *q, const void *k, const void *v, const float *g, con
         cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), s);
         if (e != cudaSuccess) return cuda_fail(e);
         gdn::TcLaunch L{q, k, v, g, beta, state_in, out, state_out, cu_seqlens, uniform_len,
-                        total_tokens, num_seqs, H, workspace, err, g_wait_limit_ns, kWaitLimitNs};
+                        total_tokens, num_seqs, H, workspace, err, g_wait_limit_ns, kWaitLimitNs, nullptr};
         e = gdn::launch_prefill_tc(L, s);
         return e == cudaSuccess ? GDN_OK : cuda_fail(e);
     }
@@ -242,6 +264,117 @@ int gdn_output_gate(const void *o, const void *z, const float *norm_w, void *y, 
     if (overlaps(y, n, z, n) || overlaps(y, n, norm_w, (size_t)dv * 4)) return GDN_ERR_INVALID_ARG;
     const cudaError_t e = gdn::launch_output_gate(dtype, dv, o, z, norm_w, y, rows, gate, eps,
                                                   static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e);
+}
+
+size_t gdn_layer_prefill_workspace_size(int num_seqs, int64_t total_tokens, int H, int d, int dtype) {
+    if (num_seqs < 1 || H < 1 || total_tokens < 0) return 0;
+    if ((d != 64 && d != 128) || (dtype != GDN_F32 && dtype != GDN_BF16)) return 0;
+    return layer_ws(num_seqs, total_tokens, H, d, dtype).total;
+}
+
+int gdn_layer_prefill(const void *xq, const void *xk, const void *xv, const float *conv_w, const float *a_logit,
+                      const float *b_logit, const void *conv_state_in, void *conv_state_out, const float *state_in,
+                      float *state_out, const void *z, const float *norm_w, void *y, const int32_t *cu_seqlens,
+                      int num_seqs, int64_t total_tokens, int H, int d, int activation, int gate, float eps,
+                      int dtype, void *workspace, size_t workspace_bytes, void *stream) {
+    if (num_seqs < 1 || H < 1 || total_tokens < 0) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (activation != GDN_ACT_NONE && activation != GDN_ACT_SILU) return GDN_ERR_INVALID_ARG;
+    if (gate != GDN_GATE_SIGMOID && gate != GDN_GATE_SILU) return GDN_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || eps > 1.f) return GDN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return GDN_ERR_UNSUPPORTED;
+    if ((int64_t)num_seqs * H > (int64_t)INT32_MAX / 2) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)num_seqs * 3 * 3 * H * d > (int64_t)INT32_MAX) return GDN_ERR_INVALID_ARG;
+    if (total_tokens > (int64_t)INT32_MAX * 8) return GDN_ERR_INVALID_ARG;
+    if (!cu_seqlens && total_tokens % num_seqs != 0) return GDN_ERR_INVALID_ARG;
+    if (total_tokens > 0 && (!xq || !xk || !xv || !conv_w || !a_logit || !b_logit || !z || !y))
+        return GDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {xq, xk, xv, conv_w, a_logit, b_logit, conv_state_in, conv_state_out, state_in, state_out,
+                          z, norm_w, y, cu_seqlens, workspace};
+    for (const void *p : ptrs)
+        if (p && misaligned(p)) return GDN_ERR_INVALID_ARG;
+    const LayerWs W = layer_ws(num_seqs, total_tokens, H, d, dtype);
+    if (!workspace || workspace_bytes < W.total) return GDN_ERR_WORKSPACE;
+    const size_t es = dtype == GDN_BF16 ? 2 : 4;
+    const size_t tens = (size_t)total_tokens * H * d * es, gates = (size_t)total_tokens * H * 4;
+    const size_t cst = (size_t)num_seqs * 9 * H * d * es, st = (size_t)num_seqs * H * d * d * 4;
+    // y, the workspace and the states may not overlap the inputs or each other;
+    // the convolution and recurrent states may each be updated in place
+    const void *ins[] = {xq, xk, xv, conv_w, a_logit, b_logit, z, norm_w, cu_seqlens};
+    const size_t in_n[] = {tens, tens, tens, (size_t)3 * H * d * 16, gates, gates, tens, (size_t)d * 4,
+                           (size_t)(num_seqs + 1) * 4};
+    const void *outs[] = {y, workspace, conv_state_out, state_out};
+    const size_t out_n[] = {tens, W.total, cst, st};
+    for (int i = 0; i < 4; ++i) {
+        for (int j = 0; j < 9; ++j)
+            if (overlaps(outs[i], out_n[i], ins[j], in_n[j])) return GDN_ERR_INVALID_ARG;
+        for (int j = i + 1; j < 4; ++j)
+            if (overlaps(outs[i], out_n[i], outs[j], out_n[j])) return GDN_ERR_INVALID_ARG;
+    }
+    const void *states_in[] = {conv_state_in, state_in};
+    const size_t states_n[] = {cst, st};
+    for (int i = 0; i < 2; ++i)
+        for (int j = 0; j < 2; ++j) {
+            if (overlaps(outs[j], out_n[j], states_in[i], states_n[i])) return GDN_ERR_INVALID_ARG;
+            if (overlaps(outs[2 + j], out_n[2 + j], states_in[i], states_n[i]) &&
+                !(i == j && outs[2 + j] == states_in[i]))
+                return GDN_ERR_INVALID_ARG;   // each state in place (the same buffer) or apart
+        }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const int64_t uniform_len = cu_seqlens ? 0 : total_tokens / num_seqs;
+    cudaError_t e = cudaSuccess;
+    if (use_tc(total_tokens, d, dtype)) {
+        // one pass of prep + chain kernels; the convolution state is written
+        // after them (it may be the state they read)
+        int *err = reinterpret_cast<int *>(ws);
+        e = cudaMemsetAsync(err, 0, sizeof(int), s);
+        if (e != cudaSuccess) return cuda_fail(e);
+        gdn::TcLayer Ly;
+        Ly.xq = xq; Ly.xk = xk; Ly.xv = xv;
+        Ly.conv_w = conv_w; Ly.a_logit = a_logit; Ly.b_logit = b_logit;
+        Ly.cs_in = conv_state_in;
+        Ly.k = ws + W.prefill;
+        Ly.v = ws + W.prefill + W.tens;
+        Ly.g = reinterpret_cast<float *>(ws + W.prefill + 2 * W.tens);
+        Ly.beta = reinterpret_cast<float *>(ws + W.prefill + 2 * W.tens + W.gates);
+        Ly.activation = activation;
+        Ly.eps = eps;
+        Ly.z = z;
+        Ly.norm_w = norm_w;
+        Ly.gate = gate;
+        gdn::TcLaunch L{nullptr, nullptr, nullptr, nullptr, nullptr, state_in, y, state_out, cu_seqlens, uniform_len,
+                        total_tokens, num_seqs, H, workspace, err, g_wait_limit_ns, kWaitLimitNs, &Ly};
+        e = gdn::launch_prefill_tc(L, s);
+    } else {
+        // the three steps one after another through the workspace
+        void *q = ws, *k = ws + W.tens, *v = ws + 2 * W.tens, *o = ws + 3 * W.tens;
+        float *g = reinterpret_cast<float *>(ws + 4 * W.tens);
+        float *beta = reinterpret_cast<float *>(ws + 4 * W.tens + W.gates);
+        if (total_tokens > 0) {
+            gdn::PreprocessArgs A;
+            A.xq = xq; A.xk = xk; A.xv = xv;
+            A.conv_w = conv_w; A.a_logit = a_logit; A.b_logit = b_logit;
+            A.cs_in = conv_state_in;
+            A.q = q; A.k = k; A.v = v; A.g = g; A.beta = beta;
+            A.cs_out = nullptr;
+            A.cu_seqlens = cu_seqlens;
+            A.num_seqs = num_seqs;
+            A.total_tokens = total_tokens;
+            A.H = H; A.d = d; A.activation = activation; A.dtype = dtype;
+            A.eps = eps;
+            e = gdn::launch_preprocess(A, s);
+        }
+        if (e == cudaSuccess)
+            e = gdn::launch_prefill_simt(dtype, d, q, k, v, g, beta, state_in, o, state_out, cu_seqlens, uniform_len,
+                                         num_seqs, H, s);
+        if (e == cudaSuccess && total_tokens > 0)
+            e = gdn::launch_output_gate(dtype, d, o, z, norm_w, y, total_tokens * H, gate, eps, s);
+    }
+    if (e == cudaSuccess && conv_state_out)
+        e = gdn::launch_conv_state(dtype, d, xq, xk, xv, conv_state_in, conv_state_out, cu_seqlens, num_seqs,
+                                   total_tokens, H, s);
     return e == cudaSuccess ? GDN_OK : cuda_fail(e);
 }
 

@@ -33,6 +33,36 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(x);
 }
 
+// sigmoid and SiLU with the fast exponential and division intrinsics
+// (relative error ~1e-6, far below the bf16 storage step; a huge exp(-x)
+// gives 0, the correct limit)
+__device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
+__device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.f + __expf(-x)); }
+
+// The bf16 path's sigmoid and SiLU: sigmoid(x) = (1 + tanh(x / 2)) / 2 with
+// tanh on the special-function unit (tanh.approx.f32, relative error about
+// 2^-11): one SFU op instead of an exponential and a reciprocal, and an
+// absolute error near 2^-12 that the bf16 rounding of the results (2^-9)
+// swamps.  The fp32 path keeps sigmoid_f and silu_f.
+__device__ __forceinline__ float tanh_sfu(float x) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(x));
+    return t;
+}
+__device__ __forceinline__ float sigmoid_t(float x) { return fmaf(0.5f, tanh_sfu(0.5f * x), 0.5f); }
+__device__ __forceinline__ float silu_t(float x) {
+    const float h = 0.5f * x;
+    return fmaf(h, tanh_sfu(h), h);
+}
+// the forms for storage type T
+template <typename T> __device__ __forceinline__ float sigmoid_io(float x) { return sigmoid_f(x); }
+template <> __device__ __forceinline__ float sigmoid_io<__nv_bfloat16>(float x) { return sigmoid_t(x); }
+template <typename T> __device__ __forceinline__ float silu_io(float x) { return silu_f(x); }
+template <> __device__ __forceinline__ float silu_io<__nv_bfloat16>(float x) { return silu_t(x); }
+
+// log(sigmoid(x)) = min(x, 0) - log1p(exp(-|x|)), without overflow
+__device__ __forceinline__ float log_sigmoid_f(float x) { return fminf(x, 0.f) - log1pf(expf(-fabsf(x))); }
+
 // Records e as this host thread's last CUDA error (gdn_last_cuda_error) and
 // returns GDN_ERR_CUDA.
 int note_cuda_error(cudaError_t e);
@@ -64,6 +94,12 @@ struct PreprocessArgs {
     float eps;
 };
 cudaError_t launch_preprocess(const PreprocessArgs &A, cudaStream_t stream);
+// The convolution state after each sequence (the raw inputs at its last three
+// positions, older ones from cs_in); reads every value before writing, so
+// cs_out may equal cs_in.
+cudaError_t launch_conv_state(int dtype, int d, const void *xq, const void *xk, const void *xv, const void *cs_in,
+                              void *cs_out, const int32_t *cu_seqlens, int num_seqs, int64_t total_tokens, int H,
+                              cudaStream_t stream);
 cudaError_t launch_output_gate(int dtype, int dv, const void *o, const void *z, const float *norm_w, void *y,
                                int64_t rows, int gate, float eps, cudaStream_t stream);
 

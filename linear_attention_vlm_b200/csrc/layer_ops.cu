@@ -71,15 +71,6 @@ __device__ __forceinline__ float warp_sum(float s) {
     return s;
 }
 
-// sigmoid and SiLU with the fast exponential and division intrinsics
-// (relative error ~1e-6, far below the bf16 storage step; a huge exp(-x)
-// gives 0, the correct limit)
-__device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
-__device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.f + __expf(-x)); }
-
-// log(sigmoid(x)) = min(x, 0) - log1p(exp(-|x|)), without overflow
-__device__ __forceinline__ float log_sigmoid_f(float x) { return fminf(x, 0.f) - log1pf(expf(-fabsf(x))); }
-
 // Sequence n containing token t: the last n with bos(n) <= t (empty sequences
 // share their start with the next one and are skipped that way).
 __device__ __forceinline__ int seq_of(const SeqBounds &sb, int N, int64_t t) {
@@ -184,7 +175,7 @@ gdn_preprocess_kernel(const T *__restrict__ xq, const T *__restrict__ xk, const 
                     a = fmaf(w[X][j][1], xr[u + 1][j], a);
                     a = fmaf(w[X][j][2], xr[u + 2][j], a);
                     a = fmaf(w[X][j][3], xr[u + 3][j], a);
-                    yv[u][j] = act ? silu_f(a) : a;
+                    yv[u][j] = act ? silu_io<T>(a) : a;
                 }
             if (X < 2) {   // L2 norm per token: 8 independent warp reductions
                 float ss[kPreTokensPerWarp];
@@ -251,7 +242,7 @@ gdn_preprocess_kernel(const T *__restrict__ xq, const T *__restrict__ xk, const 
             }
             if (act) {
 #pragma unroll
-                for (int j = 0; j < CPL; ++j) y[X][j] = silu_f(y[X][j]);
+                for (int j = 0; j < CPL; ++j) y[X][j] = silu_io<T>(y[X][j]);
             }
         }
         float ss[2] = {0.f, 0.f};
@@ -342,7 +333,7 @@ gdn_output_gate_kernel(const T *__restrict__ o, const T *__restrict__ z, const f
         float res[CPL];
 #pragma unroll
         for (int j = 0; j < CPL; ++j) {
-            const float s = sigmoid_f(zv[rr][j]);
+            const float s = sigmoid_io<T>(zv[rr][j]);
             res[j] = ov[rr][j] * sc * wn[j] * (gate ? zv[rr][j] * s : s);
         }
         store_ch<T, CPL>(y + (size_t)r * D + c0, res);
@@ -380,12 +371,8 @@ cudaError_t launch_preprocess_t(const PreprocessArgs &A, cudaStream_t stream) {
     e = cudaGetLastError();
     }
     if (e != cudaSuccess || !A.cs_out) return e;
-    const int work = 3 * A.H * D;
-    const dim3 sgrid((unsigned)A.num_seqs, (unsigned)((work + 255) / 256));
-    gdn_conv_state_kernel<T><<<sgrid, 256, 0, stream>>>(
-        static_cast<const T *>(A.xq), static_cast<const T *>(A.xk), static_cast<const T *>(A.xv),
-        static_cast<const T *>(A.cs_in), static_cast<T *>(A.cs_out), sb, A.H, D);
-    return cudaGetLastError();
+    return launch_conv_state(A.dtype, D, A.xq, A.xk, A.xv, A.cs_in, A.cs_out, A.cu_seqlens, A.num_seqs,
+                             A.total_tokens, A.H, stream);
 }
 
 template <typename T, int D>
@@ -398,7 +385,29 @@ cudaError_t launch_gate_t(const void *o, const void *z, const float *norm_w, voi
     return cudaGetLastError();
 }
 
+template <typename T>
+cudaError_t launch_conv_state_t(int d, const void *xq, const void *xk, const void *xv, const void *cs_in, void *cs_out,
+                                const int32_t *cu_seqlens, int num_seqs, int64_t total_tokens, int H,
+                                cudaStream_t stream) {
+    const SeqBounds sb{cu_seqlens, cu_seqlens ? 0 : total_tokens / num_seqs};
+    const int work = 3 * H * d;
+    const dim3 sgrid((unsigned)num_seqs, (unsigned)((work + 255) / 256));
+    gdn_conv_state_kernel<T><<<sgrid, 256, 0, stream>>>(
+        static_cast<const T *>(xq), static_cast<const T *>(xk), static_cast<const T *>(xv),
+        static_cast<const T *>(cs_in), static_cast<T *>(cs_out), sb, H, d);
+    return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_conv_state(int dtype, int d, const void *xq, const void *xk, const void *xv, const void *cs_in,
+                              void *cs_out, const int32_t *cu_seqlens, int num_seqs, int64_t total_tokens, int H,
+                              cudaStream_t stream) {
+    return dtype == 1 ? launch_conv_state_t<__nv_bfloat16>(d, xq, xk, xv, cs_in, cs_out, cu_seqlens, num_seqs,
+                                                           total_tokens, H, stream)
+                      : launch_conv_state_t<float>(d, xq, xk, xv, cs_in, cs_out, cu_seqlens, num_seqs,
+                                                   total_tokens, H, stream);
+}
 
 cudaError_t launch_preprocess(const PreprocessArgs &A, cudaStream_t stream) {
     if (A.dtype == 1) return A.d == 128 ? launch_preprocess_t<__nv_bfloat16, 128>(A, stream)

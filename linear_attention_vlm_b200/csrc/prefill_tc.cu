@@ -115,7 +115,8 @@ static_assert(ChainLayout<1>::TPP + 8192 == ChainLayout<1>::STAGE, "stage layout
 // After the stages: output staging [64 t][128 dv] bf16, ChainScalars x 3 per
 // chain, mbarriers + TMEM base + abort flag.
 template <int MODE> __host__ __device__ constexpr uint32_t c_u() { return ChainLayout<MODE>::NST * ChainLayout<MODE>::STAGE; }
-template <int MODE> __host__ __device__ constexpr uint32_t c_sce() { return c_u<MODE>() + 16384; }
+// the output stage: [64 t][128 dv] bf16, or fp32 when the output gate is fused (MODE 0, the output pass)
+template <int MODE> __host__ __device__ constexpr uint32_t c_sce() { return c_u<MODE>() + (MODE == 0 ? 32768 : 16384); }
 template <int MODE> __host__ __device__ constexpr uint32_t c_scx() { return c_sce<MODE>() + 3072; }
 template <int MODE> __host__ __device__ constexpr uint32_t c_bar() { return c_scx<MODE>() + 3072; }
 template <int MODE> __host__ __device__ constexpr uint32_t c_alloc() { return c_bar<MODE>() + 256 + 1024; }
@@ -158,6 +159,7 @@ static_assert(sizeof(PrepScalars) == 1536, "scalar block size");
 
 struct PrepParams {
     CUtensorMap map_q, map_k;
+    CUtensorMap map_v;           // layer mode: the raw v projection
     const float *g, *beta;
     const int32_t *cu_seqlens;
     const int32_t *chunk_off;    // varlen: first global chunk of each sequence, [N+1]
@@ -168,6 +170,16 @@ struct PrepParams {
     int *err;
     uint64_t timeout_ns;         // bound on the waits of the work loops
     uint64_t drain_ns;           // bound on the waits that drain copies and MMAs before exit
+    // layer mode (fused pre-processing; map_q, map_k and map_v then cover the
+    // raw projections, and g, beta are unused)
+    int layer;
+    const __nv_bfloat16 *xq, *xk, *xv;     // raw projections (halo rows)
+    const float *conv_w, *a_logit, *b_logit;
+    const __nv_bfloat16 *cs_in;            // [N, 3, 3, H, 128] or null
+    __nv_bfloat16 *k_out, *v_out;          // processed k, v
+    float *g_out, *beta_out;
+    int act;
+    float eps;
 };
 
 struct ChainParams {
@@ -190,6 +202,12 @@ struct ChainParams {
     int *err;
     uint64_t timeout_ns;         // bound on the waits of the work loops
     uint64_t drain_ns;           // bound on the waits that drain copies and MMAs before exit
+    int wait_inputs;             // k, v, g, beta come from the prep kernel (layer mode): wait first
+    // output gate in the output epilogue (z null: plain outputs)
+    const __nv_bfloat16 *z;
+    const float *norm_w;
+    int gate;
+    float eps;
 };
 
 __device__ __forceinline__ uint8_t *aligned_smem(uint8_t *raw) {
@@ -401,8 +419,126 @@ gdn_chunk_offsets_kernel(const int32_t *__restrict__ cu, int N, int32_t *__restr
     if (N == 0 && threadIdx.x == 0) chunk_off[0] = 0;
 }
 
+// ---------------------------------------------------------------- layer pre-processing
+//
+// In layer mode (gdn_layer_prefill) the prep kernel forms its own inputs from
+// the raw projections of its chunk: the TMA brings the raw q, k tiles into the
+// MMA operand slots and the raw v tile into the T' region (idle until the
+// solve), the three positions before the chunk come in as halo rows (the
+// sequence's previous tokens, the carried convolution state, or zeros), and
+//   y = act(sum_i w_i x[t - 3 + i]),   q, k = y / sqrt(|y|^2 + eps),   v = y
+// is computed in place.  Thread (tg, ci) owns the 8 tokens 8 tg .. 8 tg + 7
+// and the 8 channels 8 ci .. 8 ci + 7 of a tensor; the 16 threads of a token
+// row are 16 consecutive lanes, so the L2 norm is a 16-lane butterfly.
+
+// Layer-phase scratch in the scalar block and the solve scratch (both idle
+// until the gates are scanned): two 2 KiB buffers of convolution taps, then
+// the halo rows.  Taps of channel 8 ci + c sit at float4 slot 16 c + ci, so
+// the 16 lanes of a token row read 16 consecutive slots.
+constexpr uint32_t P_LW = P_SC;              // taps, 2 x [8 c][16 ci] float4
+constexpr uint32_t P_LH = P_SC + 4096;       // halo rows [3 X][3 r][16 pieces] of 16 B
+static_assert(P_LH + 2304 <= P_BAR, "layer scratch fits before the barriers");
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// element e (0..7) of a 16-byte piece of 8 bf16
+__device__ __forceinline__ float piece_elem(const uint4 &v, int e) {
+    const uint32_t w = e < 2 ? v.x : (e < 4 ? v.y : (e < 6 ? v.z : v.w));
+    return (e & 1) ? bf16_hi(w) : bf16_lo(w);
+}
+
+// shared-memory offset of piece ci (channels 8 ci .. 8 ci + 7) of row r of
+// tensor X's tile (X: 0 q, 1 k, 2 v)
+__device__ __forceinline__ uint32_t layer_piece_off(int X, int r, int ci) {
+    const uint32_t base = X == 2 ? P_TP + (ci >> 3) * 8192 : P_KQ + (ci >> 3) * 16384 + (X == 0 ? 8192 : 0);
+    return base + sw128_chunk(r, ci & 7);
+}
+
+// the raw row 8 tg - 3 + i (i < 3) of tensor X: from the halo rows for tg = 0
+__device__ __forceinline__ void layer_halo(const uint8_t *sm, int X, int tg, int ci, uint4 (&hl)[3]) {
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+        const int r = 8 * tg - 3 + i;
+        hl[i] = r < 0 ? *reinterpret_cast<const uint4 *>(sm + P_LH + ((X * 3 + r + 3) * 16 + ci) * 16)
+                      : *reinterpret_cast<const uint4 *>(sm + layer_piece_off(X, r, ci));
+    }
+}
+
+// Taps of tensor X (2 KiB of head h) -> tap buffer `buf`, 16 bytes per
+// thread and piece, asynchronously (cp.async group).
+__device__ __forceinline__ void layer_taps_async(const PrepParams &p, uint8_t *sm, int X, int buf, int h, int H,
+                                                 int tid) {
+    for (int i = tid; i < D; i += kPrepThreads) {   // channel i
+        const uint32_t dst = smem_u32(sm + P_LW + buf * 2048 + ((i & 7) * 16 + (i >> 3)) * 16);
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(dst),
+                     "l"(reinterpret_cast<uint64_t>(p.conv_w + (((size_t)X * H + h) * D + i) * 4))
+                     : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// This thread's share of tensor X with the taps in buffer `buf` (rows past
+// the sequence end, r >= len, become 0): q and k back into their operand rows,
+// k and v to `gout` (the workspace).  Channel-outer, so that each raw value is
+// widened once and used by the four outputs it feeds.  One out-of-line copy
+// serves the three tensors: unrolled three times inline, the code no longer
+// fits the instruction cache next to the rest of the kernel.
+__device__ __noinline__ void layer_tensor(uint8_t *sm, int X, int buf, uint4 h0, uint4 h1, uint4 h2, int tg, int ci,
+                                          int h, int H, int64_t t0, int len, __nv_bfloat16 *gout, int act, float eps) {
+    uint4 raw[11];   // rows 8 tg - 3 .. 8 tg + 7
+    raw[0] = h0; raw[1] = h1; raw[2] = h2;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) raw[3 + r] = *reinterpret_cast<const uint4 *>(sm + layer_piece_off(X, 8 * tg + r, ci));
+    const float4 *taps = reinterpret_cast<const float4 *>(sm + P_LW + buf * 2048) + ci;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        float y[4][8], ss[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const float4 w = taps[16 * c];
+            float xr[7];
+#pragma unroll
+            for (int r = 0; r < 7; ++r) xr[r] = piece_elem(raw[4 * half + r], c);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                float a = w.x * xr[u];
+                a = fmaf(w.y, xr[u + 1], a);
+                a = fmaf(w.z, xr[u + 2], a);
+                a = fmaf(w.w, xr[u + 3], a);
+                a = act ? silu_t(a) : a;
+                y[u][c] = a;
+                ss[u] = fmaf(a, a, ss[u]);
+            }
+        }
+        if (X < 2) {
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], o);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float rn = rsqrtf(ss[u] + eps);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) y[u][c] *= rn;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int r = 8 * tg + 4 * half + u;
+            const bool valid = r < len;
+            const uint4 o = valid ? make_uint4(pack_bf16(y[u][0], y[u][1]), pack_bf16(y[u][2], y[u][3]),
+                                               pack_bf16(y[u][4], y[u][5]), pack_bf16(y[u][6], y[u][7]))
+                                  : make_uint4(0u, 0u, 0u, 0u);
+            if (X < 2) *reinterpret_cast<uint4 *>(sm + layer_piece_off(X, r, ci)) = o;
+            if (gout && valid) *reinterpret_cast<uint4 *>(gout + ((size_t)(t0 + r) * H + h) * D + 8 * ci) = o;
+        }
+    }
+}
+
 // ---------------------------------------------------------------- prep kernel
 
+template <bool LAYER>
 __global__ void __launch_bounds__(kPrepThreads, 4)
 gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
     extern __shared__ uint8_t smraw[];
@@ -439,13 +575,44 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
         mbar_init(bar(PB_P1), 1);
         mbar_init(bar(PB_P2), 1);
         fence_mbar_init();
-        // K, Q -> shared memory, in flight during the TMEM allocation
+        // K, Q (layer mode: raw k, q and v) -> shared memory, in flight
+        // during the TMEM allocation
         const int z = (int)t0;
-        mbar_arrive_expect_tx(bar(PB_FULL), 32768);
+        mbar_arrive_expect_tx(bar(PB_FULL), LAYER ? 49152 : 32768);
         for (int kb = 0; kb < 2; ++kb) {
             const uint32_t dst = smem_u32(sm + P_KQ + kb * 16384);
             tma_load_3d(dst, &p.map_k, kb * 64, h, z, bar(PB_FULL));
             tma_load_3d(dst + 8192, &p.map_q, kb * 64, h, z, bar(PB_FULL));
+            if (LAYER) tma_load_3d(smem_u32(sm + P_TP + kb * 8192), &p.map_v, kb * 64, h, z, bar(PB_FULL));
+        }
+    }
+    GateRegs lg{0.f, 0.f, 0.f, 0.f};   // layer mode: g, beta of this chunk (warp 1)
+    if (LAYER) {
+        // halo rows: the raw q, k, v at positions t0 - 3 .. t0 - 1 -> P_MM
+        for (int i = tid; i < 3 * 3 * 16; i += kPrepThreads) {
+            const int X = i / 48, r = (i / 16) % 3, pc = i & 15;
+            const int64_t pos = t0 - 3 + r;
+            const __nv_bfloat16 *src = nullptr;
+            if (pos >= bos) src = (X == 0 ? p.xq : (X == 1 ? p.xk : p.xv)) + ((size_t)pos * H + h) * D + pc * 8;
+            else if (p.cs_in) src = p.cs_in + ((((size_t)nseq * 3 + (pos - bos + 3)) * 3 + X) * H + h) * D + pc * 8;
+            *reinterpret_cast<uint4 *>(sm + P_LH + i * 16) =
+                src ? __ldg(reinterpret_cast<const uint4 *>(src)) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        layer_taps_async(p, sm, 1, 0, h, H, tid);   // k's taps -> buffer 0
+        layer_taps_async(p, sm, 0, 1, h, H, tid);   // q's taps -> buffer 1
+        if (warp == 1) {
+            // g = log sigmoid(a), beta = sigmoid(b) for rows lane and lane + 32
+            const int len = (int)((eos - t0) < C ? (eos - t0) : C);
+            for (int e = 0; e < 2; ++e) {
+                const int r = lane + 32 * e;
+                if (r < len) {
+                    const size_t i = (size_t)(t0 + r) * H + h;
+                    const float gv = log_sigmoid_f(__ldg(p.a_logit + i)), bv = sigmoid_f(__ldg(p.b_logit + i));
+                    p.g_out[i] = gv;
+                    p.beta_out[i] = bv;
+                    if (e == 0) { lg.g0 = gv; lg.b0 = bv; } else { lg.g1 = gv; lg.b1 = bv; }
+                }
+            }
         }
     }
     __syncwarp();
@@ -465,6 +632,29 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     float *mm = reinterpret_cast<float *>(sm + P_MM);          // 4 warps x 16 x 20 fp32
 
+    if (LAYER) {
+        ok = mbar_wait(bar(PB_FULL), 0, lim, &no_abort);   // raw tiles landed
+        asm volatile("cp.async.wait_all;" ::: "memory");  // this thread's taps
+        const int tg = tid >> 4, ci = tid & 15;
+        const int len = (int)((eos - t0) < C ? (eos - t0) : C);
+        uint4 hl[3];
+        // k, then q: every thread reads its halo rows before any rewrites them
+        // (the barrier also publishes the taps)
+        layer_halo(sm, 1, tg, ci, hl);
+        __syncthreads();
+        layer_tensor(sm, 1, 0, hl[0], hl[1], hl[2], tg, ci, h, H, t0, len, p.k_out, p.act, p.eps);
+        layer_halo(sm, 0, tg, ci, hl);
+        __syncthreads();                            // k's taps are read: v's go to buffer 0
+        layer_taps_async(p, sm, 2, 0, h, H, tid);
+        layer_tensor(sm, 0, 1, hl[0], hl[1], hl[2], tg, ci, h, H, t0, len, nullptr, p.act, p.eps);
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        __syncthreads();
+        layer_halo(sm, 2, tg, ci, hl);   // v is read from the T' region and leaves to HBM only
+        layer_tensor(sm, 2, 0, hl[0], hl[1], hl[2], tg, ci, h, H, t0, len, p.v_out, p.act, p.eps);
+        fence_proxy_async_smem();        // the K and Q rows, written here, are MMA operands
+        __syncthreads();
+    }
+
     if (tid == 0) {
         // p1 = [K; Q] K^T -> TMEM columns 0..63
         ok = mbar_wait(bar(PB_FULL), 0, lim, &no_abort);
@@ -479,7 +669,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
         }
         mma_commit(bar(PB_P1));   // also on failure, so that no thread waits out its bound
     } else if (warp == 1) {
-        const GateRegs gr = load_gates(p.g, p.beta, bos, eos, (int)j, (int)j + 1, h, H, lane);
+        const GateRegs gr = LAYER ? lg : load_gates(p.g, p.beta, bos, eos, (int)j, (int)j + 1, h, H, lane);
         float G0, G1;
         scan_gates(gr, lane, G0, G1);
         const float GC = __shfl_sync(0xffffffffu, G1, 31);
@@ -683,7 +873,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
 
 enum { MODE_OUT = 0, MODE_TRANS = 1 };
 
-template <int MODE>
+template <int MODE, bool GATED>
 __global__ void __launch_bounds__(kChainThreads, 1)
 gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
     extern __shared__ uint8_t smraw[];
@@ -739,6 +929,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
     tc_fence_after();
     const uint32_t tm = *tmem_base_ptr;
     const uint64_t lim = p.timeout_ns;
+    if (p.wait_inputs) grid_dep_wait();   // k, v, g and beta are the prep kernel's outputs
     auto fail = [&](int code) {
         *abort_flag = 1;
         if (p.err) atomicCAS(p.err, 0, code);
@@ -1029,6 +1220,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
         const int dv = tid - 128;   // TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>((warp - 4) * 32) << 16;
         __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(sm + c_u<MODE>());
+        float *stagef = reinterpret_cast<float *>(sm + c_u<MODE>());   // gated: the norm and gate take fp32 o
         float a[32], b[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) a[j] = 0.f;
@@ -1037,9 +1229,34 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
         tmem_st32(tm + lane_off + TM_O + 32, a);
         tc_fence_before();
         mbar_arrive(bar(CB_OFREE));
+        // output gate (layer mode): y = n(o) * act(z), n an RMS norm over the
+        // row's d_v values (or the identity); a thread always takes the same
+        // 8 channels (piece dv % 16) of 8 rows, the 16 pieces of a row lying
+        // in 16 consecutive lanes
+        constexpr bool gated = GATED;
+        const int piece = dv & 15;
+        float nw[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) nw[e] = (gated && p.norm_w) ? __ldg(p.norm_w + piece * 8 + e) : 1.f;
+        // z of this thread's pieces of local chunk m (rows past the end: 0)
+        auto load_z = [&](uint4 (&zz)[8], int m) {
+            const int64_t tz = bos + (int64_t)(cb + m) * C;
+            const int lz = m < nloc ? (int)((eos - tz) < C ? (eos - tz) : C) : 0;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int t = 8 * k + (dv >> 4);
+                zz[k] = t < lz ? __ldg(reinterpret_cast<const uint4 *>(p.z + ((size_t)(tz + t) * H + h) * D + piece * 8))
+                               : make_uint4(0u, 0u, 0u, 0u);
+            }
+        };
+        uint4 zr[8], zn[8];   // z of chunk n, and of chunk n + 1 in flight a whole chunk ahead
+        if constexpr (gated) load_z(zr, 0);
         for (int n = 0; n < nloc; ++n) {
             // all four warps are done with chunk n-1's staging buffer
             if (named_bar_any(3, 128, *abort_flag != 0)) break;
+            const int64_t t0 = bos + (int64_t)(cb + n) * C;
+            const int len = (int)((eos - t0) < C ? (eos - t0) : C);
+            if constexpr (gated) load_z(zn, n + 1);
             if (!mbar_wait(bar(CB_C), n & 1, lim, abort_flag)) fail(73);
             tc_fence_after();
             tmem_ld32(tm + lane_off + TM_O, a);
@@ -1053,23 +1270,51 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
             }
             tc_fence_before();
             mbar_arrive(bar(CB_OFREE));   // the MMA thread may accumulate chunk n+1's O^T
+            if constexpr (gated) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                stage[j * D + dv] = __float2bfloat16_rn(a[j]);
-                stage[(32 + j) * D + dv] = __float2bfloat16_rn(b[j]);
+                for (int j = 0; j < 32; ++j) {
+                    stagef[j * D + dv] = a[j];
+                    stagef[(32 + j) * D + dv] = b[j];
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    stage[j * D + dv] = __float2bfloat16_rn(a[j]);
+                    stage[(32 + j) * D + dv] = __float2bfloat16_rn(b[j]);
+                }
             }
             named_bar_sync(3, 128);
             // whole 16-byte pieces of the [64 t][128 dv] tile, rows t < len
-            const int64_t t0 = bos + (int64_t)(cb + n) * C;
-            const int len = (int)((eos - t0) < C ? (eos - t0) : C);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-                const int idx = k * 128 + dv;          // 1024 pieces of 16 bytes
-                const int t = idx >> 4, piece = idx & 15;
-                if (t < len) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(stage + t * D + piece * 8);
-                    *reinterpret_cast<uint4 *>(p.out + ((size_t)(t0 + t) * H + h) * D + piece * 8) = v;
+                const int t = 8 * k + (dv >> 4);       // piece k * 128 + dv of 1024
+                uint4 v;
+                if constexpr (gated) {
+                    const float4 f0 = *reinterpret_cast<const float4 *>(stagef + t * D + piece * 8);
+                    const float4 f1 = *reinterpret_cast<const float4 *>(stagef + t * D + piece * 8 + 4);
+                    const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+                    float ss = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+#pragma unroll
+                    for (int o = 1; o < 16; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                    const float sc = p.norm_w ? rsqrtf(ss * (1.f / D) + p.eps) : 1.f;
+                    float yv[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float zv = piece_elem(zr[k], e), sg = sigmoid_t(zv);
+                        yv[e] = f[e] * sc * nw[e] * (p.gate ? zv * sg : sg);
+                    }
+                    v = make_uint4(pack_bf16(yv[0], yv[1]), pack_bf16(yv[2], yv[3]), pack_bf16(yv[4], yv[5]),
+                                   pack_bf16(yv[6], yv[7]));
+                } else {
+                    v = *reinterpret_cast<const uint4 *>(stage + t * D + piece * 8);
                 }
+                if (t < len) *reinterpret_cast<uint4 *>(p.out + ((size_t)(t0 + t) * H + h) * D + piece * 8) = v;
+            }
+            if constexpr (gated) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) zr[k] = zn[k];
             }
         }
     }
@@ -1351,13 +1596,19 @@ bool set_smem_attrs() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
     if (dev >= 0 && dev < 64 && done[dev]) return true;
-    if (cudaFuncSetAttribute(gdn_chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(gdn_chunk_prep_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)P_ALLOC) != cudaSuccess ||
-        cudaFuncSetAttribute(gdn_chunk_prep_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+        cudaFuncSetAttribute(gdn_chunk_prep_kernel<false>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              100) != cudaSuccess ||
-        cudaFuncSetAttribute(gdn_chunk_chain_kernel<MODE_OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(gdn_chunk_prep_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)P_ALLOC) != cudaSuccess ||
+        cudaFuncSetAttribute(gdn_chunk_prep_kernel<true>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             100) != cudaSuccess ||
+        cudaFuncSetAttribute(gdn_chunk_chain_kernel<MODE_OUT, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)c_alloc<MODE_OUT>()) != cudaSuccess ||
-        cudaFuncSetAttribute(gdn_chunk_chain_kernel<MODE_TRANS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(gdn_chunk_chain_kernel<MODE_OUT, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)c_alloc<MODE_OUT>()) != cudaSuccess ||
+        cudaFuncSetAttribute(gdn_chunk_chain_kernel<MODE_TRANS, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)c_alloc<MODE_TRANS>()) != cudaSuccess ||
         cudaFuncSetAttribute(gdn_scan_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kCombSmem) != cudaSuccess)
@@ -1417,13 +1668,41 @@ cudaError_t launch_prefill_tc(const TcLaunch &L, cudaStream_t stream) {
     ChainParams cp;
     memset(&pp, 0, sizeof(pp));
     memset(&cp, 0, sizeof(cp));
-    if (!make_token_map(&pp.map_q, L.q, L.total_tokens, L.H) ||
-        !make_token_map(&pp.map_k, L.k, L.total_tokens, L.H) ||
-        !make_token_map(&cp.map_v, L.v, L.total_tokens, L.H))
-        return cudaErrorInvalidValue;
-    cp.map_k = pp.map_k;
-    pp.g = cp.g = L.g;
-    pp.beta = cp.beta = L.beta;
+    const TcLayer *Ly = L.layer;
+    if (Ly) {
+        // the prep kernel reads the raw projections; the chains read the
+        // k, v, g and beta it writes
+        if (!make_token_map(&pp.map_q, Ly->xq, L.total_tokens, L.H) ||
+            !make_token_map(&pp.map_k, Ly->xk, L.total_tokens, L.H) ||
+            !make_token_map(&pp.map_v, Ly->xv, L.total_tokens, L.H) ||
+            !make_token_map(&cp.map_k, Ly->k, L.total_tokens, L.H) ||
+            !make_token_map(&cp.map_v, Ly->v, L.total_tokens, L.H))
+            return cudaErrorInvalidValue;
+        pp.layer = 1;
+        pp.xq = static_cast<const __nv_bfloat16 *>(Ly->xq);
+        pp.xk = static_cast<const __nv_bfloat16 *>(Ly->xk);
+        pp.xv = static_cast<const __nv_bfloat16 *>(Ly->xv);
+        pp.conv_w = Ly->conv_w;
+        pp.a_logit = Ly->a_logit;
+        pp.b_logit = Ly->b_logit;
+        pp.cs_in = static_cast<const __nv_bfloat16 *>(Ly->cs_in);
+        pp.k_out = static_cast<__nv_bfloat16 *>(Ly->k);
+        pp.v_out = static_cast<__nv_bfloat16 *>(Ly->v);
+        pp.g_out = Ly->g;
+        pp.beta_out = Ly->beta;
+        pp.act = Ly->activation;
+        pp.eps = Ly->eps;
+        pp.g = cp.g = Ly->g;
+        pp.beta = cp.beta = Ly->beta;
+    } else {
+        if (!make_token_map(&pp.map_q, L.q, L.total_tokens, L.H) ||
+            !make_token_map(&pp.map_k, L.k, L.total_tokens, L.H) ||
+            !make_token_map(&cp.map_v, L.v, L.total_tokens, L.H))
+            return cudaErrorInvalidValue;
+        cp.map_k = pp.map_k;
+        pp.g = cp.g = L.g;
+        pp.beta = cp.beta = L.beta;
+    }
     pp.cu_seqlens = cp.cu_seqlens = L.cu_seqlens;
     pp.chunk_off = cp.chunk_off = chunk_off;
     pp.uniform_len = cp.uniform_len = L.uniform_len;
@@ -1447,7 +1726,10 @@ cudaError_t launch_prefill_tc(const TcLaunch &L, cudaStream_t stream) {
     if (!set_smem_attrs()) return cudaGetLastError() != cudaSuccess ? cudaGetLastError() : cudaErrorUnknown;
     if (varlen) gdn_chunk_offsets_kernel<<<1, 1024, 0, stream>>>(L.cu_seqlens, L.num_seqs, chunk_off);
     dim3 pgrid((unsigned)bound, (unsigned)L.H);
-    gdn_chunk_prep_kernel<<<pgrid, kPrepThreads, P_ALLOC, stream>>>(pp);
+    if (Ly)
+        gdn_chunk_prep_kernel<true><<<pgrid, kPrepThreads, P_ALLOC, stream>>>(pp);
+    else
+        gdn_chunk_prep_kernel<false><<<pgrid, kPrepThreads, P_ALLOC, stream>>>(pp);
     const unsigned units = (unsigned)L.num_seqs * (unsigned)L.H;
     // TRANS, the combine and OUT are launched with programmatic stream
     // serialization: each may start its prologue while the previous kernel
@@ -1457,7 +1739,8 @@ cudaError_t launch_prefill_tc(const TcLaunch &L, cudaStream_t stream) {
         ChainParams ct = cp;
         ct.wait_tiles = 1;
         ct.wait_start = 0;
-        cudaError_t e = launch_pdl(gdn_chunk_chain_kernel<MODE_TRANS>, dim3(units * (nseg - 1)), dim3(kChainThreads),
+        ct.wait_inputs = Ly ? 1 : 0;
+        cudaError_t e = launch_pdl(gdn_chunk_chain_kernel<MODE_TRANS, false>, dim3(units * (nseg - 1)), dim3(kChainThreads),
                                    c_alloc<MODE_TRANS>(), stream, ct);
         if (e != cudaSuccess) return e;
         e = launch_pdl(gdn_scan_combine_kernel, dim3(units, D / kCombRows), dim3(kCombThreads), kCombSmem, stream,
@@ -1468,8 +1751,17 @@ cudaError_t launch_prefill_tc(const TcLaunch &L, cudaStream_t stream) {
     ChainParams co = cp;
     co.wait_tiles = nseg > 1 ? 0 : 1;   // after the combine, the prep kernel has completed
     co.wait_start = nseg > 1 ? 1 : 0;
-    const cudaError_t e = launch_pdl(gdn_chunk_chain_kernel<MODE_OUT>, dim3(units * nseg), dim3(kChainThreads),
-                                     c_alloc<MODE_OUT>(), stream, co);
+    co.wait_inputs = (Ly && nseg == 1) ? 1 : 0;
+    if (Ly && Ly->z) {
+        co.z = static_cast<const __nv_bfloat16 *>(Ly->z);
+        co.norm_w = Ly->norm_w;
+        co.gate = Ly->gate;
+        co.eps = Ly->eps;
+    }
+    const cudaError_t e = co.z ? launch_pdl(gdn_chunk_chain_kernel<MODE_OUT, true>, dim3(units * nseg),
+                                            dim3(kChainThreads), c_alloc<MODE_OUT>(), stream, co)
+                               : launch_pdl(gdn_chunk_chain_kernel<MODE_OUT, false>, dim3(units * nseg),
+                                            dim3(kChainThreads), c_alloc<MODE_OUT>(), stream, co);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -15,6 +15,26 @@ namespace gdn {
 // in the 128-byte-swizzled shared-memory layout of the MMAs.
 constexpr size_t kTileBytes = 49152;
 
+// The layer steps fused into the prefill (gdn_layer_prefill): the prep kernel
+// forms q, k, v, g and beta from the raw projections (causal depthwise
+// convolution of window 4, optional SiLU, q/k L2 norm, beta = sigmoid(b),
+// g = log sigmoid(a)); q stays on chip, k, v, g and beta go to the buffers
+// below for the chain kernels; the output pass writes y = n(o) * act(z)
+// instead of o.
+struct TcLayer {
+    const void *xq, *xk, *xv;          // raw projections [T, H, 128] bf16
+    const float *conv_w;               // [3, H, 128, 4]
+    const float *a_logit, *b_logit;    // [T, H]
+    const void *cs_in;                 // [N, 3, 3, H, 128] bf16, or null (zeros)
+    void *k, *v;                       // processed k, v [T, H, 128] bf16 (written)
+    float *g, *beta;                   // [T, H] (written)
+    int activation;                    // GDN_ACT_NONE / GDN_ACT_SILU
+    float eps;                         // of the q/k L2 norm and of the RMS norm
+    const void *z;                     // output-gate input [T, H, 128] bf16
+    const float *norm_w;               // [128] or null (no RMS norm)
+    int gate;                          // GDN_GATE_SIGMOID / GDN_GATE_SILU
+};
+
 struct TcLaunch {
     const void *q, *k, *v;
     const float *g, *beta, *state_in;
@@ -27,6 +47,7 @@ struct TcLaunch {
     int *err;                    // device status word (0 = ok)
     uint64_t timeout_ns;         // bound on the waits of the kernels' work loops
     uint64_t drain_ns;           // bound on the waits that drain copies and MMAs before exit
+    const TcLayer *layer;        // null: plain prefill of q, k, v, g, beta into out
 };
 
 // Upper bound on the number of 64-token chunks of a packed batch.

@@ -49,21 +49,25 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? GDN_OK : gdn::note_cu
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // The layer step for `tokens` tokens per stream (0: one decode token per
-// stream), enqueued on `st` through the public entry points.
+// stream), enqueued on `st` through the public entry points: a segment is one
+// gdn_layer_prefill call (pre-processing and output gate fused into the
+// prefill kernels on the tensor-core path), a decode token is
+// gdn_preprocess -> gdn_decode_step -> gdn_output_gate.
 int enqueue_step(gdn_session *s, int tokens, cudaStream_t st) {
     const gdn_session_buffers_t &b = s->buf;
     const int B = s->B, H = s->H, d = s->d;
-    const int64_t T = (int64_t)B * (tokens > 0 ? tokens : 1);
+    if (tokens > 0) {
+        const int64_t T = (int64_t)B * tokens;
+        return gdn_layer_prefill(b.xq, b.xk, b.xv, b.conv_w, b.a, b.b, b.conv_state, b.conv_state, b.state, b.state,
+                                 b.z, b.norm_w, b.y, nullptr, B, T, H, d, s->activation, s->gate, s->eps, s->dtype,
+                                 b.workspace, b.workspace_bytes, st);
+    }
     int rc = gdn_preprocess(b.xq, b.xk, b.xv, b.conv_w, b.a, b.b, b.conv_state, b.q, b.k, b.v, b.g, b.beta,
-                            b.conv_state, nullptr, B, T, H, d, s->activation, s->eps, s->dtype, st);
+                            b.conv_state, nullptr, B, B, H, d, s->activation, s->eps, s->dtype, st);
     if (rc != GDN_OK) return rc;
-    if (tokens > 0)
-        rc = gdn_prefill(b.q, b.k, b.v, b.g, b.beta, b.state, b.o, b.state, nullptr, B, T, H, d, d, gdn::kChunk,
-                         s->dtype, b.workspace, b.workspace_bytes, st);
-    else
-        rc = gdn_decode_step(b.q, b.k, b.v, b.g, b.beta, b.state, b.state, b.o, B, H, d, d, s->dtype, st);
+    rc = gdn_decode_step(b.q, b.k, b.v, b.g, b.beta, b.state, b.state, b.o, B, H, d, d, s->dtype, st);
     if (rc != GDN_OK) return rc;
-    return gdn_output_gate(b.o, b.z, b.norm_w, b.y, T * H, d, s->gate, s->eps, s->dtype, st);
+    return gdn_output_gate(b.o, b.z, b.norm_w, b.y, (int64_t)B * H, d, s->gate, s->eps, s->dtype, st);
 }
 
 // Instantiated graph of the step for `tokens`, captured on first use.
@@ -114,7 +118,7 @@ extern "C" {
 
 size_t gdn_session_workspace_size(int num_streams, int H, int d, int seg_tokens, int dtype) {
     if (num_streams < 1 || seg_tokens < 1) return 0;
-    return gdn_prefill_workspace_size(num_streams, (int64_t)num_streams * seg_tokens, H, d, d, gdn::kChunk, dtype);
+    return gdn_layer_prefill_workspace_size(num_streams, (int64_t)num_streams * seg_tokens, H, d, dtype);
 }
 
 int gdn_session_create(int num_streams, int H, int d, int seg_tokens, int dtype, int activation, int gate,

@@ -65,6 +65,11 @@ def _load():
     lib.gdn_preprocess.restype = i32
     lib.gdn_output_gate.argtypes = [vp, vp, fp, vp, i64, i32, i32, f32, i32, vp]
     lib.gdn_output_gate.restype = i32
+    lib.gdn_layer_prefill_workspace_size.argtypes = [i32, i64, i32, i32, i32]
+    lib.gdn_layer_prefill_workspace_size.restype = sz
+    lib.gdn_layer_prefill.argtypes = [vp, vp, vp, fp, fp, fp, vp, vp, fp, fp, vp, fp, vp, vp, i32, i64, i32, i32,
+                                      i32, i32, f32, i32, vp, sz, vp]
+    lib.gdn_layer_prefill.restype = i32
     lib.gdn_rope.argtypes = [vp, vp, vp, i32, i64, i32, i32, i32, f32, i32, vp]
     lib.gdn_rope.restype = i32
     lib.gdn_swa_attention.argtypes = [vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, f32, i32, vp, vp]
@@ -368,6 +373,68 @@ def gdn_output_gate(o: torch.Tensor, z: torch.Tensor, norm_w: Optional[torch.Ten
     if st != GDN_OK:
         raise GdnError(st, "gdn_output_gate")
     return out
+
+
+def gdn_layer_prefill_workspace_size(num_seqs: int, total_tokens: int, H: int, d: int,
+                                     dtype: torch.dtype = torch.bfloat16) -> int:
+    return int(_load().gdn_layer_prefill_workspace_size(num_seqs, total_tokens, H, d, _dtype_code(dtype)))
+
+
+def gdn_layer_prefill(xq: torch.Tensor, xk: torch.Tensor, xv: torch.Tensor, conv_w: torch.Tensor,
+                      a: torch.Tensor, b: torch.Tensor, z: torch.Tensor,
+                      conv_state_in: Optional[torch.Tensor] = None, state_in: Optional[torch.Tensor] = None,
+                      norm_w: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None, *,
+                      num_seqs: Optional[int] = None, activation: int = ACT_NONE, gate: int = GATE_SIGMOID,
+                      eps: float = 1e-6, y: Optional[torch.Tensor] = None,
+                      state_out: Optional[torch.Tensor] = None, conv_state_out: Optional[torch.Tensor] = None,
+                      workspace: Optional[torch.Tensor] = None, want_state: bool = True,
+                      want_conv_state: bool = True):
+    """Raw projections -> gated output of one layer's token mixer
+    (include/gdn.h, gdn_layer_prefill).  xq, xk, xv, z [T, H, d]; conv_w
+    [3, H, d, 4] fp32; a, b [T, H] fp32 logits; conv_state_in [N, 3, 3, H, d]
+    or None; state_in [N, H, d, d] fp32 or None; norm_w [d] fp32 or None.
+    Returns (y, state_out, conv_state_out); pass state_out=state_in and
+    conv_state_out=conv_state_in to carry both states in place."""
+    T, H, d = xq.shape
+    dev = xq.device
+    if dev.type != "cuda":
+        raise ValueError("gdn_layer_prefill needs CUDA tensors")
+    for t in (xk, xv, z):
+        if t.shape != (T, H, d) or t.dtype != xq.dtype:
+            raise ValueError("xq, xk, xv and z must share shape [T, H, d] and dtype")
+    if conv_w.shape != (3, H, d, 4) or conv_w.dtype != torch.float32:
+        raise ValueError("conv_w must be fp32 [3, H, d, 4]")
+    if a.shape != (T, H) or b.shape != (T, H) or a.dtype != torch.float32 or b.dtype != torch.float32:
+        raise ValueError("a and b must be fp32 [T, H]")
+    N = _seq_count(cu_seqlens, num_seqs, dev)
+    if conv_state_in is not None and (conv_state_in.shape != (N, 3, 3, H, d) or conv_state_in.dtype != xq.dtype):
+        raise ValueError("conv_state_in must be [N, 3, 3, H, d] in the dtype of x")
+    if state_in is not None and (state_in.shape != (N, H, d, d) or state_in.dtype != torch.float32):
+        raise ValueError("state_in must be fp32 [N, H, d, d]")
+    if norm_w is not None and (norm_w.shape != (d,) or norm_w.dtype != torch.float32):
+        raise ValueError("norm_w must be fp32 [d]")
+    for t in (xk, xv, z, conv_w, a, b, conv_state_in, state_in, norm_w, cu_seqlens, y, state_out,
+              conv_state_out, workspace):
+        if t is not None and t.device != dev:
+            raise ValueError("all tensors must be on %s" % dev)
+    if y is None:
+        y = torch.empty_like(xq)
+    if state_out is None and want_state:
+        state_out = torch.empty((N, H, d, d), dtype=torch.float32, device=dev)
+    if conv_state_out is None and want_conv_state:
+        conv_state_out = torch.empty((N, 3, 3, H, d), dtype=xq.dtype, device=dev)
+    need = gdn_layer_prefill_workspace_size(N, T, H, d, xq.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = _load().gdn_layer_prefill(_ptr(xq), _ptr(xk), _ptr(xv), _ptr(conv_w), _ptr(a), _ptr(b),
+                                   _ptr(conv_state_in), _ptr(conv_state_out), _ptr(state_in), _ptr(state_out),
+                                   _ptr(z), _ptr(norm_w), _ptr(y), _ptr(cu_seqlens), N, T, H, d, int(activation),
+                                   int(gate), float(eps), _dtype_code(xq.dtype), _ptr(workspace), ws_bytes,
+                                   _stream(dev))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_layer_prefill")
+    return y, state_out, conv_state_out
 
 
 def _seq_count(cu_seqlens: Optional[torch.Tensor], num_seqs: Optional[int], dev) -> int:
