@@ -147,8 +147,11 @@ def test_long_prefill_segmented(cuda_device):
     gap_s = rel_err(np64(st), np64(st_whole))
     gap_o = rel_err(np64(outs[-1]), np64(out_whole[-64:]))
     print("segmented vs whole: state gap %.3g, last-chunk output gap %.3g" % (gap_s, gap_o))
-    assert gap_s <= 2e-2
-    assert gap_o <= 2e-2
+    # bounds: four times the gaps measured on B200 (state 5.7e-5, last-chunk
+    # output 2.1e-3), far inside the bf16 bar, so that a carried-state error at
+    # a segment or range boundary cannot hide behind it
+    assert gap_s <= 2.5e-4
+    assert gap_o <= 9e-3
     heads = [5]
     sub = W.prefill_inputs(w, seed=0, heads=heads)
     ro, rs = run_oracle(sub)
