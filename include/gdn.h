@@ -153,8 +153,8 @@ int gdn_prefill_kernel_count(int num_seqs, int64_t total_tokens, int H, int dk, 
  *
  * The function calls no cudaMalloc, cudaFree or other allocating routine.  The
  * first call on a device looks the array's device address up (with that
- * device current) and caches it; make that first call before any stream
- * capture.  Every call on a device shares the one array: calls whose work
+ * device current) and caches it.  Every call on a device shares the one
+ * array: calls whose work
  * overlaps on the GPU (different streams, or other host threads) race on it
  * and must be serialised by the caller.  Each call clears what has to start
  * at zero, so stale contents from an earlier call are harmless.

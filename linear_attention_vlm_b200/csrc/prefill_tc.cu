@@ -947,8 +947,10 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                 }
                 if (MODE == MODE_TRANS) {
                     *reinterpret_cast<float4 *>(p.trans_r + unit * D * D + (size_t)tid * D + j) = make_float4(0.f, 0.f, 0.f, 0.f);
-                    // M = I: hi = I, lo = 0; row tid, column pairs j/2, j/2 + 1
-                    uint32_t *hi = reinterpret_cast<uint32_t *>(p.trans_m + unit * D * D) + (size_t)tid * (D / 2) + j / 2;
+                    // M = I: hi = I, lo = 0; row tid, columns j .. j + 3 (in the
+                    // combine's swizzled layout: piece j / 8 stored at (j / 8) ^ (tid & 7))
+                    uint32_t *hi = reinterpret_cast<uint32_t *>(p.trans_m + unit * D * D) + (size_t)tid * (D / 2) +
+                                   4 * ((j >> 3) ^ (tid & 7)) + ((j >> 1) & 3);
                     uint32_t *lo = hi + D * D / 2;
                     hi[0] = pack_bf16(tid == j ? 1.f : 0.f, tid == j + 1 ? 1.f : 0.f);
                     hi[1] = pack_bf16(tid == j + 2 ? 1.f : 0.f, tid == j + 3 ? 1.f : 0.f);
@@ -1371,11 +1373,15 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                                             : (finish ? finish + state_off : nullptr);
             if (!dst) break;
             const float *stg = reinterpret_cast<const float *>(sm) + c * D * PITCH;
-            if (MODE == MODE_TRANS && c == 1) {   // 2 D rows of 16 pieces (hi, then lo)
+            if (MODE == MODE_TRANS && c == 1) {
+                // 2 D rows of 16 pieces (hi, then lo); piece p of row r is stored at
+                // p ^ (r & 7), the swizzle under which the combine's ldmatrix reads
+                // eight rows at one column without bank conflicts
                 const uint32_t *sh = reinterpret_cast<const uint32_t *>(stg);
                 for (int i = threadIdx.x; i < 2 * D * 16; i += blockDim.x) {
                     const int row = i >> 4, piece = i & 15;
-                    reinterpret_cast<uint4 *>(dst)[i] = *reinterpret_cast<const uint4 *>(sh + row * MPW + 4 * piece);
+                    reinterpret_cast<uint4 *>(dst)[row * 16 + (piece ^ (row & 7))] =
+                        *reinterpret_cast<const uint4 *>(sh + row * MPW + 4 * piece);
                 }
                 continue;
             }
@@ -1404,21 +1410,18 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
 // The products run on bf16 mma.sync with each fp32 operand split in two
 // (x = hi + lo, both bf16; S M ~= S_hi M_hi + S_hi M_lo + S_lo M_hi), which
 // keeps about 16 mantissa bits; accumulation is fp32.  M_j arrives already
-// split from the transition ranges (bf16 hi and lo rows [k][n]), ldmatrix
-// (.trans) turns its rows into B fragments, and it streams into the other
-// half of a double buffer (cp.async) while step j computes.
+// split from the transition ranges (bf16 hi and lo rows [k][n], each row's
+// 16-byte pieces swizzled by row % 8) and ldmatrix (.trans) turns its rows into
+// B fragments.  M_{j+1} and this CTA's rows of R_{j+1} stream into the other
+// half of a double buffer as bulk copies (one thread, an mbarrier) while step
+// j computes.
 constexpr int kCombRows = 16;
 constexpr int kCombThreads = 256;
-constexpr int kCombMB = 136, kCombSP = 136, kCombPP = 132;   // row pitches: conflict-free fragments
-constexpr size_t kCombMBuf = (size_t)2 * D * kCombMB;         // bf16 per buffer: hi then lo
-constexpr size_t kCombSmem =
-    (size_t)2 * kCombMBuf * sizeof(__nv_bfloat16) + (size_t)(kCombRows * kCombSP + 4 * kCombRows * kCombPP) * sizeof(float);
-
-__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)),
-                 "l"(reinterpret_cast<uint64_t>(src))
-                 : "memory");
-}
+constexpr int kCombSP = 136, kCombPP = 132;                     // row pitches: conflict-free fragments
+constexpr uint32_t kCombMBytes = 2 * D * D * 2;                 // M_j: hi and lo bf16 rows
+constexpr uint32_t kCombRBytes = kCombRows * D * 4;             // 16 rows of R_j
+constexpr uint32_t kCombBufBytes = kCombMBytes + kCombRBytes;
+constexpr size_t kCombSmem = (size_t)2 * kCombBufBytes + (size_t)(kCombRows * kCombSP + 4 * kCombRows * kCombPP) * 4 + 64;
 
 // four 8x8 bf16 blocks, transposed on the way: the col-major B fragments of mma.sync
 __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const __nv_bfloat16 *row) {
@@ -1439,46 +1442,64 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
 __global__ void __launch_bounds__(kCombThreads, 1)
 gdn_scan_combine_kernel(const float *__restrict__ state_in, const float *__restrict__ trans_r,
                         const float *__restrict__ trans_m, float *__restrict__ seg_start, int nseg,
-                        int *err, uint64_t timeout_ns) {
-    (void)err;
-    (void)timeout_ns;
-    extern __shared__ float smf[];
-    __nv_bfloat16 *Mb = reinterpret_cast<__nv_bfloat16 *>(smf);   // M_j hi, lo rows [k][n], two buffers
-    float *Ss = reinterpret_cast<float *>(Mb + 2 * kCombMBuf);    // S_j rows [16][D]
-    float *Ps = Ss + kCombRows * kCombSP;                          // k-slice partials [4][16][D]
+                        int *err, uint64_t timeout_ns, uint64_t drain_ns) {
+    extern __shared__ __align__(128) uint8_t smc[];
+    // [buffer 0: M hi, M lo, R rows][buffer 1: the same][S_j rows][partials][2 mbarriers, abort flag]
+    float *Ss = reinterpret_cast<float *>(smc + 2 * kCombBufBytes);   // S_j rows [16][D]
+    float *Ps = Ss + kCombRows * kCombSP;                               // k-slice partials [4][16][D]
+    uint8_t *ctl = reinterpret_cast<uint8_t *>(Ps + 4 * kCombRows * kCombPP);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(ctl + 16);
+    auto bar = [&](int b) { return smem_u32(ctl + 8 * b); };
     const int nh = blockIdx.x, r0 = blockIdx.y * kCombRows;
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31, g = lane >> 2, q = lane & 3;
     const int kg = warp >> 1, ch = warp & 1;
+    if (t == 0) {
+        mbar_init(bar(0), 1);
+        mbar_init(bar(1), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
     grid_dep_wait();     // the transitions come from the previous kernel
     grid_dep_launch();   // the output pass may launch; its first ranges do not need this grid
-    auto stage = [&](int j) {
-        // 2 x 128 rows of 256 bytes (16 pieces each) into rows of kCombMB bf16
-        const __nv_bfloat16 *src = reinterpret_cast<const __nv_bfloat16 *>(trans_m + ((size_t)nh * (nseg - 1) + j) * D * D);
-        __nv_bfloat16 *dst = Mb + (j & 1) * kCombMBuf;
-        for (int i = t; i < 2 * D * 16; i += kCombThreads) {
-            const int row = i >> 4, piece = i & 15;   // row: hi rows 0..127, then lo rows
-            cp_async16(dst + row * kCombMB + piece * 8, src + row * D + piece * 8);
-        }
-        asm volatile("cp.async.commit_group;" ::: "memory");
+    auto stage = [&](int j) {   // thread 0
+        const size_t unit = ((size_t)nh * (nseg - 1) + j) * D * D;
+        const uint32_t dst = smem_u32(smc + (j & 1) * kCombBufBytes);
+        mbar_arrive_expect_tx(bar(j & 1), kCombBufBytes);
+        for (uint32_t o = 0; o < kCombMBytes; o += 16384)
+            bulk_load(dst + o, reinterpret_cast<const uint8_t *>(trans_m + unit) + o, 16384, bar(j & 1));
+        bulk_load(dst + kCombMBytes, trans_r + unit + (size_t)r0 * D, kCombRBytes, bar(j & 1));
     };
-    if (nseg > 1) stage(0);
+    int pending = -1;   // the last step whose copies were issued and not yet waited for
+    if (nseg > 1 && t == 0) stage(0);
+    if (nseg > 1) pending = 0;
     for (int i = t; i < kCombRows * D; i += kCombThreads)
         Ss[(i >> 7) * kCombSP + (i & 127)] =
             state_in ? state_in[(size_t)nh * D * D + (size_t)(r0 + (i >> 7)) * D + (i & 127)] : 0.f;
     for (int j = 0; j + 1 < nseg; ++j) {
         const size_t u = ((size_t)nh * (nseg - 1) + j) * D * D + (size_t)r0 * D;   // rows r0.. of step j
-        float rv[kCombRows * D / kCombThreads];
-#pragma unroll
-        for (int i = 0; i < kCombRows * D / kCombThreads; ++i) rv[i] = trans_r[u + t + kCombThreads * i];
         float acc[8][4], accx[8][4];   // hi*hi terms; the two cross terms
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[nt][e] = accx[nt][e] = 0.f;
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
-        __syncthreads();   // M_j landed for every thread; S_j rows are written
-        if (j + 2 < nseg) stage(j + 1);
-        const __nv_bfloat16 *Mh = Mb + (j & 1) * kCombMBuf, *Ml = Mh + D * kCombMB;
+        if (!mbar_wait(bar(j & 1), (j >> 1) & 1, timeout_ns, abort_flag)) {
+            *abort_flag = 1;
+            if (err) atomicCAS(err, 0, 81);
+        }
+        __syncthreads();   // M_j and R_j landed (or the wait gave up); S_j rows are written
+        if (*abort_flag) break;
+        pending = -1;
+        if (j + 2 < nseg) {
+            if (t == 0) {
+                fence_proxy_async_smem();   // step j-1's reads of that buffer come before the copy
+                stage(j + 1);
+            }
+            pending = j + 1;
+        }
+        const __nv_bfloat16 *Mh = reinterpret_cast<const __nv_bfloat16 *>(smc + (j & 1) * kCombBufBytes);
+        const __nv_bfloat16 *Ml = Mh + D * D;
+        const float *Rs = reinterpret_cast<const float *>(smc + (j & 1) * kCombBufBytes + kCombMBytes);
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks) {
             const int k0 = 32 * kg + 16 * ks;
@@ -1492,15 +1513,15 @@ gdn_scan_combine_kernel(const float *__restrict__ state_in, const float *__restr
             split2(s01.x, s01.y, ah[2], al[2]);
             split2(s11.x, s11.y, ah[3], al[3]);
             // lane -> row of one of four 8x8 blocks: k0 + (lane & 7) + 8 ((lane >> 3) & 1),
-            // columns n0 + 8 (lane >> 4); .trans turns them into the B fragments
-            // {b0, b1} of n-tiles 2 pr and 2 pr + 1
-            const int krow = k0 + (lane & 7) + 8 * ((lane >> 3) & 1), ncol = 8 * (lane >> 4);
+            // 16-byte piece 8 ch + 2 pr + (lane >> 4) of that row (stored at piece ^ (row % 8));
+            // .trans turns them into the B fragments {b0, b1} of n-tiles 2 pr and 2 pr + 1
+            const int krow = k0 + (lane & 7) + 8 * ((lane >> 3) & 1);
 #pragma unroll
             for (int pr = 0; pr < 4; ++pr) {
-                const int n0 = 64 * ch + 16 * pr;
+                const int off = krow * D + (((8 * ch + 2 * pr + (lane >> 4)) ^ (krow & 7)) << 3);
                 uint32_t bh[4], bl[4];
-                ldmatrix_x4_trans(bh, Mh + krow * kCombMB + n0 + ncol);
-                ldmatrix_x4_trans(bl, Ml + krow * kCombMB + n0 + ncol);
+                ldmatrix_x4_trans(bh, Mh + off);
+                ldmatrix_x4_trans(bl, Ml + off);
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
                     const int nt = 2 * pr + u;
@@ -1523,13 +1544,16 @@ gdn_scan_combine_kernel(const float *__restrict__ state_in, const float *__restr
 #pragma unroll
         for (int i = 0; i < kCombRows * D / kCombThreads; ++i) {
             const int e = t + kCombThreads * i, row = e >> 7, col = e & 127;
-            float v = rv[i];
+            float v = Rs[e];
 #pragma unroll
             for (int s = 0; s < 4; ++s) v += Ps[(s * kCombRows + row) * kCombPP + col];
             seg_start[u + e] = v;
             Ss[row * kCombSP + col] = v;
         }
     }
+    // no bulk copy may still be landing in shared memory at exit
+    const int zero = 0;
+    if (t == 0 && pending >= 0) mbar_wait(bar(pending & 1), (pending >> 1) & 1, drain_ns, &zero);
 }
 
 // ---------------------------------------------------------------- host side
@@ -1745,7 +1769,7 @@ cudaError_t launch_prefill_tc(const TcLaunch &L, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         e = launch_pdl(gdn_scan_combine_kernel, dim3(units, D / kCombRows), dim3(kCombThreads), kCombSmem, stream,
                        L.state_in, static_cast<const float *>(cp.trans_r), static_cast<const float *>(cp.trans_m),
-                       const_cast<float *>(cp.seg_start), nseg, L.err, L.timeout_ns);
+                       const_cast<float *>(cp.seg_start), nseg, L.err, L.timeout_ns, L.drain_ns);
         if (e != cudaSuccess) return e;
     }
     ChainParams co = cp;
