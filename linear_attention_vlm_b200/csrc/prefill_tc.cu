@@ -906,7 +906,38 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                          : (seg == 0 ? p.state_in : p.seg_start + unit * D * D);
     float *finish = MODE == MODE_TRANS ? nullptr : (seg == p.nseg - 1 ? p.state_out : nullptr);
 
-    if (tid == 0) {
+    // The copies of local chunk n into its stage (K and V boxes, the prep
+    // tile or the part of it a transition range reads), completing on the
+    // stage's FULL barrier.  A transition range reads K, V, -W and T'' of
+    // chunks that the output pass reads again after the combine: it keeps them
+    // in L2 (evict_last); the output pass reads them for the last time.
+    auto issue_stage = [&](int n, uint64_t pol) {
+        const int s = n % NST;
+        const uint32_t st = smem_u32(sm + s * Lay::STAGE);
+        const int z = (int)(bos + (int64_t)(cb + n) * C);
+        const uint32_t full = bar(CB_FULL + s);
+        const uint8_t *tile = p.tiles + ((size_t)(gc0 + n) * H + h) * kTileBytes;
+        mbar_arrive_expect_tx(full, Lay::STAGE);
+        for (int kb = 0; kb < 2; ++kb) {
+            tma_load_3d_hint(st + Lay::K + kb * 8192, &p.map_k, kb * 64, h, z, full, pol);
+            tma_load_3d_hint(st + Lay::V + kb * 8192, &p.map_v, kb * 64, h, z, full, pol);
+        }
+        if (n == 0 && p.wait_tiles) grid_dep_wait();   // tiles come from the prep kernel
+        if (MODE == MODE_TRANS) {   // -W and T'' of the tile
+            bulk_load_hint(st + ChainLayout<1>::W, tile + TILE_NEGW, 8192, full, pol);
+            bulk_load_hint(st + ChainLayout<1>::W + 8192, tile + 16384 + TILE_NEGW, 8192, full, pol);
+            bulk_load_hint(st + ChainLayout<1>::TPP, tile + TILE_TPP, 8192, full, pol);
+        } else {
+            bulk_load_hint(st + ChainLayout<0>::WQ, tile, (uint32_t)kTileBytes, full, pol);
+        }
+    };
+    // When nothing upstream still writes this kernel's inputs (an output
+    // range after the combine: the tiles are complete and K, V are inputs),
+    // the load thread initialises the barriers itself and has the first
+    // stages in flight before the rest of the prologue.
+    const bool early = !p.wait_tiles && !p.wait_inputs;
+    const int n_early = early ? min(NST, nloc) : 0;
+    if (warp == 9 && lane == 0) {
         for (int i = 0; i < CB_NUM; ++i) {
             uint32_t cnt = (i == CB_SREADY || i == CB_UREADY || i == CB_SREADY2 || i == CB_UREADY2 ||
                             i == CB_OFREE) ? 128 : 1;
@@ -915,14 +946,14 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
         }
         *abort_flag = 0;
         fence_mbar_init();
+        tma_prefetch_desc(&p.map_k);
+        tma_prefetch_desc(&p.map_v);
+        const uint64_t pol0 = MODE == MODE_TRANS ? l2_evict_last_policy() : l2_evict_first_policy();
+        for (int n = 0; n < n_early; ++n) issue_stage(n, pol0);
     }
     if (warp == 8) {
         tmem_alloc(smem_u32(tmem_base_ptr), TM_COLS);
         tmem_relinquish();
-    }
-    if (warp == 9 && lane == 0) {
-        tma_prefetch_desc(&p.map_k);
-        tma_prefetch_desc(&p.map_v);
     }
     tc_fence_before();
     __syncthreads();
@@ -964,6 +995,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
         if (lane == 0) {
             const uint64_t l2pol = MODE == MODE_TRANS ? l2_evict_last_policy() : l2_evict_first_policy();
             int issued[NST] = {};
+            for (int s = 0; s < n_early; ++s) issued[s] = 1;
             // Pull chunk m's data into L2 while its stage is still in use, so
             // that the copy into shared memory, once the stage frees up, is an
             // L2 hit.
@@ -982,34 +1014,13 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                     bulk_prefetch_l2(tm_, (uint32_t)kTileBytes);
                 }
             };
-            for (int n = 0; n < nloc; ++n) {
+            for (int n = n_early; n < nloc; ++n) {
                 const int s = n % NST;
-                const uint32_t st = smem_u32(sm + s * Lay::STAGE);
-                const int z = (int)(bos + (int64_t)(cb + n) * C);
                 if (n >= NST) {
                     prefetch(n);   // (the tiles are complete: the wait below chunk 0's loads came first)
                     if (!mbar_wait(bar(CB_EMPTY + s), ((n - NST) / NST) & 1, lim, abort_flag)) { fail(61); break; }
                 }
-                const uint32_t full = bar(CB_FULL + s);
-                const uint8_t *tile = p.tiles + ((size_t)(gc0 + n) * H + h) * kTileBytes;
-                // A transition range reads K, V, -W and T'' of chunks that the
-                // output pass reads again after the combine: keep them in L2
-                // (evict_last).  The output pass reads them for the last time.
-                const uint64_t pol = l2pol;
-                // a transition range reads -W and T'' only
-                mbar_arrive_expect_tx(full, Lay::STAGE);
-                for (int kb = 0; kb < 2; ++kb) {
-                    tma_load_3d_hint(st + Lay::K + kb * 8192, &p.map_k, kb * 64, h, z, full, pol);
-                    tma_load_3d_hint(st + Lay::V + kb * 8192, &p.map_v, kb * 64, h, z, full, pol);
-                }
-                if (n == 0 && p.wait_tiles) grid_dep_wait();   // tiles come from the prep kernel
-                if (MODE == MODE_TRANS) {   // -W and T'' of the tile
-                    bulk_load_hint(st + ChainLayout<1>::W, tile + TILE_NEGW, 8192, full, pol);
-                    bulk_load_hint(st + ChainLayout<1>::W + 8192, tile + 16384 + TILE_NEGW, 8192, full, pol);
-                    bulk_load_hint(st + ChainLayout<1>::TPP, tile + TILE_TPP, 8192, full, pol);
-                } else {
-                    bulk_load_hint(st + ChainLayout<0>::WQ, tile, (uint32_t)kTileBytes, full, pol);
-                }
+                issue_stage(n, l2pol);
                 ++issued[s];
             }
             const int zero = 0;   // no copy may still be landing in shared memory at exit
