@@ -70,7 +70,7 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
 size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
 
 // Workspace of gdn_layer_prefill.  Tensor-core path: [prefill workspace]
-// [k][v] (processed, dtype) [g][beta] (fp32); otherwise [q][k][v][o][g][beta].
+// [q][k][v] (processed, dtype) [g][beta] (fp32); otherwise [q][k][v][o][g][beta].
 struct LayerWs {
     size_t prefill, tens, gates, total;
 };
@@ -82,7 +82,7 @@ LayerWs layer_ws(int num_seqs, int64_t total_tokens, int H, int d, int dtype) {
     w.gates = align256((size_t)total_tokens * H * 4);
     if (use_tc(total_tokens, d, dtype)) {
         w.prefill = align256(gdn::tc_workspace_bytes(num_seqs, total_tokens, H, /*varlen=*/true));
-        w.total = w.prefill + 2 * w.tens + 2 * w.gates;
+        w.total = w.prefill + 3 * w.tens + 2 * w.gates;
     } else {
         w.total = 4 * w.tens + 2 * w.gates;
     }
@@ -335,10 +335,11 @@ int gdn_layer_prefill(const void *xq, const void *xk, const void *xv, const floa
         Ly.xq = xq; Ly.xk = xk; Ly.xv = xv;
         Ly.conv_w = conv_w; Ly.a_logit = a_logit; Ly.b_logit = b_logit;
         Ly.cs_in = conv_state_in;
-        Ly.k = ws + W.prefill;
-        Ly.v = ws + W.prefill + W.tens;
-        Ly.g = reinterpret_cast<float *>(ws + W.prefill + 2 * W.tens);
-        Ly.beta = reinterpret_cast<float *>(ws + W.prefill + 2 * W.tens + W.gates);
+        Ly.q = ws + W.prefill;
+        Ly.k = ws + W.prefill + W.tens;
+        Ly.v = ws + W.prefill + 2 * W.tens;
+        Ly.g = reinterpret_cast<float *>(ws + W.prefill + 3 * W.tens);
+        Ly.beta = reinterpret_cast<float *>(ws + W.prefill + 3 * W.tens + W.gates);
         Ly.activation = activation;
         Ly.eps = eps;
         Ly.z = z;

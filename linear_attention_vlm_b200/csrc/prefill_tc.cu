@@ -6,36 +6,38 @@
 //
 //   A    = strict_lower(beta_r exp(G_r - G_i) k_r.k_i),   T = (I + A)^-1
 //   T'   = diag(D) T diag(beta gamma),   T'' = diag(D) T diag(beta)
-//   W    = T' K,   Qg = diag(gamma) Q,   Pt = diag(exp(G_t - G_C)) tril(Q K^T)
+//   W    = T' K,   Pt = diag(exp(G_t - G_C)) tril(Q K^T)
 //   U^T  = V^T T''^T - S W^T           (the D-scaled delta residual)
 //   S   <- gamma_C S + U^T K
-//   O^T  = S Qg^T + U^T Pt^T           (o_t = S_t q_t for every token of the chunk)
+//   O^T  = (S Q^T) diag(gamma) + U^T Pt^T   (o_t = S_t q_t for every token of the chunk)
 //
 // which is the token recurrence S_t = a_t S_{t-1}(I - b_t k_t k_t^T) +
 // b_t v_t k_t^T, o_t = S_t q_t unrolled over the chunk.
 //
 // gdn_chunk_prep_kernel: one CTA per (chunk, head), all chunks at once.
-//   TMA brings K and Q; p1 = [K;Q] K^T on tcgen05 (TMEM); four warps form A
-//   and Phat, invert I + A (16x16 diagonal blocks by substitution, the
+//   TMA brings K and Q; p1 = [K; Q] K^T on tcgen05 (TMEM); four warps form A
+//   and Pt, invert I + A (16x16 diagonal blocks by substitution, the
 //   off-diagonal blocks with tf32 mma.sync), scale T' and T''; p2 = K^T T'^T
-//   on tcgen05 gives W.  Qg and -W (interleaved per 64-column block, so that
-//   they form one 128-row operand), T'' and Pt are written to the workspace in
-//   the 128-byte-swizzled layout the chain kernel's MMAs read, so it copies
-//   them with one bulk copy per chunk.
-// gdn_chunk_chain_kernel: one CTA per (sequence, head), fp32 state in TMEM:
-//   p3 U^T = V^T T''^T, (a + c1) [O^T | U^T] += S [Qg; -W]^T as ONE N = 128
-//   MMA, (b) S += U^T K, c2 O^T += U^T Pt^T -- M = 128 tcgen05 MMAs, the S
-//   and U^T operands read from TMEM -- with a four-warp state group (residual
-//   and state epilogues, the serial chain), a four-warp output group (output
-//   epilogue, off the chain), one MMA thread and one TMA thread.  The state
-//   never leaves the SM between chunks.  A tcgen05.mma costs its issuing
-//   thread some 60 cycles whatever its width, while an M = 128, N = 64 MMA
-//   computes for 32: merging the two MMAs that share the A operand S into one
-//   of twice the width removes eight issues per chunk.
+//   on tcgen05 gives W.  -W, T'' and Pt (32 KB) are written to the workspace
+//   in the 128-byte-swizzled layout the chain kernel's MMAs read, so that it
+//   copies them with bulk copies.  Q itself is not rewritten: the chain
+//   kernel reads it from the input and applies gamma in its output epilogue.
+// gdn_chunk_chain_kernel: one CTA per (sequence, head, chunk range), fp32
+//   state in TMEM: p3 U^T = V^T T''^T, (a + c1) [O1^T | U^T] += S [Q; -W]^T
+//   as ONE N = 128 MMA, (b) S += U^T K, c2 O2^T = U^T Pt^T -- M = 128
+//   tcgen05 MMAs, the S and U^T operands read from TMEM -- with a four-warp
+//   state group (residual and state epilogues, the serial chain), a four-warp
+//   output group (o_t = gamma_t O1_t + O2_t, off the chain), one MMA thread
+//   and one TMA thread.  The state never leaves the SM between chunks.  A
+//   tcgen05.mma costs its issuing thread some 60 cycles whatever its width,
+//   while an M = 128, N = 64 MMA computes for 32: merging the two MMAs that
+//   share the A operand S into one of twice the width removes eight issues
+//   per chunk.
 //
 // Tokens past the end of a sequence inside its last chunk get g = 0 and
 // beta = 0, which zeroes their rows of W and T'' and keeps the state
 // untouched; their outputs are not stored.
+#include <stddef.h>
 #include <string.h>
 
 #include "gdn_internal.h"
@@ -65,7 +67,7 @@ enum { PB_FULL = 0, PB_P1 = 1, PB_P2 = 2, PB_NUM = 3 };
 // The lower block triangles of A and T = (I + A)^-1, as ten 16x16 fp32 blocks
 // each (block (i, j), j <= i, at index i (i + 1) / 2 + j).  A lives over the
 // T'/T'' buffers (written only after the solve), T over the Q rows of the KQ
-// tile (dead once Qg is out): five blocks in each 8 KB half.
+// tile (dead once p1 has read them): five blocks in each 8 KB half.
 constexpr int AB_P = 20, TB_P = 24;                    // row pitches: conflict-free mma fragment loads
 constexpr uint32_t P_AB = P_TP;
 // A blocks sit 1296 B apart (324 words, 4 banks of skew) so that the two
@@ -90,28 +92,34 @@ __device__ __forceinline__ float *t_blk(uint8_t *sm, int i, int j) {
 // ------------------------------------------------------------ chain kernel layout
 constexpr int kChainThreads = 352;                     // warps 0-3 chain, 4-7 output / chain X, 8 MMA, 9 TMA, 10 MMA of chain X
 // Stages of the load pipeline.  An output range needs all of a chunk's data
-// (K, V and the 48 KB prep tile: two stages of 80 KB); a transition range
-// needs K, V, W and T'' only, and runs three stages of 56 KB so that a chunk's
-// loads are issued two chunks ahead.
+// (K, Q, V and the 32 KB prep tile: two stages of 80 KB); a transition range
+// needs K, V, -W and T'' only, and runs three stages of 56 KB so that a
+// chunk's loads are issued two chunks ahead.
 template <int MODE> struct ChainLayout;
-// WQ is the tile's [Qg | -W] operand: per 64-column block, 64 rows of Qg then
-// 64 rows of -W (a 128-row K-major operand, blocks 16 KB apart).  A
-// transition range reads -W alone, as 64 rows per block (blocks 8 KB apart).
+// An output stage keeps K, Q and -W as one K-major operand of 192 rows per
+// 64-column block (K rows 0-63, Q 64-127, -W 128-191; blocks KB bytes
+// apart): rows 64-191 are the merged MMA's B = [Q; -W], rows 0-63 (as an
+// MN-major view) the B of (b).
 template <> struct ChainLayout<0> {   // MODE_OUT
     static constexpr int NST = 2;
     static constexpr uint32_t STAGE = 81920;
-    static constexpr uint32_t K = 0, V = 16384, WQ = 32768, TPP = 65536, PT = 73728;
+    static constexpr uint32_t K = 0, KB = 24576, Q = 8192, NEGW = 16384, V = 49152, TPP = 65536, PT = 73728;
+    static constexpr uint32_t LOADED = STAGE;
 };
 template <> struct ChainLayout<1> {   // MODE_TRANS
     static constexpr int NST = 3;
     static constexpr uint32_t STAGE = 57344;
-    static constexpr uint32_t K = 0, V = 16384, W = 32768, TPP = 49152;
+    static constexpr uint32_t K = 0, KB = 8192, V = 16384, W = 32768, TPP = 49152;
+    static constexpr uint32_t LOADED = STAGE;
 };
-static_assert(ChainLayout<0>::PT + 8192 == ChainLayout<0>::STAGE &&
-              ChainLayout<0>::STAGE - ChainLayout<0>::WQ == kTileBytes, "stage layout");
-// offsets inside a tile: [Qg | -W] per block (32 KB), T'' (8 KB), Pt (8 KB)
-constexpr uint32_t TILE_NEGW = 8192, TILE_TPP = 32768, TILE_PT = 40960;
-static_assert(ChainLayout<1>::TPP + 8192 == ChainLayout<1>::STAGE, "stage layout");
+static_assert(ChainLayout<0>::PT + 8192 == ChainLayout<0>::STAGE && 2 * ChainLayout<0>::KB == ChainLayout<0>::V,
+              "stage layout");
+// a tile: -W per 64-column block (8 KB each), T'' (8 KB), Pt (8 KB); a
+// transition stage takes its first 24 KB, in that order, after K and V
+constexpr uint32_t TILE_NEGW = 0, TILE_TPP = 16384, TILE_PT = 24576;
+static_assert(TILE_PT + 8192 == kTileBytes, "tile layout");
+static_assert(ChainLayout<1>::TPP + 8192 == ChainLayout<1>::STAGE &&
+              ChainLayout<1>::STAGE - ChainLayout<1>::W == TILE_PT, "stage layout");
 // After the stages: output staging [64 t][128 dv] bf16, ChainScalars x 3 per
 // chain, mbarriers + TMEM base + abort flag.
 template <int MODE> __host__ __device__ constexpr uint32_t c_u() { return ChainLayout<MODE>::NST * ChainLayout<MODE>::STAGE; }
@@ -124,14 +132,15 @@ static_assert(c_alloc<0>() <= 232448 && c_alloc<1>() <= 232448, "chain kernel sh
 // TMEM columns of the chain kernel.  The MMA A operands produced by the chain
 // itself (bf16 S and bf16 U^T) stay in TMEM: shared-memory bandwidth, not the
 // tensor core, bounds these small-N MMAs, so only B is read from shared memory.
-// O^T sits right before U^T, so that the merged MMA writes [O^T | U^T] as one
-// 128-column accumulator.
+// O1^T sits right before U^T, so that the merged MMA writes [O1^T | U^T] as
+// one 128-column accumulator.
 constexpr uint32_t TM_S = 0;       // state S (128)
-constexpr uint32_t TM_O = 128;     // O^T (64)
+constexpr uint32_t TM_O = 128;     // O1^T = S Q^T (64)
 constexpr uint32_t TM_U = 192;     // U^T accumulator (64); then U^T bf16 in its first 32
 constexpr uint32_t TM_SBF = 256;   // S bf16, two per column (64)
 // the identity chain of a transition range: its bf16 copy, U^T and state
 constexpr uint32_t TM_XSBF = 128, TM_XU = 320, TM_XS = 384;
+constexpr uint32_t TM_O2 = 320;    // an output range: O2^T = U^T Pt^T (64)
 constexpr uint32_t TM_COLS = 512;
 // Barriers that a role may complete twice before its consumer waits once are
 // per buffer (FULL/EMPTY per stage) and waited with
@@ -139,6 +148,7 @@ constexpr uint32_t TM_COLS = 512;
 enum { CB_FULL = 0, CB_EMPTY = 3, CB_A = 6, CB_B = 7, CB_C = 8, CB_SREADY = 10, CB_UREADY = 11,
        CB_FIN = 12, CB_OFREE = 13, CB_A2 = 15, CB_B2 = 16, CB_SREADY2 = 17, CB_UREADY2 = 18,
        CB_FIN2 = 19, CB_NUM = 20 };   // FULL, EMPTY: one per stage (up to 3)
+static_assert(8 * CB_NUM + 8 <= 256, "barriers, TMEM base and abort flag fit their block");
 
 struct ChainScalars {   // per chunk, state group
     float gC;           // exp(G_C)
@@ -152,10 +162,10 @@ struct PrepScalars {
     float beta[C];
     float bg[C];        // beta * gamma
     float Dd[C];        // exp(G_C - G_t)
-    float gam[C];       // exp(G_t)
     float invD[C];      // exp(G_t - G_C)
+    float gam[C];       // exp(G_t) (layer mode: the q buffer gets diag(gamma) q)
 };
-static_assert(sizeof(PrepScalars) == 1536, "scalar block size");
+static_assert(sizeof(PrepScalars) <= 1536, "scalar block size");
 
 struct PrepParams {
     CUtensorMap map_q, map_k;
@@ -176,14 +186,14 @@ struct PrepParams {
     const __nv_bfloat16 *xq, *xk, *xv;     // raw projections (halo rows)
     const float *conv_w, *a_logit, *b_logit;
     const __nv_bfloat16 *cs_in;            // [N, 3, 3, H, 128] or null
-    __nv_bfloat16 *k_out, *v_out;          // processed k, v
+    __nv_bfloat16 *q_out, *k_out, *v_out;  // processed q, k, v
     float *g_out, *beta_out;
     int act;
     float eps;
 };
 
 struct ChainParams {
-    CUtensorMap map_k, map_v;
+    CUtensorMap map_k, map_v, map_q;   // map_q: output ranges only
     const float *g, *beta, *state_in;
     float *state_out;
     __nv_bfloat16 *out;
@@ -202,7 +212,7 @@ struct ChainParams {
     int *err;
     uint64_t timeout_ns;         // bound on the waits of the work loops
     uint64_t drain_ns;           // bound on the waits that drain copies and MMAs before exit
-    int wait_inputs;             // k, v, g, beta come from the prep kernel (layer mode): wait first
+    int wait_inputs;             // q, k, v, g, beta come from the prep kernel (layer mode): wait first
     // output gate in the output epilogue (z null: plain outputs)
     const __nv_bfloat16 *z;
     const float *norm_w;
@@ -268,6 +278,23 @@ __device__ __forceinline__ GateRegs load_gates(const float *__restrict__ g, cons
             r.g1 = __ldg(g + (size_t)(t0 + lane + 32) * H + h);
             r.b1 = __ldg(beta + (size_t)(t0 + lane + 32) * H + h);
         }
+    }
+    return r;
+}
+
+// load_gates for g alone, with loads issued where the call stands (a plain
+// load may be sunk to its first use, a chunk later, exposing its latency).
+__device__ __forceinline__ GateRegs load_gates_pinned(const float *__restrict__ g, int64_t bos, int64_t eos, int m,
+                                                      int nchunks, int h, int H, int lane) {
+    GateRegs r{0.f, 0.f, 0.f, 0.f};
+    if (m < nchunks) {
+        const int64_t t0 = bos + (int64_t)m * C;
+        const int64_t rem = eos - t0;
+        const int len = rem < C ? (int)rem : C;
+        if (lane < len)
+            asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(r.g0) : "l"(g + (size_t)(t0 + lane) * H + h));
+        if (lane + 32 < len)
+            asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(r.g1) : "l"(g + (size_t)(t0 + lane + 32) * H + h));
     }
     return r;
 }
@@ -427,7 +454,9 @@ gdn_chunk_offsets_kernel(const int32_t *__restrict__ cu, int N, int32_t *__restr
 // solve), the three positions before the chunk come in as halo rows (the
 // sequence's previous tokens, the carried convolution state, or zeros), and
 //   y = act(sum_i w_i x[t - 3 + i]),   q, k = y / sqrt(|y|^2 + eps),   v = y
-// is computed in place.  Thread (tg, ci) owns the 8 tokens 8 tg .. 8 tg + 7
+// is computed: q and k back into their operand rows, k and v to the
+// workspace for the chain kernels, and q to it as diag(gamma) q once the
+// gates are scanned (the gated output pass's Q operand).  Thread (tg, ci) owns the 8 tokens 8 tg .. 8 tg + 7
 // and the 8 channels 8 ci .. 8 ci + 7 of a tensor; the 16 threads of a token
 // row are 16 consecutive lanes, so the L2 norm is a 16-lane butterfly.
 
@@ -628,7 +657,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
     const int no_abort = 0;   // CTA-local failures end each wait by its own bound
     bool ok = true;
     PrepScalars *sc = reinterpret_cast<PrepScalars *>(sm + P_SC);
-    uint8_t *tile = p.tiles + ((size_t)gc * H + h) * kTileBytes;   // [Qg|-W 32K][T'' 8K][Pt 8K]
+    uint8_t *tile = p.tiles + ((size_t)gc * H + h) * kTileBytes;   // [-W 16K][T'' 8K][Pt 8K]
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     float *mm = reinterpret_cast<float *>(sm + P_MM);          // 4 warps x 16 x 20 fp32
 
@@ -656,7 +685,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
     }
 
     if (tid == 0) {
-        // p1 = [K; Q] K^T -> TMEM columns 0..63
+        // p1 = [K; Q] K^T -> TMEM columns 0..63: K K^T in lanes 0..63, Q K^T in 64..127
         ok = mbar_wait(bar(PB_FULL), 0, lim, &no_abort);
         if (ok) {
             tc_fence_after();
@@ -677,23 +706,31 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
         sc->beta[lane] = gr.b0; sc->beta[lane + 32] = gr.b1;
         sc->bg[lane] = gr.b0 * expf(G0); sc->bg[lane + 32] = gr.b1 * expf(G1);
         sc->Dd[lane] = expf(GC - G0); sc->Dd[lane + 32] = expf(GC - G1);
-        sc->gam[lane] = expf(G0); sc->gam[lane + 32] = expf(G1);
         sc->invD[lane] = expf(G0 - GC); sc->invD[lane + 32] = expf(G1 - GC);
+        if (LAYER) { sc->gam[lane] = expf(G0); sc->gam[lane + 32] = expf(G1); }
     }
     __syncwarp();
     __syncthreads();   // gates scanned; K and Q landed (thread 0 waited for them)
-    float x[64];       // this lane's row of p1
+    float x[64];       // this lane's row of p1 (rows 64..127: Q K^T, kept for Pt)
     {
         float (&x0)[32] = *reinterpret_cast<float (*)[32]>(&x[0]);
         float (&x1)[32] = *reinterpret_cast<float (*)[32]>(&x[32]);
-        if (tid >= 64) {
-            // Qg = diag(gamma) Q straight to the tile, read while p1 runs.  The
-            // swizzled bytes keep their positions; consecutive threads take
-            // consecutive 16-byte pieces, so every warp writes 512 contiguous bytes.
-            ok = mbar_wait(bar(PB_FULL), 0, lim, &no_abort);   // complete: makes the TMA data visible here
+        ok = mbar_wait(bar(PB_P1), 0, lim, &no_abort) && ok;
+        tc_fence_after();
+        tmem_ld32(tm + lane_off, x0);
+        tmem_ld32(tm + lane_off + 32, x1);
+    }
+    if (LAYER && tid >= 64) {
+        // layer mode: diag(gamma) Q of the sequence's rows to the q buffer, the
+        // output pass's Q operand (its gated epilogue then needs no gamma),
+        // before T goes over the Q rows.  Thread tid takes the swizzled 16-byte
+        // pieces tid - 64 + 64 k: piece pc of row r holds channels
+        // 8 (pc ^ (r % 8)) .. + 7 of its 64-channel block.
+        const int len = (int)((eos - t0) < C ? (eos - t0) : C);
 #pragma unroll 4
-            for (int k = 0; k < 16; ++k) {
-                const int q = (tid - 64) + 64 * k, kb = q >> 9, r = (q >> 3) & 63, pc = q & 7;
+        for (int k = 0; k < 16; ++k) {
+            const int q = (tid - 64) + 64 * k, kb = q >> 9, r = (q >> 3) & 63, pc = q & 7;
+            if (r < len) {
                 const float gr = sc->gam[r];
                 uint4 v = *reinterpret_cast<const uint4 *>(sm + P_KQ + kb * 16384 + 8192 + r * 128 + pc * 16);
                 __nv_bfloat162 *hv = reinterpret_cast<__nv_bfloat162 *>(&v);
@@ -702,37 +739,33 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
                     const float2 f = __bfloat1622float2(hv[e]);
                     hv[e] = __floats2bfloat162_rn(gr * f.x, gr * f.y);
                 }
-                *reinterpret_cast<uint4 *>(tile + kb * 16384 + r * 128 + pc * 16) = v;
+                *reinterpret_cast<uint4 *>(p.q_out + ((size_t)(t0 + r) * H + h) * D + kb * 64 + ((pc ^ (r & 7)) << 3)) = v;
             }
         }
-        ok = mbar_wait(bar(PB_P1), 0, lim, &no_abort) && ok;
-        tc_fence_after();
-        tmem_ld32(tm + lane_off, x0);
-        tmem_ld32(tm + lane_off + 32, x1);
-        if (tid < 64) {
-            // A[r][i] = beta_r exp(G_r - G_i) k_r.k_i = (beta_r gamma_r) exp(-G_i) KK[r][i], i < r
-            const int r = tid, rb = r >> 4;
-            const float bgr = sc->bg[r];
+    }
+    if (tid < 64) {
+        // A[r][i] = beta_r exp(G_r - G_i) k_r.k_i = (beta_r gamma_r) exp(-G_i) KK[r][i], i < r
+        const int r = tid, rb = r >> 4;
+        const float bgr = sc->bg[r];
 #pragma unroll
-            for (int jb = 0; jb < 4; ++jb) {
-                if (jb > rb) break;
-                float *dst = a_blk(sm, rb, jb) + (r & 15) * AB_P;
+        for (int jb = 0; jb < 4; ++jb) {
+            if (jb > rb) break;
+            float *dst = a_blk(sm, rb, jb) + (r & 15) * AB_P;
 #pragma unroll
-                for (int c = 0; c < 16; c += 4) {
-                    const int i = 16 * jb + c;
-                    const float4 iv = *reinterpret_cast<const float4 *>(&sc->inv[i]);
-                    float4 a;
-                    a.x = (i < r) ? bgr * iv.x * x[i] : 0.f;
-                    a.y = (i + 1 < r) ? bgr * iv.y * x[i + 1] : 0.f;
-                    a.z = (i + 2 < r) ? bgr * iv.z * x[i + 2] : 0.f;
-                    a.w = (i + 3 < r) ? bgr * iv.w * x[i + 3] : 0.f;
-                    *reinterpret_cast<float4 *>(dst + c) = a;
-                }
+            for (int c = 0; c < 16; c += 4) {
+                const int i = 16 * jb + c;
+                const float4 iv = *reinterpret_cast<const float4 *>(&sc->inv[i]);
+                float4 a;
+                a.x = (i < r) ? bgr * iv.x * x[i] : 0.f;
+                a.y = (i + 1 < r) ? bgr * iv.y * x[i + 1] : 0.f;
+                a.z = (i + 2 < r) ? bgr * iv.z * x[i + 2] : 0.f;
+                a.w = (i + 3 < r) ? bgr * iv.w * x[i + 3] : 0.f;
+                *reinterpret_cast<float4 *>(dst + c) = a;
             }
         }
     }
     tc_fence_before();
-    __syncthreads();   // A complete; Q no longer read (T goes over it)
+    __syncthreads();   // A complete; p1 has read the Q rows (T goes over them)
     if (tid < 64) {
         // T = (I + A)^-1: 16x16 diagonal blocks by forward substitution
         const int b = tid >> 4, c = tid & 15;
@@ -839,9 +872,8 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
-        bulk_store(tile + TILE_NEGW, smem_u32(sm + P_TP), 8192);              // -W, first block
-        bulk_store(tile + 16384 + TILE_NEGW, smem_u32(sm + P_TP + 8192), 8192); // -W, second block
-        bulk_store(tile + TILE_PT, smem_u32(sm + P_KQ + 8192), 8192);         // Pt
+        bulk_store(tile + TILE_NEGW, smem_u32(sm + P_TP), 16384);   // -W, both blocks
+        bulk_store(tile + TILE_PT, smem_u32(sm + P_KQ + 8192), 8192);  // Pt
         bulk_commit_wait_read();
     }
     if (!ok && p.err) atomicCAS(p.err, 0, 52);
@@ -917,18 +949,21 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
         const int z = (int)(bos + (int64_t)(cb + n) * C);
         const uint32_t full = bar(CB_FULL + s);
         const uint8_t *tile = p.tiles + ((size_t)(gc0 + n) * H + h) * kTileBytes;
-        mbar_arrive_expect_tx(full, Lay::STAGE);
+        mbar_arrive_expect_tx(full, Lay::LOADED);
         for (int kb = 0; kb < 2; ++kb) {
-            tma_load_3d_hint(st + Lay::K + kb * 8192, &p.map_k, kb * 64, h, z, full, pol);
+            tma_load_3d_hint(st + Lay::K + kb * Lay::KB, &p.map_k, kb * 64, h, z, full, pol);
             tma_load_3d_hint(st + Lay::V + kb * 8192, &p.map_v, kb * 64, h, z, full, pol);
+            if (MODE == MODE_OUT)
+                tma_load_3d_hint(st + ChainLayout<0>::Q + kb * ChainLayout<0>::KB, &p.map_q, kb * 64, h, z, full, pol);
         }
         if (n == 0 && p.wait_tiles) grid_dep_wait();   // tiles come from the prep kernel
-        if (MODE == MODE_TRANS) {   // -W and T'' of the tile
-            bulk_load_hint(st + ChainLayout<1>::W, tile + TILE_NEGW, 8192, full, pol);
-            bulk_load_hint(st + ChainLayout<1>::W + 8192, tile + 16384 + TILE_NEGW, 8192, full, pol);
-            bulk_load_hint(st + ChainLayout<1>::TPP, tile + TILE_TPP, 8192, full, pol);
-        } else {
-            bulk_load_hint(st + ChainLayout<0>::WQ, tile, (uint32_t)kTileBytes, full, pol);
+        if (MODE == MODE_TRANS) {   // -W and T'': the tile's first 24 KB
+            bulk_load_hint(st + ChainLayout<1>::W, tile, TILE_PT, full, pol);
+        } else {                    // -W per block after K and Q, then T'' and Pt
+            for (int kb = 0; kb < 2; ++kb)
+                bulk_load_hint(st + ChainLayout<0>::NEGW + kb * ChainLayout<0>::KB, tile + TILE_NEGW + kb * 8192,
+                               8192, full, pol);
+            bulk_load_hint(st + ChainLayout<0>::TPP, tile + TILE_TPP, 16384, full, pol);   // T'', Pt
         }
     };
     // When nothing upstream still writes this kernel's inputs (an output
@@ -948,6 +983,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
         fence_mbar_init();
         tma_prefetch_desc(&p.map_k);
         tma_prefetch_desc(&p.map_v);
+        if (MODE == MODE_OUT) tma_prefetch_desc(&p.map_q);
         const uint64_t pol0 = MODE == MODE_TRANS ? l2_evict_last_policy() : l2_evict_first_policy();
         for (int n = 0; n < n_early; ++n) issue_stage(n, pol0);
     }
@@ -1005,14 +1041,10 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                 for (int kb = 0; kb < 2; ++kb) {
                     tma_prefetch_3d(&p.map_k, kb * 64, h, zm);
                     tma_prefetch_3d(&p.map_v, kb * 64, h, zm);
+                    if (MODE == MODE_OUT) tma_prefetch_3d(&p.map_q, kb * 64, h, zm);
                 }
-                const uint8_t *tm_ = p.tiles + ((size_t)(gc0 + m) * H + h) * kTileBytes;
-                if (MODE == MODE_TRANS) {
-                    bulk_prefetch_l2(tm_ + TILE_NEGW, 8192);
-                    bulk_prefetch_l2(tm_ + 16384 + TILE_NEGW, 16384);   // second -W block and T''
-                } else {
-                    bulk_prefetch_l2(tm_, (uint32_t)kTileBytes);
-                }
+                bulk_prefetch_l2(p.tiles + ((size_t)(gc0 + m) * H + h) * kTileBytes,
+                                 MODE == MODE_TRANS ? TILE_PT : (uint32_t)kTileBytes);
             };
             for (int n = n_early; n < nloc; ++n) {
                 const int s = n % NST;
@@ -1040,7 +1072,8 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
             const uint32_t id_b = idesc_bf16(128, 128, false, true);
             // descriptors are built once; a byte offset o inside the stages adds o >> 4
             const uint64_t dSTk = desc_sw128(smem_u32(sm), 16, 1024);      // K-major views of stage data
-            const uint64_t dSTm = desc_sw128(smem_u32(sm), 8192, 1024);    // MN-major views of K and V
+            const uint64_t dSTm = desc_sw128(smem_u32(sm), 8192, 1024);    // MN-major views of V (and K, MODE_TRANS)
+            const uint64_t dKm = desc_sw128(smem_u32(sm), Lay::KB, 1024);  // MN-major view of K
             const int zero = 0;
             bool ok = true;
             // transition ranges: U^T (+)= S (-W)^T, -W as 64 rows per block, 8 KB apart
@@ -1054,7 +1087,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
             // (b): S += U^T K  (A = U^T bf16 in TMEM; B = K tile MN-major)
             auto issue_b = [&](uint32_t col_s, uint32_t col_u, uint32_t st) {
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ts(tm + col_s, tm + col_u + 8 * ks, dSTm + ((st + Lay::K + ks * 2048) >> 4), id_b, 1);
+                    mma_bf16_ts(tm + col_s, tm + col_u + 8 * ks, dKm + ((st + Lay::K + ks * 2048) >> 4), id_b, 1);
             };
             for (int n = 0; ok && n < nloc; ++n) {
                 const int s = n % NST;
@@ -1091,10 +1124,11 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                     mma_commit(bar(CB_B));
                     mma_commit(bar(CB_EMPTY + s));
                 } else {
-                    // (a) and c1 share A = S: [O^T | U^T] += S [Qg; -W]^T as one N = 128 MMA per
-                    // K step (O^T starts cleared, U^T holds p3)
+                    // (a) and c1 share A = S: [O1^T | U^T] += S [Q; -W]^T as one N = 128 MMA
+                    // per K step, B = rows 64-191 of the stage's operand block (O1^T
+                    // starts cleared, U^T holds p3)
                     for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t off = st + ChainLayout<0>::WQ + (ks >> 2) * 16384 + (ks & 3) * 32;
+                        const uint32_t off = st + ChainLayout<0>::Q + (ks >> 2) * ChainLayout<0>::KB + (ks & 3) * 32;
                         mma_bf16_ts(tm + TM_O, tm + TM_SBF + 8 * ks, dSTk + (off >> 4), id_n128, 1);
                     }
                     mma_commit(bar(CB_A));
@@ -1102,10 +1136,11 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                     tc_fence_after();
                     issue_b(TM_S, TM_U, st);
                     mma_commit(bar(CB_B));
-                    // c2: O^T += U^T Pt^T
+                    // c2: O2^T = U^T Pt^T (gated: Q is diag(gamma) Q, and c2 accumulates onto O1^T)
                     for (int ks = 0; ks < 4; ++ks)
-                        mma_bf16_ts(tm + TM_O, tm + TM_U + 8 * ks,
-                                    dSTk + ((st + ChainLayout<0>::PT + ks * 32) >> 4), id_n64, 1);
+                        mma_bf16_ts(tm + (GATED ? TM_O : TM_O2), tm + TM_U + 8 * ks,
+                                    dSTk + ((st + ChainLayout<0>::PT + ks * 32) >> 4), id_n64,
+                                    GATED ? 1u : (ks > 0 ? 1u : 0u));
                     mma_commit(bar(CB_C));
                     mma_commit(bar(CB_EMPTY + s));
                 }
@@ -1114,7 +1149,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
             mma_commit(bar(fin));   // every issued MMA completes before TMEM is released
             mbar_wait(bar(fin), 0, p.drain_ns, &zero);
         }
-    } else if (warp < 4 || MODE == MODE_TRANS) {
+    } else if (warp < 4 || (MODE == MODE_TRANS && warp < 8)) {
         // ------------------------------------------------------------ state group(s)
         // warps 0-3: the state chain (R in MODE_TRANS); warps 4-7 in MODE_TRANS: chain X
         const bool xchain = warp >= 4;
@@ -1227,17 +1262,24 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                 }
             }
         }
-    } else {
+    } else if (MODE == MODE_OUT && warp < 8) {
         // ------------------------------------------------------------ output group (MODE_OUT)
-        // O^T (lane dv, 64 t) -> bf16 rows of out; off the state chain
+        // o_t = gamma_t O1_t + O2_t (lane dv, 64 t) -> bf16 rows of out; off the
+        // state chain.  O2 of chunk n is read before OFREE(n + 1) is signalled,
+        // and c2(n + 1), which overwrites it, is issued after the merged MMA
+        // that waits for OFREE(n + 1).  Gated (layer mode), the q buffer holds
+        // diag(gamma) q and c2 accumulates onto O1, so that o_t = O1_t.
         const int dv = tid - 128;   // TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>((warp - 4) * 32) << 16;
+        float *gam = reinterpret_cast<float *>(sm + c_scx<MODE>()) + (warp - 4) * C;   // this warp's gamma_t
+        GateRegs gn{0.f, 0.f, 0.f, 0.f};
+        if constexpr (!GATED) gn = load_gates_pinned(p.g, bos, eos, cb, ce, h, H, lane);
         __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(sm + c_u<MODE>());
         float *stagef = reinterpret_cast<float *>(sm + c_u<MODE>());   // gated: the norm and gate take fp32 o
-        float a[32], b[32];
+        float a[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) a[j] = 0.f;
-        // O^T starts cleared: the merged MMA accumulates c1 onto it
+        // O1^T starts cleared: the merged MMA accumulates c1 onto it
         tmem_st32(tm + lane_off + TM_O, a);
         tmem_st32(tm + lane_off + TM_O + 32, a);
         tc_fence_before();
@@ -1251,15 +1293,20 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
         float nw[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) nw[e] = (gated && p.norm_w) ? __ldg(p.norm_w + piece * 8 + e) : 1.f;
-        // z of this thread's pieces of local chunk m (rows past the end: 0)
+        // z of this thread's pieces of local chunk m (rows past the end: 0),
+        // issued where it stands (a plain load may be sunk to its use, a chunk
+        // later, which would expose its latency there)
         auto load_z = [&](uint4 (&zz)[8], int m) {
             const int64_t tz = bos + (int64_t)(cb + m) * C;
             const int lz = m < nloc ? (int)((eos - tz) < C ? (eos - tz) : C) : 0;
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 const int t = 8 * k + (dv >> 4);
-                zz[k] = t < lz ? __ldg(reinterpret_cast<const uint4 *>(p.z + ((size_t)(tz + t) * H + h) * D + piece * 8))
-                               : make_uint4(0u, 0u, 0u, 0u);
+                zz[k] = make_uint4(0u, 0u, 0u, 0u);
+                if (t < lz)
+                    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(zz[k].x), "=r"(zz[k].y), "=r"(zz[k].z), "=r"(zz[k].w)
+                                 : "l"(p.z + ((size_t)(tz + t) * H + h) * D + piece * 8));
             }
         };
         uint4 zr[8], zn[8];   // z of chunk n, and of chunk n + 1 in flight a whole chunk ahead
@@ -1269,33 +1316,49 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
             if (named_bar_any(3, 128, *abort_flag != 0)) break;
             const int64_t t0 = bos + (int64_t)(cb + n) * C;
             const int len = (int)((eos - t0) < C ? (eos - t0) : C);
+            if constexpr (!gated) {
+                // gamma_t = exp(G_t) of chunk n (the state group's scan of the same
+                // gates), before this iteration's loads are issued: a wait for the
+                // gates must not also wait for them
+                float G0, G1;
+                scan_gates(gn, lane, G0, G1);
+                gam[lane] = expf(G0);
+                gam[lane + 32] = expf(G1);
+                __syncwarp();
+                gn = load_gates_pinned(p.g, bos, eos, cb + n + 1, ce, h, H, lane);
+            }
             if constexpr (gated) load_z(zn, n + 1);
             if (!mbar_wait(bar(CB_C), n & 1, lim, abort_flag)) fail(73);
             tc_fence_after();
-            tmem_ld32(tm + lane_off + TM_O, a);
-            tmem_ld32(tm + lane_off + TM_O + 32, b);
-            {
-                float z[32];
+            // o_t = gamma_t O1_t + O2_t (gated: O1_t), 32 columns t at a time, into
+            // the staging tile
 #pragma unroll
-                for (int j = 0; j < 32; ++j) z[j] = 0.f;
-                tmem_st32(tm + lane_off + TM_O, z);
-                tmem_st32(tm + lane_off + TM_O + 32, z);
+            for (int hh = 0; hh < 2; ++hh) {
+                tmem_ld32(tm + lane_off + TM_O + 32 * hh, a);
+                if constexpr (!gated) {
+                    float o2[32];
+                    tmem_ld32(tm + lane_off + TM_O2 + 32 * hh, o2);
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4) {
+                        const float4 gv = *reinterpret_cast<const float4 *>(gam + 32 * hh + j);
+                        a[j] = fmaf(gv.x, a[j], o2[j]);
+                        a[j + 1] = fmaf(gv.y, a[j + 1], o2[j + 1]);
+                        a[j + 2] = fmaf(gv.z, a[j + 2], o2[j + 2]);
+                        a[j + 3] = fmaf(gv.w, a[j + 3], o2[j + 3]);
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    if constexpr (gated) stagef[(32 * hh + j) * D + dv] = a[j];
+                    else stage[(32 * hh + j) * D + dv] = __float2bfloat16_rn(a[j]);
+                }
             }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) a[j] = 0.f;
+            tmem_st32(tm + lane_off + TM_O, a);
+            tmem_st32(tm + lane_off + TM_O + 32, a);
             tc_fence_before();
-            mbar_arrive(bar(CB_OFREE));   // the MMA thread may accumulate chunk n+1's O^T
-            if constexpr (gated) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    stagef[j * D + dv] = a[j];
-                    stagef[(32 + j) * D + dv] = b[j];
-                }
-            } else {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    stage[j * D + dv] = __float2bfloat16_rn(a[j]);
-                    stage[(32 + j) * D + dv] = __float2bfloat16_rn(b[j]);
-                }
-            }
+            mbar_arrive(bar(CB_OFREE));   // the MMA thread may accumulate chunk n+1's O1^T
             named_bar_sync(3, 128);
             // whole 16-byte pieces of the [64 t][128 dv] tile, rows t < len
 #pragma unroll
@@ -1706,10 +1769,11 @@ cudaError_t launch_prefill_tc(const TcLaunch &L, cudaStream_t stream) {
     const TcLayer *Ly = L.layer;
     if (Ly) {
         // the prep kernel reads the raw projections; the chains read the
-        // k, v, g and beta it writes
+        // q, k, v, g and beta it writes
         if (!make_token_map(&pp.map_q, Ly->xq, L.total_tokens, L.H) ||
             !make_token_map(&pp.map_k, Ly->xk, L.total_tokens, L.H) ||
             !make_token_map(&pp.map_v, Ly->xv, L.total_tokens, L.H) ||
+            !make_token_map(&cp.map_q, Ly->q, L.total_tokens, L.H) ||
             !make_token_map(&cp.map_k, Ly->k, L.total_tokens, L.H) ||
             !make_token_map(&cp.map_v, Ly->v, L.total_tokens, L.H))
             return cudaErrorInvalidValue;
@@ -1721,6 +1785,7 @@ cudaError_t launch_prefill_tc(const TcLaunch &L, cudaStream_t stream) {
         pp.a_logit = Ly->a_logit;
         pp.b_logit = Ly->b_logit;
         pp.cs_in = static_cast<const __nv_bfloat16 *>(Ly->cs_in);
+        pp.q_out = static_cast<__nv_bfloat16 *>(Ly->q);
         pp.k_out = static_cast<__nv_bfloat16 *>(Ly->k);
         pp.v_out = static_cast<__nv_bfloat16 *>(Ly->v);
         pp.g_out = Ly->g;
@@ -1734,6 +1799,7 @@ cudaError_t launch_prefill_tc(const TcLaunch &L, cudaStream_t stream) {
             !make_token_map(&pp.map_k, L.k, L.total_tokens, L.H) ||
             !make_token_map(&cp.map_v, L.v, L.total_tokens, L.H))
             return cudaErrorInvalidValue;
+        cp.map_q = pp.map_q;
         cp.map_k = pp.map_k;
         pp.g = cp.g = L.g;
         pp.beta = cp.beta = L.beta;

@@ -10,23 +10,22 @@
 namespace gdn {
 
 // Bytes of per-chunk factors the prep kernel hands to the chain kernel for
-// one (chunk, head): W (64 x 128 bf16), diag(gamma) Q (64 x 128 bf16),
-// T'' (64 x 64 bf16) and the scaled QK^T triangle (64 x 64 bf16), each already
-// in the 128-byte-swizzled shared-memory layout of the MMAs.
-constexpr size_t kTileBytes = 49152;
+// one (chunk, head): -W (64 x 128 bf16), T'' (64 x 64 bf16) and the scaled
+// QK^T triangle Pt (64 x 64 bf16), already in the 128-byte-swizzled
+// shared-memory layout of the MMAs.
+constexpr size_t kTileBytes = 32768;
 
 // The layer steps fused into the prefill (gdn_layer_prefill): the prep kernel
 // forms q, k, v, g and beta from the raw projections (causal depthwise
 // convolution of window 4, optional SiLU, q/k L2 norm, beta = sigmoid(b),
-// g = log sigmoid(a)); q stays on chip, k, v, g and beta go to the buffers
-// below for the chain kernels; the output pass writes y = n(o) * act(z)
-// instead of o.
+// g = log sigmoid(a)); q, k, v, g and beta go to the buffers below for the
+// chain kernels; the output pass writes y = n(o) * act(z) instead of o.
 struct TcLayer {
     const void *xq, *xk, *xv;          // raw projections [T, H, 128] bf16
     const float *conv_w;               // [3, H, 128, 4]
     const float *a_logit, *b_logit;    // [T, H]
     const void *cs_in;                 // [N, 3, 3, H, 128] bf16, or null (zeros)
-    void *k, *v;                       // processed k, v [T, H, 128] bf16 (written)
+    void *q, *k, *v;                   // processed q, k, v [T, H, 128] bf16 (written)
     float *g, *beta;                   // [T, H] (written)
     int activation;                    // GDN_ACT_NONE / GDN_ACT_SILU
     float eps;                         // of the q/k L2 norm and of the RMS norm
