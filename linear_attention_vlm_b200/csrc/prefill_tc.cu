@@ -90,7 +90,9 @@ __device__ __forceinline__ float *t_blk(uint8_t *sm, int i, int j) {
 }
 
 // ------------------------------------------------------------ chain kernel layout
-constexpr int kChainThreads = 352;                     // warps 0-3 chain, 4-7 output / chain X, 8 MMA, 9 TMA, 10 MMA of chain X
+// warps 0-3 chain, 4-7 output / chain X, 8 MMA, 9 TMA, 10 MMA of chain X /
+// output stores, 11 output stores
+constexpr int kChainThreads = 384;
 // Stages of the load pipeline.  An output range needs all of a chunk's data
 // (K, Q, V and the 32 KB prep tile: two stages of 80 KB); a transition range
 // needs K, V, -W and T'' only, and runs three stages of 56 KB so that a
@@ -1059,7 +1061,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
             for (int s = 0; s < NST; ++s)
                 if (issued[s]) mbar_wait(bar(CB_FULL + s), (issued[s] - 1) & 1, p.drain_ns, &zero);
         }
-    } else if (warp == 8 || warp == 10) {
+    } else if (warp == 8 || (MODE == MODE_TRANS && warp == 10)) {
         // ------------------------------------------------------------ MMA issuers
         // warp 8: the state chain (p3, the residual and state products and,
         // for outputs, c1 and c2); warp 10 (MODE_TRANS): the identity chain,
@@ -1262,46 +1264,58 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                 }
             }
         }
-    } else if (MODE == MODE_OUT && warp < 8) {
+    } else if (MODE == MODE_OUT && warp != 8 && warp != 9) {
         // ------------------------------------------------------------ output group (MODE_OUT)
         // o_t = gamma_t O1_t + O2_t (lane dv, 64 t) -> bf16 rows of out; off the
-        // state chain.  O2 of chunk n is read before OFREE(n + 1) is signalled,
-        // and c2(n + 1), which overwrites it, is issued after the merged MMA
-        // that waits for OFREE(n + 1).  Gated (layer mode), the q buffer holds
-        // diag(gamma) q and c2 accumulates onto O1, so that o_t = O1_t.
-        const int dv = tid - 128;   // TMEM lane
-        const uint32_t lane_off = static_cast<uint32_t>((warp - 4) * 32) << 16;
-        float *gam = reinterpret_cast<float *>(sm + c_scx<MODE>()) + (warp - 4) * C;   // this warp's gamma_t
+        // state chain.  Warps 4-7 (TMEM lanes dv) stage the tile; warps 10-11
+        // join them for the stores (and the output gate, the longest part of
+        // the gated pass).  O2 of chunk n is read before OFREE(n + 1) is
+        // signalled, and c2(n + 1), which overwrites it, is issued after the
+        // merged MMA that waits for OFREE(n + 1).  Gated (layer mode), the q
+        // buffer holds diag(gamma) q and c2 accumulates onto O1, so that
+        // o_t = O1_t.
+        constexpr int kOut = 192;                    // output threads
+        constexpr int kRows = kOut / 16;             // rows per store pass (16 pieces a row)
+        constexpr int kPasses = (C + kRows - 1) / kRows;
+        const bool tw = warp < 8;                    // a TMEM warp
+        const int dv = tid - 128;                    // TMEM lane (warps 4-7)
+        const int so = tw ? dv : 128 + (warp - 10) * 32 + lane;   // 0 .. kOut - 1
+        const int piece = so & 15, rsub = so >> 4;   // 16-byte piece, and row within a pass
+        const uint32_t lane_off = static_cast<uint32_t>(tw ? (warp - 4) * 32 : 0) << 16;
+        float *gam = reinterpret_cast<float *>(sm + c_scx<MODE>()) + (tw ? warp - 4 : 0) * C;   // this warp's gamma_t
         GateRegs gn{0.f, 0.f, 0.f, 0.f};
-        if constexpr (!GATED) gn = load_gates_pinned(p.g, bos, eos, cb, ce, h, H, lane);
+        if constexpr (!GATED) {
+            if (tw) gn = load_gates_pinned(p.g, bos, eos, cb, ce, h, H, lane);
+        }
         __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(sm + c_u<MODE>());
         float *stagef = reinterpret_cast<float *>(sm + c_u<MODE>());   // gated: the norm and gate take fp32 o
         float a[32];
+        if (tw) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) a[j] = 0.f;
-        // O1^T starts cleared: the merged MMA accumulates c1 onto it
-        tmem_st32(tm + lane_off + TM_O, a);
-        tmem_st32(tm + lane_off + TM_O + 32, a);
-        tc_fence_before();
-        mbar_arrive(bar(CB_OFREE));
+            for (int j = 0; j < 32; ++j) a[j] = 0.f;
+            // O1^T starts cleared: the merged MMA accumulates c1 onto it
+            tmem_st32(tm + lane_off + TM_O, a);
+            tmem_st32(tm + lane_off + TM_O + 32, a);
+            tc_fence_before();
+            mbar_arrive(bar(CB_OFREE));
+        }
         // output gate (layer mode): y = n(o) * act(z), n an RMS norm over the
         // row's d_v values (or the identity); a thread always takes the same
-        // 8 channels (piece dv % 16) of 8 rows, the 16 pieces of a row lying
-        // in 16 consecutive lanes
+        // 8 channels (piece) of its rows, the 16 pieces of a row lying in 16
+        // consecutive lanes
         constexpr bool gated = GATED;
-        const int piece = dv & 15;
         float nw[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) nw[e] = (gated && p.norm_w) ? __ldg(p.norm_w + piece * 8 + e) : 1.f;
         // z of this thread's pieces of local chunk m (rows past the end: 0),
         // issued where it stands (a plain load may be sunk to its use, a chunk
         // later, which would expose its latency there)
-        auto load_z = [&](uint4 (&zz)[8], int m) {
+        auto load_z = [&](uint4 (&zz)[kPasses], int m) {
             const int64_t tz = bos + (int64_t)(cb + m) * C;
             const int lz = m < nloc ? (int)((eos - tz) < C ? (eos - tz) : C) : 0;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int t = 8 * k + (dv >> 4);
+            for (int k = 0; k < kPasses; ++k) {
+                const int t = kRows * k + rsub;
                 zz[k] = make_uint4(0u, 0u, 0u, 0u);
                 if (t < lz)
                     asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -1309,65 +1323,71 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                                  : "l"(p.z + ((size_t)(tz + t) * H + h) * D + piece * 8));
             }
         };
-        uint4 zr[8], zn[8];   // z of chunk n, and of chunk n + 1 in flight a whole chunk ahead
+        uint4 zr[kPasses], zn[kPasses];   // z of chunk n, and of chunk n + 1 in flight a whole chunk ahead
         if constexpr (gated) load_z(zr, 0);
         for (int n = 0; n < nloc; ++n) {
-            // all four warps are done with chunk n-1's staging buffer
-            if (named_bar_any(3, 128, *abort_flag != 0)) break;
+            // all output warps are done with chunk n-1's staging buffer
+            if (named_bar_any(3, kOut, *abort_flag != 0)) break;
             const int64_t t0 = bos + (int64_t)(cb + n) * C;
             const int len = (int)((eos - t0) < C ? (eos - t0) : C);
             if constexpr (!gated) {
-                // gamma_t = exp(G_t) of chunk n (the state group's scan of the same
-                // gates), before this iteration's loads are issued: a wait for the
-                // gates must not also wait for them
-                float G0, G1;
-                scan_gates(gn, lane, G0, G1);
-                gam[lane] = expf(G0);
-                gam[lane + 32] = expf(G1);
-                __syncwarp();
-                gn = load_gates_pinned(p.g, bos, eos, cb + n + 1, ce, h, H, lane);
+                if (tw) {
+                    // gamma_t = exp(G_t) of chunk n (the state group's scan of the same
+                    // gates), before this iteration's loads are issued: a wait for the
+                    // gates must not also wait for them
+                    float G0, G1;
+                    scan_gates(gn, lane, G0, G1);
+                    gam[lane] = expf(G0);
+                    gam[lane + 32] = expf(G1);
+                    __syncwarp();
+                    gn = load_gates_pinned(p.g, bos, eos, cb + n + 1, ce, h, H, lane);
+                }
             }
             if constexpr (gated) load_z(zn, n + 1);
-            if (!mbar_wait(bar(CB_C), n & 1, lim, abort_flag)) fail(73);
-            tc_fence_after();
-            // o_t = gamma_t O1_t + O2_t (gated: O1_t), 32 columns t at a time, into
-            // the staging tile
+            if (tw) {
+                if (!mbar_wait(bar(CB_C), n & 1, lim, abort_flag)) fail(73);
+                tc_fence_after();
+                // o_t = gamma_t O1_t + O2_t (gated: O1_t), 32 columns t at a time,
+                // into the staging tile
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                tmem_ld32(tm + lane_off + TM_O + 32 * hh, a);
-                if constexpr (!gated) {
-                    float o2[32];
-                    tmem_ld32(tm + lane_off + TM_O2 + 32 * hh, o2);
+                for (int hh = 0; hh < 2; ++hh) {
+                    tmem_ld32(tm + lane_off + TM_O + 32 * hh, a);
+                    if constexpr (!gated) {
+                        float o2[32];
+                        tmem_ld32(tm + lane_off + TM_O2 + 32 * hh, o2);
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4) {
-                        const float4 gv = *reinterpret_cast<const float4 *>(gam + 32 * hh + j);
-                        a[j] = fmaf(gv.x, a[j], o2[j]);
-                        a[j + 1] = fmaf(gv.y, a[j + 1], o2[j + 1]);
-                        a[j + 2] = fmaf(gv.z, a[j + 2], o2[j + 2]);
-                        a[j + 3] = fmaf(gv.w, a[j + 3], o2[j + 3]);
+                        for (int j = 0; j < 32; j += 4) {
+                            const float4 gv = *reinterpret_cast<const float4 *>(gam + 32 * hh + j);
+                            a[j] = fmaf(gv.x, a[j], o2[j]);
+                            a[j + 1] = fmaf(gv.y, a[j + 1], o2[j + 1]);
+                            a[j + 2] = fmaf(gv.z, a[j + 2], o2[j + 2]);
+                            a[j + 3] = fmaf(gv.w, a[j + 3], o2[j + 3]);
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        if constexpr (gated) stagef[(32 * hh + j) * D + dv] = a[j];
+                        else stage[(32 * hh + j) * D + dv] = __float2bfloat16_rn(a[j]);
                     }
                 }
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    if constexpr (gated) stagef[(32 * hh + j) * D + dv] = a[j];
-                    else stage[(32 * hh + j) * D + dv] = __float2bfloat16_rn(a[j]);
-                }
+                for (int j = 0; j < 32; ++j) a[j] = 0.f;
+                tmem_st32(tm + lane_off + TM_O, a);
+                tmem_st32(tm + lane_off + TM_O + 32, a);
+                tc_fence_before();
+                mbar_arrive(bar(CB_OFREE));   // the MMA thread may accumulate chunk n+1's O1^T
             }
+            named_bar_sync(3, kOut);
+            // whole 16-byte pieces of the [64 t][128 dv] tile, rows t < len (a row
+            // past 63 in the last pass is read as row 63, so that every lane takes
+            // part in the shuffles, and not stored)
 #pragma unroll
-            for (int j = 0; j < 32; ++j) a[j] = 0.f;
-            tmem_st32(tm + lane_off + TM_O, a);
-            tmem_st32(tm + lane_off + TM_O + 32, a);
-            tc_fence_before();
-            mbar_arrive(bar(CB_OFREE));   // the MMA thread may accumulate chunk n+1's O1^T
-            named_bar_sync(3, 128);
-            // whole 16-byte pieces of the [64 t][128 dv] tile, rows t < len
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int t = 8 * k + (dv >> 4);       // piece k * 128 + dv of 1024
+            for (int k = 0; k < kPasses; ++k) {
+                const int t = kRows * k + rsub, tc = t < C ? t : C - 1;
                 uint4 v;
                 if constexpr (gated) {
-                    const float4 f0 = *reinterpret_cast<const float4 *>(stagef + t * D + piece * 8);
-                    const float4 f1 = *reinterpret_cast<const float4 *>(stagef + t * D + piece * 8 + 4);
+                    const float4 f0 = *reinterpret_cast<const float4 *>(stagef + tc * D + piece * 8);
+                    const float4 f1 = *reinterpret_cast<const float4 *>(stagef + tc * D + piece * 8 + 4);
                     const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
                     float ss = 0.f;
 #pragma unroll
@@ -1384,13 +1404,13 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                     v = make_uint4(pack_bf16(yv[0], yv[1]), pack_bf16(yv[2], yv[3]), pack_bf16(yv[4], yv[5]),
                                    pack_bf16(yv[6], yv[7]));
                 } else {
-                    v = *reinterpret_cast<const uint4 *>(stage + t * D + piece * 8);
+                    v = *reinterpret_cast<const uint4 *>(stage + tc * D + piece * 8);
                 }
                 if (t < len) *reinterpret_cast<uint4 *>(p.out + ((size_t)(t0 + t) * H + h) * D + piece * 8) = v;
             }
             if constexpr (gated) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k) zr[k] = zn[k];
+                for (int k = 0; k < kPasses; ++k) zr[k] = zn[k];
             }
         }
     }
