@@ -289,10 +289,11 @@ int gdn_output_gate(const void *o, const void *z, const float *norm_w, void *y, 
  *
  * On the tensor-core path (GDN_BF16, d = 128, total_tokens > 0) the steps
  * are fused: the chunk-prep kernel forms q, k, v, g and beta from its chunk's
- * raw projections (q never leaves the chip; k, v, g and beta go to the
- * workspace for the state and output passes), and the output pass writes y
- * in place of o.  Otherwise the three steps run one after another through
- * the workspace.
+ * raw projections and leaves them in the workspace for the state and output
+ * passes (q already scaled, row by row, by the decay exp(G_t) from the start
+ * of its 64-token chunk, the form the output pass consumes), and the output
+ * pass writes y in place of o.  Otherwise the three steps run one after
+ * another through the workspace.
  *
  *   xq, xk, xv, conv_w, a_logit, b_logit, conv_state_in, conv_state_out,
  *   activation   as in gdn_preprocess (conv_state_out may equal

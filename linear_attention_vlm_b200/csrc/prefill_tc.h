@@ -25,7 +25,8 @@ struct TcLayer {
     const float *conv_w;               // [3, H, 128, 4]
     const float *a_logit, *b_logit;    // [T, H]
     const void *cs_in;                 // [N, 3, 3, H, 128] bf16, or null (zeros)
-    void *q, *k, *v;                   // processed q, k, v [T, H, 128] bf16 (written)
+    void *q, *k, *v;                   // processed q (rows scaled by exp(G_t) of their chunk), k, v
+                                       // [T, H, 128] bf16 (written)
     float *g, *beta;                   // [T, H] (written)
     int activation;                    // GDN_ACT_NONE / GDN_ACT_SILU
     float eps;                         // of the q/k L2 norm and of the RMS norm
