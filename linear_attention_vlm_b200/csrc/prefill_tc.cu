@@ -579,22 +579,27 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
     const int gc = blockIdx.x;
     grid_dep_launch();   // the next kernel may stage its prologue while this grid drains
 
-    // which sequence and which of its chunks this CTA prepares
+    // which sequence and which of its chunks global chunk c is (false: a
+    // padding chunk past the last sequence of a packed batch)
+    auto locate = [&](int c, int &nseq_, int64_t &j_) {
+        if (p.chunk_off) {
+            if (c >= p.chunk_off[p.num_seqs]) return false;
+            int lo = 0, hi = p.num_seqs - 1;                 // last n with chunk_off[n] <= c
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (p.chunk_off[mid] <= c) lo = mid; else hi = mid - 1;
+            }
+            nseq_ = lo;
+            j_ = c - p.chunk_off[lo];
+        } else {
+            nseq_ = c / p.cps;
+            j_ = c % p.cps;
+        }
+        return true;
+    };
     int nseq;
     int64_t j;
-    if (p.chunk_off) {
-        if (gc >= p.chunk_off[p.num_seqs]) return;          // uniform across the CTA
-        int lo = 0, hi = p.num_seqs - 1;                     // last n with chunk_off[n] <= gc
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (p.chunk_off[mid] <= gc) lo = mid; else hi = mid - 1;
-        }
-        nseq = lo;
-        j = gc - p.chunk_off[lo];
-    } else {
-        nseq = gc / p.cps;
-        j = gc % p.cps;
-    }
+    if (!locate(gc, nseq, j)) return;                        // uniform across the CTA
     int64_t bos, eos;
     SeqBounds{p.cu_seqlens, p.uniform_len}.get(nseq, bos, eos);
     const int64_t t0 = bos + j * C;
@@ -1499,8 +1504,9 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
 // Start state of every range after the first: S_{j+1} = S_j M_j + R_j,
 // sequentially over the ranges of one (sequence, head).  Rows of S are
 // independent, so a CTA owns 16 of them: grid (N*H, 8), eight warps.  Warp w
-// multiplies the k-slice [32 (w/2), +32) of S_j against column half w%2 of
-// M_j; the four k-slice partials meet in shared memory, where R_j is added.
+// computes columns [16 w, +16) of S_{j+1} over the whole k range and adds R_j
+// to them, so that no partial sums cross warps; S_j and S_{j+1} alternate
+// between two shared-memory row buffers.
 // The products run on bf16 mma.sync with each fp32 operand split in two
 // (x = hi + lo, both bf16; S M ~= S_hi M_hi + S_hi M_lo + S_lo M_hi), which
 // keeps about 16 mantissa bits; accumulation is fp32.  M_j arrives already
@@ -1511,11 +1517,11 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
 // j computes.
 constexpr int kCombRows = 16;
 constexpr int kCombThreads = 256;
-constexpr int kCombSP = 136, kCombPP = 132;                     // row pitches: conflict-free fragments
+constexpr int kCombSP = 136;                                    // row pitch: conflict-free fragments
 constexpr uint32_t kCombMBytes = 2 * D * D * 2;                 // M_j: hi and lo bf16 rows
 constexpr uint32_t kCombRBytes = kCombRows * D * 4;             // 16 rows of R_j
 constexpr uint32_t kCombBufBytes = kCombMBytes + kCombRBytes;
-constexpr size_t kCombSmem = (size_t)2 * kCombBufBytes + (size_t)(kCombRows * kCombSP + 4 * kCombRows * kCombPP) * 4 + 64;
+constexpr size_t kCombSmem = (size_t)2 * kCombBufBytes + (size_t)2 * kCombRows * kCombSP * 4 + 64;
 
 // four 8x8 bf16 blocks, transposed on the way: the col-major B fragments of mma.sync
 __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const __nv_bfloat16 *row) {
@@ -1538,15 +1544,13 @@ gdn_scan_combine_kernel(const float *__restrict__ state_in, const float *__restr
                         const float *__restrict__ trans_m, float *__restrict__ seg_start, int nseg,
                         int *err, uint64_t timeout_ns, uint64_t drain_ns) {
     extern __shared__ __align__(128) uint8_t smc[];
-    // [buffer 0: M hi, M lo, R rows][buffer 1: the same][S_j rows][partials][2 mbarriers, abort flag]
-    float *Ss = reinterpret_cast<float *>(smc + 2 * kCombBufBytes);   // S_j rows [16][D]
-    float *Ps = Ss + kCombRows * kCombSP;                               // k-slice partials [4][16][D]
-    uint8_t *ctl = reinterpret_cast<uint8_t *>(Ps + 4 * kCombRows * kCombPP);
+    // [buffer 0: M hi, M lo, R rows][buffer 1: the same][S rows, two buffers][2 mbarriers, abort flag]
+    float *Ss = reinterpret_cast<float *>(smc + 2 * kCombBufBytes);   // S_j rows [2][16][D] (pitch kCombSP)
+    uint8_t *ctl = reinterpret_cast<uint8_t *>(Ss + 2 * kCombRows * kCombSP);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(ctl + 16);
     auto bar = [&](int b) { return smem_u32(ctl + 8 * b); };
     const int nh = blockIdx.x, r0 = blockIdx.y * kCombRows;
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31, g = lane >> 2, q = lane & 3;
-    const int kg = warp >> 1, ch = warp & 1;
     if (t == 0) {
         mbar_init(bar(0), 1);
         mbar_init(bar(1), 1);
@@ -1572,16 +1576,16 @@ gdn_scan_combine_kernel(const float *__restrict__ state_in, const float *__restr
             state_in ? state_in[(size_t)nh * D * D + (size_t)(r0 + (i >> 7)) * D + (i & 127)] : 0.f;
     for (int j = 0; j + 1 < nseg; ++j) {
         const size_t u = ((size_t)nh * (nseg - 1) + j) * D * D + (size_t)r0 * D;   // rows r0.. of step j
-        float acc[8][4], accx[8][4];   // hi*hi terms; the two cross terms
+        float acc[2][4], accx[2][4];   // hi*hi terms; the two cross terms
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
+        for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[nt][e] = accx[nt][e] = 0.f;
         if (!mbar_wait(bar(j & 1), (j >> 1) & 1, timeout_ns, abort_flag)) {
             *abort_flag = 1;
             if (err) atomicCAS(err, 0, 81);
         }
-        __syncthreads();   // M_j and R_j landed (or the wait gave up); S_j rows are written
+        __syncthreads();   // M_j and R_j landed (or the wait gave up); S_j rows are written, S_{j-1} read
         if (*abort_flag) break;
         pending = -1;
         if (j + 2 < nseg) {
@@ -1594,55 +1598,47 @@ gdn_scan_combine_kernel(const float *__restrict__ state_in, const float *__restr
         const __nv_bfloat16 *Mh = reinterpret_cast<const __nv_bfloat16 *>(smc + (j & 1) * kCombBufBytes);
         const __nv_bfloat16 *Ml = Mh + D * D;
         const float *Rs = reinterpret_cast<const float *>(smc + (j & 1) * kCombBufBytes + kCombMBytes);
+        const float *Sc = Ss + (j & 1) * kCombRows * kCombSP;          // S_j
+        float *Sn = Ss + ((j + 1) & 1) * kCombRows * kCombSP;          // S_{j+1}
 #pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-            const int k0 = 32 * kg + 16 * ks;
+        for (int ks = 0; ks < D / 16; ++ks) {
+            const int k0 = 16 * ks;
             uint32_t ah[4], al[4];
-            const float2 s00 = *reinterpret_cast<const float2 *>(Ss + g * kCombSP + k0 + 2 * q);
-            const float2 s10 = *reinterpret_cast<const float2 *>(Ss + (g + 8) * kCombSP + k0 + 2 * q);
-            const float2 s01 = *reinterpret_cast<const float2 *>(Ss + g * kCombSP + k0 + 2 * q + 8);
-            const float2 s11 = *reinterpret_cast<const float2 *>(Ss + (g + 8) * kCombSP + k0 + 2 * q + 8);
+            const float2 s00 = *reinterpret_cast<const float2 *>(Sc + g * kCombSP + k0 + 2 * q);
+            const float2 s10 = *reinterpret_cast<const float2 *>(Sc + (g + 8) * kCombSP + k0 + 2 * q);
+            const float2 s01 = *reinterpret_cast<const float2 *>(Sc + g * kCombSP + k0 + 2 * q + 8);
+            const float2 s11 = *reinterpret_cast<const float2 *>(Sc + (g + 8) * kCombSP + k0 + 2 * q + 8);
             split2(s00.x, s00.y, ah[0], al[0]);
             split2(s10.x, s10.y, ah[1], al[1]);
             split2(s01.x, s01.y, ah[2], al[2]);
             split2(s11.x, s11.y, ah[3], al[3]);
             // lane -> row of one of four 8x8 blocks: k0 + (lane & 7) + 8 ((lane >> 3) & 1),
-            // 16-byte piece 8 ch + 2 pr + (lane >> 4) of that row (stored at piece ^ (row % 8));
-            // .trans turns them into the B fragments {b0, b1} of n-tiles 2 pr and 2 pr + 1
+            // 16-byte piece 2 w + (lane >> 4) of that row (stored at piece ^ (row % 8));
+            // .trans turns them into the B fragments {b0, b1} of n-tiles 0 and 1
             const int krow = k0 + (lane & 7) + 8 * ((lane >> 3) & 1);
+            const int off = krow * D + (((2 * warp + (lane >> 4)) ^ (krow & 7)) << 3);
+            uint32_t bh[4], bl[4];
+            ldmatrix_x4_trans(bh, Mh + off);
+            ldmatrix_x4_trans(bl, Ml + off);
 #pragma unroll
-            for (int pr = 0; pr < 4; ++pr) {
-                const int off = krow * D + (((8 * ch + 2 * pr + (lane >> 4)) ^ (krow & 7)) << 3);
-                uint32_t bh[4], bl[4];
-                ldmatrix_x4_trans(bh, Mh + off);
-                ldmatrix_x4_trans(bl, Ml + off);
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int nt = 2 * pr + u;
-                    mma_bf16_16816(accx[nt], al[0], al[1], al[2], al[3], bh[2 * u], bh[2 * u + 1]);
-                    mma_bf16_16816(accx[nt], ah[0], ah[1], ah[2], ah[3], bl[2 * u], bl[2 * u + 1]);
-                    mma_bf16_16816(acc[nt], ah[0], ah[1], ah[2], ah[3], bh[2 * u], bh[2 * u + 1]);
-                }
+            for (int nt = 0; nt < 2; ++nt) {
+                mma_bf16_16816(accx[nt], al[0], al[1], al[2], al[3], bh[2 * nt], bh[2 * nt + 1]);
+                mma_bf16_16816(accx[nt], ah[0], ah[1], ah[2], ah[3], bl[2 * nt], bl[2 * nt + 1]);
+                mma_bf16_16816(acc[nt], ah[0], ah[1], ah[2], ah[3], bh[2 * nt], bh[2 * nt + 1]);
             }
         }
-        float *P = Ps + kg * kCombRows * kCombPP;
+        // S_{j+1} = S_j M_j + R_j: rows g and g + 8, columns 16 w + 8 nt + 2 q, + 1
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            const int col = 64 * ch + 8 * nt + 2 * q;
-            *reinterpret_cast<float2 *>(P + g * kCombPP + col) =
-                make_float2(acc[nt][0] + accx[nt][0], acc[nt][1] + accx[nt][1]);
-            *reinterpret_cast<float2 *>(P + (g + 8) * kCombPP + col) =
-                make_float2(acc[nt][2] + accx[nt][2], acc[nt][3] + accx[nt][3]);
-        }
-        __syncthreads();   // partials complete; every warp has read S_j
-#pragma unroll
-        for (int i = 0; i < kCombRows * D / kCombThreads; ++i) {
-            const int e = t + kCombThreads * i, row = e >> 7, col = e & 127;
-            float v = Rs[e];
-#pragma unroll
-            for (int s = 0; s < 4; ++s) v += Ps[(s * kCombRows + row) * kCombPP + col];
-            seg_start[u + e] = v;
-            Ss[row * kCombSP + col] = v;
+        for (int nt = 0; nt < 2; ++nt) {
+            const int col = 16 * warp + 8 * nt + 2 * q;
+            const float2 ra = *reinterpret_cast<const float2 *>(Rs + g * D + col);
+            const float2 rb = *reinterpret_cast<const float2 *>(Rs + (g + 8) * D + col);
+            const float2 va = make_float2(acc[nt][0] + accx[nt][0] + ra.x, acc[nt][1] + accx[nt][1] + ra.y);
+            const float2 vb = make_float2(acc[nt][2] + accx[nt][2] + rb.x, acc[nt][3] + accx[nt][3] + rb.y);
+            *reinterpret_cast<float2 *>(seg_start + u + g * D + col) = va;
+            *reinterpret_cast<float2 *>(seg_start + u + (g + 8) * D + col) = vb;
+            *reinterpret_cast<float2 *>(Sn + g * kCombSP + col) = va;
+            *reinterpret_cast<float2 *>(Sn + (g + 8) * kCombSP + col) = vb;
         }
     }
     // no bulk copy may still be landing in shared memory at exit
