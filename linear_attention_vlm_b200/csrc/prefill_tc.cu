@@ -184,6 +184,7 @@ struct PrepParams {
     uint64_t drain_ns;           // bound on the waits that drain copies and MMAs before exit
     // layer mode (fused pre-processing; map_q, map_k and map_v then cover the
     // raw projections, and g, beta are unused)
+    int keep_tiles;              // all tiles fit in L2 beside the streams: keep them there for the chain passes
     int layer;
     const __nv_bfloat16 *xq, *xk, *xv;     // raw projections (halo rows)
     const float *conv_w, *a_logit, *b_logit;
@@ -215,6 +216,7 @@ struct ChainParams {
     uint64_t timeout_ns;         // bound on the waits of the work loops
     uint64_t drain_ns;           // bound on the waits that drain copies and MMAs before exit
     int wait_inputs;             // q, k, v, g, beta come from the prep kernel (layer mode): wait first
+    int keep_tiles;              // the prep kernel left the tiles in L2 (see PrepParams)
     // output gate in the output epilogue (z null: plain outputs)
     const __nv_bfloat16 *z;
     const float *norm_w;
@@ -250,6 +252,27 @@ __device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t byt
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
                  ::"l"(reinterpret_cast<uint64_t>(dst)), "r"(src), "r"(bytes)
                  : "memory");
+}
+
+// bulk_store with an L2 eviction-priority policy for the lines it writes.
+__device__ __forceinline__ void bulk_store_hint(void *dst, uint32_t src, uint32_t bytes, uint64_t policy) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;"
+                 ::"l"(reinterpret_cast<uint64_t>(dst)), "r"(src), "r"(bytes), "l"(policy)
+                 : "memory");
+}
+
+// A 16-byte global store with an L2 eviction-priority policy.
+__device__ __forceinline__ void st_global_v4_hint(void *dst, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                                  uint64_t policy) {
+    asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;"
+                 ::"l"(reinterpret_cast<uint64_t>(dst)), "r"(a), "r"(b), "r"(c), "r"(d), "l"(policy)
+                 : "memory");
+}
+
+// Drop a 128-byte line of workspace data that nothing reads again from L2
+// without writing it back (its memory contents become indeterminate).
+__device__ __forceinline__ void l2_discard_line(const void *p) {
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(reinterpret_cast<uint64_t>(p)) : "memory");
 }
 
 // Commit this thread's bulk stores and wait until they have read shared memory.
@@ -612,13 +635,21 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
         mbar_init(bar(PB_P2), 1);
         fence_mbar_init();
         // K, Q (layer mode: raw k, q and v) -> shared memory, in flight
-        // during the TMEM allocation
+        // during the TMEM allocation.  L2, when the tiles are kept there: the
+        // inputs are streamed (the chain passes read them again far later), so
+        // that they do not push out the tiles this CTA writes.
         const int z = (int)t0;
         mbar_arrive_expect_tx(bar(PB_FULL), LAYER ? 49152 : 32768);
         for (int kb = 0; kb < 2; ++kb) {
             const uint32_t dst = smem_u32(sm + P_KQ + kb * 16384);
-            tma_load_3d(dst, &p.map_k, kb * 64, h, z, bar(PB_FULL));
-            tma_load_3d(dst + 8192, &p.map_q, kb * 64, h, z, bar(PB_FULL));
+            if (p.keep_tiles) {
+                const uint64_t stream_pol = l2_evict_first_policy();
+                tma_load_3d_hint(dst, &p.map_k, kb * 64, h, z, bar(PB_FULL), stream_pol);
+                tma_load_3d_hint(dst + 8192, &p.map_q, kb * 64, h, z, bar(PB_FULL), stream_pol);
+            } else {
+                tma_load_3d(dst, &p.map_k, kb * 64, h, z, bar(PB_FULL));
+                tma_load_3d(dst + 8192, &p.map_q, kb * 64, h, z, bar(PB_FULL));
+            }
             if (LAYER) tma_load_3d(smem_u32(sm + P_TP + kb * 8192), &p.map_v, kb * 64, h, z, bar(PB_FULL));
         }
     }
@@ -665,6 +696,8 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
     bool ok = true;
     PrepScalars *sc = reinterpret_cast<PrepScalars *>(sm + P_SC);
     uint8_t *tile = p.tiles + ((size_t)gc * H + h) * kTileBytes;   // [-W 16K][T'' 8K][Pt 8K]
+    // the tile stays in L2 for the chain passes when all tiles fit beside the streams
+    const uint64_t keep_pol = l2_evict_last_policy();
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     float *mm = reinterpret_cast<float *>(sm + P_MM);          // 4 warps x 16 x 20 fp32
 
@@ -823,7 +856,8 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
         const uint32_t off = r * 128 + pc * 16;
         st_shared_v4(smem_u32(sm + P_TP + off), a0, a1, a2, a3);
         st_shared_v4(smem_u32(sm + P_TP + 8192 + off), a0, a1, a2, a3);
-        *reinterpret_cast<uint4 *>(tile + TILE_TPP + off) = make_uint4(b0, b1, b2, b3);
+        if (p.keep_tiles) st_global_v4_hint(tile + TILE_TPP + off, b0, b1, b2, b3, keep_pol);
+        else *reinterpret_cast<uint4 *>(tile + TILE_TPP + off) = make_uint4(b0, b1, b2, b3);
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -879,8 +913,13 @@ gdn_chunk_prep_kernel(const __grid_constant__ PrepParams p) {
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
-        bulk_store(tile + TILE_NEGW, smem_u32(sm + P_TP), 16384);   // -W, both blocks
-        bulk_store(tile + TILE_PT, smem_u32(sm + P_KQ + 8192), 8192);  // Pt
+        if (p.keep_tiles) {
+            bulk_store_hint(tile + TILE_NEGW, smem_u32(sm + P_TP), 16384, keep_pol);   // -W, both blocks
+            bulk_store_hint(tile + TILE_PT, smem_u32(sm + P_KQ + 8192), 8192, keep_pol);  // Pt
+        } else {
+            bulk_store(tile + TILE_NEGW, smem_u32(sm + P_TP), 16384);
+            bulk_store(tile + TILE_PT, smem_u32(sm + P_KQ + 8192), 8192);
+        }
         bulk_commit_wait_read();
     }
     if (!ok && p.err) atomicCAS(p.err, 0, 52);
@@ -947,10 +986,12 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
 
     // The copies of local chunk n into its stage (K and V boxes, the prep
     // tile or the part of it a transition range reads), completing on the
-    // stage's FULL barrier.  A transition range reads K, V, -W and T'' of
-    // chunks that the output pass reads again after the combine: it keeps them
-    // in L2 (evict_last); the output pass reads them for the last time.
-    auto issue_stage = [&](int n, uint64_t pol) {
+    // stage's FULL barrier.  L2 policies: a transition range keeps what the
+    // output pass reads again (ptile, evict_last): the tiles, and also K and V
+    // (pin) when the tiles are too many to stay in L2 from the prep kernel on;
+    // otherwise the inputs are streamed (evict_first) so that the kept tiles
+    // stay, and the output pass drops each tile unwritten once it is read.
+    auto issue_stage = [&](int n, uint64_t pin, uint64_t ptile) {
         const int s = n % NST;
         const uint32_t st = smem_u32(sm + s * Lay::STAGE);
         const int z = (int)(bos + (int64_t)(cb + n) * C);
@@ -958,19 +999,19 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
         const uint8_t *tile = p.tiles + ((size_t)(gc0 + n) * H + h) * kTileBytes;
         mbar_arrive_expect_tx(full, Lay::LOADED);
         for (int kb = 0; kb < 2; ++kb) {
-            tma_load_3d_hint(st + Lay::K + kb * Lay::KB, &p.map_k, kb * 64, h, z, full, pol);
-            tma_load_3d_hint(st + Lay::V + kb * 8192, &p.map_v, kb * 64, h, z, full, pol);
+            tma_load_3d_hint(st + Lay::K + kb * Lay::KB, &p.map_k, kb * 64, h, z, full, pin);
+            tma_load_3d_hint(st + Lay::V + kb * 8192, &p.map_v, kb * 64, h, z, full, pin);
             if (MODE == MODE_OUT)
-                tma_load_3d_hint(st + ChainLayout<0>::Q + kb * ChainLayout<0>::KB, &p.map_q, kb * 64, h, z, full, pol);
+                tma_load_3d_hint(st + ChainLayout<0>::Q + kb * ChainLayout<0>::KB, &p.map_q, kb * 64, h, z, full, pin);
         }
         if (n == 0 && p.wait_tiles) grid_dep_wait();   // tiles come from the prep kernel
         if (MODE == MODE_TRANS) {   // -W and T'': the tile's first 24 KB
-            bulk_load_hint(st + ChainLayout<1>::W, tile, TILE_PT, full, pol);
+            bulk_load_hint(st + ChainLayout<1>::W, tile, TILE_PT, full, ptile);
         } else {                    // -W per block after K and Q, then T'' and Pt
             for (int kb = 0; kb < 2; ++kb)
                 bulk_load_hint(st + ChainLayout<0>::NEGW + kb * ChainLayout<0>::KB, tile + TILE_NEGW + kb * 8192,
-                               8192, full, pol);
-            bulk_load_hint(st + ChainLayout<0>::TPP, tile + TILE_TPP, 16384, full, pol);   // T'', Pt
+                               8192, full, ptile);
+            bulk_load_hint(st + ChainLayout<0>::TPP, tile + TILE_TPP, 16384, full, ptile);   // T'', Pt
         }
     };
     // When nothing upstream still writes this kernel's inputs (an output
@@ -991,8 +1032,9 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
         tma_prefetch_desc(&p.map_k);
         tma_prefetch_desc(&p.map_v);
         if (MODE == MODE_OUT) tma_prefetch_desc(&p.map_q);
-        const uint64_t pol0 = MODE == MODE_TRANS ? l2_evict_last_policy() : l2_evict_first_policy();
-        for (int n = 0; n < n_early; ++n) issue_stage(n, pol0);
+        const uint64_t pin = MODE == MODE_TRANS && !p.keep_tiles ? l2_evict_last_policy() : l2_evict_first_policy();
+        const uint64_t ptile = MODE == MODE_TRANS ? l2_evict_last_policy() : l2_evict_first_policy();
+        for (int n = 0; n < n_early; ++n) issue_stage(n, pin, ptile);
     }
     if (warp == 8) {
         tmem_alloc(smem_u32(tmem_base_ptr), TM_COLS);
@@ -1036,7 +1078,8 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
     } else if (warp == 9) {
         // ------------------------------------------------------------ TMA / bulk producer
         if (lane == 0) {
-            const uint64_t l2pol = MODE == MODE_TRANS ? l2_evict_last_policy() : l2_evict_first_policy();
+            const uint64_t pin = MODE == MODE_TRANS && !p.keep_tiles ? l2_evict_last_policy() : l2_evict_first_policy();
+            const uint64_t ptile = MODE == MODE_TRANS ? l2_evict_last_policy() : l2_evict_first_policy();
             int issued[NST] = {};
             for (int s = 0; s < n_early; ++s) issued[s] = 1;
             // Pull chunk m's data into L2 while its stage is still in use, so
@@ -1059,7 +1102,7 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                     prefetch(n);   // (the tiles are complete: the wait below chunk 0's loads came first)
                     if (!mbar_wait(bar(CB_EMPTY + s), ((n - NST) / NST) & 1, lim, abort_flag)) { fail(61); break; }
                 }
-                issue_stage(n, l2pol);
+                issue_stage(n, pin, ptile);
                 ++issued[s];
             }
             const int zero = 0;   // no copy may still be landing in shared memory at exit
@@ -1383,6 +1426,12 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
                 mbar_arrive(bar(CB_OFREE));   // the MMA thread may accumulate chunk n+1's O1^T
             }
             named_bar_sync(3, kOut);
+            if (p.keep_tiles) {
+                // chunk n's prep tile, kept in L2, has been read for the last time
+                // (its copies completed before c2(n)): drop it without a write-back
+                const uint8_t *tl = p.tiles + ((size_t)(gc0 + n) * H + h) * kTileBytes;
+                for (int i = so; i < (int)(kTileBytes / 128); i += kOut) l2_discard_line(tl + 128 * i);
+            }
             // whole 16-byte pieces of the [64 t][128 dv] tile, rows t < len (a row
             // past 63 in the last pass is read as row 63, so that every lane takes
             // part in the shuffles, and not stored)
@@ -1681,6 +1730,8 @@ bool make_token_map(CUtensorMap *m, const void *base, int64_t T, int H) {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+constexpr size_t kKeepTileBytes = (size_t)96 << 20;   // tiles kept in L2 up to this size
+
 size_t chunk_off_bytes(int num_seqs) { return align_up(4 * (size_t)(num_seqs + 1), 1024); }
 
 // units of the range-transition arrays (R, M, start states)
@@ -1825,6 +1876,9 @@ cudaError_t launch_prefill_tc(const TcLaunch &L, cudaStream_t stream) {
     pp.uniform_len = cp.uniform_len = L.uniform_len;
     pp.cps = cp.cps = cps;
     pp.num_seqs = L.num_seqs;
+    // tiles of at most three quarters of the 126 MB L2 stay there from the prep
+    // kernel to the chain passes (evict_last); larger sets stream
+    pp.keep_tiles = cp.keep_tiles = (size_t)bound * L.H * kTileBytes <= kKeepTileBytes ? 1 : 0;
     pp.H = cp.H = L.H;
     pp.tiles = tiles;
     cp.tiles = tiles;
