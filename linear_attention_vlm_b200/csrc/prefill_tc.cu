@@ -1561,16 +1561,25 @@ gdn_chunk_chain_kernel(const __grid_constant__ ChainParams p) {
 // keeps about 16 mantissa bits; accumulation is fp32.  M_j arrives already
 // split from the transition ranges (bf16 hi and lo rows [k][n], each row's
 // 16-byte pieces swizzled by row % 8) and ldmatrix (.trans) turns its rows into
-// B fragments.  M_{j+1} and this CTA's rows of R_{j+1} stream into the other
-// half of a double buffer as bulk copies (one thread, an mbarrier) while step
-// j computes.
+// B fragments.  S_{j+1} is split once, by the warp that computes it, into bf16
+// hi and lo rows, from which every warp takes its A fragments with ldmatrix.
+// M_{j+1} and this CTA's rows of R_{j+1} stream into the other half of a
+// double buffer as bulk copies (one thread, an mbarrier) while step j computes.
 constexpr int kCombRows = 16;
 constexpr int kCombThreads = 256;
-constexpr int kCombSP = 136;                                    // row pitch: conflict-free fragments
+constexpr int kCombAP = 136;                                    // bf16 row pitch of S: conflict-free ldmatrix
+constexpr uint32_t kCombSBytes = 2 * kCombRows * kCombAP * 2;   // one S buffer: hi rows, then lo rows
 constexpr uint32_t kCombMBytes = 2 * D * D * 2;                 // M_j: hi and lo bf16 rows
 constexpr uint32_t kCombRBytes = kCombRows * D * 4;             // 16 rows of R_j
 constexpr uint32_t kCombBufBytes = kCombMBytes + kCombRBytes;
-constexpr size_t kCombSmem = (size_t)2 * kCombBufBytes + (size_t)2 * kCombRows * kCombSP * 4 + 64;
+constexpr size_t kCombSmem = (size_t)2 * kCombBufBytes + (size_t)2 * kCombSBytes + 64;
+
+// four 8x8 bf16 blocks as they are stored: the row-major A fragments of mma.sync
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const __nv_bfloat16 *row) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(row)));
+}
 
 // four 8x8 bf16 blocks, transposed on the way: the col-major B fragments of mma.sync
 __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const __nv_bfloat16 *row) {
@@ -1593,9 +1602,9 @@ gdn_scan_combine_kernel(const float *__restrict__ state_in, const float *__restr
                         const float *__restrict__ trans_m, float *__restrict__ seg_start, int nseg,
                         int *err, uint64_t timeout_ns, uint64_t drain_ns) {
     extern __shared__ __align__(128) uint8_t smc[];
-    // [buffer 0: M hi, M lo, R rows][buffer 1: the same][S rows, two buffers][2 mbarriers, abort flag]
-    float *Ss = reinterpret_cast<float *>(smc + 2 * kCombBufBytes);   // S_j rows [2][16][D] (pitch kCombSP)
-    uint8_t *ctl = reinterpret_cast<uint8_t *>(Ss + 2 * kCombRows * kCombSP);
+    // [buffer 0: M hi, M lo, R rows][buffer 1: the same][S hi and lo rows, two buffers][2 mbarriers, abort flag]
+    __nv_bfloat16 *Ss = reinterpret_cast<__nv_bfloat16 *>(smc + 2 * kCombBufBytes);   // [2][hi, lo][16][kCombAP]
+    uint8_t *ctl = smc + 2 * kCombBufBytes + 2 * kCombSBytes;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(ctl + 16);
     auto bar = [&](int b) { return smem_u32(ctl + 8 * b); };
     const int nh = blockIdx.x, r0 = blockIdx.y * kCombRows;
@@ -1620,16 +1629,24 @@ gdn_scan_combine_kernel(const float *__restrict__ state_in, const float *__restr
     int pending = -1;   // the last step whose copies were issued and not yet waited for
     if (nseg > 1 && t == 0) stage(0);
     if (nseg > 1) pending = 0;
-    for (int i = t; i < kCombRows * D; i += kCombThreads)
-        Ss[(i >> 7) * kCombSP + (i & 127)] =
-            state_in ? state_in[(size_t)nh * D * D + (size_t)(r0 + (i >> 7)) * D + (i & 127)] : 0.f;
+    // S_0: this CTA's rows of the initial state, split into buffer 0
+    for (int i = t; i < kCombRows * D / 2; i += kCombThreads) {
+        const int row = i >> 6, col = 2 * (i & 63);
+        const float2 v = state_in ? *reinterpret_cast<const float2 *>(state_in + (size_t)nh * D * D +
+                                                                       (size_t)(r0 + row) * D + col)
+                                  : make_float2(0.f, 0.f);
+        uint32_t hi, lo;
+        split2(v.x, v.y, hi, lo);
+        *reinterpret_cast<uint32_t *>(Ss + row * kCombAP + col) = hi;
+        *reinterpret_cast<uint32_t *>(Ss + (kCombRows + row) * kCombAP + col) = lo;
+    }
     for (int j = 0; j + 1 < nseg; ++j) {
         const size_t u = ((size_t)nh * (nseg - 1) + j) * D * D + (size_t)r0 * D;   // rows r0.. of step j
-        float acc[2][4], accx[2][4];   // hi*hi terms; the two cross terms
+        float acc[2][4], accx[2][4], accy[2][4];   // hi*hi terms; lo*hi; hi*lo
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[nt][e] = accx[nt][e] = 0.f;
+            for (int e = 0; e < 4; ++e) acc[nt][e] = accx[nt][e] = accy[nt][e] = 0.f;
         if (!mbar_wait(bar(j & 1), (j >> 1) & 1, timeout_ns, abort_flag)) {
             *abort_flag = 1;
             if (err) atomicCAS(err, 0, 81);
@@ -1647,20 +1664,17 @@ gdn_scan_combine_kernel(const float *__restrict__ state_in, const float *__restr
         const __nv_bfloat16 *Mh = reinterpret_cast<const __nv_bfloat16 *>(smc + (j & 1) * kCombBufBytes);
         const __nv_bfloat16 *Ml = Mh + D * D;
         const float *Rs = reinterpret_cast<const float *>(smc + (j & 1) * kCombBufBytes + kCombMBytes);
-        const float *Sc = Ss + (j & 1) * kCombRows * kCombSP;          // S_j
-        float *Sn = Ss + ((j + 1) & 1) * kCombRows * kCombSP;          // S_{j+1}
+        const __nv_bfloat16 *Sc = Ss + (j & 1) * (kCombSBytes / 2);         // S_j: hi rows, lo rows
+        __nv_bfloat16 *Sn = Ss + ((j + 1) & 1) * (kCombSBytes / 2);         // S_{j+1}
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
             const int k0 = 16 * ks;
+            // lane -> row lane & 15 of the 16-row block, columns k0 + 8 (lane >> 4) ..: the four
+            // 8x8 blocks {rows 0-7, 8-15} x {k0, k0 + 8} are the A fragments {a0, a1, a2, a3}
+            const int aoff = (lane & 15) * kCombAP + k0 + 8 * (lane >> 4);
             uint32_t ah[4], al[4];
-            const float2 s00 = *reinterpret_cast<const float2 *>(Sc + g * kCombSP + k0 + 2 * q);
-            const float2 s10 = *reinterpret_cast<const float2 *>(Sc + (g + 8) * kCombSP + k0 + 2 * q);
-            const float2 s01 = *reinterpret_cast<const float2 *>(Sc + g * kCombSP + k0 + 2 * q + 8);
-            const float2 s11 = *reinterpret_cast<const float2 *>(Sc + (g + 8) * kCombSP + k0 + 2 * q + 8);
-            split2(s00.x, s00.y, ah[0], al[0]);
-            split2(s10.x, s10.y, ah[1], al[1]);
-            split2(s01.x, s01.y, ah[2], al[2]);
-            split2(s11.x, s11.y, ah[3], al[3]);
+            ldmatrix_x4(ah, Sc + aoff);
+            ldmatrix_x4(al, Sc + kCombRows * kCombAP + aoff);
             // lane -> row of one of four 8x8 blocks: k0 + (lane & 7) + 8 ((lane >> 3) & 1),
             // 16-byte piece 2 w + (lane >> 4) of that row (stored at piece ^ (row % 8));
             // .trans turns them into the B fragments {b0, b1} of n-tiles 0 and 1
@@ -1672,7 +1686,7 @@ gdn_scan_combine_kernel(const float *__restrict__ state_in, const float *__restr
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
                 mma_bf16_16816(accx[nt], al[0], al[1], al[2], al[3], bh[2 * nt], bh[2 * nt + 1]);
-                mma_bf16_16816(accx[nt], ah[0], ah[1], ah[2], ah[3], bl[2 * nt], bl[2 * nt + 1]);
+                mma_bf16_16816(accy[nt], ah[0], ah[1], ah[2], ah[3], bl[2 * nt], bl[2 * nt + 1]);
                 mma_bf16_16816(acc[nt], ah[0], ah[1], ah[2], ah[3], bh[2 * nt], bh[2 * nt + 1]);
             }
         }
@@ -1682,12 +1696,19 @@ gdn_scan_combine_kernel(const float *__restrict__ state_in, const float *__restr
             const int col = 16 * warp + 8 * nt + 2 * q;
             const float2 ra = *reinterpret_cast<const float2 *>(Rs + g * D + col);
             const float2 rb = *reinterpret_cast<const float2 *>(Rs + (g + 8) * D + col);
-            const float2 va = make_float2(acc[nt][0] + accx[nt][0] + ra.x, acc[nt][1] + accx[nt][1] + ra.y);
-            const float2 vb = make_float2(acc[nt][2] + accx[nt][2] + rb.x, acc[nt][3] + accx[nt][3] + rb.y);
+            const float2 va = make_float2(acc[nt][0] + (accx[nt][0] + accy[nt][0]) + ra.x,
+                                          acc[nt][1] + (accx[nt][1] + accy[nt][1]) + ra.y);
+            const float2 vb = make_float2(acc[nt][2] + (accx[nt][2] + accy[nt][2]) + rb.x,
+                                          acc[nt][3] + (accx[nt][3] + accy[nt][3]) + rb.y);
             *reinterpret_cast<float2 *>(seg_start + u + g * D + col) = va;
             *reinterpret_cast<float2 *>(seg_start + u + (g + 8) * D + col) = vb;
-            *reinterpret_cast<float2 *>(Sn + g * kCombSP + col) = va;
-            *reinterpret_cast<float2 *>(Sn + (g + 8) * kCombSP + col) = vb;
+            uint32_t hi, lo;
+            split2(va.x, va.y, hi, lo);
+            *reinterpret_cast<uint32_t *>(Sn + g * kCombAP + col) = hi;
+            *reinterpret_cast<uint32_t *>(Sn + (kCombRows + g) * kCombAP + col) = lo;
+            split2(vb.x, vb.y, hi, lo);
+            *reinterpret_cast<uint32_t *>(Sn + (g + 8) * kCombAP + col) = hi;
+            *reinterpret_cast<uint32_t *>(Sn + (kCombRows + g + 8) * kCombAP + col) = lo;
         }
     }
     // no bulk copy may still be landing in shared memory at exit
