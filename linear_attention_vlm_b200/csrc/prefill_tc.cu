@@ -1666,28 +1666,31 @@ gdn_scan_combine_kernel(const float *__restrict__ state_in, const float *__restr
         const float *Rs = reinterpret_cast<const float *>(smc + (j & 1) * kCombBufBytes + kCombMBytes);
         const __nv_bfloat16 *Sc = Ss + (j & 1) * (kCombSBytes / 2);         // S_j: hi rows, lo rows
         __nv_bfloat16 *Sn = Ss + ((j + 1) & 1) * (kCombSBytes / 2);         // S_{j+1}
+        // without an initial state S_0 = 0, so S_1 = R_0: the first step has no products
+        if (j > 0 || state_in) {
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-            const int k0 = 16 * ks;
-            // lane -> row lane & 15 of the 16-row block, columns k0 + 8 (lane >> 4) ..: the four
-            // 8x8 blocks {rows 0-7, 8-15} x {k0, k0 + 8} are the A fragments {a0, a1, a2, a3}
-            const int aoff = (lane & 15) * kCombAP + k0 + 8 * (lane >> 4);
-            uint32_t ah[4], al[4];
-            ldmatrix_x4(ah, Sc + aoff);
-            ldmatrix_x4(al, Sc + kCombRows * kCombAP + aoff);
-            // lane -> row of one of four 8x8 blocks: k0 + (lane & 7) + 8 ((lane >> 3) & 1),
-            // 16-byte piece 2 w + (lane >> 4) of that row (stored at piece ^ (row % 8));
-            // .trans turns them into the B fragments {b0, b1} of n-tiles 0 and 1
-            const int krow = k0 + (lane & 7) + 8 * ((lane >> 3) & 1);
-            const int off = krow * D + (((2 * warp + (lane >> 4)) ^ (krow & 7)) << 3);
-            uint32_t bh[4], bl[4];
-            ldmatrix_x4_trans(bh, Mh + off);
-            ldmatrix_x4_trans(bl, Ml + off);
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const int k0 = 16 * ks;
+                // lane -> row lane & 15 of the 16-row block, columns k0 + 8 (lane >> 4) ..: the four
+                // 8x8 blocks {rows 0-7, 8-15} x {k0, k0 + 8} are the A fragments {a0, a1, a2, a3}
+                const int aoff = (lane & 15) * kCombAP + k0 + 8 * (lane >> 4);
+                uint32_t ah[4], al[4];
+                ldmatrix_x4(ah, Sc + aoff);
+                ldmatrix_x4(al, Sc + kCombRows * kCombAP + aoff);
+                // lane -> row of one of four 8x8 blocks: k0 + (lane & 7) + 8 ((lane >> 3) & 1),
+                // 16-byte piece 2 w + (lane >> 4) of that row (stored at piece ^ (row % 8));
+                // .trans turns them into the B fragments {b0, b1} of n-tiles 0 and 1
+                const int krow = k0 + (lane & 7) + 8 * ((lane >> 3) & 1);
+                const int off = krow * D + (((2 * warp + (lane >> 4)) ^ (krow & 7)) << 3);
+                uint32_t bh[4], bl[4];
+                ldmatrix_x4_trans(bh, Mh + off);
+                ldmatrix_x4_trans(bl, Ml + off);
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                mma_bf16_16816(accx[nt], al[0], al[1], al[2], al[3], bh[2 * nt], bh[2 * nt + 1]);
-                mma_bf16_16816(accy[nt], ah[0], ah[1], ah[2], ah[3], bl[2 * nt], bl[2 * nt + 1]);
-                mma_bf16_16816(acc[nt], ah[0], ah[1], ah[2], ah[3], bh[2 * nt], bh[2 * nt + 1]);
+                for (int nt = 0; nt < 2; ++nt) {
+                    mma_bf16_16816(accx[nt], al[0], al[1], al[2], al[3], bh[2 * nt], bh[2 * nt + 1]);
+                    mma_bf16_16816(accy[nt], ah[0], ah[1], ah[2], ah[3], bl[2 * nt], bl[2 * nt + 1]);
+                    mma_bf16_16816(acc[nt], ah[0], ah[1], ah[2], ah[3], bh[2 * nt], bh[2 * nt + 1]);
+                }
             }
         }
         // S_{j+1} = S_j M_j + R_j: rows g and g + 8, columns 16 w + 8 nt + 2 q, + 1
