@@ -26,7 +26,7 @@
 //   state in TMEM: p3 U^T = V^T T''^T, (a + c1) [O1^T | U^T] += S [Q; -W]^T
 //   as ONE N = 128 MMA, (b) S += U^T K, c2 O2^T = U^T Pt^T -- M = 128
 //   tcgen05 MMAs, the S and U^T operands read from TMEM -- with a four-warp
-//   state group (residual and state epilogues, the serial chain), a four-warp
+//   state group (residual and state epilogues, the serial chain), a six-warp
 //   output group (o_t = gamma_t O1_t + O2_t, off the chain), one MMA thread
 //   and one TMA thread.  The state never leaves the SM between chunks.  A
 //   tcgen05.mma costs its issuing thread some 60 cycles whatever its width,
@@ -1618,12 +1618,15 @@ gdn_scan_combine_kernel(const float *__restrict__ state_in, const float *__restr
     __syncthreads();
     grid_dep_wait();     // the transitions come from the previous kernel
     grid_dep_launch();   // the output pass may launch; its first ranges do not need this grid
+    // without an initial state S_0 = 0, so S_1 = R_0: step 0 neither reads M_0 nor forms products
+    auto has_products = [&](int j) { return j > 0 || state_in != nullptr; };
     auto stage = [&](int j) {   // thread 0
         const size_t unit = ((size_t)nh * (nseg - 1) + j) * D * D;
         const uint32_t dst = smem_u32(smc + (j & 1) * kCombBufBytes);
-        mbar_arrive_expect_tx(bar(j & 1), kCombBufBytes);
-        for (uint32_t o = 0; o < kCombMBytes; o += 16384)
-            bulk_load(dst + o, reinterpret_cast<const uint8_t *>(trans_m + unit) + o, 16384, bar(j & 1));
+        mbar_arrive_expect_tx(bar(j & 1), has_products(j) ? kCombBufBytes : kCombRBytes);
+        if (has_products(j))
+            for (uint32_t o = 0; o < kCombMBytes; o += 16384)
+                bulk_load(dst + o, reinterpret_cast<const uint8_t *>(trans_m + unit) + o, 16384, bar(j & 1));
         bulk_load(dst + kCombMBytes, trans_r + unit + (size_t)r0 * D, kCombRBytes, bar(j & 1));
     };
     int pending = -1;   // the last step whose copies were issued and not yet waited for
@@ -1666,8 +1669,7 @@ gdn_scan_combine_kernel(const float *__restrict__ state_in, const float *__restr
         const float *Rs = reinterpret_cast<const float *>(smc + (j & 1) * kCombBufBytes + kCombMBytes);
         const __nv_bfloat16 *Sc = Ss + (j & 1) * (kCombSBytes / 2);         // S_j: hi rows, lo rows
         __nv_bfloat16 *Sn = Ss + ((j + 1) & 1) * (kCombSBytes / 2);         // S_{j+1}
-        // without an initial state S_0 = 0, so S_1 = R_0: the first step has no products
-        if (j > 0 || state_in) {
+        if (has_products(j)) {
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
                 const int k0 = 16 * ks;
