@@ -82,6 +82,7 @@ KERNEL_SOURCES = {
     "prefill": [os.path.join(_CSRC, f) for f in ("prefill_tc.cu", "prefill_tc.h", "sm100.cuh")],
     "swa": [os.path.join(_CSRC, f) for f in ("swa.cu", "sm100.cuh")],
     "decode": [os.path.join(_CSRC, "decode.cu")],
+    "layer": [os.path.join(_CSRC, "layer_ops.cu")],
 }
 
 
@@ -583,10 +584,12 @@ def run_native(args):
                                      note="part of the state can stay in the 126 MB L2 between steps")},
         "preprocess": {"metric": "pre-processing tokens/s (conv4 + SiLU + q/k L2 norm + gates), prefill shapes",
                        "value": aggregate_throughput(T, world, ms_pre), "unit": "tokens/s", "ms_per_step": ms_pre,
-                       "roofline": hbm_roofline("gdn_preprocess_kernel", pre_bytes, ms_pre)},
+                       "roofline": hbm_roofline("gdn_preprocess_kernel", pre_bytes, ms_pre,
+                                                traffic=measured_traffic("preprocess_prefill_shapes", "layer"))},
         "output_gate": {"metric": "output gate tokens/s (RMS norm + sigmoid gate), prefill shapes",
                         "value": aggregate_throughput(T, world, ms_gate), "unit": "tokens/s", "ms_per_step": ms_gate,
-                        "roofline": hbm_roofline("gdn_output_gate_kernel", gate_bytes, ms_gate)},
+                        "roofline": hbm_roofline("gdn_output_gate_kernel", gate_bytes, ms_gate,
+                                                 traffic=measured_traffic("output_gate_prefill_shapes", "layer"))},
         "layer": {"metric": "GDN layer token mixer tokens/s at the prefill shapes: raw projections -> "
                             "pre-processing -> recurrence -> output gate",
                   "value": aggregate_throughput(T, world, ms_layer_fused), "unit": "tokens/s",
