@@ -74,15 +74,17 @@ def peaks():
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per call or
 # launch, measured by ncu and recorded in profiles/dram_traffic.txt together
-# with a hash of the kernel's sources at the time of the capture.  A figure
-# whose sources have changed since is not reported (traffic: null).
+# with a hash of the kernel's sources at the time of the capture: its .cu file
+# and the headers whose device code it uses (the decode kernel takes only the
+# dtype conversions from gdn_internal.h).  A figure whose sources have changed
+# since is not reported (traffic: null).
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 _CSRC = os.path.join("linear_attention_vlm_b200", "csrc")
 KERNEL_SOURCES = {
-    "prefill": [os.path.join(_CSRC, f) for f in ("prefill_tc.cu", "prefill_tc.h", "sm100.cuh")],
-    "swa": [os.path.join(_CSRC, f) for f in ("swa.cu", "sm100.cuh")],
+    "prefill": [os.path.join(_CSRC, f) for f in ("prefill_tc.cu", "prefill_tc.h", "sm100.cuh", "gdn_internal.h")],
+    "swa": [os.path.join(_CSRC, f) for f in ("swa.cu", "sm100.cuh", "gdn_internal.h")],
     "decode": [os.path.join(_CSRC, "decode.cu")],
-    "layer": [os.path.join(_CSRC, "layer_ops.cu")],
+    "layer": [os.path.join(_CSRC, f) for f in ("layer_ops.cu", "gdn_internal.h")],
 }
 
 
