@@ -32,3 +32,27 @@ def test_algorithmic_bytes():
     assert bench.prefill_bytes(T, H, d, d, 1, with_state_in=True) == T * H * per + 2 * H * d * d * 4
     # decode: the state read and written once, one token in and out
     assert bench.decode_bytes(3, 2, d, d) == 3 * 2 * (2 * d * d * 4 + 3 * d * 2 + 8 + d * 2)
+
+
+def test_committed_traffic_records_are_well_formed():
+    """Every record names a key bench.py asks for, a 16-digit source hash,
+    a byte count and the profile summary it comes from; every key bench.py
+    asks for has a record."""
+    import os
+    import re
+    src = open(os.path.join(bench.ROOT, "bench.py")).read()
+    asked = set(re.findall(r'measured_traffic\("([a-z0-9_]+)", "([a-z]+)"\)', src))
+    keys = {}
+    with open(bench.TRAFFIC_FILE) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            key, h, nbytes, what = line.split(None, 3)
+            assert re.fullmatch(r"[0-9a-f]{16}", h), line
+            assert float(nbytes) > 0, line
+            ref = re.search(r"\(([\w.]+\.md)\)\s*$", what)
+            assert ref and os.path.exists(os.path.join(bench.ROOT, "profiles", ref.group(1))), line
+            keys[key] = h
+    for key, kind in asked:
+        assert kind in bench.KERNEL_SOURCES, (key, kind)
+        assert key in keys, key
